@@ -1,0 +1,325 @@
+"""Benchmark of the neighbor-list hot path on B200.
+
+One step = nl_sort_hilbert + nl_build + nl_skin_check on the 10.29M-atom
+salt-solution workload (rigid water + 0.15 M NaCl on 151^3 sites, cutoff
+5.75 A, skin 1.0 A, capacity 256), inputs resident in HBM.  Prints one JSON
+line (rank 0).  `--impl reference` times the CPU oracle instead, on a
+bounded sample of the same workload recipe.
+
+Multi-GPU: the path does not shard across GPUs in this build (one problem per
+GPU), so `--gpus N` under torchrun runs N independent replicas; `value` is
+the atoms of all replicas over the slowest replica's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "neighbor-list build atoms/s and pairs/s at 1 B200; % of HBM roofline"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(steps: int = 1) -> dict:
+    """The CPU oracle, as it stands, on a bounded sample of the salt-solution
+    recipe (60^3 sites, ~0.65M atoms): curve sort + neighbor list + skin
+    check per step, single-threaded."""
+    import oracle
+    from neighbor_list_construction_b200 import workloads
+    w = workloads.make("saltwater_n60", seed=4)
+    oracle.lib()
+    t0 = time.perf_counter()
+    pairs = 0
+    for _ in range(steps):
+        perm, _ = oracle.sort(w.pos, w.box)
+        ps = w.pos[perm]
+        nbr, cnt, _ = oracle.build(ps, w.box, w.cutoff, w.skin, w.capacity)
+        oracle.skin_check(ps, ps, w.box, w.skin)
+        pairs += int(cnt.sum())
+    dt = time.perf_counter() - t0
+    return {"value": steps * w.n / dt, "unit": "atoms/s", "cores": 1, "kind": "oracle",
+            "sample": f"{w.n} atoms, salt-solution recipe on 60^3 sites (same density, "
+                      f"cutoff 5.75, skin 1.0, capacity 256), sort+build+skin x{steps}, "
+                      f"{dt:.1f} s single-threaded",
+            "pairs_per_s": pairs / dt, "seconds": dt}
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    steps = max(1, min(args.steps, 3))
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample(1)
+    r = oracle_sample(steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "atoms/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * r["seconds"] / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "saltwater10m recipe, bounded sample", "parallelism": "replicas"},
+        "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "e2e": {"value": r["value"], "unit": "atoms/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "pairs_per_s": r["pairs_per_s"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+    from neighbor_list_construction_b200 import nl, workloads
+
+    torch.cuda.set_device(local_rank)
+    w = workloads.make(args.workload)
+    n, K = w.n, w.capacity
+    box = w.box
+    pos_host = torch.from_numpy(w.pos).pin_memory()
+    pos = pos_host.cuda()
+    ctx = nl.Context(n, K)
+    h = ctx.handle
+    perm = torch.empty(n, dtype=torch.int32, device="cuda")
+    ps = torch.empty(n, 4, dtype=torch.float32, device="cuda")
+    nbr = torch.empty(n, K, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(n, dtype=torch.int32, device="cuda")
+    rb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cnt_host = torch.empty(n, dtype=torch.int32).pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def step(src):
+        nl.nl_sort_hilbert(h, src, box, perm, ps, None, stream)
+        nl.nl_build(h, ps, box, w.cutoff, w.skin, K, nbr, cnt, stream)
+        nl.nl_skin_check(h, ps, box, w.skin, rb, None, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(pos)
+    st = ctx.sync_status()
+    if st < 0:
+        raise RuntimeError(nl.nl_status_string(st))
+    info = nl.nl_last_build_info(h)
+    pairs = int(cnt.to(torch.int64).sum().item())
+    nl.nl_profile_read(h)
+
+    # ---- device-resident timed region
+    clocks = ClockSampler(local_rank)
+    nl.nl_profile_enable(h, True)
+    barrier()
+    clocks.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(pos)
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    phases = nl.nl_profile_read(h)
+    nl.nl_profile_enable(h, False)
+    ms_max = max_over_ranks(ms)
+
+    # ---- end to end through the public API with host buffers
+    barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        pos.copy_(pos_host, non_blocking=True)
+        step(pos)
+        cnt_host.copy_(cnt, non_blocking=True)
+    f1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps)
+    st = ctx.sync_status()
+
+    if rank == 0:
+        peaks = measured_peaks()
+        pair_ms, pair_launches = phases.get("pair_search", (0.0, 0))
+        fb_ms, fb_launches = phases.get("pair_search_per_atom", (0.0, 0))
+        dom = "pair_search" if pair_launches else "pair_search_per_atom"
+        dom_ms = (pair_ms / pair_launches) if pair_launches else (fb_ms / max(fb_launches, 1))
+        bytes_per_atom = 16 + 4 * K + 4
+        alg_bytes = n * bytes_per_atom
+        achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
+        build_ms = sum(phases.get(p, (0.0, 0))[0] for p in
+                       ("bin_count", "cell_scan", "bin_scatter", "cell_sort", "pair_search",
+                        "pair_search_per_atom")) / args.steps
+        sort_ms = sum(phases.get(p, (0.0, 0))[0] for p in
+                      ("keys", "key_scan", "radix_sort", "gather")) / args.steps
+        launches_per_step = sum(v[1] for v in phases.values()) / args.steps
+        line = {
+            "metric": METRIC,
+            "value": world * n / (ms_max * 1e-3),
+            "unit": "atoms/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {w.description}", "atoms": n,
+                       "cutoff": w.cutoff, "skin": w.skin, "capacity": K,
+                       "step": "nl_sort_hilbert + nl_build + nl_skin_check",
+                       "cells": info[:3], "staged_pair_kernel": bool(info[3]),
+                       "l2": "inputs larger than L2 (positions 165 MB, rows "
+                             f"{n * K * 4 / 1e9:.1f} GB per step)",
+                       "parallelism": "replicas" if world > 1 else "single"},
+            "pairs_per_s": world * pairs / (ms_max * 1e-3),
+            "directed_pairs": pairs,
+            "build": {"ms": build_ms, "atoms_per_s": n / (build_ms * 1e-3),
+                      "pairs_per_s": pairs / (build_ms * 1e-3),
+                      "bytes": alg_bytes,
+                      "frac_of_8TBs": alg_bytes / (build_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+                      "frac_of_measured": alg_bytes / (build_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "sort_ms": sort_ms,
+            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved,
+                         "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": None,
+                         "bytes_per_atom": bytes_per_atom, "launch_ms": dom_ms},
+            "phases_ms": {k: v[0] / args.steps for k, v in phases.items() if v[1]},
+            "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "atoms/s",
+                    "h2d_bytes_per_step": n * 16, "d2h_bytes_per_step": n * 4,
+                    "ms_per_step": e2e_ms},
+            "clocks": clk,
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "status": nl.nl_status_string(st),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            cb = oracle_sample(1)
+            line["cpu_baseline"] = {"value": cb["value"], "unit": "atoms/s", "cores": cb["cores"],
+                                    "kind": "oracle", "sample": cb["sample"]}
+        print(json.dumps(line), flush=True)
+    ctx.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="saltwater10m")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

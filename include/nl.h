@@ -1,0 +1,161 @@
+/*
+ * nl.h -- C ABI of libnl.so, the B200 (sm_100a) periodic neighbor-list build.
+ *
+ * Method source: "Ab Initio Accuracy Beyond the Cutoff: Distributed
+ * Message-Passing Equivariant Attention at Tens-of-Millions-of-Atom Scale"
+ * (Tessera), abstract.  The runtime described there sorts atoms along a
+ * space-filling curve, searches neighbors through a multi-level structure,
+ * keeps tensor shapes fixed between rebuilds with a conservative neighbor
+ * skin, and replays each rebuild interval as one CUDA Graph.  The pages give
+ * no formulas or API; the definitions below are this library's readings.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Positions      `pos` is a DEVICE pointer to n x 4 floats (float4 per atom,
+ *                16-byte aligned): x, y, z in angstrom; the 4th float is
+ *                ignored on input.  Coordinates must be finite; they may lie
+ *                outside the box (they are wrapped, see below).
+ * Box            `box` is a HOST pointer to 3 floats (Lx, Ly, Lz), an
+ *                orthorhombic periodic box with its corner at the origin.
+ * Wrap           w = x - L*floor(x/L) in fp32, then one fold into [0, L)
+ *                (add L if negative, subtract L if >= L, 0 if still outside).
+ * Distance       d = w_j - w_i; d = d - L*rintf(d/L) per axis;
+ *                r2 = (dx*dx + dy*dy) + dz*dz, every operation an fp32
+ *                round-to-nearest-even without fused multiply-add.
+ * Neighbors      N(i) = { j != i : r2 < rl*rl }, rl = fl(cutoff + skin),
+ *                strict inequality; a full (directed) list.
+ * Streams        `stream` is a cudaStream_t (NULL = the legacy default
+ *                stream).  Every call only enqueues work on it and returns;
+ *                no call synchronizes except nl_sync_status.
+ * Ownership      all array arguments are caller-owned device buffers; the
+ *                context owns all scratch.  After nl_create no call
+ *                allocates device memory.
+ * Errors         the return value reports argument and launch errors only.
+ *                Conditions found on the device (row overflow, a bounded
+ *                spin that gave up) are accumulated in the context and
+ *                returned, then cleared, by nl_sync_status.
+ */
+#ifndef NL_H
+#define NL_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct nl_ctx nl_ctx;
+
+typedef enum {
+    NL_OK = 0,
+    NL_OVERFLOW = 1,       /* some atom has more than `capacity` neighbors:
+                              counts are true counts, such rows hold `capacity`
+                              of them, every other row is complete */
+    NL_ERR_ARG = -1,       /* NULL pointer, n < 0, bad float, misaligned pos */
+    NL_ERR_BOX = -2,       /* box narrower than three cells of width rl on
+                              some axis (a cell must be at least rl wide) */
+    NL_ERR_CUDA = -3,      /* a CUDA runtime call failed */
+    NL_ERR_TIMEOUT = -4,   /* a bounded device-side wait gave up; results of
+                              that call are not valid */
+    NL_ERR_CAPACITY = -5   /* n > max_atoms or capacity > max_capacity */
+} nl_status;
+
+/* Creates a context on the current CUDA device and allocates all scratch for
+ * up to `max_atoms` atoms (<= 2^30) and rows of up to `max_capacity`
+ * neighbors.  Returns NL_ERR_CUDA if the allocation fails. */
+nl_status nl_create(nl_ctx **ctx, int64_t max_atoms, int32_t max_capacity);
+
+/* Frees the context and its scratch.  Waits for the context's work. */
+void nl_destroy(nl_ctx *ctx);
+
+/* Space-filling-curve order (Tessera abstract: atoms are sorted along a
+ * space-filling curve).  Per atom: wrap, quantize each axis to 21 bits as
+ * q = min(floor(w * fl(2^21/L)), 2^21-1), form the 63-bit 3-D Hilbert index
+ * of (qx, qy, qz) (J. Skilling, "Programming the Hilbert curve", 2004:
+ * axes-to-transpose, index bits from the top level down, x first in each
+ * triple), then sort (key, original index) pairs ascending with a stable
+ * LSD radix sort, so equal keys keep index order.
+ * Outputs (device): perm_out[k] = original index of the k-th atom (int32,
+ * n entries); pos_sorted_out[k] = (x, y, z of atom perm_out[k] as given,
+ * 4th float = perm_out[k] as int32 bits) (n float4); keys_out[k] = its key
+ * (uint64, may be NULL). */
+nl_status nl_sort_hilbert(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                          int32_t *perm_out, float *pos_sorted_out, uint64_t *keys_out,
+                          void *stream);
+
+/* As nl_sort_hilbert with the Morton (Z-order) key instead: key bit 3l+2 =
+ * bit l of qx, 3l+1 = qy, 3l = qz.  The baseline order the Tessera abstract
+ * compares against. */
+nl_status nl_sort_morton(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                         int32_t *perm_out, float *pos_sorted_out, uint64_t *keys_out,
+                         void *stream);
+
+/* Fixed-capacity neighbor list (Tessera abstract: workload shapes fixed
+ * between rebuilds; neighbor search through curve order, cells and pairs).
+ * Outputs (device): nbr_out is n x capacity int32, row-major; row i holds
+ * the indices (into `pos`) of N(i) in an unspecified order, then -1 up to
+ * `capacity`; if |N(i)| > capacity the row holds `capacity` members of N(i).
+ * counts_out[i] = |N(i)| (true count, int32).  Also snapshots `pos` as the
+ * reference positions of nl_skin_check.  Requires every box side to hold at
+ * least three cells of width rl (else NL_ERR_BOX); rl <= 0 or capacity < 1
+ * is NL_ERR_ARG. */
+nl_status nl_build(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                   float cutoff, float skin, int32_t capacity,
+                   int32_t *nbr_out, int32_t *counts_out, void *stream);
+
+/* Skin check (Tessera abstract: a conservative neighbor skin preserves the
+ * topology across updates).  m = max over atoms of the squared minimum-image
+ * displacement between `pos` and the positions of the last nl_build (raw,
+ * unwrapped coordinates, same fp32 formula as above);
+ * *rebuild_out = (m > fl(h*h)) with h = fl(skin * 0.5), strict.
+ * rebuild_out: device int32[1]; max_d2_out: device float[1] or NULL.
+ * `n` must equal the n of the last nl_build. */
+nl_status nl_skin_check(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                        float skin, int32_t *rebuild_out, float *max_d2_out, void *stream);
+
+/* One rebuild interval replayed as one CUDA Graph (Tessera abstract: each
+ * rebuild interval replays as one CUDA Graph).  Runs n_steps iterations of
+ *     [step_graph] -> skin check -> if rebuild: nl_build (same arguments)
+ * inside a single graph launch (a conditional WHILE node around an IF node),
+ * and records decisions_out[t] = 1 if iteration t rebuilt, else 0 (device
+ * int32[n_steps]).  step_graph is a cudaGraph_t with the caller's per-step
+ * work (it may read the iteration index from nl_step_counter); NULL means no
+ * per-step work.  nl_build must have run on `pos` before (it sets the
+ * reference positions).  The executable graph is cached in the context and
+ * rebuilt when any argument changes. */
+nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps,
+                    int64_t n, float *pos, const float *box, float cutoff, float skin,
+                    int32_t capacity, int32_t *nbr, int32_t *counts,
+                    int32_t *decisions_out, void *stream);
+
+/* Device pointer to the 0-based iteration index that nl_replay maintains
+ * while its graph runs (int32[1], owned by the context). */
+const int32_t *nl_step_counter(nl_ctx *ctx);
+
+/* Synchronizes `stream`, returns the device-detected status accumulated
+ * since the last call (NL_ERR_TIMEOUT, else NL_OVERFLOW, else NL_OK) and
+ * clears it. */
+nl_status nl_sync_status(nl_ctx *ctx, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *nl_status_string(nl_status s);
+
+/* Build statistics of the last nl_build (host values, no synchronization):
+ * out[0..2] = cells per axis, out[3] = 1 if the staged pair-search kernel
+ * was used (0 = the per-atom kernel), out[4] = cells in total. */
+nl_status nl_last_build_info(nl_ctx *ctx, int64_t out[8]);
+
+/* Per-kernel timing with CUDA events recorded on the call's stream.
+ * nl_profile_enable(ctx, 1) starts recording; nl_profile_read synchronizes
+ * the device, writes for each phase p < max_phases the summed milliseconds
+ * ms_out[p] and launches launches_out[p] since the last read, and returns the
+ * number of phases.  Phase names: nl_profile_phase_name. */
+nl_status nl_profile_enable(nl_ctx *ctx, int on);
+int32_t nl_profile_read(nl_ctx *ctx, double *ms_out, int64_t *launches_out, int32_t max_phases);
+const char *nl_profile_phase_name(int32_t phase);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NL_H */

@@ -1,0 +1,250 @@
+// nl_cells.cu -- cell binning: count, single-pass scan, scatter, in-cell sort.
+//
+// The cells are the middle level of the neighbor search (Tessera abstract:
+// "three-level neighbor search"; read here as curve order -> cells -> pairs).
+// Cells are at least rl wide on every axis, numbered x fastest, so the three
+// cells (cx-1, cx, cx+1) of one (cy, cz) row are contiguous in memory.
+// Inside a cell atoms are ordered by (wrapped x, index), which makes every
+// such row sorted by x and the result independent of atomic ordering.
+#include "nl_internal.cuh"
+
+namespace nl {
+namespace {
+
+// Largest cell the in-cell sort handles (8 atoms per lane).
+constexpr int kCellSortMax = 256;
+
+__global__ void __launch_bounds__(256)
+k_bin_count(const float4 *__restrict__ pos, int64_t n, CellGrid g, uint32_t *__restrict__ atom_cell,
+            uint32_t *__restrict__ atom_rank, int32_t *__restrict__ cell_count,
+            float4 *__restrict__ ref)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) - lane;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const uint32_t lt = lanemask_lt();
+    for (int64_t b = warp0; b < n; b += stride) {
+        const int64_t i = b + lane;
+        uint32_t c = 0xffffffffu;
+        if (i < n) {
+            const float4 p = pos[i];
+            ref[i] = p;
+            const int cx = cell_coord(wrap_coord(p.x, g.Lx), g.Tx, g.nx);
+            const int cy = cell_coord(wrap_coord(p.y, g.Ly), g.Ty, g.ny);
+            const int cz = cell_coord(wrap_coord(p.z, g.Lz), g.Tz, g.nz);
+            c = (uint32_t)(((int64_t)cz * g.ny + cy) * g.nx + cx);
+        }
+        // warp-aggregated increment: one atomic per distinct cell
+        const uint32_t peers = __match_any_sync(0xffffffffu, c);
+        const int leader = __ffs(peers) - 1;
+        uint32_t old = 0u;
+        if (lane == leader && c != 0xffffffffu)
+            old = (uint32_t)atomicAdd(&cell_count[c], __popc(peers));
+        old = __shfl_sync(0xffffffffu, old, leader);
+        if (i < n) {
+            atom_cell[i] = c;
+            atom_rank[i] = old + __popc(peers & lt);
+        }
+    }
+}
+
+// Exclusive scan of cell_count[0, ncell) into cell_start[0, ncell], with
+// cell_start[ncell] = total, in one pass: tiles by ticket, decoupled
+// look-back on one status word per tile.
+__global__ void __launch_bounds__(kScanThreads)
+k_cell_scan(const int32_t *__restrict__ count, int32_t *__restrict__ start, int64_t ncell,
+            uint32_t *status, uint32_t *ticket, uint32_t *flags)
+{
+    __shared__ uint32_t s_tile;
+    __shared__ uint32_t s_wtot[kScanThreads / 32];
+    __shared__ uint32_t s_excl;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    if (t == 0) s_tile = atomicAdd(ticket, 1u);
+    __syncthreads();
+    const uint32_t tile = s_tile;
+    const int64_t base = (int64_t)tile * kScanTile + (int64_t)t * kScanItems;
+
+    uint32_t v[kScanItems];
+    uint32_t sum = 0u;
+#pragma unroll
+    for (int k = 0; k < kScanItems; ++k) {
+        v[k] = base + k < ncell ? (uint32_t)count[base + k] : 0u;
+        sum += v[k];
+    }
+    uint32_t x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_wtot[w] = x;
+    __syncthreads();
+    uint32_t wbefore = 0u, total = 0u;
+#pragma unroll
+    for (int i = 0; i < kScanThreads / 32; ++i) {
+        if (i < w) wbefore += s_wtot[i];
+        total += s_wtot[i];
+    }
+    if (t == 0) {
+        uint32_t excl = 0u;
+        uint32_t *st = status + tile;
+        if (tile == 0) {
+            st_volatile_u32(st, kStPrefix | total);
+        } else {
+            st_volatile_u32(st, kStAggregate | total);
+            int64_t j = (int64_t)tile - 1;
+            uint32_t spins = 0u;
+            while (j >= 0) {
+                const uint32_t s = ld_volatile_u32(status + j);
+                const uint32_t f = s & ~kStValue;
+                if (f == 0u) {
+                    if (++spins >= kSpinLimit) {
+                        atomicOr(flags, kFlagTimeout);
+                        break;
+                    }
+                    if (spins > 64u) __nanosleep(64);
+                    continue;
+                }
+                excl += s & kStValue;
+                if (f == kStPrefix) break;
+                --j;
+            }
+            st_volatile_u32(st, kStPrefix | ((excl + total) & kStValue));
+        }
+        s_excl = excl;
+    }
+    __syncthreads();
+    uint32_t run = s_excl + wbefore + x - sum;
+#pragma unroll
+    for (int k = 0; k < kScanItems; ++k) {
+        if (base + k < ncell) start[base + k] = (int32_t)run;
+        if (base + k == ncell - 1) start[ncell] = (int32_t)(run + v[k]);
+        run += v[k];
+    }
+}
+
+__global__ void __launch_bounds__(256)
+k_bin_scatter(const float4 *__restrict__ pos, int64_t n, CellGrid g,
+              const uint32_t *__restrict__ atom_cell, const uint32_t *__restrict__ atom_rank,
+              const int32_t *__restrict__ cell_start, float4 *__restrict__ cell_pos)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const float4 p = pos[i];
+        const int64_t dst = (int64_t)cell_start[atom_cell[i]] + atom_rank[i];
+        cell_pos[dst] = make_float4(wrap_coord(p.x, g.Lx), wrap_coord(p.y, g.Ly),
+                                    wrap_coord(p.z, g.Lz), __int_as_float((int)i));
+    }
+}
+
+__device__ __forceinline__ bool before_xi(float xa, int ia, float xb, int ib)
+{
+    return xa < xb || (xa == xb && ia < ib);
+}
+
+// One warp per cell: rank every atom of the cell by (x, index) with shuffles
+// and store it at its rank.  Cells above kCellSortMax stay in scatter order.
+__global__ void __launch_bounds__(256)
+k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t c = warp; c < ncell; c += nwarps) {
+        const int32_t s = cell_start[c];
+        const int m = cell_start[c + 1] - s;
+        if (m <= 1 || m > kCellSortMax) continue;
+        if (m <= 32) {
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (lane < m) v = cell_pos[s + lane];
+            const int id = __float_as_int(v.w);
+            int r = 0;
+            for (int j = 0; j < m; ++j) {
+                const float xj = __shfl_sync(0xffffffffu, v.x, j);
+                const int ij = __shfl_sync(0xffffffffu, id, j);
+                r += before_xi(xj, ij, v.x, id) ? 1 : 0;
+            }
+            __syncwarp();
+            if (lane < m) cell_pos[s + r] = v;
+        } else {
+            constexpr int E = kCellSortMax / 32;
+            float4 v[E];
+            int r[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                r[e] = 0;
+                v[e] = e * 32 + lane < m ? cell_pos[s + e * 32 + lane]
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int es = 0; es < E; ++es) {
+                if (es * 32 >= m) break;
+                const float xs = v[es].x;
+                const int is = __float_as_int(v[es].w);
+                const int lim = m - es * 32 < 32 ? m - es * 32 : 32;
+                for (int l = 0; l < lim; ++l) {
+                    const float xj = __shfl_sync(0xffffffffu, xs, l);
+                    const int ij = __shfl_sync(0xffffffffu, is, l);
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        r[e] += before_xi(xj, ij, v[e].x, __float_as_int(v[e].w)) ? 1 : 0;
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                if (e * 32 + lane < m) cell_pos[s + r[e]] = v[e];
+        }
+    }
+}
+
+unsigned grid_for(int64_t work, int threads, int64_t cap)
+{
+    int64_t b = (work + threads - 1) / threads;
+    if (b < 1) b = 1;
+    if (b > cap) b = cap;
+    return (unsigned)b;
+}
+
+}  // namespace
+
+cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const CellGrid &g,
+                           cudaStream_t s)
+{
+    const int64_t cap = (int64_t)ctx->sm_count * 8;
+    const int64_t scan_tiles = (g.ncell + kScanTile - 1) / kScanTile;
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->cell_count, 0, sizeof(int32_t) * g.ncell, s));
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->scan_status, 0, sizeof(uint32_t) * scan_tiles, s));
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->scan_ctr, 0, sizeof(uint32_t), s));
+    {
+        ProfScope ps(ctx, PH_BIN_COUNT, s);
+        if (n > 0)
+            k_bin_count<<<grid_for(n, 256, cap), 256, 0, s>>>(pos, n, g, ctx->atom_cell,
+                                                               ctx->atom_rank, ctx->cell_count,
+                                                               ctx->ref);
+        NL_CUDA_TRY(cudaGetLastError());
+    }
+    {
+        ProfScope ps(ctx, PH_CELL_SCAN, s);
+        k_cell_scan<<<(unsigned)scan_tiles, kScanThreads, 0, s>>>(
+            ctx->cell_count, ctx->cell_start, g.ncell, ctx->scan_status, ctx->scan_ctr, ctx->flags);
+        NL_CUDA_TRY(cudaGetLastError());
+    }
+    if (n <= 0) return cudaSuccess;
+    {
+        ProfScope ps(ctx, PH_BIN_SCATTER, s);
+        k_bin_scatter<<<grid_for(n, 256, cap), 256, 0, s>>>(pos, n, g, ctx->atom_cell,
+                                                             ctx->atom_rank, ctx->cell_start,
+                                                             ctx->cell_pos);
+        NL_CUDA_TRY(cudaGetLastError());
+    }
+    {
+        ProfScope ps(ctx, PH_CELL_SORT, s);
+        k_cell_sort<<<grid_for(g.ncell * 32, 256, cap), 256, 0, s>>>(ctx->cell_pos,
+                                                                      ctx->cell_start, g.ncell);
+        NL_CUDA_TRY(cudaGetLastError());
+    }
+    return cudaSuccess;
+}
+
+}  // namespace nl

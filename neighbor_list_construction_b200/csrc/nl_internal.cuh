@@ -1,0 +1,220 @@
+// nl_internal.cuh -- shared declarations of the libnl CUDA sources.
+//
+// Everything here is internal to libnl.so; the public C ABI is include/nl.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nl.h"
+
+namespace nl {
+
+// ----------------------------------------------------------------- constants
+constexpr int kQBits = 21;                    // bits per axis of the curve grid
+constexpr uint32_t kQMax = (1u << kQBits) - 1u;
+constexpr int kRadixBits = 8;                 // LSD digit width
+constexpr int kRadixBins = 1 << kRadixBits;
+constexpr int kKeyPasses = 8;                 // 63-bit keys: 8 digits of 8 bits
+
+// Onesweep tile: 256 threads x 16 keys.
+constexpr int kSortThreads = 256;
+constexpr int kSortItems = 16;
+constexpr int kSortTile = kSortThreads * kSortItems;
+
+// Cell-count scan tile: 256 threads x 16 cells.
+constexpr int kScanThreads = 256;
+constexpr int kScanItems = 16;
+constexpr int kScanTile = kScanThreads * kScanItems;
+
+// Look-back status words: 2 flag bits over a 30-bit count.
+constexpr uint32_t kStAggregate = 1u << 30;
+constexpr uint32_t kStPrefix = 2u << 30;
+constexpr uint32_t kStValue = (1u << 30) - 1u;
+// Polls of one status word before a bounded wait gives up.
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+// Device-detected conditions, accumulated in ctx->flags.
+constexpr uint32_t kFlagOverflow = 1u;
+constexpr uint32_t kFlagTimeout = 2u;
+
+enum Phase {
+    PH_KEYS = 0,
+    PH_KEY_SCAN,
+    PH_SORT,
+    PH_GATHER,
+    PH_BIN_COUNT,
+    PH_CELL_SCAN,
+    PH_BIN_SCATTER,
+    PH_CELL_SORT,
+    PH_PAIRS,
+    PH_PAIRS_FALLBACK,
+    PH_SKIN,
+    PH_COUNT
+};
+
+// Cell grid of one build, all values computed on the host.
+struct CellGrid {
+    int nx, ny, nz;          // cells per axis (>= 3)
+    float Lx, Ly, Lz;        // box
+    float Tx, Ty, Tz;        // fl(n_a / L_a): cell coordinate = floor(w * T)
+    float rl2;               // fl(rl * rl)
+    int64_t ncell;
+    int literal;             // 1: some axis has < 5 cells -> literal min image
+};
+
+}  // namespace nl
+
+// ------------------------------------------------------------------ context
+struct nl_ctx {
+    int device = 0;
+    int sm_count = 148;
+    int64_t max_atoms = 0;
+    int32_t max_capacity = 0;
+    int64_t max_cells = 0;
+
+    // radix sort
+    uint64_t *keys[2] = {nullptr, nullptr};
+    uint32_t *vals[2] = {nullptr, nullptr};
+    uint32_t *hist = nullptr;          // [8][256] counts, then exclusive starts
+    uint32_t *sort_status = nullptr;   // [8][max_sort_tiles][256] look-back
+    uint32_t *sort_ctr = nullptr;      // [8] tile tickets
+    int64_t max_sort_tiles = 0;
+
+    // cells
+    int32_t *cell_count = nullptr;     // [max_cells]
+    int32_t *cell_start = nullptr;     // [max_cells + 1]
+    uint32_t *scan_status = nullptr;   // [max_scan_tiles]
+    uint32_t *scan_ctr = nullptr;      // [1]
+    int64_t max_scan_tiles = 0;
+    uint32_t *atom_cell = nullptr;     // [max_atoms]
+    uint32_t *atom_rank = nullptr;     // [max_atoms]
+    float4 *cell_pos = nullptr;        // [max_atoms] wrapped xyz + index bits
+    float4 *ref = nullptr;             // [max_atoms] reference positions
+
+    // status and small state
+    uint32_t *flags = nullptr;         // [1]
+    uint32_t *skin_acc = nullptr;      // [2]: max bits, block ticket
+    int32_t *step = nullptr;           // [1] replay iteration index
+    int32_t *rebuild_tmp = nullptr;    // [1]
+    uint32_t *zero_block = nullptr;    // one allocation holding the small state
+
+    // last build
+    int64_t last_n = -1;
+    nl::CellGrid last_grid{};
+    int last_fast = 0;
+
+    // replay cache
+    cudaGraph_t replay_graph = nullptr;
+    cudaGraphExec_t replay_exec = nullptr;
+    unsigned char replay_key[128] = {0};
+    int replay_key_len = 0;
+
+    // profiling
+    int prof_on = 0;
+    static const int kProfSlots = 8192;
+    cudaEvent_t *prof_ev = nullptr;    // [2 * kProfSlots]
+    int *prof_phase = nullptr;         // [kProfSlots]
+    int prof_used = 0;
+    int prof_dropped = 0;
+    double prof_ms[nl::PH_COUNT] = {0};
+    int64_t prof_launches[nl::PH_COUNT] = {0};
+};
+
+namespace nl {
+
+// -------------------------------------------------------------- profiling
+// Returns a slot (or -1) and records its start event on `s`.
+int prof_begin(nl_ctx *ctx, int phase, cudaStream_t s);
+void prof_end(nl_ctx *ctx, int slot, cudaStream_t s);
+
+struct ProfScope {
+    nl_ctx *ctx;
+    cudaStream_t s;
+    int slot;
+    ProfScope(nl_ctx *c, int phase, cudaStream_t st) : ctx(c), s(st), slot(prof_begin(c, phase, st)) {}
+    ~ProfScope() { prof_end(ctx, slot, s); }
+};
+
+// ------------------------------------------------------------- launchers
+// Curve keys of all atoms into ctx->keys[0]/vals[0] and the 8 digit
+// histograms into ctx->hist (which must be zero); curve 0 Hilbert, 1 Morton.
+cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
+                        float Lz, float Sx, float Sy, float Sz, int curve, cudaStream_t s);
+// Exclusive scan of the 8 histograms in place.
+cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s);
+// 8 onesweep passes; the last writes keys to keys_final (may be ctx->keys[0])
+// and indices to vals_final.
+cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
+                                uint32_t *vals_final, cudaStream_t s);
+cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, float4 *out,
+                          cudaStream_t s);
+
+// Cell binning of `pos` into ctx->cell_pos (cell order, x-sorted in cells).
+cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const CellGrid &g,
+                           cudaStream_t s);
+// Pair search over the binned atoms.
+cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
+                         int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast);
+
+// Skin check.  decisions/step may be NULL; cond_handle 0 = none.
+cudaError_t launch_skin(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
+                        float Lz, float h2, int32_t *rebuild_out, float *max_d2_out,
+                        int32_t *decisions, const int32_t *step,
+                        unsigned long long cond_handle, cudaStream_t s);
+
+// ------------------------------------------------------- device helpers
+__device__ __forceinline__ float wrap_coord(float x, float L)
+{
+    // w = x - L*floor(x/L), one fold into [0, L), else 0
+    float t = floorf(__fdiv_rn(x, L));
+    float w = __fsub_rn(x, __fmul_rn(L, t));
+    if (w < 0.0f) w = __fadd_rn(w, L);
+    if (w >= L) w = __fsub_rn(w, L);
+    if (!(w >= 0.0f && w < L)) w = 0.0f;
+    return w;
+}
+
+// Literal minimum image d - L*rintf(d/L).
+__device__ __forceinline__ float min_image_literal(float d, float L)
+{
+    float r = rintf(__fdiv_rn(d, L));
+    return __fsub_rn(d, __fmul_rn(L, r));
+}
+
+__device__ __forceinline__ float r2_of(float dx, float dy, float dz)
+{
+    return __fadd_rn(__fadd_rn(__fmul_rn(dx, dx), __fmul_rn(dy, dy)), __fmul_rn(dz, dz));
+}
+
+__device__ __forceinline__ int cell_coord(float w, float T, int n)
+{
+    float f = floorf(__fmul_rn(w, T));
+    int c = f >= 0.0f ? (int)f : 0;
+    return c < n ? c : n - 1;
+}
+
+__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t *p)
+{
+    return *(const volatile uint32_t *)p;
+}
+
+__device__ __forceinline__ void st_volatile_u32(uint32_t *p, uint32_t v)
+{
+    *(volatile uint32_t *)p = v;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt()
+{
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+}  // namespace nl
+
+#define NL_CUDA_TRY(expr)                                   \
+    do {                                                    \
+        cudaError_t _e = (expr);                            \
+        if (_e != cudaSuccess) return _e;                   \
+    } while (0)

@@ -1,0 +1,190 @@
+// nl_sort.cu -- onesweep LSD radix sort of (63-bit key, 32-bit index) pairs.
+//
+// One kernel launch per 8-bit digit.  Each CTA takes the next tile from an
+// atomic ticket (so a tile only ever waits on tiles whose CTAs are already
+// running), ranks its keys stably with warp match/popc, publishes its per-
+// digit counts, and finds the counts of all earlier tiles by decoupled
+// look-back over per-(tile, digit) status words.  The global digit starts
+// come from histograms computed once, in the key kernel.  Waits on a status
+// word are bounded: past kSpinLimit polls the kernel records kFlagTimeout
+// and carries on, so a stuck predecessor cannot hang the device.
+#include "nl_internal.cuh"
+
+namespace nl {
+namespace {
+
+constexpr int kWarps = kSortThreads / 32;
+constexpr size_t kSortDynSmem = (size_t)kSortTile * (sizeof(uint64_t) + sizeof(uint32_t));
+
+template <bool WRITE_KEYS>
+__global__ void __launch_bounds__(kSortThreads)
+k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
+           uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, int64_t n,
+           int shift, const uint32_t *__restrict__ digit_start, uint32_t *status,
+           uint32_t *ticket, uint32_t *flags)
+{
+    extern __shared__ __align__(16) unsigned char sort_smem[];
+    uint64_t *s_keys = reinterpret_cast<uint64_t *>(sort_smem);
+    uint32_t *s_vals = reinterpret_cast<uint32_t *>(sort_smem + sizeof(uint64_t) * kSortTile);
+    __shared__ uint32_t s_whist[kWarps][kRadixBins];  // per-warp counts -> prefixes
+    __shared__ uint32_t s_tdig[kRadixBins];           // digit start inside the tile
+    __shared__ uint32_t s_gbase[kRadixBins];          // global start of digit in tile
+    __shared__ uint32_t s_wtot[kWarps];
+    __shared__ uint32_t s_tile;
+
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    if (t == 0) s_tile = atomicAdd(ticket, 1u);
+    for (int i = t; i < kWarps * kRadixBins; i += kSortThreads) (&s_whist[0][0])[i] = 0u;
+    __syncthreads();
+    const uint32_t tile = s_tile;
+    const int64_t base = (int64_t)tile * kSortTile;
+
+    // warp w owns elements [base + 512w, base + 512w + 512); item k of lane l
+    // is element base + 512w + 32k + l, so (k, lane) order is index order.
+    uint64_t key[kSortItems];
+    uint32_t val[kSortItems];
+    uint32_t rank[kSortItems];
+#pragma unroll
+    for (int k = 0; k < kSortItems; ++k) {
+        const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
+        if (idx < n) {
+            key[k] = keys_in[idx];
+            val[k] = vals_in[idx];
+        } else {
+            key[k] = ~0ull;  // digit 255 in every pass, never written
+            val[k] = 0u;
+        }
+    }
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int k = 0; k < kSortItems; ++k) {
+        const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
+        const uint32_t d = idx < n ? (uint32_t)(key[k] >> shift) & 0xffu : 0x100u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, d);
+        const int leader = __ffs(peers) - 1;
+        uint32_t before = 0u;
+        if (lane == leader && d < 0x100u) {
+            before = s_whist[w][d];
+            s_whist[w][d] = before + __popc(peers);
+        }
+        before = __shfl_sync(0xffffffffu, before, leader);
+        rank[k] = before + __popc(peers & lt);
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // thread t now owns digit t
+    uint32_t cnt = 0u;
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) {
+        const uint32_t c = s_whist[ww][t];
+        s_whist[ww][t] = cnt;
+        cnt += c;
+    }
+    uint32_t *st = status + (size_t)tile * kRadixBins + t;
+    uint32_t excl = 0u;
+    if (tile == 0) {
+        st_volatile_u32(st, kStPrefix | cnt);
+    } else {
+        st_volatile_u32(st, kStAggregate | cnt);
+        int64_t j = (int64_t)tile - 1;
+        uint32_t spins = 0u;
+        while (j >= 0) {
+            const uint32_t s = ld_volatile_u32(status + (size_t)j * kRadixBins + t);
+            const uint32_t f = s & ~kStValue;
+            if (f == 0u) {
+                if (++spins >= kSpinLimit) {
+                    atomicOr(flags, kFlagTimeout);
+                    break;
+                }
+                if (spins > 64u) __nanosleep(64);
+                continue;
+            }
+            excl += s & kStValue;
+            if (f == kStPrefix) break;
+            --j;
+        }
+        st_volatile_u32(st, kStPrefix | ((excl + cnt) & kStValue));
+    }
+    s_gbase[t] = digit_start[t] + excl;
+
+    // exclusive scan of the tile's digit counts
+    uint32_t x = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_wtot[w] = x;
+    __syncthreads();
+    uint32_t before = 0u;
+    for (int i = 0; i < w; ++i) before += s_wtot[i];
+    s_tdig[t] = before + x - cnt;
+    __syncthreads();
+
+    // stage the tile in digit order
+#pragma unroll
+    for (int k = 0; k < kSortItems; ++k) {
+        const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
+        if (idx < n) {
+            const uint32_t d = (uint32_t)(key[k] >> shift) & 0xffu;
+            const uint32_t p = s_tdig[d] + s_whist[w][d] + rank[k];
+            s_keys[p] = key[k];
+            s_vals[p] = val[k];
+        }
+    }
+    __syncthreads();
+
+    // runs of equal digits go to consecutive global addresses
+    const int64_t rem = n - base;
+    const int tile_n = rem < kSortTile ? (int)rem : kSortTile;
+    for (int p = t; p < tile_n; p += kSortThreads) {
+        const uint64_t k = s_keys[p];
+        const uint32_t d = (uint32_t)(k >> shift) & 0xffu;
+        const uint32_t out = s_gbase[d] + ((uint32_t)p - s_tdig[d]);
+        if (WRITE_KEYS) keys_out[out] = k;
+        vals_out[out] = s_vals[p];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
+                                uint32_t *vals_final, cudaStream_t s)
+{
+    if (n <= 0) return cudaSuccess;
+    const int64_t tiles = (n + kSortTile - 1) / kSortTile;
+    static bool attr_set = false;
+    if (!attr_set) {
+        NL_CUDA_TRY(cudaFuncSetAttribute(k_onesweep<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSortDynSmem));
+        NL_CUDA_TRY(cudaFuncSetAttribute(k_onesweep<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSortDynSmem));
+        attr_set = true;
+    }
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_status, 0,
+                                sizeof(uint32_t) * kKeyPasses * tiles * kRadixBins, s));
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_ctr, 0, sizeof(uint32_t) * kKeyPasses, s));
+    int src = 0;
+    for (int p = 0; p < kKeyPasses; ++p) {
+        const bool last = p == kKeyPasses - 1;
+        uint64_t *ko = last ? (keys_final ? keys_final : ctx->keys[1 - src]) : ctx->keys[1 - src];
+        uint32_t *vo = last ? vals_final : ctx->vals[1 - src];
+        uint32_t *status = ctx->sort_status + (size_t)p * tiles * kRadixBins;
+        if (last && !keys_final)
+            k_onesweep<false><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
+                ctx->keys[src], ctx->vals[src], ko, vo, n, kRadixBits * p,
+                ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags);
+        else
+            k_onesweep<true><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
+                ctx->keys[src], ctx->vals[src], ko, vo, n, kRadixBits * p,
+                ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags);
+        NL_CUDA_TRY(cudaGetLastError());
+        src = 1 - src;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace nl

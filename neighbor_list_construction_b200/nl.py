@@ -1,0 +1,242 @@
+"""Python binding of libnl.so (C ABI in include/nl.h): argument marshalling only.
+
+Every function here mirrors one C entry point of the same name and forwards
+torch CUDA tensors as raw device pointers; all work runs in libnl's kernels.
+Importing this module loads the library and raises ImportError if it has not
+been built (``python -m neighbor_list_construction_b200.build_lib``): there is
+no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnl.so")
+
+NL_OK, NL_OVERFLOW = 0, 1
+NL_ERR_ARG, NL_ERR_BOX, NL_ERR_CUDA, NL_ERR_TIMEOUT, NL_ERR_CAPACITY = -1, -2, -3, -4, -5
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libnl.so not built at {LIB_PATH}; run "
+                      "`python -m neighbor_list_construction_b200.build_lib`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i32, _i64, _f32, _u64 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                              ctypes.c_uint64)
+_SIGS = {
+    "nl_create": (_i32, [ctypes.POINTER(_vp), _i64, _i32]),
+    "nl_destroy": (None, [_vp]),
+    "nl_sort_hilbert": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "nl_sort_morton": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "nl_build": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
+    "nl_skin_check": (_i32, [_vp, _i64, _vp, _vp, _f32, _vp, _vp, _vp]),
+    "nl_replay": (_i32, [_vp, _vp, _i32, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp, _vp]),
+    "nl_step_counter": (_vp, [_vp]),
+    "nl_sync_status": (_i32, [_vp, _vp]),
+    "nl_status_string": (ctypes.c_char_p, [_i32]),
+    "nl_last_build_info": (_i32, [_vp, _vp]),
+    "nl_profile_enable": (_i32, [_vp, ctypes.c_int]),
+    "nl_profile_read": (_i32, [_vp, _vp, _vp, _i32]),
+    "nl_profile_phase_name": (ctypes.c_char_p, [_i32]),
+    "nls_displace": (_i32, [_i64, _vp, _u64, _i64, _vp, _f32, _vp]),
+    "nls_step_graph": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _u64, _vp, _f32]),
+    "nls_graph_destroy": (None, [_vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTS = tuple(_SIGS)
+
+
+class NLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {nl_status_string(status)}")
+        self.status = status
+
+
+def nl_status_string(status: int) -> str:
+    return _lib.nl_status_string(status).decode()
+
+
+def _check(status: int, where: str) -> int:
+    if status < 0:
+        raise NLError(status, where)
+    return status
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _box(box) -> ctypes.Array:
+    b = [float(v) for v in (box.tolist() if hasattr(box, "tolist") else box)]
+    if len(b) != 3:
+        raise ValueError("box must have 3 entries")
+    return (ctypes.c_float * 3)(*b)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _pos(pos: torch.Tensor) -> torch.Tensor:
+    if pos.dtype != torch.float32 or pos.dim() != 2 or pos.shape[1] != 4:
+        raise ValueError("positions must be a float32 [n, 4] CUDA tensor")
+    return pos
+
+
+# --------------------------------------------------------------- C mirrors
+def nl_create(max_atoms: int, max_capacity: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_lib.nl_create(ctypes.byref(h), int(max_atoms), int(max_capacity)), "nl_create")
+    return h
+
+
+def nl_destroy(ctx) -> None:
+    _lib.nl_destroy(ctx)
+
+
+def nl_sort_hilbert(ctx, pos, box, perm_out, pos_sorted_out, keys_out=None, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_sort_hilbert(ctx, pos.shape[0], _ptr(pos), _box(box), _ptr(perm_out),
+                                       _ptr(pos_sorted_out), _ptr(keys_out), _stream(stream)),
+                  "nl_sort_hilbert")
+
+
+def nl_sort_morton(ctx, pos, box, perm_out, pos_sorted_out, keys_out=None, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_sort_morton(ctx, pos.shape[0], _ptr(pos), _box(box), _ptr(perm_out),
+                                      _ptr(pos_sorted_out), _ptr(keys_out), _stream(stream)),
+                  "nl_sort_morton")
+
+
+def nl_build(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_build(ctx, pos.shape[0], _ptr(pos), _box(box), float(cutoff),
+                                float(skin), int(capacity), _ptr(nbr_out), _ptr(counts_out),
+                                _stream(stream)), "nl_build")
+
+
+def nl_skin_check(ctx, pos, box, skin, rebuild_out, max_d2_out=None, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_skin_check(ctx, pos.shape[0], _ptr(pos), _box(box), float(skin),
+                                     _ptr(rebuild_out), _ptr(max_d2_out), _stream(stream)),
+                  "nl_skin_check")
+
+
+def nl_replay(ctx, step_graph, n_steps, pos, box, cutoff, skin, capacity, nbr, counts,
+              decisions_out, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_replay(ctx, step_graph, int(n_steps), pos.shape[0], _ptr(pos),
+                                 _box(box), float(cutoff), float(skin), int(capacity), _ptr(nbr),
+                                 _ptr(counts), _ptr(decisions_out), _stream(stream)), "nl_replay")
+
+
+def nl_step_counter(ctx) -> int:
+    return _lib.nl_step_counter(ctx)
+
+
+def nl_sync_status(ctx, stream=None) -> int:
+    return _check(_lib.nl_sync_status(ctx, _stream(stream)), "nl_sync_status")
+
+
+def nl_last_build_info(ctx) -> list[int]:
+    out = (ctypes.c_int64 * 8)()
+    _check(_lib.nl_last_build_info(ctx, out), "nl_last_build_info")
+    return list(out)
+
+
+def nl_profile_enable(ctx, on: bool = True) -> None:
+    _check(_lib.nl_profile_enable(ctx, 1 if on else 0), "nl_profile_enable")
+
+
+def nl_profile_read(ctx) -> dict[str, tuple[float, int]]:
+    ms = (ctypes.c_double * 32)()
+    ln = (ctypes.c_int64 * 32)()
+    n = _lib.nl_profile_read(ctx, ms, ln, 32)
+    if n < 0:
+        raise NLError(NL_ERR_CUDA, "nl_profile_read")
+    return {_lib.nl_profile_phase_name(p).decode(): (ms[p], ln[p]) for p in range(n)}
+
+
+def nl_profile_phase_name(phase: int) -> str:
+    return _lib.nl_profile_phase_name(int(phase)).decode()
+
+
+def nls_displace(pos, seed: int, step: int, sigma: float, step_dev: int | None = None,
+                 stream=None) -> None:
+    _pos(pos)
+    _check(_lib.nls_displace(pos.shape[0], _ptr(pos), int(seed) & (2 ** 64 - 1), int(step),
+                             ctypes.c_void_p(step_dev) if step_dev else None, float(sigma),
+                             _stream(stream)), "nls_displace")
+
+
+def nls_step_graph(pos, seed: int, step_dev: int, sigma: float) -> ctypes.c_void_p:
+    _pos(pos)
+    g = ctypes.c_void_p()
+    _check(_lib.nls_step_graph(ctypes.byref(g), pos.shape[0], _ptr(pos), int(seed) & (2 ** 64 - 1),
+                               ctypes.c_void_p(step_dev), float(sigma)), "nls_step_graph")
+    return g
+
+
+def nls_graph_destroy(graph) -> None:
+    _lib.nls_graph_destroy(graph)
+
+
+# ------------------------------------------------------------ convenience
+class Context:
+    """Owns an nl_ctx and allocates output tensors for the common calls."""
+
+    def __init__(self, max_atoms: int, max_capacity: int):
+        self.handle = nl_create(max_atoms, max_capacity)
+
+    def close(self) -> None:
+        if self.handle:
+            nl_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def sort(self, pos, box, curve: str = "hilbert", keys: bool = False, stream=None):
+        n = pos.shape[0]
+        perm = torch.empty(n, dtype=torch.int32, device=pos.device)
+        ps = torch.empty(n, 4, dtype=torch.float32, device=pos.device)
+        ks = torch.empty(n, dtype=torch.int64, device=pos.device) if keys else None
+        fn = nl_sort_hilbert if curve == "hilbert" else nl_sort_morton
+        fn(self.handle, pos, box, perm, ps, ks, stream)
+        return perm, ps, ks
+
+    def build(self, pos, box, cutoff, skin, capacity, nbr=None, counts=None, stream=None):
+        n = pos.shape[0]
+        if nbr is None:
+            nbr = torch.empty(n, capacity, dtype=torch.int32, device=pos.device)
+        if counts is None:
+            counts = torch.empty(n, dtype=torch.int32, device=pos.device)
+        nl_build(self.handle, pos, box, cutoff, skin, capacity, nbr, counts, stream)
+        return nbr, counts
+
+    def skin_check(self, pos, box, skin, stream=None):
+        rb = torch.zeros(1, dtype=torch.int32, device=pos.device)
+        md = torch.zeros(1, dtype=torch.float32, device=pos.device)
+        nl_skin_check(self.handle, pos, box, skin, rb, md, stream)
+        return rb, md
+
+    def sync_status(self, stream=None) -> int:
+        return nl_sync_status(self.handle, stream)

@@ -1,0 +1,294 @@
+"""GPU path vs the CPU oracle, through the C ABI (bit-exact).
+
+Curve order: the permutation (ties by index) and keys equal the oracle's at
+every size.  Neighbor lists: canonicalised rows and counts equal the
+oracle's; at the 1M and 10M workloads on sampled rows plus size-independent
+properties.  All inputs are the seeded workloads of
+neighbor_list_construction_b200.workloads.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nl():
+    from neighbor_list_construction_b200 import nl as _nl
+    return _nl
+
+
+@pytest.fixture(scope="module")
+def ctx(nl):
+    c = nl.Context(10_400_000, 320)
+    yield c
+    c.close()
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def gpu_sort(ctx, pos, box, curve="hilbert"):
+    perm, ps, ks = ctx.sort(dev(pos), box, curve, keys=True)
+    assert ctx.sync_status() == 0
+    return perm.cpu().numpy(), ps.cpu().numpy(), ks.cpu().numpy().view(np.uint64)
+
+
+def gpu_build(ctx, pos, box, cutoff, skin, K):
+    nbr, cnt = ctx.build(dev(pos), box, cutoff, skin, K)
+    st = ctx.sync_status()
+    return nbr.cpu().numpy(), cnt.cpu().numpy(), st
+
+
+# ------------------------------------------------------------------ curve order
+@pytest.mark.parametrize("name", ["uniform4k", "lattice60k", "saltwater_n20"])
+@pytest.mark.parametrize("curve", ["hilbert", "morton"])
+def test_sort_matches_oracle(ctx, oracle, name, curve):
+    w = gu.workload(name)
+    perm, ps, ks = gpu_sort(ctx, w.pos, w.box, curve)
+    o_perm, o_ks = oracle.sort(w.pos, w.box, curve)
+    np.testing.assert_array_equal(ks, o_ks)
+    np.testing.assert_array_equal(perm, o_perm)
+    np.testing.assert_array_equal(ps[:, :3], w.pos[o_perm, :3])
+    np.testing.assert_array_equal(ps[:, 3].view(np.int32), o_perm)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 31, 33, 4095, 4096, 4097, 12289, 65537])
+def test_sort_ragged_sizes(ctx, oracle, n):
+    rng = np.random.default_rng(n)
+    box = np.array([50.0, 61.5, 43.25], np.float32)
+    pos = np.zeros((n, 4), np.float32)
+    pos[:, :3] = rng.uniform(-0.5, 1.5, (n, 3)) * box  # some outside the box
+    if n > 8:
+        pos[: n // 4, :3] = pos[n // 4: 2 * (n // 4), :3]  # duplicates -> equal keys
+    perm, ps, ks = gpu_sort(ctx, pos, box)
+    o_perm, o_ks = oracle.sort(pos, box)
+    np.testing.assert_array_equal(ks, o_ks)
+    np.testing.assert_array_equal(perm, o_perm)
+
+
+def test_sort_full_size_salt_solution(ctx, oracle):
+    w = gu.workload("saltwater10m")
+    perm, ps, ks = gpu_sort(ctx, w.pos, w.box)
+    o_perm, o_ks = oracle.sort(w.pos, w.box)
+    np.testing.assert_array_equal(ks, o_ks)
+    np.testing.assert_array_equal(perm, o_perm)
+
+
+# --------------------------------------------------------------- neighbor lists
+def test_build_uniform4k_equals_bruteforce(ctx, oracle):
+    w = gu.workload("uniform4k")
+    nbr, cnt, st = gpu_build(ctx, w.pos, w.box, w.cutoff, w.skin, w.capacity)
+    o_nbr, o_cnt, o_ov = oracle.bruteforce(w.pos, w.box, w.cutoff, w.skin, w.capacity)
+    assert st == 0 and not o_ov
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+
+
+@pytest.mark.parametrize("name", ["lattice60k", "saltwater_n20", "uniform4k"])
+def test_build_matches_oracle_on_sorted_positions(ctx, oracle, name):
+    w = gu.workload(name)
+    _, ps, _ = gpu_sort(ctx, w.pos, w.box)
+    nbr, cnt, st = gpu_build(ctx, ps, w.box, w.cutoff, w.skin, w.capacity)
+    o_nbr, o_cnt, o_ov = oracle.build(ps, w.box, w.cutoff, w.skin, w.capacity)
+    assert st == (1 if o_ov else 0)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+
+
+@pytest.mark.parametrize("box,cutoff,skin", [
+    ([7.5, 7.5, 7.5], 2.0, 0.5),        # exactly 3 rl: 2 cells -> error (margin)
+    ([7.6, 7.6, 7.6], 2.0, 0.5),        # 3 cells per axis, literal min image
+    ([10.1, 10.1, 10.1], 2.0, 0.5),     # 4 cells per axis, literal
+    ([13.0, 10.1, 7.6], 2.0, 0.5),      # orthorhombic, mixed
+    ([12.6, 20.0, 31.0], 2.0, 0.5),     # >= 5 cells everywhere: shifted path
+])
+def test_build_small_boxes(ctx, oracle, box, cutoff, skin):
+    rng = np.random.default_rng(5)
+    box = np.array(box, np.float32)
+    n = int(0.1 * np.prod(box)) + 7
+    pos = np.zeros((n, 4), np.float32)
+    pos[:, :3] = rng.random((n, 3)) * box
+    edge = np.array([[0, 0, 0], [-0.0, 0, 0], [box[0], 0, 0], [box[0] + 2.0, 0, 0],
+                     [2.5, 0, 0], [box[0] - 1e-3, box[1] - 1e-3, box[2] - 1e-3],
+                     [-1e-8, -1e-8, -1e-8]], np.float32)
+    pos[:7, :3] = edge
+    o_nbr, o_cnt, o_ov = oracle.bruteforce(pos, box, cutoff, skin, 64)
+    if box[0] == np.float32(7.5):
+        from neighbor_list_construction_b200 import nl as _nl
+        with pytest.raises(_nl.NLError) as e:
+            ctx.build(dev(pos), box, cutoff, skin, 64)
+        assert e.value.status == _nl.NL_ERR_BOX
+        return
+    nbr, cnt, st = gpu_build(ctx, pos, box, cutoff, skin, 64)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+
+
+def test_build_golden_fixtures(ctx):
+    import glob
+    import json
+    import os
+    for path in sorted(glob.glob(os.path.join(os.path.dirname(__file__), "golden", "tiny_*.json"))):
+        g = json.load(open(path))
+        pos = np.zeros((len(g["positions"]), 4), np.float32)
+        pos[:, :3] = np.array(g["positions"], np.float32)
+        # the fixtures' boxes hold 3-4 cells: they exercise the literal path
+        nbr, cnt, st = gpu_build(ctx, pos, g["box"], g["cutoff"], g["skin"], g["capacity"])
+        np.testing.assert_array_equal(cnt, np.array(g["counts"], np.int32))
+        exp = np.array(g["rows"], np.int32)
+        ok = cnt <= g["capacity"]
+        np.testing.assert_array_equal(gu.canonical(nbr)[ok], exp[ok])
+        assert st == (1 if g.get("overflow") else 0)
+
+
+def test_overflow_status_and_rows(ctx, oracle):
+    rng = np.random.default_rng(18)
+    box = np.array([20.0, 20.0, 20.0], np.float32)
+    pos = np.zeros((300, 4), np.float32)
+    pos[:, :3] = rng.random((300, 3)) * 3.0 + 5.0
+    nbr, cnt, st = gpu_build(ctx, pos, box, 2.0, 0.5, 16)
+    o_nbr, o_cnt, o_ov = oracle.build(pos, box, 2.0, 0.5, 16)
+    full, fcnt, _ = oracle.build(pos, box, 2.0, 0.5, 400)
+    sets = [set(full[i, :fcnt[i]].tolist()) for i in range(300)]
+    assert o_ov and st == 1
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt, full_sets=sets)
+
+
+@pytest.mark.parametrize("name", ["saltwater1m", "saltwater10m", "shell10m"])
+def test_build_full_size_sampled(ctx, oracle, name):
+    """Full-size workloads, in the order the benchmark uses (curve-sorted):
+    sampled rows against the oracle, symmetry of the sampled rows, and the
+    global pair count parity."""
+    w = gu.workload(name)
+    perm, ps, _ = gpu_sort(ctx, w.pos, w.box)
+    nbr_t, cnt_t = ctx.build(dev(ps), w.box, w.cutoff, w.skin, w.capacity)
+    st = ctx.sync_status()
+    assert st in (0, 1)
+    cnt = cnt_t.cpu().numpy()
+    rng = np.random.default_rng(123)
+    n = w.n
+    sample = np.unique(np.concatenate([rng.choice(n, 3000, replace=False),
+                                       np.arange(0, 64), np.arange(n - 64, n)]))
+    nbr_s = nbr_t[torch.from_numpy(sample).cuda()].cpu().numpy()
+    o_nbr, o_cnt, o_ov = oracle.rows(ps, w.box, w.cutoff, w.skin, w.capacity, sample)
+    gu.assert_rows_match(nbr_s, cnt[sample], o_nbr, o_cnt)
+    assert (st == 1) == bool((cnt > w.capacity).any())
+    # every directed pair has its reverse: total is even, and sampled rows
+    # appear in their neighbors' rows
+    assert int(cnt.astype(np.int64).sum()) % 2 == 0
+    sub = sample[:200]
+    rows = nbr_t[torch.from_numpy(sub).cuda()].cpu().numpy()
+    for i, row in zip(sub, rows):
+        js = row[row >= 0]
+        back = nbr_t[torch.from_numpy(js.astype(np.int64)).cuda()].cpu().numpy()
+        assert np.all((back == i).sum(axis=1) == 1)
+
+
+# ------------------------------------------------------------------ skin check
+def test_skin_special_cases(ctx, nl):
+    box = [10.0, 10.0, 10.0]
+    ref = np.zeros((10, 4), np.float32)
+    ref[:, :3] = 1.0
+    r = dev(ref)
+    ctx.build(r, box, 2.0, 1.0, 32)
+    rb, md = ctx.skin_check(r, box, 1.0)
+    assert rb.item() == 0 and md.item() == 0.0
+    p = ref.copy()
+    p[3, 0] = 1.5  # exactly h = 0.5 -> r2 = 0.25 = h^2, strict -> no rebuild
+    rb, md = ctx.skin_check(dev(p), box, 1.0)
+    assert rb.item() == 0 and md.item() == 0.25
+    p[3, 0] = np.nextafter(np.float32(1.5), np.float32(2))
+    rb, md = ctx.skin_check(dev(p), box, 1.0)
+    assert rb.item() == 1 and md.item() > 0.25
+    assert ctx.sync_status() == 0
+
+
+def test_skin_matches_oracle(ctx, oracle):
+    w = gu.workload("lattice60k")
+    p0 = dev(w.pos)
+    ctx.build(p0, w.box, w.cutoff, w.skin, w.capacity)
+    rng = np.random.default_rng(9)
+    for scale in (0.05, 0.2, 0.35, 0.6):
+        moved = w.pos.copy()
+        moved[:, :3] += rng.normal(0, scale, (w.n, 3)).astype(np.float32)
+        moved[:5, :3] += w.box  # a few atoms crossed the box: min image
+        rb, md = ctx.skin_check(dev(moved), w.box, w.skin)
+        o_m, o_rb = oracle.skin_check(moved, w.pos, w.box, w.skin)
+        assert md.item() == o_m and bool(rb.item()) == o_rb
+
+
+def test_displacement_stand_in_matches_oracle(ctx, nl, oracle):
+    w = gu.workload("lattice60k")
+    p = dev(w.pos)
+    for step in (1, 2, 17):
+        nl.nls_displace(p, 77, step, 0.02)
+    exp = w.pos.copy()
+    for step in (1, 2, 17):
+        exp = oracle.displace(exp, 77, step, 0.02)
+    np.testing.assert_array_equal(p.cpu().numpy()[:, :3], exp[:, :3])
+
+
+# ------------------------------------------------------------------ replay
+def _replay(ctx, nl, oracle, name, steps, seed=2024, check_lists=True):
+    w = gu.workload(name)
+    _, ps, _ = gpu_sort(ctx, w.pos, w.box)
+    p = dev(ps)
+    nbr, cnt = ctx.build(p, w.box, w.cutoff, w.skin, w.capacity)
+    g = nl.nls_step_graph(p, seed, nl.nl_step_counter(ctx.handle), w.sigma_step)
+    dec = torch.full((steps,), -1, dtype=torch.int32, device="cuda")
+    try:
+        nl.nl_replay(ctx.handle, g, steps, p, w.box, w.cutoff, w.skin, w.capacity, nbr, cnt, dec)
+        st = ctx.sync_status()
+    finally:
+        nl.nls_graph_destroy(g)
+    o_dec, o_final, o_ref = oracle.md_decisions(ps, w.box, w.skin, seed, w.sigma_step, steps)
+    np.testing.assert_array_equal(dec.cpu().numpy(), o_dec)
+    np.testing.assert_array_equal(p.cpu().numpy()[:, :3], o_final[:, :3])
+    if check_lists:
+        o_nbr, o_cnt, o_ov = oracle.build(o_ref, w.box, w.cutoff, w.skin, w.capacity)
+        assert st == (1 if o_ov else 0)
+        gu.assert_rows_match(nbr.cpu().numpy(), cnt.cpu().numpy(), o_nbr, o_cnt)
+    return o_dec
+
+
+def test_replay_lattice60k_50_steps(ctx, nl, oracle):
+    dec = _replay(ctx, nl, oracle, "lattice60k", 50)
+    assert dec.sum() >= 1
+
+
+def test_replay_twice_reuses_graph(ctx, nl, oracle):
+    _replay(ctx, nl, oracle, "uniform4k", 30, seed=5)
+    _replay(ctx, nl, oracle, "uniform4k", 30, seed=5)
+
+
+def test_replay_salt_solution_200_steps(ctx, nl, oracle):
+    dec = _replay(ctx, nl, oracle, "saltwater10m", 200, check_lists=False)
+    assert 3 <= dec.sum() <= 40
+
+
+# ------------------------------------------------------------------ errors
+def test_argument_errors(ctx, nl):
+    p = dev(np.zeros((10, 4), np.float32))
+    with pytest.raises(nl.NLError) as e:
+        ctx.build(p, [10, 10, 10], 2.0, 0.5, 400)
+    assert e.value.status == nl.NL_ERR_CAPACITY
+    with pytest.raises(nl.NLError) as e:
+        ctx.build(p, [10, 10, 10], -1.0, 0.5, 16)
+    assert e.value.status == nl.NL_ERR_ARG
+    with pytest.raises(nl.NLError) as e:
+        ctx.build(p, [10, 0, 10], 2.0, 0.5, 16)
+    assert e.value.status == nl.NL_ERR_ARG
+    with pytest.raises(nl.NLError) as e:
+        ctx.build(p, [5, 10, 10], 2.0, 0.5, 16)
+    assert e.value.status == nl.NL_ERR_BOX
+    assert ctx.sync_status() == 0
+
+
+def test_empty_input(ctx, nl):
+    p = torch.zeros((0, 4), dtype=torch.float32, device="cuda")
+    nbr, cnt = ctx.build(p, [10, 10, 10], 2.0, 0.5, 16)
+    perm, ps, _ = ctx.sort(p, [10, 10, 10])
+    rb, md = ctx.skin_check(p, [10, 10, 10], 0.5)
+    assert rb.item() == 0 and ctx.sync_status() == 0
