@@ -145,6 +145,24 @@ const char *nl_status_string(nl_status s);
  * was used (0 = the per-atom kernel), out[4] = cells in total. */
 nl_status nl_last_build_info(nl_ctx *ctx, int64_t out[8]);
 
+/* Curve sort that allocates nothing.  The paper has no counterpart: this
+ * entry point exists for callers that cannot call cudaMalloc (code running
+ * inside a framework that owns all device memory, or a plugin whose host
+ * forbids allocation).  It computes exactly what nl_sort_hilbert computes,
+ * with the same arguments and outputs and no context; its scratch lives in a
+ * static device array inside libnl.so (about 26 MiB, held by every GPU that
+ * loads the library until the process exits), which bounds n to at most
+ * 2^20 = 1,048,576 atoms: larger n returns NL_ERR_CAPACITY without touching
+ * the GPU.  The first call on each device looks up the array's device
+ * address (with that device current); make that first call before any
+ * stream capture.  All calls share the array, so calls whose work overlaps
+ * on the GPU race; order them on one stream.  status_out (device int32[1],
+ * may be NULL) receives NL_OK, or NL_ERR_TIMEOUT if a bounded device wait
+ * gave up during this call. */
+nl_status nl_sort_hilbert_noalloc(int64_t n, const float *pos, const float *box,
+                                  int32_t *perm_out, float *pos_sorted_out, uint64_t *keys_out,
+                                  int32_t *status_out, void *stream);
+
 /* Per-kernel timing with CUDA events recorded on the call's stream.
  * nl_profile_enable(ctx, 1) starts recording; nl_profile_read synchronizes
  * the device, writes for each phase p < max_phases the summed milliseconds

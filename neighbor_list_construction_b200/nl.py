@@ -41,6 +41,7 @@ _SIGS = {
     "nl_profile_enable": (_i32, [_vp, ctypes.c_int]),
     "nl_profile_read": (_i32, [_vp, _vp, _vp, _i32]),
     "nl_profile_phase_name": (ctypes.c_char_p, [_i32]),
+    "nl_sort_hilbert_noalloc": (_i32, [_i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nls_displace": (_i32, [_i64, _vp, _u64, _i64, _vp, _f32, _vp]),
     "nls_step_graph": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _u64, _vp, _f32]),
     "nls_graph_destroy": (None, [_vp]),
@@ -121,6 +122,15 @@ def nl_sort_morton(ctx, pos, box, perm_out, pos_sorted_out, keys_out=None, strea
     return _check(_lib.nl_sort_morton(ctx, pos.shape[0], _ptr(pos), _box(box), _ptr(perm_out),
                                       _ptr(pos_sorted_out), _ptr(keys_out), _stream(stream)),
                   "nl_sort_morton")
+
+
+def nl_sort_hilbert_noalloc(pos, box, perm_out, pos_sorted_out, keys_out=None, status_out=None,
+                            stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_sort_hilbert_noalloc(pos.shape[0], _ptr(pos), _box(box), _ptr(perm_out),
+                                               _ptr(pos_sorted_out), _ptr(keys_out),
+                                               _ptr(status_out), _stream(stream)),
+                  "nl_sort_hilbert_noalloc")
 
 
 def nl_build(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, stream=None) -> int:
