@@ -31,7 +31,8 @@ void free_ctx(nl_ctx *c)
     if (c->replay_graph) cudaGraphDestroy(c->replay_graph);
     void *bufs[] = {c->keys[0], c->keys[1], c->vals[0], c->vals[1], c->hist, c->sort_status,
                     c->sort_ctr, c->cell_count, c->cell_start, c->scan_status, c->scan_ctr,
-                    c->atom_cell, c->atom_rank, c->cell_pos, c->ref, c->zero_block};
+                    c->atom_cell, c->atom_rank, c->cell_pos, c->ref, c->zero_block,
+                    c->fb_list};
     for (void *b : bufs)
         if (b) cudaFree(b);
     if (c->prof_ev) {
@@ -371,11 +372,15 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
     ok &= alloc(&c->cell_pos, N) == cudaSuccess;
     ok &= alloc(&c->ref, N) == cudaSuccess;
     ok &= alloc(&c->zero_block, 64) == cudaSuccess;
+    ok &= alloc(&c->fb_list, c->max_cells) == cudaSuccess;
     if (ok) {
         c->flags = c->zero_block;
         c->skin_acc = c->zero_block + 4;
         c->step = reinterpret_cast<int32_t *>(c->zero_block + 8);
         c->rebuild_tmp = reinterpret_cast<int32_t *>(c->zero_block + 9);
+        c->unsorted = c->zero_block + 12;
+        c->fb_count = c->zero_block + 13;
+        ok &= pairs_set_attributes() == cudaSuccess;
         ok &= cudaMemset(c->zero_block, 0, 64 * sizeof(uint32_t)) == cudaSuccess;
         ok &= cudaDeviceSynchronize() == cudaSuccess;
     }

@@ -145,7 +145,8 @@ __device__ __forceinline__ bool before_xi(float xa, int ia, float xb, int ib)
 // One warp per cell: rank every atom of the cell by (x, index) with shuffles
 // and store it at its rank.  Cells above kCellSortMax stay in scatter order.
 __global__ void __launch_bounds__(256)
-k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell)
+k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell,
+            uint32_t *unsorted)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -153,7 +154,11 @@ k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_star
     for (int64_t c = warp; c < ncell; c += nwarps) {
         const int32_t s = cell_start[c];
         const int m = cell_start[c + 1] - s;
-        if (m <= 1 || m > kCellSortMax) continue;
+        if (m > kCellSortMax) {
+            if (lane == 0) atomicOr(unsorted, 1u);
+            continue;
+        }
+        if (m <= 1) continue;
         if (m <= 32) {
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (lane < m) v = cell_pos[s + lane];
@@ -216,6 +221,7 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
     NL_CUDA_TRY(cudaMemsetAsync(ctx->cell_count, 0, sizeof(int32_t) * g.ncell, s));
     NL_CUDA_TRY(cudaMemsetAsync(ctx->scan_status, 0, sizeof(uint32_t) * scan_tiles, s));
     NL_CUDA_TRY(cudaMemsetAsync(ctx->scan_ctr, 0, sizeof(uint32_t), s));
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->unsorted, 0, sizeof(uint32_t), s));
     {
         ProfScope ps(ctx, PH_BIN_COUNT, s);
         if (n > 0)
@@ -240,8 +246,8 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
     }
     {
         ProfScope ps(ctx, PH_CELL_SORT, s);
-        k_cell_sort<<<grid_for(g.ncell * 32, 256, cap), 256, 0, s>>>(ctx->cell_pos,
-                                                                      ctx->cell_start, g.ncell);
+        k_cell_sort<<<grid_for(g.ncell * 32, 256, cap), 256, 0, s>>>(
+            ctx->cell_pos, ctx->cell_start, g.ncell, ctx->unsorted);
         NL_CUDA_TRY(cudaGetLastError());
     }
     return cudaSuccess;

@@ -97,6 +97,9 @@ struct nl_ctx {
     uint32_t *skin_acc = nullptr;      // [2]: max bits, block ticket
     int32_t *step = nullptr;           // [1] replay iteration index
     int32_t *rebuild_tmp = nullptr;    // [1]
+    uint32_t *unsorted = nullptr;      // [1] 1 if a cell was too large for the in-cell sort
+    uint32_t *fb_count = nullptr;      // [1] tiles listed for the per-atom search
+    uint32_t *fb_list = nullptr;       // [max_cells] their ids
     uint32_t *zero_block = nullptr;    // one allocation holding the small state
 
     // last build
@@ -153,6 +156,8 @@ cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, flo
 // Cell binning of `pos` into ctx->cell_pos (cell order, x-sorted in cells).
 cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const CellGrid &g,
                            cudaStream_t s);
+// One-time kernel attributes of the pair search (large dynamic shared memory).
+cudaError_t pairs_set_attributes();
 // Pair search over the binned atoms.
 cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
                          int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast);

@@ -156,6 +156,30 @@ def test_overflow_status_and_rows(ctx, oracle):
     gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt, full_sets=sets)
 
 
+def test_build_mixed_density_uses_both_paths(ctx, nl, oracle):
+    """A dense slab whose tiles overflow the shared-memory stage (listed for
+    the per-atom search) beside sparse tiles that are staged; rows with more
+    neighbors than the capacity are checked as subsets."""
+    rng = np.random.default_rng(44)
+    box = np.array([25.0, 25.0, 25.0], np.float32)
+    # 9 cells of 2.78 A per axis; the slab fills x-cells 0 and 1 with ~200
+    # atoms per cell, so a tile's 9 rows hold ~3,600 atoms (over the stage)
+    sparse = rng.random((1600, 3)) * box
+    dense = rng.random((32400, 3)) * np.array([5.5, 25.0, 25.0])
+    pos = np.zeros((34000, 4), np.float32)
+    pos[:, :3] = np.concatenate([sparse, dense])[rng.permutation(34000)]
+    K = 256
+    nbr, cnt, st = gpu_build(ctx, pos, box, 2.0, 0.5, K)
+    info = nl.nl_last_build_info(ctx.handle)
+    assert info[3] == 1  # staged kernel ran (dense tiles went to the listed path)
+    full, fcnt, _ = oracle.build(pos, box, 2.0, 0.5, 1024)
+    o_nbr = full[:, :K]
+    sets = [set(full[i, :fcnt[i]].tolist()) for i in range(pos.shape[0])]
+    assert st == (1 if (fcnt > K).any() else 0)
+    gu.assert_rows_match(nbr, cnt, np.where(np.arange(K) < fcnt[:, None], o_nbr, -1), fcnt,
+                         full_sets=sets)
+
+
 @pytest.mark.parametrize("name", ["saltwater1m", "saltwater10m", "shell10m"])
 def test_build_full_size_sampled(ctx, oracle, name):
     """Full-size workloads, in the order the benchmark uses (curve-sorted):
