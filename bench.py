@@ -47,7 +47,9 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+        # nvidia-smi numbers GPUs physically; map through CUDA_VISIBLE_DEVICES
+        vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+        self.gpu = vis[gpu_index] if gpu_index < len(vis) else str(gpu_index)
         self.proc = None
         self.lines: list[str] = []
         self.thread = None
@@ -66,12 +68,21 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
-    def stop(self) -> dict:
+    def window(self, t0: float, t1: float) -> dict:
+        """Median clocks and active throttle reasons of the samples taken
+        between host times t0 and t1 (the sampler keeps running)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        deadline = time.monotonic() + 1.0
+        while time.monotonic() < deadline and (not self.lines or self.lines[-1][0] < t1):
+            time.sleep(0.05)
+        return self._summary([ln for (t, ln) in list(self.lines) if t0 <= t <= t1 + 0.15])
+
+    def stop(self) -> None:
+        if self.proc is None:
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -79,9 +90,11 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
+
+    def _summary(self, lines) -> dict:
         sm, mx, reasons = [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -150,11 +163,93 @@ def run_reference(args, rank: int, world: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def interval_timing(nl, torch, h, ps_src, w, K, steps: int, seed: int = 2024) -> dict:
+    """The skin-check interval: `steps` iterations of [stand-in MD step ->
+    skin check -> rebuild if needed], once as one replayed CUDA graph
+    (nl_replay) and once eagerly from the host (launch, read the decision,
+    rebuild).  Device time per step for each."""
+    n = ps_src.shape[0]
+    stream = torch.cuda.current_stream()
+    nbr = torch.empty(n, K, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(n, dtype=torch.int32, device="cuda")
+    dec = torch.zeros(steps, dtype=torch.int32, device="cuda")
+    rb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = {}
+    # graph
+    p = ps_src.clone()
+    nl.nl_build(h, p, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+    g = nl.nls_step_graph(p, seed, nl.nl_step_counter(h), w.sigma_step)
+    try:
+        nl.nl_replay(h, g, steps, p, w.box, w.cutoff, w.skin, K, nbr, cnt, dec, stream)  # warm
+        p.copy_(ps_src)
+        nl.nl_build(h, p, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        nl.nl_replay(h, g, steps, p, w.box, w.cutoff, w.skin, K, nbr, cnt, dec, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out["graph_ms_per_step"] = e0.elapsed_time(e1) / steps
+        out["rebuilds"] = int(dec.sum().item())
+    finally:
+        nl.nls_graph_destroy(g)
+    # eager
+    p.copy_(ps_src)
+    nl.nl_build(h, p, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+    torch.cuda.synchronize()
+    rbh = torch.zeros(1, dtype=torch.int32).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    rebuilds = 0
+    for t in range(1, steps + 1):
+        nl.nls_displace(p, seed, t, w.sigma_step, None, stream)
+        nl.nl_skin_check(h, p, w.box, w.skin, rb, None, stream)
+        rbh.copy_(rb, non_blocking=True)
+        stream.synchronize()
+        if rbh.item():
+            rebuilds += 1
+            nl.nl_build(h, p, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    out["eager_ms_per_step"] = e0.elapsed_time(e1) / steps
+    out["eager_rebuilds"] = rebuilds
+    out["steps"] = steps
+    out["graph_speedup"] = out["eager_ms_per_step"] / out["graph_ms_per_step"]
+    return out
+
+
+def curve_comparison(nl, torch, h, pos, w, K, reps: int = 5) -> dict:
+    """nl_build time after a Hilbert sort vs after a Morton sort (same atoms)."""
+    n = pos.shape[0]
+    stream = torch.cuda.current_stream()
+    perm = torch.empty(n, dtype=torch.int32, device="cuda")
+    ps = torch.empty(n, 4, dtype=torch.float32, device="cuda")
+    nbr = torch.empty(n, K, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(n, dtype=torch.int32, device="cuda")
+    res = {}
+    for curve, fn in (("hilbert", nl.nl_sort_hilbert), ("morton", nl.nl_sort_morton)):
+        fn(h, pos, w.box, perm, ps, None, stream)
+        nl.nl_build(h, ps, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            nl.nl_build(h, ps, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res[f"{curve}_build_ms"] = e0.elapsed_time(e1) / reps
+    return res
+
+
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
     from neighbor_list_construction_b200 import nl, workloads
 
+    # nvidia-smi starts before this process touches the GPU, so its start-up
+    # never overlaps a timed region; samples are matched to regions by time.
+    clocks = ClockSampler(local_rank)
+    clocks.start()
     torch.cuda.set_device(local_rank)
     w = workloads.make(args.workload)
     n, K = w.n, w.capacity
@@ -198,11 +293,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     nl.nl_profile_read(h)
 
     # ---- device-resident timed region
-    clocks = ClockSampler(local_rank)
     nl.nl_profile_enable(h, True)
     barrier()
-    clocks.start()
-    time.sleep(0.3)
+    t_host0 = time.monotonic()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -210,7 +303,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         step(pos)
     e1.record(stream)
     barrier()
-    clk = clocks.stop()
+    clk = clocks.window(t_host0, time.monotonic())
     ms = e0.elapsed_time(e1) / args.steps
     phases = nl.nl_profile_read(h)
     nl.nl_profile_enable(h, False)
@@ -283,11 +376,15 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             "gpu_launches": int(round(launches_per_step * args.steps)),
             "status": nl.nl_status_string(st),
         }
+        if args.extras and world == 1:
+            line["interval"] = interval_timing(nl, torch, h, ps, w, K, w.steps or 200)
+            line["curves"] = curve_comparison(nl, torch, h, pos, w, K)
         if world == 1 and not args.no_cpu_baseline:
             cb = oracle_sample(1)
             line["cpu_baseline"] = {"value": cb["value"], "unit": "atoms/s", "cores": cb["cores"],
                                     "kind": "oracle", "sample": cb["sample"]}
         print(json.dumps(line), flush=True)
+    clocks.stop()
     ctx.close()
 
 
@@ -299,6 +396,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="saltwater10m")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extras", action="store_true",
+                    help="also time the replayed skin-check interval (graph vs eager) "
+                         "and nl_build after Hilbert vs Morton order")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -32,7 +32,7 @@ void free_ctx(nl_ctx *c)
     void *bufs[] = {c->keys[0], c->keys[1], c->vals[0], c->vals[1], c->hist, c->sort_status,
                     c->sort_ctr, c->cell_count, c->cell_start, c->scan_status, c->scan_ctr,
                     c->atom_cell, c->atom_rank, c->cell_pos, c->ref, c->zero_block,
-                    c->fb_list};
+                    c->fb_list, c->cell_tab};
     for (void *b : bufs)
         if (b) cudaFree(b);
     if (c->prof_ev) {
@@ -55,10 +55,15 @@ nl_status check_box(const float *box)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Cell grid: n_a = floor(L_a / (rl (1 + 2^-20) + L_a 2^-20)) cells per axis,
-// so that a cell stays wider than rl even after the fp32 rounding of the
-// cell assignment floor(w * fl(n/L)) (which moves an atom by at most a few
-// ulp of L); coarsened if the grid would exceed the context's cell budget.
+// Cell grid.  Preferred ("column") grid: cells at least rl wide along x and
+// rl/2 wide along y and z, so a neighbor lies within +-1 cell in x and +-2
+// cells in y and z; it needs >= 5 cells in x and >= 7 in y and z so that the
+// periodic shift of every stencil cell is known (see nl_pairs.cu).  Smaller
+// boxes get cells at least rl wide on every axis (>= 3 per axis, else
+// NL_ERR_BOX) and the literal minimum image.  A cell's width carries a margin
+// of rl*2^-20 + L*2^-20 over its nominal minimum, so the fp32 rounding of the
+// cell assignment floor(w * fl(n/L)) never moves a neighbor outside the
+// stencil.  Grids above the context's cell budget are coarsened.
 nl_status make_grid(nl_ctx *ctx, const float *box, float cutoff, float skin, CellGrid *g)
 {
     if (!std::isfinite(cutoff) || !std::isfinite(skin) || cutoff < 0.0f || skin < 0.0f)
@@ -66,20 +71,37 @@ nl_status make_grid(nl_ctx *ctx, const float *box, float cutoff, float skin, Cel
     volatile float rl = cutoff + skin;
     if (!(rl > 0.0f)) return NL_ERR_ARG;
     volatile float rl2 = rl * rl;
-    int64_t n[3];
-    for (int a = 0; a < 3; ++a) {
+    const double eps = std::ldexp(1.0, -20);
+    auto cells = [&](int a, double width) {
         const double L = box[a];
-        const double side = (double)rl * (1.0 + std::ldexp(1.0, -20)) + L * std::ldexp(1.0, -20);
-        const double m = std::floor(L / side);
-        n[a] = m > 4096.0 ? 4096 : (int64_t)m;
-        if (n[a] < 3) return NL_ERR_BOX;
+        const double m = std::floor(L / (width * (1.0 + eps) + L * eps));
+        return m > 8192.0 ? (int64_t)8192 : (int64_t)m;
+    };
+    int64_t n[3];
+    int wy = 2, wz = 2, literal = 0;
+    n[0] = cells(0, (double)rl);
+    n[1] = cells(1, 0.5 * (double)rl);
+    n[2] = cells(2, 0.5 * (double)rl);
+    bool columns = n[0] >= 5 && n[1] >= 7 && n[2] >= 7;
+    if (columns) {
+        while (n[0] * n[1] * n[2] > ctx->max_cells) {
+            int a = n[0] > n[1] ? (n[0] > n[2] ? 0 : 2) : (n[1] > n[2] ? 1 : 2);
+            n[a] = n[a] * 7 / 8;
+        }
+        columns = n[0] >= 5 && n[1] >= 7 && n[2] >= 7;
     }
-    while (n[0] * n[1] * n[2] > ctx->max_cells) {
-        int a = 0;
-        for (int b = 1; b < 3; ++b)
-            if (n[b] > n[a]) a = b;
-        n[a] = n[a] * 7 / 8;
-        if (n[a] < 3) return NL_ERR_BOX;
+    if (!columns) {
+        wy = wz = 1;
+        for (int a = 0; a < 3; ++a) {
+            n[a] = cells(a, (double)rl);
+            if (n[a] < 3) return NL_ERR_BOX;
+        }
+        while (n[0] * n[1] * n[2] > ctx->max_cells) {
+            int a = n[0] > n[1] ? (n[0] > n[2] ? 0 : 2) : (n[1] > n[2] ? 1 : 2);
+            n[a] = n[a] * 7 / 8;
+            if (n[a] < 3) return NL_ERR_BOX;
+        }
+        literal = (n[0] < 5 || n[1] < 5 || n[2] < 5) ? 1 : 0;
     }
     g->nx = (int)n[0];
     g->ny = (int)n[1];
@@ -95,7 +117,9 @@ nl_status make_grid(nl_ctx *ctx, const float *box, float cutoff, float skin, Cel
     g->Tz = tz;
     g->rl2 = rl2;
     g->ncell = n[0] * n[1] * n[2];
-    g->literal = (n[0] < 5 || n[1] < 5 || n[2] < 5) ? 1 : 0;
+    g->wy = wy;
+    g->wz = wz;
+    g->literal = literal;
     return NL_OK;
 }
 
@@ -373,6 +397,7 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
     ok &= alloc(&c->ref, N) == cudaSuccess;
     ok &= alloc(&c->zero_block, 64) == cudaSuccess;
     ok &= alloc(&c->fb_list, c->max_cells) == cudaSuccess;
+    ok &= alloc(&c->cell_tab, (size_t)c->max_cells * 16) == cudaSuccess;
     if (ok) {
         c->flags = c->zero_block;
         c->skin_acc = c->zero_block + 4;

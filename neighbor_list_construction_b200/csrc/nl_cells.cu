@@ -143,10 +143,14 @@ __device__ __forceinline__ bool before_xi(float xa, int ia, float xb, int ib)
 }
 
 // One warp per cell: rank every atom of the cell by (x, index) with shuffles
-// and store it at its rank.  Cells above kCellSortMax stay in scatter order.
+// and store it at its rank.  Also writes the cell's x sub-bin table: byte b
+// (b = 0..15) = number of the cell's atoms whose x lies below the cell's low
+// x face plus b/16 of its width (bin of an atom = floor((x - face) * 16 /
+// width), clamped to 0..15).  The pair search reads these to find x-windows.
+// Cells above kCellSortMax stay in scatter order and raise `unsorted`.
 __global__ void __launch_bounds__(256)
 k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell,
-            uint32_t *unsorted)
+            int nx, float side_x, float inv_bin, uint8_t *__restrict__ cell_tab, uint32_t *unsorted)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -158,38 +162,46 @@ k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_star
             if (lane == 0) atomicOr(unsorted, 1u);
             continue;
         }
-        if (m <= 1) continue;
+        const float face = (float)(int)(c % nx) * side_x;
+        int below = 0;  // lanes 0..15: atoms with bin < lane
         if (m <= 32) {
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (lane < m) v = cell_pos[s + lane];
             const int id = __float_as_int(v.w);
+            const int bin = max(0, min(15, (int)floorf((v.x - face) * inv_bin)));
             int r = 0;
             for (int j = 0; j < m; ++j) {
                 const float xj = __shfl_sync(0xffffffffu, v.x, j);
                 const int ij = __shfl_sync(0xffffffffu, id, j);
+                const int bj = __shfl_sync(0xffffffffu, bin, j);
                 r += before_xi(xj, ij, v.x, id) ? 1 : 0;
+                below += bj < lane ? 1 : 0;
             }
             __syncwarp();
-            if (lane < m) cell_pos[s + r] = v;
+            if (lane < m && m > 1) cell_pos[s + r] = v;
         } else {
             constexpr int E = kCellSortMax / 32;
             float4 v[E];
-            int r[E];
+            int r[E], bin[E];
 #pragma unroll
             for (int e = 0; e < E; ++e) {
                 r[e] = 0;
                 v[e] = e * 32 + lane < m ? cell_pos[s + e * 32 + lane]
                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                bin[e] = max(0, min(15, (int)floorf((v[e].x - face) * inv_bin)));
             }
 #pragma unroll
             for (int es = 0; es < E; ++es) {
                 if (es * 32 >= m) break;
                 const float xs = v[es].x;
                 const int is = __float_as_int(v[es].w);
+                const int bs = bin[es];
                 const int lim = m - es * 32 < 32 ? m - es * 32 : 32;
                 for (int l = 0; l < lim; ++l) {
                     const float xj = __shfl_sync(0xffffffffu, xs, l);
                     const int ij = __shfl_sync(0xffffffffu, is, l);
+                    const int bj = __shfl_sync(0xffffffffu, bs, l);
+                    below += bj < lane ? 1 : 0;
 #pragma unroll
                     for (int e = 0; e < E; ++e)
                         r[e] += before_xi(xj, ij, v[e].x, __float_as_int(v[e].w)) ? 1 : 0;
@@ -200,6 +212,7 @@ k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_star
             for (int e = 0; e < E; ++e)
                 if (e * 32 + lane < m) cell_pos[s + r[e]] = v[e];
         }
+        if (lane < 16) cell_tab[c * 16 + lane] = (uint8_t)below;
     }
 }
 
@@ -246,8 +259,10 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
     }
     {
         ProfScope ps(ctx, PH_CELL_SORT, s);
+        const float side_x = g.Lx / (float)g.nx;
         k_cell_sort<<<grid_for(g.ncell * 32, 256, cap), 256, 0, s>>>(
-            ctx->cell_pos, ctx->cell_start, g.ncell, ctx->unsorted);
+            ctx->cell_pos, ctx->cell_start, g.ncell, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
+            ctx->unsorted);
         NL_CUDA_TRY(cudaGetLastError());
     }
     return cudaSuccess;

@@ -55,12 +55,13 @@ enum Phase {
 
 // Cell grid of one build, all values computed on the host.
 struct CellGrid {
-    int nx, ny, nz;          // cells per axis (>= 3)
+    int nx, ny, nz;          // cells per axis
     float Lx, Ly, Lz;        // box
     float Tx, Ty, Tz;        // fl(n_a / L_a): cell coordinate = floor(w * T)
     float rl2;               // fl(rl * rl)
     int64_t ncell;
-    int literal;             // 1: some axis has < 5 cells -> literal min image
+    int wy, wz;              // stencil half-width in y and z (x is always 1)
+    int literal;             // 1: literal minimum image (small boxes)
 };
 
 }  // namespace nl
@@ -90,6 +91,7 @@ struct nl_ctx {
     uint32_t *atom_cell = nullptr;     // [max_atoms]
     uint32_t *atom_rank = nullptr;     // [max_atoms]
     float4 *cell_pos = nullptr;        // [max_atoms] wrapped xyz + index bits
+    uint8_t *cell_tab = nullptr;       // [max_cells][16] x sub-bin tables
     float4 *ref = nullptr;             // [max_atoms] reference positions
 
     // status and small state
