@@ -142,77 +142,113 @@ __device__ __forceinline__ bool before_xi(float xa, int ia, float xb, int ib)
     return xa < xb || (xa == xb && ia < ib);
 }
 
-// One warp per cell: rank every atom of the cell by (x, index) with shuffles
-// and store it at its rank.  Also writes the cell's x sub-bin table: byte b
-// (b = 0..15) = number of the cell's atoms whose x lies below the cell's low
-// x face plus b/16 of its width (bin of an atom = floor((x - face) * 16 /
-// width), clamped to 0..15).  The pair search reads these to find x-windows.
-// Cells above kCellSortMax stay in scatter order and raise `unsorted`.
+// Sorts the atoms of cell c by (x, index) in place and writes the cell's x
+// sub-bin table: byte b (b = 0..15) = number of the cell's atoms whose x is
+// below the cell's low x face plus b/16 of its width (bin of an atom =
+// floor((x - face) * 16 / width), clamped to 0..15).  The pair search reads
+// these to find x-windows.  Half-warp version for cells of at most 16 atoms:
+// lane hl of the half owns atom hl, ranks it with shuffles inside the half
+// and computes table entry hl.
+__device__ __forceinline__ void sort_small_cell(float4 *__restrict__ cell_pos, int32_t s, int m,
+                                                float face, float inv_bin, uint8_t *tab, int hl,
+                                                bool real)
+{
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (hl < m) v = cell_pos[s + hl];
+    const int id = __float_as_int(v.w);
+    const int bin = max(0, min(15, (int)floorf((v.x - face) * inv_bin)));
+    int r = 0, below = 0;
+    for (int j = 0; j < 16; ++j) {
+        const float xj = __shfl_sync(0xffffffffu, v.x, j, 16);
+        const int ij = __shfl_sync(0xffffffffu, id, j, 16);
+        const int bj = __shfl_sync(0xffffffffu, bin, j, 16);
+        if (j < m) {
+            r += before_xi(xj, ij, v.x, id) ? 1 : 0;
+            below += bj < hl ? 1 : 0;
+        }
+    }
+    __syncwarp();
+    if (!real) return;   // a half with no cell only takes part in the shuffles
+    if (hl < m && m > 1) cell_pos[s + r] = v;
+    tab[hl] = (uint8_t)below;
+}
+
+// Full-warp version for cells of 17..kCellSortMax atoms (8 atoms per lane).
+__device__ __forceinline__ void sort_large_cell(float4 *__restrict__ cell_pos, int32_t s, int m,
+                                                float face, float inv_bin, uint8_t *tab, int lane)
+{
+    constexpr int E = kCellSortMax / 32;
+    float4 v[E];
+    int r[E], bin[E];
+    int below = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        r[e] = 0;
+        v[e] = e * 32 + lane < m ? cell_pos[s + e * 32 + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+        bin[e] = max(0, min(15, (int)floorf((v[e].x - face) * inv_bin)));
+    }
+#pragma unroll
+    for (int es = 0; es < E; ++es) {
+        if (es * 32 >= m) break;
+        const float xs = v[es].x;
+        const int is = __float_as_int(v[es].w);
+        const int bs = bin[es];
+        const int lim = m - es * 32 < 32 ? m - es * 32 : 32;
+        for (int l = 0; l < lim; ++l) {
+            const float xj = __shfl_sync(0xffffffffu, xs, l);
+            const int ij = __shfl_sync(0xffffffffu, is, l);
+            const int bj = __shfl_sync(0xffffffffu, bs, l);
+            below += bj < lane ? 1 : 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                r[e] += before_xi(xj, ij, v[e].x, __float_as_int(v[e].w)) ? 1 : 0;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (e * 32 + lane < m) cell_pos[s + r[e]] = v[e];
+    if (lane < 16) tab[lane] = (uint8_t)below;
+}
+
+// Two cells per warp (one per half); a cell above 16 atoms is redone by the
+// whole warp, and one above kCellSortMax stays in scatter order and raises
+// `unsorted`.
 __global__ void __launch_bounds__(256)
 k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell,
             int nx, float side_x, float inv_bin, uint8_t *__restrict__ cell_tab, uint32_t *unsorted)
 {
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t c = warp; c < ncell; c += nwarps) {
-        const int32_t s = cell_start[c];
-        const int m = cell_start[c + 1] - s;
-        if (m > kCellSortMax) {
-            if (lane == 0) atomicOr(unsorted, 1u);
+    for (int64_t c0 = 2 * warp; c0 < ncell; c0 += 2 * nwarps) {
+        const int64_t c = c0 + half;
+        const bool have = c < ncell;
+        const int32_t s = have ? cell_start[c] : 0;
+        const int m = have ? cell_start[c + 1] - s : 0;
+        const float face = (float)(int)(c % nx) * side_x;
+        const bool small = m <= 16;
+        if (__all_sync(0xffffffffu, small)) {
+            sort_small_cell(cell_pos, s, m, face, inv_bin, cell_tab + (have ? c : 0) * 16, hl, have);
             continue;
         }
-        const float face = (float)(int)(c % nx) * side_x;
-        int below = 0;  // lanes 0..15: atoms with bin < lane
-        if (m <= 32) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (lane < m) v = cell_pos[s + lane];
-            const int id = __float_as_int(v.w);
-            const int bin = max(0, min(15, (int)floorf((v.x - face) * inv_bin)));
-            int r = 0;
-            for (int j = 0; j < m; ++j) {
-                const float xj = __shfl_sync(0xffffffffu, v.x, j);
-                const int ij = __shfl_sync(0xffffffffu, id, j);
-                const int bj = __shfl_sync(0xffffffffu, bin, j);
-                r += before_xi(xj, ij, v.x, id) ? 1 : 0;
-                below += bj < lane ? 1 : 0;
+        // at least one of the two cells is large: whole warp, one cell at a time
+        for (int h = 0; h < 2; ++h) {
+            const int64_t cc = c0 + h;
+            if (cc >= ncell) break;
+            const int32_t ss = cell_start[cc];
+            const int mm = cell_start[cc + 1] - ss;
+            const float ff = (float)(int)(cc % nx) * side_x;
+            if (mm > kCellSortMax) {
+                if (lane == 0) atomicOr(unsorted, 1u);
+            } else if (mm <= 16) {
+                // half 0 sorts; half 1 only pairs the shuffles
+                sort_small_cell(cell_pos, ss, half == 0 ? mm : 0, ff, inv_bin, cell_tab + cc * 16, hl,
+                                half == 0);
+            } else {
+                sort_large_cell(cell_pos, ss, mm, ff, inv_bin, cell_tab + cc * 16, lane);
             }
-            __syncwarp();
-            if (lane < m && m > 1) cell_pos[s + r] = v;
-        } else {
-            constexpr int E = kCellSortMax / 32;
-            float4 v[E];
-            int r[E], bin[E];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                r[e] = 0;
-                v[e] = e * 32 + lane < m ? cell_pos[s + e * 32 + lane]
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                bin[e] = max(0, min(15, (int)floorf((v[e].x - face) * inv_bin)));
-            }
-#pragma unroll
-            for (int es = 0; es < E; ++es) {
-                if (es * 32 >= m) break;
-                const float xs = v[es].x;
-                const int is = __float_as_int(v[es].w);
-                const int bs = bin[es];
-                const int lim = m - es * 32 < 32 ? m - es * 32 : 32;
-                for (int l = 0; l < lim; ++l) {
-                    const float xj = __shfl_sync(0xffffffffu, xs, l);
-                    const int ij = __shfl_sync(0xffffffffu, is, l);
-                    const int bj = __shfl_sync(0xffffffffu, bs, l);
-                    below += bj < lane ? 1 : 0;
-#pragma unroll
-                    for (int e = 0; e < E; ++e)
-                        r[e] += before_xi(xj, ij, v[e].x, __float_as_int(v[e].w)) ? 1 : 0;
-                }
-            }
-            __syncwarp();
-#pragma unroll
-            for (int e = 0; e < E; ++e)
-                if (e * 32 + lane < m) cell_pos[s + r[e]] = v[e];
         }
-        if (lane < 16) cell_tab[c * 16 + lane] = (uint8_t)below;
     }
 }
 

@@ -311,6 +311,51 @@ __device__ __forceinline__ float cand_r2(const float4 q, const float4 me, int s,
     return r2_of(dx, dy, dz);
 }
 
+// One candidate, no periodic shift, as explicit PTX: three fp32
+// differences, three products, two sums, all round-to-nearest with no
+// contraction; on r2 < rl2 (and, for the home row, idx != self) append idx
+// to the row buffer.  Only used with FAST (no lane can pass B).
+template <bool SELF>
+__device__ __forceinline__ void test_plain(const float4 c, const float4 me, float rl2,
+                                           uint32_t self, uint32_t &bp)
+{
+    if (SELF)
+        asm volatile(
+            "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
+            "sub.rn.f32 dx, %1, %5;\n\t"
+            "sub.rn.f32 dy, %2, %6;\n\t"
+            "sub.rn.f32 dz, %3, %7;\n\t"
+            "mul.rn.f32 dx, dx, dx;\n\t"
+            "mul.rn.f32 dy, dy, dy;\n\t"
+            "mul.rn.f32 dz, dz, dz;\n\t"
+            "add.rn.f32 s, dx, dy;\n\t"
+            "add.rn.f32 s, s, dz;\n\t"
+            "setp.lt.f32 p, s, %8;\n\t"
+            "setp.ne.and.u32 p, %4, %9, p;\n\t"
+            "@p st.shared.b32 [%0], %4;\n\t"
+            "@p add.u32 %0, %0, 4;\n\t}"
+            : "+r"(bp)
+            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "f"(me.x), "f"(me.y),
+              "f"(me.z), "f"(rl2), "r"(self));
+    else
+        asm volatile(
+            "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
+            "sub.rn.f32 dx, %1, %5;\n\t"
+            "sub.rn.f32 dy, %2, %6;\n\t"
+            "sub.rn.f32 dz, %3, %7;\n\t"
+            "mul.rn.f32 dx, dx, dx;\n\t"
+            "mul.rn.f32 dy, dy, dy;\n\t"
+            "mul.rn.f32 dz, dz, dz;\n\t"
+            "add.rn.f32 s, dx, dy;\n\t"
+            "add.rn.f32 s, s, dz;\n\t"
+            "setp.lt.f32 p, s, %8;\n\t"
+            "@p st.shared.b32 [%0], %4;\n\t"
+            "@p add.u32 %0, %0, 4;\n\t}"
+            : "+r"(bp)
+            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "f"(me.x), "f"(me.y),
+              "f"(me.z), "f"(rl2));
+}
+
 // Tests L consecutive candidates q[0..L) of one row (stage slots slot0 ..)
 // against this lane's atom: groups of 8, then of 4, then single ones.
 template <bool XS, bool YZ, bool SELF, bool FAST>
@@ -320,6 +365,19 @@ __device__ __forceinline__ void scan_row(const float4 *__restrict__ q, int slot0
 {
     const uint32_t self = (uint32_t)__float_as_int(me.w);
     int k = 0;
+    if (!XS && !YZ && FAST) {
+        uint32_t bp = o.bp;
+        for (; k + 8 <= L; k += 8) {
+            float4 c[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) c[u] = q[k + u];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) test_plain<SELF>(c[u], me, rl2, self, bp);
+        }
+        for (; k < L; ++k) test_plain<SELF>(q[k], me, rl2, self, bp);
+        o.bp = bp;
+        return;
+    }
     for (; k + 8 <= L; k += 8) {
         float4 c[8];
 #pragma unroll
