@@ -95,59 +95,76 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Staged column search (column grid only: cells rl wide in x, rl/2 in y, z).
+// Staged tile search (column grid only: cells >= rl wide in x, >= rl/2 in y
+// and z, so the stencil is +-1 cell in x and +-2 cells in y and z).
 //
-// A tile is kTileCells consecutive cells along x of one (cy, cz) column.
-// Its 25 neighbor rows (dy, dz in -2..2), each covering cells cx0-1 ..
-// cx0+G along x (plus one periodic image cell at either end of the box), are
-// contiguous ranges of the cell-ordered array; one warp lane per row issues
-// their cp.async.bulk copies into shared memory, completing on one mbarrier.
-// Atoms of a row are sorted by x, so the candidates of a home atom in a row
-// lie in the index window of [x - h, x + h], h = sqrt(rl^2 - d_perp^2) from
-// the atom's distance to the row's (y, z) cell face, plus a margin.  The
-// window ends come from a per-row table of first indices at 1/16-cell steps
-// in x (conservative: a window never loses a candidate).  Each lane owns one
-// home atom of the tile (the tile's home atoms are x-sorted and share one
-// narrow (y, z) column, so their windows have similar lengths); every lane
-// walks the warp's longest window length from its own start, so a lane may
-// test atoms beyond its window -- harmless, since every tested pair is
-// decided by the exact predicate.  Hits are kept as 16-bit stage slots in a
-// per-lane row in shared memory and written out as full 16-byte row vectors.
+// A tile is kTX x kTY x kTZ home cells.  Its 36 staged rows (y and z from
+// two cells below to two cells above the home block) each cover the
+// conceptual cells cx0-1 .. cx0+Gx along x, with a periodic image cell at
+// either end of the box.  Every row is a contiguous range of the
+// cell-ordered array; one lane per row issues its cp.async.bulk copies into
+// shared memory, all completing on one mbarrier.  Rows are separated by
+// kGap slots of NaN (a NaN candidate never passes r2 < rl2).
+//
+// A home atom meets 25 rows (dy, dz in -2..2).  Atoms of a row are sorted by
+// x, so its candidates in a row lie in the slot window of [x - h, x + h],
+// h = sqrt(rl^2 - d_perp^2) from the atom's distance to the row's (y, z)
+// cell face plus a margin; the window ends come from per-cell tables of
+// first slots at 1/16-cell steps in x (conservative: no candidate is lost).
+// Each window becomes a segment of whole groups of 4 slots (extended into
+// the row or into the NaN gap; an extra tested atom is decided by the exact
+// predicate like any other).  The home row's window is split around the
+// atom's own slot, so self never reaches the predicate.  A lane walks the
+// concatenation of its segments; the warp runs for the largest lane total.
+//
+// Hits go to a per-lane buffer of two halves in shared memory; every 16
+// slots a lane with >= kFlushAt pending entries sends its whole 16-byte
+// vectors to its global row with one cp.async.bulk copy and continues in the
+// other half.  Rows are finished with -1 from a shared block of -1.
 // ---------------------------------------------------------------------------
-constexpr int kTileCells = 8;          // G: cells per tile along x
-constexpr int kRows = 25;              // (dy, dz) in -2..2
-constexpr int kCenterRow = 12;         // dy = dz = 0
-constexpr int kBinsPerCell = 16;       // x sub-bins per cell (tables built by k_cell_sort)
-constexpr int kRowCells = kTileCells + 2;
-constexpr int kStageMin = 2048;        // fewest staged atoms worth a launch
+constexpr int kTX = 5, kTY = 2, kTZ = 2;   // home cells per tile
+constexpr int kSY = kTY + 4, kSZ = kTZ + 4;
+constexpr int kSRows = kSY * kSZ;           // 36 staged rows
+constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
+constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
+constexpr int kRowTab = kSCells * kBinsPerCell;
+constexpr int kGap = 4;                     // NaN slots before, between and after rows
+constexpr int kSeg = 27;                    // segment descriptors per lane (25 rows, self split, end)
+constexpr int kHalf = 28;                   // entries per half of a lane's hit buffer
+constexpr int kFlushAt = 12;                // pending entries that trigger a flush
+constexpr int kTileWarps = 6;
+constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
-struct ColTile {
-    int row_off[kRows];
-    int row_len[kRows];
-    int row_lend[kRows];   // [0, lend): periodic image cell at the low x end (shift -Lx)
-    int row_rbeg[kRows];   // [rbeg, len): periodic image cell at the high x end (shift +Lx)
-    float row_sy[kRows];
-    float row_sz[kRows];
-    int row_cell[kRows][kRowCells + 1];   // staged start of each conceptual cell, then len
-    int total;
-    int home_begin, home_end;
+// Segment descriptor: first slot (14 bits), groups of 4 slots (12 bits),
+// staged row (6 bits).
+__host__ __device__ constexpr uint32_t seg_pack(uint32_t slot, uint32_t ng, uint32_t row)
+{
+    return slot | (ng << 14) | (row << 26);
+}
+
+struct TileRows {
+    int off[kSRows];                 // slot of the row's first atom
+    int len[kSRows];
+    int cell[kSRows][kSCells + 1];   // row-local start of conceptual cell k
+    int home_begin[4];               // slot of the first home atom of home row h
+    int home_pref[5];                // home atoms before home row h
+    int total;                       // staged slots, gaps included
     int fallback;
 };
 
-struct ColParams {
+struct TileParams {
     const float4 *cell_pos;
     const int32_t *cell_start;
+    const uint8_t *cell_tab;
     int32_t *nbr;
     int32_t *counts;
     uint32_t *flags;
     const uint32_t *unsorted;
     uint32_t *fb_list;
     uint32_t *fb_count;
-    const uint8_t *cell_tab;
-    int tiles_x;
+    int tiles_x, tiles_y;
     int K;
-    int B;              // row entries kept in shared memory (multiple of 4, <= K)
-    int stage_max;      // staged atoms per tile
+    int stage_max;      // staged slots per tile, gaps included
     float side_x, side_y, side_z;
     float inv_bin;      // kBinsPerCell / side_x (as in k_cell_sort)
     float eps;          // window margin (A)
@@ -157,20 +174,6 @@ struct ColParams {
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ float4 lds_f4(uint32_t addr)
-{
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ void sts_u16(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"((unsigned short)v) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
@@ -211,59 +214,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
-// Row output of one lane: the first B neighbor indices go to the lane's
-// buffer in shared memory (bp = next free byte, bufend = its end); entries
-// B .. K-1 of long rows go straight to the lane's global row (byte address of
-// entry e = gmap + smem address of entry e); entries past K are only counted.
-struct RowOut {
-    uint32_t bp, bufend, rowend;
-    uint64_t gmap;
-};
-
-// Appends `idx` when r2 < rl2 (and, for the home row, idx != self).  FAST:
-// no lane can pass B in this row -- one predicated shared store and a
-// predicated bump, no branch.  Otherwise also the global spill and the
-// capacity cut-off.
-template <bool SELF, bool FAST>
-__device__ __forceinline__ void append_if_hit(float r2, float rl2, uint32_t idx, uint32_t self,
-                                              RowOut &o)
-{
-    if (FAST) {
-        if (SELF)
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "setp.lt.f32 p, %1, %2;\n\t"
-                "setp.ne.and.u32 p, %3, %4, p;\n\t"
-                "@p st.shared.b32 [%0], %3;\n\t"
-                "@p add.u32 %0, %0, 4;\n\t}"
-                : "+r"(o.bp)
-                : "f"(r2), "f"(rl2), "r"(idx), "r"(self));
-        else
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "setp.lt.f32 p, %1, %2;\n\t"
-                "@p st.shared.b32 [%0], %3;\n\t"
-                "@p add.u32 %0, %0, 4;\n\t}"
-                : "+r"(o.bp)
-                : "f"(r2), "f"(rl2), "r"(idx));
-    } else {
-        const uint64_t ga = o.gmap + (uint64_t)o.bp;
-        asm volatile(
-            "{\n\t.reg .pred p, ps, pg;\n\t"
-            "setp.lt.f32 p, %1, %2;\n\t"
-            "setp.ne.and.u32 p, %3, %4, p;\n\t"
-            "setp.lt.and.u32 ps, %0, %5, p;\n\t"
-            "setp.ge.and.u32 pg, %0, %5, p;\n\t"
-            "setp.lt.and.u32 pg, %0, %6, pg;\n\t"
-            "@ps st.shared.b32 [%0], %3;\n\t"
-            "@pg st.global.b32 [%7], %3;\n\t"
-            "@p add.u32 %0, %0, 4;\n\t}"
-            : "+r"(o.bp)
-            : "f"(r2), "f"(rl2), "r"(idx), "r"(SELF ? self : 0xffffffffu), "r"(o.bufend),
-              "r"(o.rowend), "l"(ga));
-    }
-}
-
 // One contiguous shared -> global copy (16-byte aligned, 16-byte multiple),
 // tracked in this thread's bulk group.
 __device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes)
@@ -278,10 +228,11 @@ __device__ __forceinline__ void bulk_commit()
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-// Waits until this thread's bulk copies have read their shared-memory source.
+// Waits until at most N of this thread's bulk groups still read shared memory.
+template <int N>
 __device__ __forceinline__ void bulk_wait_read()
 {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void bulk_wait_all()
@@ -294,49 +245,55 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// r2 of one candidate against this lane's atom, with the row's periodic
-// shifts (XS: x image cells at the row ends; YZ: the row's y/z shift).
-template <bool XS, bool YZ>
-__device__ __forceinline__ float cand_r2(const float4 q, const float4 me, int s, float Lx,
-                                         int lend_slot, int rbeg_slot, float sy, float sz)
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr)
 {
-    float dx = __fsub_rn(q.x, me.x);
-    float dy = __fsub_rn(q.y, me.y);
-    float dz = __fsub_rn(q.z, me.z);
-    if (XS) dx = __fadd_rn(dx, s < lend_slot ? -Lx : (s >= rbeg_slot ? Lx : 0.0f));
-    if (YZ) {
-        dy = __fadd_rn(dy, sy);
-        dz = __fadd_rn(dz, sz);
-    }
-    return r2_of(dx, dy, dz);
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
-// One candidate, no periodic shift, as explicit PTX: three fp32
-// differences, three products, two sums, all round-to-nearest with no
-// contraction; on r2 < rl2 (and, for the home row, idx != self) append idx
-// to the row buffer.  Only used with FAST (no lane can pass B).
-template <bool SELF>
-__device__ __forceinline__ void test_plain(const float4 c, const float4 me, float rl2,
-                                           uint32_t self, uint32_t &bp)
+__device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v)
 {
-    if (SELF)
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// One candidate: three fp32 differences (each followed by its periodic
+// shift when GEN), three products, two sums, all round-to-nearest with no
+// contraction; on r2 < rl2 the candidate's atom index is appended at bp.
+template <bool GEN>
+__device__ __forceinline__ void test_cand(const float4 c, const float4 me, float sx, float sy,
+                                          float sz, float rl2, uint32_t &bp)
+{
+    if (GEN)
         asm volatile(
             "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
             "sub.rn.f32 dx, %1, %5;\n\t"
             "sub.rn.f32 dy, %2, %6;\n\t"
             "sub.rn.f32 dz, %3, %7;\n\t"
+            "add.rn.f32 dx, dx, %9;\n\t"
+            "add.rn.f32 dy, dy, %10;\n\t"
+            "add.rn.f32 dz, dz, %11;\n\t"
             "mul.rn.f32 dx, dx, dx;\n\t"
             "mul.rn.f32 dy, dy, dy;\n\t"
             "mul.rn.f32 dz, dz, dz;\n\t"
             "add.rn.f32 s, dx, dy;\n\t"
             "add.rn.f32 s, s, dz;\n\t"
             "setp.lt.f32 p, s, %8;\n\t"
-            "setp.ne.and.u32 p, %4, %9, p;\n\t"
             "@p st.shared.b32 [%0], %4;\n\t"
             "@p add.u32 %0, %0, 4;\n\t}"
             : "+r"(bp)
             : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "f"(me.x), "f"(me.y),
-              "f"(me.z), "f"(rl2), "r"(self));
+              "f"(me.z), "f"(rl2), "f"(sx), "f"(sy), "f"(sz));
     else
         asm volatile(
             "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
@@ -356,185 +313,297 @@ __device__ __forceinline__ void test_plain(const float4 c, const float4 me, floa
               "f"(me.z), "f"(rl2));
 }
 
-// Tests L consecutive candidates q[0..L) of one row (stage slots slot0 ..)
-// against this lane's atom: groups of 8, then of 4, then single ones.
-template <bool XS, bool YZ, bool SELF, bool FAST>
-__device__ __forceinline__ void scan_row(const float4 *__restrict__ q, int slot0, int L,
-                                         const float4 me, float Lx, int lend_slot, int rbeg_slot,
-                                         float sy, float sz, float rl2, RowOut &o)
+// Output state of one lane: hits are appended at bp in the current half
+// `cur` of the lane's buffer (halves h0, h1); gfl bytes of the atom's row
+// are already on their way to global memory.
+struct LaneOut {
+    uint32_t bp, cur, h0, h1, gfl, Kb;
+    char *grow;
+};
+
+// Every 16 slots: with >= kFlushAt entries pending, send the whole 16-byte
+// vectors to the row (entries past the capacity are only counted) and move
+// the partial vector to the start of the other half, whose previous copy
+// has finished reading by then.
+__device__ __forceinline__ void flush_check(LaneOut &o)
 {
-    const uint32_t self = (uint32_t)__float_as_int(me.w);
-    int k = 0;
-    if (!XS && !YZ && FAST) {
-        uint32_t bp = o.bp;
-        for (; k + 8 <= L; k += 8) {
-            float4 c[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) c[u] = q[k + u];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) test_plain<SELF>(c[u], me, rl2, self, bp);
+    const uint32_t u = o.bp - o.cur;
+    if (u >= 4u * kFlushAt) {
+        const uint32_t nv = u & ~15u;
+        if (o.gfl < o.Kb) {
+            fence_proxy_async_smem();
+            bulk_s2g(o.grow + o.gfl, o.cur, min(nv, o.Kb - o.gfl));
         }
-        for (; k < L; ++k) test_plain<SELF>(q[k], me, rl2, self, bp);
-        o.bp = bp;
-        return;
-    }
-    for (; k + 8 <= L; k += 8) {
-        float4 c[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) c[u] = q[k + u];
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-            append_if_hit<SELF, FAST>(
-                cand_r2<XS, YZ>(c[u], me, slot0 + k + u, Lx, lend_slot, rbeg_slot, sy, sz), rl2,
-                (uint32_t)__float_as_int(c[u].w), self, o);
-    }
-    if (k + 4 <= L) {
-        float4 c[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) c[u] = q[k + u];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            append_if_hit<SELF, FAST>(
-                cand_r2<XS, YZ>(c[u], me, slot0 + k + u, Lx, lend_slot, rbeg_slot, sy, sz), rl2,
-                (uint32_t)__float_as_int(c[u].w), self, o);
-        k += 4;
-    }
-    for (; k < L; ++k) {
-        const float4 c = q[k];
-        append_if_hit<SELF, FAST>(
-            cand_r2<XS, YZ>(c, me, slot0 + k, Lx, lend_slot, rbeg_slot, sy, sz), rl2,
-            (uint32_t)__float_as_int(c.w), self, o);
+        bulk_commit();
+        bulk_wait_read<1>();
+        const uint32_t oth = o.cur == o.h0 ? o.h1 : o.h0;
+        sts_u4(oth, lds_u4(o.cur + nv));
+        o.gfl += nv;
+        o.bp = oth + (u - nv);
+        o.cur = oth;
     }
 }
 
-__global__ void __launch_bounds__(64)
-k_pairs_columns(const CellGrid g, const ColParams P)
+// Walks this lane's segments (descriptors dsc[0], dsc[32], ...; entry nseg
+// is the end marker, a group of NaN slots that repeats) for G4 groups of 4
+// slots, G4 a multiple of 4.  GEN: periodic shifts per slot (x image cells
+// at the row ends) and per row (y, z), from rinfo.
+template <bool GEN>
+__device__ __forceinline__ void walk_segments(const float4 *__restrict__ stage,
+                                              const uint32_t *__restrict__ dsc, int nseg, int G4,
+                                              const float4 me, float rl2, const int4 *rinfo,
+                                              float Lx, LaneOut &o)
 {
-    extern __shared__ __align__(16) unsigned char col_smem[];
-    float4 *stage = reinterpret_cast<float4 *>(col_smem);
-    uint8_t *tabs = col_smem + sizeof(float4) * P.stage_max;   // [kRows][kRowCells][16]
-    int32_t *rows = reinterpret_cast<int32_t *>(tabs + kRows * kRowCells * kBinsPerCell);
-    __shared__ ColTile ti;
+    const uint32_t d0 = dsc[0];
+    int sl = (int)(d0 & 0x3FFFu);
+    int se = sl + 4 * (int)((d0 >> 14) & 0xFFFu);
+    int sidx = nseg < 1 ? nseg : 1;
+    uint32_t nd = dsc[sidx * 32];
+    int4 ri = make_int4(0, 0, 0, 0), nri = make_int4(0, 0, 0, 0);
+    if (GEN) {
+        ri = rinfo[d0 >> 26];
+        nri = rinfo[nd >> 26];
+    }
+    for (int g = 0; g < G4; g += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float4 c[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) c[k] = stage[sl + k];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float sx = 0.0f, sy = 0.0f, sz = 0.0f;
+                if (GEN) {
+                    sx = sl + k < ri.x ? -Lx : (sl + k >= ri.y ? Lx : 0.0f);
+                    sy = __int_as_float(ri.z);
+                    sz = __int_as_float(ri.w);
+                }
+                test_cand<GEN>(c[k], me, sx, sy, sz, rl2, o.bp);
+            }
+            sl += 4;
+            const bool adv = sl == se;
+            const int nsl = (int)(nd & 0x3FFFu);
+            const int nse = nsl + 4 * (int)((nd >> 14) & 0xFFFu);
+            sl = adv ? nsl : sl;
+            se = adv ? nse : se;
+            if (GEN) ri = adv ? nri : ri;
+            sidx = adv ? (sidx + 1 < nseg ? sidx + 1 : nseg) : sidx;
+            nd = dsc[sidx * 32];
+            if (GEN) nri = rinfo[nd >> 26];
+        }
+        flush_check(o);
+    }
+}
+
+// Staged row R of a tile: conceptual cells cx0-1 .. cx0+Gx of the (y, z)
+// column two cells below .. above the home block, as up to three
+// contiguous pieces of the cell-ordered array (the low periodic image cell
+// nx-1, the in-box cells, the high periodic image cell 0).
+struct RowSrc {
+    int need;
+    int has_lo, has_hi;         // image cells present (cx0 == 0; cx0 + Gx == nx)
+    int lo_src, lo_cnt;
+    int mid_src, mid_cnt;
+    int mid_cells;
+    int hi_src, hi_cnt;
+    int64_t rowc;               // cell index of x = 0 in this (y, z) column
+    int first;                  // first in-box cell
+    int len, lend, rbeg;        // slots; [0, lend) low image, [rbeg, len) high image
+    float sy, sz;               // periodic shifts of the row
+};
+
+__device__ __forceinline__ void describe_row(const CellGrid &g, const int32_t *__restrict__ cs,
+                                             int R, int cx0, int cy0, int cz0, int Gx, int Gy,
+                                             int Gz, RowSrc &rs, int *cell)
+{
+    const int ry = R % kSY, rz = R / kSY;
+    rs.need = R < kSRows && ry < Gy + 4 && rz < Gz + 4;
+    rs.has_lo = rs.has_hi = 0;
+    rs.lo_cnt = rs.mid_cnt = rs.hi_cnt = 0;
+    rs.lo_src = rs.mid_src = rs.hi_src = 0;
+    rs.mid_cells = 0;
+    rs.rowc = 0;
+    rs.first = 0;
+    rs.len = rs.lend = rs.rbeg = 0;
+    rs.sy = rs.sz = 0.0f;
+    if (!rs.need) return;
+    int y = cy0 - 2 + ry, z = cz0 - 2 + rz;
+    if (y < 0) { y += g.ny; rs.sy = -g.Ly; } else if (y >= g.ny) { y -= g.ny; rs.sy = g.Ly; }
+    if (z < 0) { z += g.nz; rs.sz = -g.Lz; } else if (z >= g.nz) { z -= g.nz; rs.sz = g.Lz; }
+    const int64_t rowc = ((int64_t)z * g.ny + y) * g.nx;
+    rs.rowc = rowc;
+    int k = 0, len = 0;
+    if (cx0 == 0) {   // conceptual cell -1 is cell nx-1
+        const int a = cs[rowc + g.nx - 1], b = cs[rowc + g.nx];
+        rs.has_lo = 1;
+        rs.lo_src = a;
+        rs.lo_cnt = b - a;
+        cell[k++] = 0;
+        len = b - a;
+    }
+    rs.lend = len;
+    const int first = cx0 == 0 ? 0 : cx0 - 1;
+    const int last = cx0 + Gx <= g.nx - 1 ? cx0 + Gx : g.nx - 1;
+    const int a = cs[rowc + first];
+    for (int cc = first; cc <= last; ++cc) cell[k++] = len + (cs[rowc + cc] - a);
+    const int b = cs[rowc + last + 1];
+    rs.first = first;
+    rs.mid_src = a;
+    rs.mid_cnt = b - a;
+    rs.mid_cells = last - first + 1;
+    len += b - a;
+    rs.rbeg = len;
+    if (cx0 + Gx == g.nx) {   // conceptual cell nx is cell 0
+        const int a2 = cs[rowc], b2 = cs[rowc + 1];
+        rs.has_hi = 1;
+        rs.hi_src = a2;
+        rs.hi_cnt = b2 - a2;
+        cell[k++] = len;
+        len += b2 - a2;
+    }
+    cell[k] = len;   // k == Gx + 2
+    rs.len = len;
+}
+
+// Issues the copies of one staged row: its atoms to stage slot `off`, the x
+// tables of its Gx + 2 conceptual cells to `tdst`; all complete on `bar`.
+__device__ __forceinline__ void copy_row(const RowSrc &rs, const TileParams &P, const CellGrid &g,
+                                         uint32_t stage_base, int off, uint32_t tdst, uint64_t *bar)
+{
+    if (!rs.need) return;
+    uint32_t dst = stage_base + 16u * (uint32_t)off;
+    if (rs.lo_cnt > 0) bulk_g2s(dst, P.cell_pos + rs.lo_src, 16u * (uint32_t)rs.lo_cnt, bar);
+    dst += 16u * (uint32_t)rs.lo_cnt;
+    if (rs.mid_cnt > 0) bulk_g2s(dst, P.cell_pos + rs.mid_src, 16u * (uint32_t)rs.mid_cnt, bar);
+    dst += 16u * (uint32_t)rs.mid_cnt;
+    if (rs.hi_cnt > 0) bulk_g2s(dst, P.cell_pos + rs.hi_src, 16u * (uint32_t)rs.hi_cnt, bar);
+    const uint32_t tb = (uint32_t)kBinsPerCell;
+    if (rs.has_lo) {
+        bulk_g2s(tdst, P.cell_tab + (rs.rowc + g.nx - 1) * kBinsPerCell, tb, bar);
+        tdst += tb;
+    }
+    bulk_g2s(tdst, P.cell_tab + (rs.rowc + rs.first) * kBinsPerCell, tb * (uint32_t)rs.mid_cells,
+             bar);
+    tdst += tb * (uint32_t)rs.mid_cells;
+    if (rs.has_hi) bulk_g2s(tdst, P.cell_tab + rs.rowc * kBinsPerCell, tb, bar);
+}
+
+// Bytes copy_row moves for a row.
+__device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
+{
+    if (!rs.need) return 0u;
+    return 16u * (uint32_t)rs.len +
+           (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
+}
+
+__global__ void __launch_bounds__(kTileWarps * 32, 2)
+k_pairs_tiles(const CellGrid g, const TileParams P)
+{
+    extern __shared__ __align__(16) unsigned char tile_smem[];
+    float4 *stage = reinterpret_cast<float4 *>(tile_smem);
+    uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
+    uint32_t *desc = reinterpret_cast<uint32_t *>(tabs + kSRows * kRowTab);   // [W][kSeg][32]
+    int32_t *hits = reinterpret_cast<int32_t *>(desc + kTileWarps * kSeg * 32);  // [W*32][2*kHalf]
+    int32_t *negs = hits + kTileWarps * 32 * 2 * kHalf;                // P.K entries of -1
+    __shared__ TileRows tr;
+    __shared__ int4 rinfo[kSRows];   // GEN: x image bounds (slots) and y, z shifts per row
     __shared__ __align__(8) uint64_t bar;
 
-    const int W = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int B = P.B;        // neighbor indices kept in shared memory per row
-    const int RS = B + 4;     // row stride in words (rows 16-byte aligned for bulk copies)
-    int32_t *negs = rows + W * 32 * RS;   // P.K entries of -1, the padding source
     for (int e = threadIdx.x; e < P.K; e += blockDim.x) negs[e] = -1;
-    const int tile = blockIdx.x;
-    const int tx = tile % P.tiles_x;
-    const int rest = tile / P.tiles_x;
-    const int cy = rest % g.ny;
-    const int cz = rest / g.ny;
-    const int cx0 = tx * kTileCells;
-    const int G = min(kTileCells, g.nx - cx0);
-    const uint32_t stage_base = smem_u32(stage);
+    fence_proxy_async_smem();   // -1 block is read by bulk copies of any thread
 
-    // ---- row table: lane r of warp 0 describes row r (its atoms and the
-    //      x tables of its G+2 conceptual cells cx0-1 .. cx0+G)
+    int t = blockIdx.x;
+    const int tx = t % P.tiles_x;
+    t /= P.tiles_x;
+    const int ty = t % P.tiles_y, tz = t / P.tiles_y;
+    const int cx0 = tx * kTX, cy0 = ty * kTY, cz0 = tz * kTZ;
+    const int Gx = min(kTX, g.nx - cx0), Gy = min(kTY, g.ny - cy0), Gz = min(kTZ, g.nz - cz0);
+    const uint32_t stage_base = smem_u32(stage);
+    const bool general = cx0 == 0 || cx0 + Gx == g.nx || cy0 < 2 || cy0 + Gy + 2 > g.ny ||
+                         cz0 < 2 || cz0 + Gz + 2 > g.nz;
+
     if (warp == 0) {
-        int seg_src[3] = {0, 0, 0}, seg_cnt[3] = {0, 0, 0};
-        int64_t tab_src[3] = {0, 0, 0};
-        int tab_cnt[3] = {0, 0, 0};
-        int nseg = 0, len = 0;
         if (lane == 0) mbar_init(&bar, 1);
-        if (lane < kRows) {
-            const int dy = lane % 5 - 2, dz = lane / 5 - 2;
-            int y = cy + dy, z = cz + dz;
-            float sy = 0.0f, sz = 0.0f;
-            if (y < 0) { y += g.ny; sy = -g.Ly; } else if (y >= g.ny) { y -= g.ny; sy = g.Ly; }
-            if (z < 0) { z += g.nz; sz = -g.Lz; } else if (z >= g.nz) { z -= g.nz; sz = g.Lz; }
-            const int64_t rowc = ((int64_t)z * g.ny + y) * g.nx;
-            int k = 0;
-            if (cx0 == 0) {  // conceptual cell -1 is cell nx-1
-                const int a = P.cell_start[rowc + g.nx - 1], b = P.cell_start[rowc + g.nx];
-                seg_src[nseg] = a;
-                seg_cnt[nseg] = b - a;
-                tab_src[nseg] = rowc + g.nx - 1;
-                tab_cnt[nseg] = 1;
-                ++nseg;
-                ti.row_cell[lane][k++] = 0;
-                len += b - a;
-            }
-            ti.row_lend[lane] = len;
-            const int first = cx0 == 0 ? 0 : cx0 - 1;
-            const int last = cx0 + G <= g.nx - 1 ? cx0 + G : g.nx - 1;
-            const int a = P.cell_start[rowc + first];
-            for (int cc = first; cc <= last; ++cc)
-                ti.row_cell[lane][k++] = len + (P.cell_start[rowc + cc] - a);
-            const int b = P.cell_start[rowc + last + 1];
-            seg_src[nseg] = a;
-            seg_cnt[nseg] = b - a;
-            tab_src[nseg] = rowc + first;
-            tab_cnt[nseg] = last - first + 1;
-            ++nseg;
-            if (lane == kCenterRow) {
-                ti.home_begin = len + (P.cell_start[rowc + cx0] - a);
-                ti.home_end = len + (P.cell_start[rowc + cx0 + G] - a);
-            }
-            len += b - a;
-            ti.row_rbeg[lane] = len;
-            if (cx0 + G == g.nx) {  // conceptual cell nx is cell 0
-                const int a2 = P.cell_start[rowc], b2 = P.cell_start[rowc + 1];
-                seg_src[nseg] = a2;
-                seg_cnt[nseg] = b2 - a2;
-                tab_src[nseg] = rowc;
-                tab_cnt[nseg] = 1;
-                ++nseg;
-                ti.row_cell[lane][k++] = len;
-                len += b2 - a2;
-            }
-            ti.row_cell[lane][k] = len;   // k == G + 2
-            ti.row_len[lane] = len;
-            ti.row_sy[lane] = sy;
-            ti.row_sz[lane] = sz;
-        }
-        __syncwarp();
-        // exclusive scan of the row lengths -> row offsets
-        int x = len;
+        RowSrc ra, rb;   // rows lane and lane + 32
+        int cell_scratch[kSCells + 1];
+        describe_row(g, P.cell_start, lane, cx0, cy0, cz0, Gx, Gy, Gz, ra, tr.cell[lane]);
+        describe_row(g, P.cell_start, lane + 32, cx0, cy0, cz0, Gx, Gy, Gz, rb,
+                     lane + 32 < kSRows ? tr.cell[lane + 32] : cell_scratch);
+        // offsets: kGap NaN slots before every row and after the last
+        const int va = ra.len + kGap, vb = lane + 32 < kSRows ? rb.len + kGap : 0;
+        int xa = va, xb = vb;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+            const int ya = __shfl_up_sync(0xffffffffu, xa, o);
+            const int yb = __shfl_up_sync(0xffffffffu, xb, o);
+            if (lane >= o) {
+                xa += ya;
+                xb += yb;
+            }
         }
-        const int off = x - len;
-        const int total = __shfl_sync(0xffffffffu, x, 31);
-        if (lane < kRows) ti.row_off[lane] = off;
-        if (lane == kCenterRow) {
-            ti.home_begin += off;
-            ti.home_end += off;
+        const int suma = __shfl_sync(0xffffffffu, xa, 31);
+        const int sumb = __shfl_sync(0xffffffffu, xb, 31);
+        const int offa = kGap + xa - va;
+        const int offb = kGap + suma + xb - vb;
+        const int total = kGap + suma + sumb;
+        tr.off[lane] = offa;
+        tr.len[lane] = ra.len;
+        rinfo[lane] = make_int4(offa + ra.lend, offa + ra.rbeg, __float_as_int(ra.sy),
+                                __float_as_int(ra.sz));
+        if (lane + 32 < kSRows) {
+            tr.off[lane + 32] = offb;
+            tr.len[lane + 32] = rb.len;
+            rinfo[lane + 32] = make_int4(offb + rb.lend, offb + rb.rbeg, __float_as_int(rb.sy),
+                                         __float_as_int(rb.sz));
         }
+        // home rows h = hy + 2 hz are staged rows (hy + 2) + kSY (hz + 2), all below 32
+        const int h = lane == 14 ? 0 : lane == 15 ? 1 : lane == 20 ? 2 : lane == 21 ? 3 : -1;
+        int hcnt = 0;
+        if (h >= 0) {
+            const bool valid = (h & 1) < Gy && (h >> 1) < Gz;
+            tr.home_begin[h] = offa + tr.cell[lane][1];
+            hcnt = valid ? tr.cell[lane][Gx + 1] - tr.cell[lane][1] : 0;
+        }
+        const int c0 = __shfl_sync(0xffffffffu, hcnt, 14), c1 = __shfl_sync(0xffffffffu, hcnt, 15);
+        const int c2 = __shfl_sync(0xffffffffu, hcnt, 20), c3 = __shfl_sync(0xffffffffu, hcnt, 21);
+        const uint32_t bytes = __reduce_add_sync(0xffffffffu, row_bytes(ra) + row_bytes(rb));
         const int fb = (total > P.stage_max || *P.unsorted != 0u) ? 1 : 0;
         if (lane == 0) {
-            ti.total = total;
-            ti.fallback = fb;
+            tr.home_pref[0] = 0;
+            tr.home_pref[1] = c0;
+            tr.home_pref[2] = c0 + c1;
+            tr.home_pref[3] = c0 + c1 + c2;
+            tr.home_pref[4] = c0 + c1 + c2 + c3;
+            tr.total = total;
+            tr.fallback = fb;
             if (fb) {
                 const uint32_t slot = atomicAdd(P.fb_count, 1u);
-                P.fb_list[slot] = (uint32_t)tile;
+                P.fb_list[slot] = (uint32_t)blockIdx.x;
             } else {
                 asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-                mbar_arrive_expect_tx(
-                    &bar, (uint32_t)total * 16u + (uint32_t)(kRows * (G + 2) * kBinsPerCell));
+                mbar_arrive_expect_tx(&bar, bytes);
             }
         }
         __syncwarp();
-        if (!fb && lane < kRows) {
-            uint32_t dst = stage_base + 16u * (uint32_t)off;
-            uint32_t tdst = smem_u32(tabs) + (uint32_t)(lane * kRowCells * kBinsPerCell);
-            for (int sg = 0; sg < nseg; ++sg) {
-                if (seg_cnt[sg] > 0)
-                    bulk_g2s(dst, P.cell_pos + seg_src[sg], (uint32_t)seg_cnt[sg] * 16u, &bar);
-                dst += 16u * (uint32_t)seg_cnt[sg];
-                bulk_g2s(tdst, P.cell_tab + tab_src[sg] * kBinsPerCell,
-                         (uint32_t)(tab_cnt[sg] * kBinsPerCell), &bar);
-                tdst += (uint32_t)(tab_cnt[sg] * kBinsPerCell);
-            }
+        if (!fb) {
+            copy_row(ra, P, g, stage_base, offa, smem_u32(tabs) + (uint32_t)(lane * kRowTab), &bar);
+            copy_row(rb, P, g, stage_base, offb, smem_u32(tabs) + (uint32_t)((lane + 32) * kRowTab),
+                     &bar);
         }
     }
     __syncthreads();
-    if (ti.fallback) return;
+    if (tr.fallback) return;
+    // NaN in the gaps (disjoint from the copies still in flight)
+    {
+        const float qn = __int_as_float(0x7fc00000);
+        const float4 nan4 = make_float4(qn, qn, qn, qn);
+        for (int e = threadIdx.x; e < (kSRows + 1) * kGap; e += blockDim.x) {
+            const int q = e / kGap, j = e % kGap;
+            stage[(q < kSRows ? tr.off[q] : tr.total) - kGap + j] = nan4;
+        }
+    }
+    __syncthreads();
     {
         uint32_t spins = 0;
         while (!mbar_try_wait(&bar, 0)) {
@@ -546,169 +615,163 @@ k_pairs_columns(const CellGrid g, const ColParams P)
     }
 
     const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
-    const int nbins = (G + 2) * kBinsPerCell;
+    const int nbins = (Gx + 2) * kBinsPerCell;
     const float rl2 = g.rl2;
-    const int nhome = ti.home_end - ti.home_begin;
-    const int nchunks = (nhome + 31) >> 5;
-    const uint32_t mybuf = smem_u32(rows) + 4u * (uint32_t)((warp * 32 + lane) * RS);
-    const float ylo = (float)cy * P.side_y, yhi = (float)(cy + 1) * P.side_y;
-    const float zlo = (float)cz * P.side_z, zhi = (float)(cz + 1) * P.side_z;
+    const int nhome = tr.home_pref[4];
+    uint32_t *dsc = desc + warp * kSeg * 32 + lane;   // this lane's descriptors, stride 32
+    const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * 2 * kHalf * 4);
+    const uint32_t negs_addr = smem_u32(negs);
 
-    for (int c = warp; c < nchunks; c += W) {
-        const int a = ti.home_begin + c * 32 + lane;
-        const bool valid = a < ti.home_end;
-        const float4 me =
-            valid ? stage[a] : make_float4(-1e30f, -1e30f, -1e30f, __int_as_float(-1));
+    for (int c = warp; c * 32 < nhome; c += kTileWarps) {
+        const int a = c * 32 + lane;
+        const bool valid = a < nhome;
+        int h = 0;
+        while (h < 3 && a >= tr.home_pref[h + 1]) ++h;
+        const int slot = tr.home_begin[h] + (a - tr.home_pref[h]);
+        const float qn = __int_as_float(0x7fc00000);
+        const float4 me = valid ? stage[slot] : make_float4(qn, qn, qn, qn);
+        const int hy = h & 1, hz = h >> 1;
+        const float ylo = (float)(cy0 + hy) * P.side_y, yhi = (float)(cy0 + hy + 1) * P.side_y;
+        const float zlo = (float)(cz0 + hz) * P.side_z, zhi = (float)(cz0 + hz + 1) * P.side_z;
         const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
         const float dz_lo = me.z - zlo, dz_hi = zhi - me.z;
-        const int myid = __float_as_int(me.w);
-        bulk_wait_read();   // the previous chunk's rows have left this buffer
-        RowOut o;
-        o.bp = mybuf;
-        o.bufend = mybuf + 4u * (uint32_t)B;
-        o.rowend = mybuf + 4u * (uint32_t)P.K;
-        o.gmap = (uint64_t)(uintptr_t)(P.nbr + (int64_t)(valid ? myid : 0) * P.K) - (uint64_t)mybuf;
-        for (int r = 0; r < kRows; ++r) {
-            const int dy = r % 5 - 2, dz = r / 5 - 2;
-            const int off = ti.row_off[r], len = ti.row_len[r];
-            if (len == 0) continue;
-            float py = dy > 0 ? dy_hi + (float)(dy - 1) * P.side_y
-                              : (dy < 0 ? dy_lo + (float)(-dy - 1) * P.side_y : 0.0f);
-            float pz = dz > 0 ? dz_hi + (float)(dz - 1) * P.side_z
-                              : (dz < 0 ? dz_lo + (float)(-dz - 1) * P.side_z : 0.0f);
-            py = fmaxf(py - P.eps, 0.0f);
-            pz = fmaxf(pz - P.eps, 0.0f);
-            const float h2 = P.rl2_margin - (py * py + pz * pz);
-            int lo = 0, hi = 0;
-            if (valid && h2 > 0.0f) {
-                // first index at or above bin b = start of b's cell + cell table entry
+
+        // ---- this lane's segments
+        int nseg = 0, tot = 0;
+        if (valid) {
+            for (int r = 0; r < 25; ++r) {
+                const int dy = r % 5 - 2, dz = r / 5 - 2;
+                const int R = (hy + dy + 2) + kSY * (hz + dz + 2);
+                const int len = tr.len[R];
+                if (len == 0) continue;
+                float py = dy > 0 ? dy_hi + (float)(dy - 1) * P.side_y
+                                  : (dy < 0 ? dy_lo + (float)(-dy - 1) * P.side_y : 0.0f);
+                float pz = dz > 0 ? dz_hi + (float)(dz - 1) * P.side_z
+                                  : (dz < 0 ? dz_lo + (float)(-dz - 1) * P.side_z : 0.0f);
+                py = fmaxf(py - P.eps, 0.0f);
+                pz = fmaxf(pz - P.eps, 0.0f);
+                const float h2 = P.rl2_margin - (py * py + pz * pz);
+                if (!(h2 > 0.0f)) continue;
+                // first slot at or above bin b = start of b's cell + cell table entry;
                 // approximate root (relative error ~1e-6): the margin absorbs it
-                const float h = h2 * rsqrtf(h2) + P.eps;
-                const uint8_t *tb = tabs + r * (kRowCells * kBinsPerCell);
-                const int *rc = ti.row_cell[r];
-                const int b0 = max(0, min((int)floorf((me.x - h - X0) * P.inv_bin), nbins - 1));
-                const int b1 = (int)floorf((me.x + h - X0) * P.inv_bin) + 1;
-                lo = rc[b0 >> 4] + tb[b0];
-                hi = b1 >= nbins ? len : (b1 <= 0 ? 0 : rc[b1 >> 4] + tb[b1]);
-                if (hi < lo) hi = lo;
-            }
-            const int Lmax = __reduce_max_sync(0xffffffffu, hi - lo);
-            if (Lmax == 0) continue;
-            // whole groups of 4 when the row is long enough (extra tests are harmless)
-            const int L = min((Lmax + 3) & ~3, len);
-            const int st = lo < len - L ? lo : len - L;
-            const int lend = ti.row_lend[r], rbeg = ti.row_rbeg[r];
-            // image shifts are needed as soon as any lane's tested range
-            // [st, st + L) reaches an image cell (not only its exact window):
-            // an unshifted image copy of a cell could otherwise pair with a
-            // home atom that also meets the cell's own copy
-            const bool xs = __any_sync(0xffffffffu, st < lend || st + L > rbeg);
-            const bool yz = ti.row_sy[r] != 0.0f || ti.row_sz[r] != 0.0f;
-            const bool fast = !__any_sync(0xffffffffu, o.bp + 4u * (uint32_t)L > o.bufend);
-            const float sy = ti.row_sy[r], sz = ti.row_sz[r];
-            const float4 *a0 = stage + off + st;
-            const int slot0 = off + st;
-            const int ls = off + lend, rs = off + rbeg;
-            const float Lx = g.Lx;
-            if (r == kCenterRow) {
-                if (xs) {
-                    if (fast) scan_row<true, false, true, true>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                    else scan_row<true, false, true, false>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
+                const float hw = h2 * rsqrtf(h2) + P.eps;
+                const uint8_t *tb = tabs + R * kRowTab;
+                const int *rc = tr.cell[R];
+                const int b0 = max(0, min((int)floorf((me.x - hw - X0) * P.inv_bin), nbins - 1));
+                const int b1 = (int)floorf((me.x + hw - X0) * P.inv_bin) + 1;
+                const int lo = rc[b0 >> 4] + tb[b0];
+                const int hi = b1 >= nbins ? len : (b1 <= 0 ? 0 : rc[b1 >> 4] + tb[b1]);
+                if (hi <= lo) continue;
+                const int base = tr.off[R];
+                if (r == 12) {   // home row: around the atom's own slot
+                    const int s = slot - base;
+                    const int e1 = min(hi, s);
+                    if (e1 > lo) {
+                        const int ng = (e1 - lo + 3) >> 2;
+                        dsc[32 * nseg++] = seg_pack((uint32_t)(base + e1 - 4 * ng), ng, R);
+                        tot += ng;
+                    }
+                    const int s1 = max(lo, s + 1);
+                    if (hi > s1) {
+                        const int ng = (hi - s1 + 3) >> 2;
+                        dsc[32 * nseg++] = seg_pack((uint32_t)(base + s1), ng, R);
+                        tot += ng;
+                    }
                 } else {
-                    if (fast) scan_row<false, false, true, true>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                    else scan_row<false, false, true, false>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                }
-            } else if (!yz) {
-                if (xs) {
-                    if (fast) scan_row<true, false, false, true>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                    else scan_row<true, false, false, false>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                } else {
-                    if (fast) scan_row<false, false, false, true>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                    else scan_row<false, false, false, false>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                }
-            } else {
-                if (xs) {
-                    if (fast) scan_row<true, true, false, true>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                    else scan_row<true, true, false, false>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                } else {
-                    if (fast) scan_row<false, true, false, true>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
-                    else scan_row<false, true, false, false>(a0, slot0, L, me, Lx, ls, rs, sy, sz, rl2, o);
+                    const int ng = (hi - lo + 3) >> 2;
+                    dsc[32 * nseg++] = seg_pack((uint32_t)(base + lo), ng, R);
+                    tot += ng;
                 }
             }
         }
-        const int cnt = (int)((o.bp - mybuf) >> 2);
+        dsc[32 * nseg] = seg_pack(0u, 1u, 0u);   // end marker: the first gap, repeated
+        const int G4 = (__reduce_max_sync(0xffffffffu, tot) + 3) & ~3;
+
+        // ---- walk
+        bulk_wait_read<0>();   // the previous chunk's copies have left this buffer
+        LaneOut o;
+        o.h0 = hb;
+        o.h1 = hb + 4u * kHalf;
+        o.cur = o.h0;
+        o.bp = o.h0;
+        o.gfl = 0u;
+        o.Kb = 4u * (uint32_t)P.K;
+        const int myid = __float_as_int(me.w);
+        o.grow = reinterpret_cast<char *>(P.nbr + (int64_t)(valid ? myid : 0) * P.K);
+        if (general)
+            walk_segments<true>(stage, dsc, nseg, G4, me, rl2, rinfo, g.Lx, o);
+        else
+            walk_segments<false>(stage, dsc, nseg, G4, me, rl2, rinfo, g.Lx, o);
+
+        // ---- finish the row: pending hits to a whole vector with -1, then
+        //      -1 from the shared block up to the capacity
         if (valid) {
+            const uint32_t u = o.bp - o.cur;
+            for (uint32_t b = u; (b & 15u) != 0u; b += 4u) sts_u32(o.cur + b, 0xffffffffu);
+            const uint32_t nv = (u + 15u) & ~15u;
+            fence_proxy_async_smem();
+            if (nv > 0u && o.gfl < o.Kb) bulk_s2g(o.grow + o.gfl, o.cur, min(nv, o.Kb - o.gfl));
+            const uint32_t pf = o.gfl + nv;
+            if (pf < o.Kb) bulk_s2g(o.grow + pf, negs_addr, o.Kb - pf);
+            bulk_commit();
+            const int cnt = (int)((o.gfl + u) >> 2);
             P.counts[myid] = cnt;
             if (cnt > P.K) atomicOr(P.flags, kFlagOverflow);
-            // the lane's row leaves by bulk copies: buffered hits rounded up to a
-            // whole 16-byte vector with -1, then -1 from `negs` up to K; entries
-            // B .. min(cnt, K)-1 of a long row are already in global memory
-            int32_t *rowbuf = rows + (warp * 32 + lane) * RS;
-            int32_t *grow = P.nbr + (int64_t)myid * P.K;
-            const int nsm = cnt < B ? cnt : B;
-            const int n1 = (nsm + 3) & ~3;
-            for (int e = nsm; e < n1; ++e) rowbuf[e] = -1;
-            int npad_from = n1;
-            if (cnt > B) {
-                const int ntot = cnt < P.K ? cnt : P.K;
-                npad_from = (ntot + 3) & ~3;
-                for (int e = ntot; e < npad_from; ++e) grow[e] = -1;
-            }
-            fence_proxy_async_smem();
-            if (n1 > 0) bulk_s2g(grow, mybuf, 4u * (uint32_t)n1);
-            if (P.K > npad_from)
-                bulk_s2g(grow + npad_from, smem_u32(negs), 4u * (uint32_t)(P.K - npad_from));
-            bulk_commit();
         }
     }
     bulk_wait_all();
 }
 
-// Rows of the tiles the staged kernel listed: per-atom search over their
-// home atoms.
+// Home atoms of the tiles the staged kernel listed (stage too small or cells
+// unsorted): per-atom search straight from global memory.
 __global__ void __launch_bounds__(128)
 k_pairs_listed(const float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start,
                const uint32_t *__restrict__ atom_cell, CellGrid g, int32_t K, int tiles_x,
-               const uint32_t *__restrict__ fb_list, const uint32_t *__restrict__ fb_count,
-               int32_t *__restrict__ nbr, int32_t *__restrict__ counts, uint32_t *flags)
+               int tiles_y, const uint32_t *__restrict__ fb_list,
+               const uint32_t *__restrict__ fb_count, int32_t *__restrict__ nbr,
+               int32_t *__restrict__ counts, uint32_t *flags)
 {
     const uint32_t nlisted = *fb_count;
     for (uint32_t e = blockIdx.x; e < nlisted; e += gridDim.x) {
-        const int tile = (int)fb_list[e];
-        const int tx = tile % tiles_x;
-        const int rest = tile / tiles_x;
-        const int cy = rest % g.ny;
-        const int cz = rest / g.ny;
-        const int cx0 = tx * kTileCells;
-        const int G = min(kTileCells, g.nx - cx0);
-        const int64_t rowc = ((int64_t)cz * g.ny + cy) * g.nx;
-        const int32_t k0 = cell_start[rowc + cx0], k1 = cell_start[rowc + cx0 + G];
-        for (int32_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
-            pair_row_per_atom<false>(k, cell_pos, cell_start, atom_cell, g, K, nbr, counts, flags);
+        int t = (int)fb_list[e];
+        const int tx = t % tiles_x;
+        t /= tiles_x;
+        const int ty = t % tiles_y, tz = t / tiles_y;
+        const int cx0 = tx * kTX, cy0 = ty * kTY, cz0 = tz * kTZ;
+        const int Gx = min(kTX, g.nx - cx0), Gy = min(kTY, g.ny - cy0), Gz = min(kTZ, g.nz - cz0);
+        for (int hz = 0; hz < Gz; ++hz)
+            for (int hy = 0; hy < Gy; ++hy) {
+                const int64_t rowc = ((int64_t)(cz0 + hz) * g.ny + (cy0 + hy)) * g.nx;
+                const int32_t k0 = cell_start[rowc + cx0], k1 = cell_start[rowc + cx0 + Gx];
+                for (int32_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
+                    pair_row_per_atom<false>(k, cell_pos, cell_start, atom_cell, g, K, nbr, counts,
+                                             flags);
+            }
     }
 }
 
-constexpr size_t kColSmemCap = 200 * 1024;
-constexpr int kColWarps = 2;
+constexpr int kSlotLimit = 16000;   // descriptor slot field is 14 bits
 
-constexpr int kRowBuffer = 128;   // row entries kept in shared memory
-
-int row_buffer(int K) { return K < kRowBuffer ? K : kRowBuffer; }
-
-size_t col_fixed_smem(int W, int K)
+size_t tile_fixed_smem(int K)
 {
-    const size_t tabs = (size_t)kRows * kRowCells * kBinsPerCell;
-    const size_t rows = (size_t)W * 32 * (size_t)(row_buffer(K) + 4) * sizeof(int32_t);
-    const size_t negs = (size_t)K * sizeof(int32_t);
-    return tabs + rows + negs;
+    return (size_t)kSRows * kRowTab + (size_t)kTileWarps * kSeg * 32 * sizeof(uint32_t) +
+           (size_t)kTileWarps * 32 * 2 * kHalf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
 }  // namespace
 
 cudaError_t pairs_set_attributes()
 {
-    return cudaFuncSetAttribute(k_pairs_columns, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kColSmemCap);
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, k_pairs_tiles);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_pairs_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin - (int)fa.sharedSizeBytes);
 }
 
 cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
@@ -717,41 +780,52 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
     *used_fast = 0;
     if (n <= 0) return cudaSuccess;
     // Staged kernel: column grid and rows of whole 16-byte vectors.  The
-    // stage must hold a typical tile (25 rows x (G+2) cells at the mean cell
-    // occupancy) with 25 % to spare; take the smallest shared-memory budget
-    // (3, 2 or 1 CTAs per SM) that does.  Denser tiles fall back per atom.
+    // stage must hold a typical tile (36 rows x (kTX + 2) cells at the mean
+    // cell occupancy, plus the gaps) with 10 % to spare; take the largest
+    // number of CTAs per SM whose shared-memory share still does.  Denser
+    // tiles are listed and searched per atom.
     int stage_max = 0;
-    const int W = kColWarps;
-    if (g.wy == 2 && !g.literal && capacity % 4 == 0 &&
+    if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
         (reinterpret_cast<uintptr_t>(nbr) & 15u) == 0 && n < (int64_t(1) << 31)) {
-        const size_t fixed = col_fixed_smem(W, capacity);
+        int dev = 0, per_sm = 0, reserved = 0, optin = 0;
+        NL_CUDA_TRY(cudaGetDevice(&dev));
+        NL_CUDA_TRY(cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev));
+        NL_CUDA_TRY(cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev));
+        NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+        cudaFuncAttributes fa;
+        NL_CUDA_TRY(cudaFuncGetAttributes(&fa, k_pairs_tiles));
+        const size_t fixed = tile_fixed_smem(capacity);
         const double per_cell = (double)n / (double)g.ncell;
-        const int want = (int)(1.1 * per_cell * kRows * (kTileCells + 2)) + 32;
+        const int want =
+            (int)(1.1 * per_cell * kSRows * kSCells) + (kSRows + 1) * kGap + 32;
         const int need = want > kStageMin ? want : kStageMin;
-        // per-SM 228 KB less 1 KB per CTA and the static tile table
-        for (size_t budget : {size_t(73) * 1024, size_t(110) * 1024, kColSmemCap}) {
-            const int fit = budget > fixed ? (int)((budget - fixed) / sizeof(float4)) : 0;
-            if (fit >= need || budget == kColSmemCap) {
-                stage_max = fit < 8192 ? fit : 8192;
+        for (int ctas = 3; ctas >= 1; --ctas) {
+            long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
+            const long cap = (long)optin - (long)fa.sharedSizeBytes;
+            if (budget > cap) budget = cap;
+            const long fit = budget > (long)fixed ? (budget - (long)fixed) / (long)sizeof(float4) : 0;
+            if (fit >= need || ctas == 1) {
+                stage_max = (int)(fit < kSlotLimit ? fit : kSlotLimit);
                 break;
             }
         }
         if (stage_max < 256) stage_max = 0;
     }
     if (stage_max > 0) {
-        ColParams P;
+        TileParams P;
         P.cell_pos = ctx->cell_pos;
         P.cell_start = ctx->cell_start;
+        P.cell_tab = ctx->cell_tab;
         P.nbr = nbr;
         P.counts = counts;
         P.flags = ctx->flags;
         P.unsorted = ctx->unsorted;
         P.fb_list = ctx->fb_list;
         P.fb_count = ctx->fb_count;
-        P.cell_tab = ctx->cell_tab;
-        P.tiles_x = (g.nx + kTileCells - 1) / kTileCells;
+        P.tiles_x = (g.nx + kTX - 1) / kTX;
+        P.tiles_y = (g.ny + kTY - 1) / kTY;
+        const int tiles_z = (g.nz + kTZ - 1) / kTZ;
         P.K = capacity;
-        P.B = row_buffer(capacity);
         P.stage_max = stage_max;
         P.side_x = g.Lx / (float)g.nx;
         P.side_y = g.Ly / (float)g.ny;
@@ -761,19 +835,19 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         const float Lmax = fmaxf(g.Lx, fmaxf(g.Ly, g.Lz));
         P.eps = 1e-3f * rl + 4e-6f * Lmax;
         P.rl2_margin = g.rl2 * (1.0f + 1e-4f);
-        const int64_t ntiles = (int64_t)P.tiles_x * g.ny * g.nz;
-        const size_t smem = sizeof(float4) * (size_t)stage_max + col_fixed_smem(W, capacity);
+        const int64_t ntiles = (int64_t)P.tiles_x * P.tiles_y * tiles_z;
+        const size_t smem = sizeof(float4) * (size_t)stage_max + tile_fixed_smem(capacity);
         NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, sizeof(uint32_t), s));
         {
             ProfScope ps(ctx, PH_PAIRS, s);
-            k_pairs_columns<<<(unsigned)ntiles, W * 32, smem, s>>>(g, P);
+            k_pairs_tiles<<<(unsigned)ntiles, kTileWarps * 32, smem, s>>>(g, P);
             NL_CUDA_TRY(cudaGetLastError());
         }
         *used_fast = 1;
         ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
         k_pairs_listed<<<(unsigned)(ctx->sm_count * 4), 128, 0, s>>>(
-            ctx->cell_pos, ctx->cell_start, ctx->atom_cell, g, capacity, P.tiles_x, ctx->fb_list,
-            ctx->fb_count, nbr, counts, ctx->flags);
+            ctx->cell_pos, ctx->cell_start, ctx->atom_cell, g, capacity, P.tiles_x, P.tiles_y,
+            ctx->fb_list, ctx->fb_count, nbr, counts, ctx->flags);
         return cudaGetLastError();
     }
     ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
