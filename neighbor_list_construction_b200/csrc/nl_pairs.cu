@@ -117,12 +117,12 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // atom's own slot, so self never reaches the predicate.  A lane walks the
 // concatenation of its segments; the warp runs for the largest lane total.
 //
-// Hits go to a per-lane buffer of two halves in shared memory; every 16
-// slots a lane with >= kFlushAt pending entries sends its whole 16-byte
-// vectors to its global row with one cp.async.bulk copy and continues in the
-// other half.  Rows are finished with -1 from a shared block of -1.
+// Hits go to a small per-lane buffer in shared memory; every 16 slots a
+// lane stores its whole 16-byte vectors to its global row and moves the
+// partial vector to the buffer's start.  Rows are finished with one
+// cp.async.bulk copy from a shared block of -1.
 // ---------------------------------------------------------------------------
-constexpr int kTX = 5, kTY = 2, kTZ = 2;   // home cells per tile
+constexpr int kTX = 4, kTY = 2, kTZ = 2;   // home cells per tile
 constexpr int kSY = kTY + 4, kSZ = kTZ + 4;
 constexpr int kSRows = kSY * kSZ;           // 36 staged rows
 constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
@@ -130,9 +130,8 @@ constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built
 constexpr int kRowTab = kSCells * kBinsPerCell;
 constexpr int kGap = 4;                     // NaN slots before, between and after rows
 constexpr int kSeg = 27;                    // segment descriptors per lane (25 rows, self split, end)
-constexpr int kHalf = 28;                   // entries per half of a lane's hit buffer
-constexpr int kFlushAt = 12;                // pending entries that trigger a flush
-constexpr int kTileWarps = 6;
+constexpr int kBuf = 20;                    // entries of a lane's hit buffer
+constexpr int kTileWarps = 5;
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
 // Segment descriptor: first slot (14 bits), groups of 4 slots (12 bits),
@@ -235,11 +234,6 @@ __device__ __forceinline__ void bulk_wait_read()
     asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ void bulk_wait_all()
-{
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -262,10 +256,6 @@ __device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v)
                  : "memory");
 }
 
-__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
 
 // One candidate: three fp32 differences (each followed by its periodic
 // shift when GEN), three products, two sums, all round-to-nearest with no
@@ -313,34 +303,35 @@ __device__ __forceinline__ void test_cand(const float4 c, const float4 me, float
               "f"(me.z), "f"(rl2));
 }
 
-// Output state of one lane: hits are appended at bp in the current half
-// `cur` of the lane's buffer (halves h0, h1); gfl bytes of the atom's row
-// are already on their way to global memory.
+__device__ __forceinline__ void stg_u4(char *p, uint4 v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+// Output state of one lane: hits are appended at bp in the lane's buffer
+// (shared memory from `buf`); the first gfl bytes of the atom's row are
+// stored; Kb = capacity in bytes.
 struct LaneOut {
-    uint32_t bp, cur, h0, h1, gfl, Kb;
+    uint32_t bp, buf, gfl, Kb;
     char *grow;
 };
 
-// Every 16 slots: with >= kFlushAt entries pending, send the whole 16-byte
-// vectors to the row (entries past the capacity are only counted) and move
-// the partial vector to the start of the other half, whose previous copy
-// has finished reading by then.
+// Every 16 slots (at most 16 new hits, so at most 3 + 16 pending): store the
+// whole 16-byte vectors to the row (entries past the capacity are only
+// counted) and move the partial vector to the buffer's start.
 __device__ __forceinline__ void flush_check(LaneOut &o)
 {
-    const uint32_t u = o.bp - o.cur;
-    if (u >= 4u * kFlushAt) {
-        const uint32_t nv = u & ~15u;
-        if (o.gfl < o.Kb) {
-            fence_proxy_async_smem();
-            bulk_s2g(o.grow + o.gfl, o.cur, min(nv, o.Kb - o.gfl));
-        }
-        bulk_commit();
-        bulk_wait_read<1>();
-        const uint32_t oth = o.cur == o.h0 ? o.h1 : o.h0;
-        sts_u4(oth, lds_u4(o.cur + nv));
+    const uint32_t u = o.bp - o.buf;
+    const uint32_t nv = u & ~15u;
+    if (nv != 0u) {
+#pragma unroll
+        for (uint32_t b = 0; b < 64u; b += 16u)
+            if (b < nv && o.gfl + b < o.Kb) stg_u4(o.grow + o.gfl + b, lds_u4(o.buf + b));
+        sts_u4(o.buf, lds_u4(o.buf + nv));
         o.gfl += nv;
-        o.bp = oth + (u - nv);
-        o.cur = oth;
+        o.bp -= nv;
     }
 }
 
@@ -496,15 +487,15 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-__global__ void __launch_bounds__(kTileWarps * 32, 2)
+__global__ void __launch_bounds__(kTileWarps * 32, 3)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
     extern __shared__ __align__(16) unsigned char tile_smem[];
     float4 *stage = reinterpret_cast<float4 *>(tile_smem);
     uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
     uint32_t *desc = reinterpret_cast<uint32_t *>(tabs + kSRows * kRowTab);   // [W][kSeg][32]
-    int32_t *hits = reinterpret_cast<int32_t *>(desc + kTileWarps * kSeg * 32);  // [W*32][2*kHalf]
-    int32_t *negs = hits + kTileWarps * 32 * 2 * kHalf;                // P.K entries of -1
+    int32_t *hits = reinterpret_cast<int32_t *>(desc + kTileWarps * kSeg * 32);  // [W*32][kBuf]
+    int32_t *negs = hits + kTileWarps * 32 * kBuf;                     // P.K entries of -1
     __shared__ TileRows tr;
     __shared__ int4 rinfo[kSRows];   // GEN: x image bounds (slots) and y, z shifts per row
     __shared__ __align__(8) uint64_t bar;
@@ -619,7 +610,7 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     const float rl2 = g.rl2;
     const int nhome = tr.home_pref[4];
     uint32_t *dsc = desc + warp * kSeg * 32 + lane;   // this lane's descriptors, stride 32
-    const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * 2 * kHalf * 4);
+    const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * kBuf * 4);
     const uint32_t negs_addr = smem_u32(negs);
 
     for (int c = warp; c * 32 < nhome; c += kTileWarps) {
@@ -688,12 +679,9 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         const int G4 = (__reduce_max_sync(0xffffffffu, tot) + 3) & ~3;
 
         // ---- walk
-        bulk_wait_read<0>();   // the previous chunk's copies have left this buffer
         LaneOut o;
-        o.h0 = hb;
-        o.h1 = hb + 4u * kHalf;
-        o.cur = o.h0;
-        o.bp = o.h0;
+        o.buf = hb;
+        o.bp = hb;
         o.gfl = 0u;
         o.Kb = 4u * (uint32_t)P.K;
         const int myid = __float_as_int(me.w);
@@ -703,15 +691,20 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         else
             walk_segments<false>(stage, dsc, nseg, G4, me, rl2, rinfo, g.Lx, o);
 
-        // ---- finish the row: pending hits to a whole vector with -1, then
-        //      -1 from the shared block up to the capacity
+        // ---- finish the row (the walk ends with a flush: at most 3 entries
+        //      pending): the partial vector completed with -1, then -1 from
+        //      the shared block up to the capacity
         if (valid) {
-            const uint32_t u = o.bp - o.cur;
-            for (uint32_t b = u; (b & 15u) != 0u; b += 4u) sts_u32(o.cur + b, 0xffffffffu);
-            const uint32_t nv = (u + 15u) & ~15u;
-            fence_proxy_async_smem();
-            if (nv > 0u && o.gfl < o.Kb) bulk_s2g(o.grow + o.gfl, o.cur, min(nv, o.Kb - o.gfl));
-            const uint32_t pf = o.gfl + nv;
+            const uint32_t u = o.bp - o.buf;
+            uint32_t pf = o.gfl;
+            if (u != 0u) {
+                uint4 v = lds_u4(o.buf);
+                if (u <= 4u) v.y = 0xffffffffu;
+                if (u <= 8u) v.z = 0xffffffffu;
+                v.w = 0xffffffffu;
+                if (o.gfl < o.Kb) stg_u4(o.grow + o.gfl, v);
+                pf += 16u;
+            }
             if (pf < o.Kb) bulk_s2g(o.grow + pf, negs_addr, o.Kb - pf);
             bulk_commit();
             const int cnt = (int)((o.gfl + u) >> 2);
@@ -719,7 +712,7 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
             if (cnt > P.K) atomicOr(P.flags, kFlagOverflow);
         }
     }
-    bulk_wait_all();
+    bulk_wait_read<0>();   // the -1 block stays readable until the copies are done
 }
 
 // Home atoms of the tiles the staged kernel listed (stage too small or cells
@@ -755,7 +748,7 @@ constexpr int kSlotLimit = 16000;   // descriptor slot field is 14 bits
 size_t tile_fixed_smem(int K)
 {
     return (size_t)kSRows * kRowTab + (size_t)kTileWarps * kSeg * 32 * sizeof(uint32_t) +
-           (size_t)kTileWarps * 32 * 2 * kHalf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
+           (size_t)kTileWarps * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
 }  // namespace
