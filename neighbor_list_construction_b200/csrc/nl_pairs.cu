@@ -128,6 +128,7 @@ constexpr int kSRows = kSY * kSZ;           // 36 staged rows
 constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
 constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
 constexpr int kRowTab = kSCells * kBinsPerCell;
+constexpr int kBinStride = kRowTab + 2;     // slot-table entries per row (bins and the row end)
 constexpr int kGap = 4;                     // NaN slots before, between and after rows
 constexpr int kSeg = 27;                    // segment descriptors per lane (25 rows, self split, end)
 constexpr int kBuf = 20;                    // entries of a lane's hit buffer
@@ -493,7 +494,8 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     extern __shared__ __align__(16) unsigned char tile_smem[];
     float4 *stage = reinterpret_cast<float4 *>(tile_smem);
     uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
-    uint32_t *desc = reinterpret_cast<uint32_t *>(tabs + kSRows * kRowTab);   // [W][kSeg][32]
+    uint16_t *sbin = reinterpret_cast<uint16_t *>(tabs + kSRows * kRowTab);   // [kSRows][kBinStride]
+    uint32_t *desc = reinterpret_cast<uint32_t *>(sbin + kSRows * kBinStride);   // [W][kSeg][32]
     int32_t *hits = reinterpret_cast<int32_t *>(desc + kTileWarps * kSeg * 32);  // [W*32][kBuf]
     int32_t *negs = hits + kTileWarps * 32 * kBuf;                     // P.K entries of -1
     __shared__ TileRows tr;
@@ -596,17 +598,26 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     }
     __syncthreads();
     {
-        uint32_t spins = 0;
-        while (!mbar_try_wait(&bar, 0)) {
-            if (++spins >= 4096u) {   // ~4 s
-                if (threadIdx.x == 0) atomicOr(P.flags, kFlagTimeout);
-                return;
-            }
+        bool done = false;
+        for (uint32_t spins = 0; spins < 4096u && !done; ++spins)   // ~4 s
+            done = mbar_try_wait(&bar, 0);
+        if (__syncthreads_or(!done)) {
+            if (threadIdx.x == 0) atomicOr(P.flags, kFlagTimeout);
+            return;
         }
     }
+    const int nbins = (Gx + 2) * kBinsPerCell;
+    // slot table: sbin[R][b] = first staged slot of row R at or above x bin
+    // b (start of b's cell + the cell's table entry); b >= nbins: row end
+    for (int e = threadIdx.x; e < kSRows * kBinStride; e += blockDim.x) {
+        const int R = e / kBinStride, b = e - R * kBinStride;
+        const int v = b < nbins ? tr.off[R] + tr.cell[R][b >> 4] + tabs[R * kRowTab + b]
+                                : tr.off[R] + tr.len[R];
+        sbin[e] = (uint16_t)v;
+    }
+    __syncthreads();
 
     const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
-    const int nbins = (Gx + 2) * kBinsPerCell;
     const float rl2 = g.rl2;
     const int nhome = tr.home_pref[4];
     uint32_t *dsc = desc + warp * kSeg * 32 + lane;   // this lane's descriptors, stride 32
@@ -627,52 +638,56 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
         const float dz_lo = me.z - zlo, dz_hi = zhi - me.z;
 
-        // ---- this lane's segments
+        // ---- this lane's segments: for each of the 25 rows, squared distance
+        //      (less the margin) from the atom to the row's (y, z) cell column,
+        //      x half-width h of the window, its bins and slots
+        float py2[5], pz2[5];
+#pragma unroll
+        for (int d = -2; d <= 2; ++d) {
+            float py = d > 0 ? dy_hi + (float)(d - 1) * P.side_y
+                             : (d < 0 ? dy_lo + (float)(-d - 1) * P.side_y : 0.0f);
+            float pz = d > 0 ? dz_hi + (float)(d - 1) * P.side_z
+                             : (d < 0 ? dz_lo + (float)(-d - 1) * P.side_z : 0.0f);
+            py = fmaxf(py - P.eps, 0.0f);
+            pz = fmaxf(pz - P.eps, 0.0f);
+            py2[d + 2] = py * py;
+            pz2[d + 2] = pz * pz;
+        }
+        const float mxr = me.x - X0;
+        const int Rh = (hy + 2) + kSY * (hz + 2);
         int nseg = 0, tot = 0;
-        if (valid) {
-            for (int r = 0; r < 25; ++r) {
-                const int dy = r % 5 - 2, dz = r / 5 - 2;
-                const int R = (hy + dy + 2) + kSY * (hz + dz + 2);
-                const int len = tr.len[R];
-                if (len == 0) continue;
-                float py = dy > 0 ? dy_hi + (float)(dy - 1) * P.side_y
-                                  : (dy < 0 ? dy_lo + (float)(-dy - 1) * P.side_y : 0.0f);
-                float pz = dz > 0 ? dz_hi + (float)(dz - 1) * P.side_z
-                                  : (dz < 0 ? dz_lo + (float)(-dz - 1) * P.side_z : 0.0f);
-                py = fmaxf(py - P.eps, 0.0f);
-                pz = fmaxf(pz - P.eps, 0.0f);
-                const float h2 = P.rl2_margin - (py * py + pz * pz);
-                if (!(h2 > 0.0f)) continue;
-                // first slot at or above bin b = start of b's cell + cell table entry;
-                // approximate root (relative error ~1e-6): the margin absorbs it
-                const float hw = h2 * rsqrtf(h2) + P.eps;
-                const uint8_t *tb = tabs + R * kRowTab;
-                const int *rc = tr.cell[R];
-                const int b0 = max(0, min((int)floorf((me.x - hw - X0) * P.inv_bin), nbins - 1));
-                const int b1 = (int)floorf((me.x + hw - X0) * P.inv_bin) + 1;
-                const int lo = rc[b0 >> 4] + tb[b0];
-                const int hi = b1 >= nbins ? len : (b1 <= 0 ? 0 : rc[b1 >> 4] + tb[b1]);
-                if (hi <= lo) continue;
-                const int base = tr.off[R];
-                if (r == 12) {   // home row: around the atom's own slot
-                    const int s = slot - base;
-                    const int e1 = min(hi, s);
-                    if (e1 > lo) {
-                        const int ng = (e1 - lo + 3) >> 2;
-                        dsc[32 * nseg++] = seg_pack((uint32_t)(base + e1 - 4 * ng), ng, R);
-                        tot += ng;
-                    }
-                    const int s1 = max(lo, s + 1);
-                    if (hi > s1) {
-                        const int ng = (hi - s1 + 3) >> 2;
-                        dsc[32 * nseg++] = seg_pack((uint32_t)(base + s1), ng, R);
-                        tot += ng;
-                    }
-                } else {
-                    const int ng = (hi - lo + 3) >> 2;
-                    dsc[32 * nseg++] = seg_pack((uint32_t)(base + lo), ng, R);
-                    tot += ng;
-                }
+#pragma unroll
+        for (int r = 0; r < 25; ++r) {
+            const int dy = r % 5 - 2, dz = r / 5 - 2;
+            const int R = Rh + dy + kSY * dz;
+            const float h2 = P.rl2_margin - (py2[dy + 2] + pz2[dz + 2]);
+            const bool ok = valid && h2 > 0.0f;
+            // approximate root (relative error ~1e-6): the margin absorbs it
+            const float hc = fmaxf(h2, 1e-20f);
+            const float hw = hc * rsqrtf(hc) + P.eps;
+            const int b0 = min(max(__float2int_rd((mxr - hw) * P.inv_bin), 0), nbins - 1);
+            const int b1 = min(max(__float2int_rd((mxr + hw) * P.inv_bin) + 1, 0), nbins);
+            const uint16_t *tb = sbin + R * kBinStride;
+            const int lo = tb[b0], hi = tb[b1];
+            if (r == 12) {   // home row: around the atom's own slot
+                const int e1 = min(hi, slot);
+                const int n1 = ok ? e1 - lo : 0;
+                const int ng1 = n1 > 0 ? (n1 + 3) >> 2 : 0;
+                dsc[32 * nseg] = seg_pack((uint32_t)(e1 - 4 * ng1), (uint32_t)ng1, (uint32_t)R);
+                nseg += ng1 > 0 ? 1 : 0;
+                tot += ng1;
+                const int s1 = max(lo, slot + 1);
+                const int n2 = ok ? hi - s1 : 0;
+                const int ng2 = n2 > 0 ? (n2 + 3) >> 2 : 0;
+                dsc[32 * nseg] = seg_pack((uint32_t)s1, (uint32_t)ng2, (uint32_t)R);
+                nseg += ng2 > 0 ? 1 : 0;
+                tot += ng2;
+            } else {
+                const int n = ok ? hi - lo : 0;
+                const int ng = n > 0 ? (n + 3) >> 2 : 0;
+                dsc[32 * nseg] = seg_pack((uint32_t)lo, (uint32_t)ng, (uint32_t)R);
+                nseg += ng > 0 ? 1 : 0;
+                tot += ng;
             }
         }
         dsc[32 * nseg] = seg_pack(0u, 1u, 0u);   // end marker: the first gap, repeated
@@ -747,7 +762,8 @@ constexpr int kSlotLimit = 16000;   // descriptor slot field is 14 bits
 
 size_t tile_fixed_smem(int K)
 {
-    return (size_t)kSRows * kRowTab + (size_t)kTileWarps * kSeg * 32 * sizeof(uint32_t) +
+    return (size_t)kSRows * kRowTab + (size_t)kSRows * kBinStride * sizeof(uint16_t) +
+           (size_t)kTileWarps * kSeg * 32 * sizeof(uint32_t) +
            (size_t)kTileWarps * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
