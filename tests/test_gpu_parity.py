@@ -156,6 +156,28 @@ def test_overflow_status_and_rows(ctx, oracle):
     gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt, full_sets=sets)
 
 
+def test_build_cutoff_shell_pairs(ctx, oracle):
+    """Partners placed within a few ulps of the cutoff radius: every pair
+    decision sits on the r2 < rl2 boundary, so any change in rounding (a
+    fused multiply-add, a reordered sum) flips some of them."""
+    rng = np.random.default_rng(17)
+    L, cutoff, skin = 48.0, 5.75, 1.0
+    rl = np.float64(np.float32(cutoff + skin))
+    nb = 6000
+    base = rng.random((nb, 3)) * L
+    u = rng.normal(size=(nb, 3))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    r = rl * (1.0 + rng.uniform(-3e-7, 3e-7, size=(nb, 1)))
+    pos = np.zeros((2 * nb, 4), np.float32)
+    pos[:nb, :3] = base
+    pos[nb:, :3] = base + r * u
+    box = np.array([L, L, L], np.float32)
+    nbr, cnt, st = gpu_build(ctx, pos, box, cutoff, skin, 256)
+    o_nbr, o_cnt, o_ov = oracle.build(pos, box, cutoff, skin, 256)
+    assert st == (1 if o_ov else 0)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+
+
 def test_build_mixed_density_uses_both_paths(ctx, nl, oracle):
     """A dense slab whose tiles overflow the shared-memory stage (listed for
     the per-atom search) beside sparse tiles that are staged; rows with more
