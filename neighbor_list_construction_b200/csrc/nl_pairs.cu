@@ -132,7 +132,7 @@ constexpr int kBinStride = kRowTab + 2;     // slot-table entries per row (bins 
 constexpr int kGap = 4;                     // NaN slots before, between and after rows
 constexpr int kSeg = 27;                    // segment descriptors per lane (25 rows, self split, end)
 constexpr int kBuf = 20;                    // entries of a lane's hit buffer
-constexpr int kTileWarps = 3;
+constexpr int kTileWarps = 5;
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
 // Segment descriptor: first slot (14 bits), groups of 4 slots (12 bits),
@@ -147,8 +147,7 @@ struct TileRows {
     int len[kSRows];
     int cell[kSRows][kSCells + 1];   // row-local start of conceptual cell k
     int home_begin[4];               // slot of the first home atom of home row h
-    int home_cnt[4];                 // home atoms of home row h
-    int pair_pref[5];                // lane pairs (two adjacent home atoms) before home row h
+    int home_pref[5];                // home atoms before home row h
     int total;                       // staged slots, gaps included
     int fallback;
 };
@@ -251,11 +250,6 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr)
     return v;
 }
 
-__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
 __device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v)
 {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
@@ -264,85 +258,50 @@ __device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v)
 }
 
 
-// Two fp32 values in one 64-bit register (element 0 in the low half).
-__device__ __forceinline__ uint64_t pack2(float a, float b)
-{
-    return ((uint64_t)__float_as_uint(b) << 32) | (uint64_t)__float_as_uint(a);
-}
-
-// One candidate c against the lane's two atoms A and B (coordinates packed
-// as {A, B}): per atom three fp32 differences (each followed by its periodic
-// shift when GEN) and three products with the packed f32x2 operations (each
-// half rounded as its own binary32 operation), then the two sums as scalar
-// round-to-nearest adds.  The sums stay scalar: ptxas fuses a packed product
-// that feeds a packed add into one packed fma even with .rn and no fmad,
-// which moves r2 by an ulp near the cutoff.  On r2 < rl2 the candidate's
-// atom index is appended to that atom's buffer.
+// One candidate: three fp32 differences (each followed by its periodic
+// shift when GEN), three products, two sums, all round-to-nearest with no
+// contraction; on r2 < rl2 the candidate's atom index is appended at bp.
 template <bool GEN>
-__device__ __forceinline__ void test_pair(const float4 c, uint64_t mx, uint64_t my, uint64_t mz,
-                                          float sx, uint64_t syz_y, uint64_t syz_z, float rl2,
-                                          uint32_t &bpa, uint32_t &bpb)
+__device__ __forceinline__ void test_cand(const float4 c, const float4 me, float sx, float sy,
+                                          float sz, float rl2, uint32_t &bp)
 {
     if (GEN)
         asm volatile(
-            "{\n\t.reg .b64 q, dx, dy, dz;\n\t.reg .f32 ra, rb, xa, xb, ya, yb, za, zb;\n\t.reg .pred pa, pb;\n\t"
-            "mov.b64 q, {%2, %2};\n\t"
-            "sub.rn.f32x2 dx, q, %6;\n\t"
-            "mov.b64 q, {%3, %3};\n\t"
-            "sub.rn.f32x2 dy, q, %7;\n\t"
-            "mov.b64 q, {%4, %4};\n\t"
-            "sub.rn.f32x2 dz, q, %8;\n\t"
-            "mov.b64 q, {%10, %10};\n\t"
-            "add.rn.f32x2 dx, dx, q;\n\t"
-            "add.rn.f32x2 dy, dy, %11;\n\t"
-            "add.rn.f32x2 dz, dz, %12;\n\t"
-            "mul.rn.f32x2 dx, dx, dx;\n\t"
-            "mul.rn.f32x2 dy, dy, dy;\n\t"
-            "mul.rn.f32x2 dz, dz, dz;\n\t"
-            "mov.b64 {xa, xb}, dx;\n\t"
-            "mov.b64 {ya, yb}, dy;\n\t"
-            "mov.b64 {za, zb}, dz;\n\t"
-            "add.rn.f32 ra, xa, ya;\n\t"
-            "add.rn.f32 rb, xb, yb;\n\t"
-            "add.rn.f32 ra, ra, za;\n\t"
-            "add.rn.f32 rb, rb, zb;\n\t"
-            "setp.lt.f32 pa, ra, %9;\n\t"
-            "setp.lt.f32 pb, rb, %9;\n\t"
-            "@pa st.shared.b32 [%0], %5;\n\t"
-            "@pa add.u32 %0, %0, 4;\n\t"
-            "@pb st.shared.b32 [%1], %5;\n\t"
-            "@pb add.u32 %1, %1, 4;\n\t}"
-            : "+r"(bpa), "+r"(bpb)
-            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "l"(mx), "l"(my), "l"(mz),
-              "f"(rl2), "f"(sx), "l"(syz_y), "l"(syz_z));
+            "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
+            "sub.rn.f32 dx, %1, %5;\n\t"
+            "sub.rn.f32 dy, %2, %6;\n\t"
+            "sub.rn.f32 dz, %3, %7;\n\t"
+            "add.rn.f32 dx, dx, %9;\n\t"
+            "add.rn.f32 dy, dy, %10;\n\t"
+            "add.rn.f32 dz, dz, %11;\n\t"
+            "mul.rn.f32 dx, dx, dx;\n\t"
+            "mul.rn.f32 dy, dy, dy;\n\t"
+            "mul.rn.f32 dz, dz, dz;\n\t"
+            "add.rn.f32 s, dx, dy;\n\t"
+            "add.rn.f32 s, s, dz;\n\t"
+            "setp.lt.f32 p, s, %8;\n\t"
+            "@p st.shared.b32 [%0], %4;\n\t"
+            "@p add.u32 %0, %0, 4;\n\t}"
+            : "+r"(bp)
+            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "f"(me.x), "f"(me.y),
+              "f"(me.z), "f"(rl2), "f"(sx), "f"(sy), "f"(sz));
     else
         asm volatile(
-            "{\n\t.reg .b64 q, dx, dy, dz;\n\t.reg .f32 ra, rb, xa, xb, ya, yb, za, zb;\n\t.reg .pred pa, pb;\n\t"
-            "mov.b64 q, {%2, %2};\n\t"
-            "sub.rn.f32x2 dx, q, %6;\n\t"
-            "mov.b64 q, {%3, %3};\n\t"
-            "sub.rn.f32x2 dy, q, %7;\n\t"
-            "mov.b64 q, {%4, %4};\n\t"
-            "sub.rn.f32x2 dz, q, %8;\n\t"
-            "mul.rn.f32x2 dx, dx, dx;\n\t"
-            "mul.rn.f32x2 dy, dy, dy;\n\t"
-            "mul.rn.f32x2 dz, dz, dz;\n\t"
-            "mov.b64 {xa, xb}, dx;\n\t"
-            "mov.b64 {ya, yb}, dy;\n\t"
-            "mov.b64 {za, zb}, dz;\n\t"
-            "add.rn.f32 ra, xa, ya;\n\t"
-            "add.rn.f32 rb, xb, yb;\n\t"
-            "add.rn.f32 ra, ra, za;\n\t"
-            "add.rn.f32 rb, rb, zb;\n\t"
-            "setp.lt.f32 pa, ra, %9;\n\t"
-            "setp.lt.f32 pb, rb, %9;\n\t"
-            "@pa st.shared.b32 [%0], %5;\n\t"
-            "@pa add.u32 %0, %0, 4;\n\t"
-            "@pb st.shared.b32 [%1], %5;\n\t"
-            "@pb add.u32 %1, %1, 4;\n\t}"
-            : "+r"(bpa), "+r"(bpb)
-            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "l"(mx), "l"(my), "l"(mz),
-              "f"(rl2));
+            "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
+            "sub.rn.f32 dx, %1, %5;\n\t"
+            "sub.rn.f32 dy, %2, %6;\n\t"
+            "sub.rn.f32 dz, %3, %7;\n\t"
+            "mul.rn.f32 dx, dx, dx;\n\t"
+            "mul.rn.f32 dy, dy, dy;\n\t"
+            "mul.rn.f32 dz, dz, dz;\n\t"
+            "add.rn.f32 s, dx, dy;\n\t"
+            "add.rn.f32 s, s, dz;\n\t"
+            "setp.lt.f32 p, s, %8;\n\t"
+            "@p st.shared.b32 [%0], %4;\n\t"
+            "@p add.u32 %0, %0, 4;\n\t}"
+            : "+r"(bp)
+            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "f"(me.x), "f"(me.y),
+              "f"(me.z), "f"(rl2));
 }
 
 __device__ __forceinline__ void stg_u4(char *p, uint4 v)
@@ -352,9 +311,9 @@ __device__ __forceinline__ void stg_u4(char *p, uint4 v)
                  : "memory");
 }
 
-// Output state of one atom's row: hits are appended at bp in its buffer
-// (shared memory from `buf`); the first gfl bytes of the row are stored;
-// Kb = capacity in bytes.
+// Output state of one lane: hits are appended at bp in the lane's buffer
+// (shared memory from `buf`); the first gfl bytes of the atom's row are
+// stored; Kb = capacity in bytes.
 struct LaneOut {
     uint32_t bp, buf, gfl, Kb;
     char *grow;
@@ -379,15 +338,13 @@ __device__ __forceinline__ void flush_check(LaneOut &o)
 
 // Walks this lane's segments (descriptors dsc[0], dsc[32], ...; entry nseg
 // is the end marker, a group of NaN slots that repeats) for G4 groups of 4
-// slots, G4 a multiple of 4, testing every slot against both atoms.  GEN:
-// periodic shifts per slot (x image cells at the row ends) and per row (y,
-// z), from rinfo.
+// slots, G4 a multiple of 4.  GEN: periodic shifts per slot (x image cells
+// at the row ends) and per row (y, z), from rinfo.
 template <bool GEN>
 __device__ __forceinline__ void walk_segments(const float4 *__restrict__ stage,
                                               const uint32_t *__restrict__ dsc, int nseg, int G4,
-                                              uint64_t mx, uint64_t my, uint64_t mz, float rl2,
-                                              const int4 *rinfo, float Lx, LaneOut &oa,
-                                              LaneOut &ob)
+                                              const float4 me, float rl2, const int4 *rinfo,
+                                              float Lx, LaneOut &o)
 {
     const uint32_t d0 = dsc[0];
     int sl = (int)(d0 & 0x3FFFu);
@@ -405,16 +362,15 @@ __device__ __forceinline__ void walk_segments(const float4 *__restrict__ stage,
             float4 c[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) c[k] = stage[sl + k];
-            uint64_t sy2 = 0, sz2 = 0;
-            if (GEN) {
-                sy2 = pack2(__int_as_float(ri.z), __int_as_float(ri.z));
-                sz2 = pack2(__int_as_float(ri.w), __int_as_float(ri.w));
-            }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                float sx = 0.0f;
-                if (GEN) sx = sl + k < ri.x ? -Lx : (sl + k >= ri.y ? Lx : 0.0f);
-                test_pair<GEN>(c[k], mx, my, mz, sx, sy2, sz2, rl2, oa.bp, ob.bp);
+                float sx = 0.0f, sy = 0.0f, sz = 0.0f;
+                if (GEN) {
+                    sx = sl + k < ri.x ? -Lx : (sl + k >= ri.y ? Lx : 0.0f);
+                    sy = __int_as_float(ri.z);
+                    sz = __int_as_float(ri.w);
+                }
+                test_cand<GEN>(c[k], me, sx, sy, sz, rl2, o.bp);
             }
             sl += 4;
             const bool adv = sl == se;
@@ -427,8 +383,7 @@ __device__ __forceinline__ void walk_segments(const float4 *__restrict__ stage,
             nd = dsc[sidx * 32];
             if (GEN) nri = rinfo[nd >> 26];
         }
-        flush_check(oa);
-        flush_check(ob);
+        flush_check(o);
     }
 }
 
@@ -533,51 +488,6 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-// Squared distances (less the margin, clamped at 0) from an atom to the
-// (y, z) cell columns d = -2..2 away from its home cell [ylo, yhi) x [zlo, zhi).
-__device__ __forceinline__ void perp_terms(const float4 me, float ylo, float yhi, float zlo,
-                                           float zhi, const TileParams &P, float (&py2)[5],
-                                           float (&pz2)[5])
-{
-    const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
-    const float dz_lo = me.z - zlo, dz_hi = zhi - me.z;
-#pragma unroll
-    for (int d = -2; d <= 2; ++d) {
-        float py = d > 0 ? dy_hi + (float)(d - 1) * P.side_y
-                         : (d < 0 ? dy_lo + (float)(-d - 1) * P.side_y : 0.0f);
-        float pz = d > 0 ? dz_hi + (float)(d - 1) * P.side_z
-                         : (d < 0 ? dz_lo + (float)(-d - 1) * P.side_z : 0.0f);
-        py = fmaxf(py - P.eps, 0.0f);
-        pz = fmaxf(pz - P.eps, 0.0f);
-        py2[d + 2] = py * py;
-        pz2[d + 2] = pz * pz;
-    }
-}
-
-// Finishes one atom's row (the walk ends with a flush: at most 3 entries
-// pending): the partial vector completed with -1, then -1 from the shared
-// block up to the capacity; the count, and the overflow flag past it.
-__device__ __forceinline__ void finish_row(LaneOut &o, uint32_t negs_addr, const TileParams &P,
-                                           int id)
-{
-    const uint32_t u = o.bp - o.buf;
-    uint32_t pf = o.gfl;
-    if (u != 0u) {
-        uint4 v = lds_u4(o.buf);
-        if (u <= 4u) v.y = 0xffffffffu;
-        if (u <= 8u) v.z = 0xffffffffu;
-        v.w = 0xffffffffu;
-        if (o.gfl < o.Kb) stg_u4(o.grow + o.gfl, v);
-        pf += 16u;
-    }
-    if (pf < o.Kb) bulk_s2g(o.grow + pf, negs_addr, o.Kb - pf);
-    bulk_commit();
-    const int cnt = (int)((o.gfl + u) >> 2);
-    P.counts[id] = cnt;
-    if (cnt > P.K) atomicOr(P.flags, kFlagOverflow);
-}
-
-
 __global__ void __launch_bounds__(kTileWarps * 32, 3)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
@@ -586,8 +496,8 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
     uint16_t *sbin = reinterpret_cast<uint16_t *>(tabs + kSRows * kRowTab);   // [kSRows][kBinStride]
     uint32_t *desc = reinterpret_cast<uint32_t *>(sbin + kSRows * kBinStride);   // [W][kSeg][32]
-    int32_t *hits = reinterpret_cast<int32_t *>(desc + kTileWarps * kSeg * 32);  // [W*32][2][kBuf]
-    int32_t *negs = hits + kTileWarps * 32 * 2 * kBuf;                 // P.K entries of -1
+    int32_t *hits = reinterpret_cast<int32_t *>(desc + kTileWarps * kSeg * 32);  // [W*32][kBuf]
+    int32_t *negs = hits + kTileWarps * 32 * kBuf;                     // P.K entries of -1
     __shared__ TileRows tr;
     __shared__ int4 rinfo[kSRows];   // GEN: x image bounds (slots) and y, z shifts per row
     __shared__ __align__(8) uint64_t bar;
@@ -653,15 +563,11 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         const uint32_t bytes = __reduce_add_sync(0xffffffffu, row_bytes(ra) + row_bytes(rb));
         const int fb = (total > P.stage_max || *P.unsorted != 0u) ? 1 : 0;
         if (lane == 0) {
-            tr.home_cnt[0] = c0;
-            tr.home_cnt[1] = c1;
-            tr.home_cnt[2] = c2;
-            tr.home_cnt[3] = c3;
-            tr.pair_pref[0] = 0;
-            tr.pair_pref[1] = (c0 + 1) >> 1;
-            tr.pair_pref[2] = tr.pair_pref[1] + ((c1 + 1) >> 1);
-            tr.pair_pref[3] = tr.pair_pref[2] + ((c2 + 1) >> 1);
-            tr.pair_pref[4] = tr.pair_pref[3] + ((c3 + 1) >> 1);
+            tr.home_pref[0] = 0;
+            tr.home_pref[1] = c0;
+            tr.home_pref[2] = c0 + c1;
+            tr.home_pref[3] = c0 + c1 + c2;
+            tr.home_pref[4] = c0 + c1 + c2 + c3;
             tr.total = total;
             tr.fallback = fb;
             if (fb) {
@@ -713,69 +619,64 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
 
     const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
     const float rl2 = g.rl2;
-    const int npairs = tr.pair_pref[4];
+    const int nhome = tr.home_pref[4];
     uint32_t *dsc = desc + warp * kSeg * 32 + lane;   // this lane's descriptors, stride 32
-    const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * 2 * kBuf * 4);
+    const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * kBuf * 4);
     const uint32_t negs_addr = smem_u32(negs);
-    const float qn = __int_as_float(0x7fc00000);
-    const float4 nan4 = make_float4(qn, qn, qn, qn);
 
-    for (int c = warp; c * 32 < npairs; c += kTileWarps) {
-        // ---- this lane's atoms: A and, unless A ends an odd home row, the
-        //      next atom B of the same home row (x-sorted, so their windows
-        //      nearly coincide)
-        const int p = c * 32 + lane;
-        const bool valid = p < npairs;
+    for (int c = warp; c * 32 < nhome; c += kTileWarps) {
+        const int a = c * 32 + lane;
+        const bool valid = a < nhome;
         int h = 0;
-        while (h < 3 && p >= tr.pair_pref[h + 1]) ++h;
-        const int m = 2 * (p - tr.pair_pref[h]);
-        const int sa = tr.home_begin[h] + m;
-        const bool vb = valid && m + 1 < tr.home_cnt[h];
-        const int sb = vb ? sa + 1 : sa;
-        const float4 ma = valid ? stage[sa] : nan4;
-        const float4 mb = vb ? stage[sb] : nan4;
+        while (h < 3 && a >= tr.home_pref[h + 1]) ++h;
+        const int slot = tr.home_begin[h] + (a - tr.home_pref[h]);
+        const float qn = __int_as_float(0x7fc00000);
+        const float4 me = valid ? stage[slot] : make_float4(qn, qn, qn, qn);
         const int hy = h & 1, hz = h >> 1;
         const float ylo = (float)(cy0 + hy) * P.side_y, yhi = (float)(cy0 + hy + 1) * P.side_y;
         const float zlo = (float)(cz0 + hz) * P.side_z, zhi = (float)(cz0 + hz + 1) * P.side_z;
-        float ay2[5], az2[5], by2[5], bz2[5];
-        perp_terms(ma, ylo, yhi, zlo, zhi, P, ay2, az2);
-        perp_terms(mb, ylo, yhi, zlo, zhi, P, by2, bz2);
+        const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
+        const float dz_lo = me.z - zlo, dz_hi = zhi - me.z;
 
-        // ---- segments: per row the union of both atoms' windows (x half
-        //      width h from the squared distance to the row's (y, z) cell
-        //      column, less the margin), as bins, then slots
-        const float mxa = ma.x - X0, mxb = mb.x - X0;
+        // ---- this lane's segments: for each of the 25 rows, squared distance
+        //      (less the margin) from the atom to the row's (y, z) cell column,
+        //      x half-width h of the window, its bins and slots
+        float py2[5], pz2[5];
+#pragma unroll
+        for (int d = -2; d <= 2; ++d) {
+            float py = d > 0 ? dy_hi + (float)(d - 1) * P.side_y
+                             : (d < 0 ? dy_lo + (float)(-d - 1) * P.side_y : 0.0f);
+            float pz = d > 0 ? dz_hi + (float)(d - 1) * P.side_z
+                             : (d < 0 ? dz_lo + (float)(-d - 1) * P.side_z : 0.0f);
+            py = fmaxf(py - P.eps, 0.0f);
+            pz = fmaxf(pz - P.eps, 0.0f);
+            py2[d + 2] = py * py;
+            pz2[d + 2] = pz * pz;
+        }
+        const float mxr = me.x - X0;
         const int Rh = (hy + 2) + kSY * (hz + 2);
         int nseg = 0, tot = 0;
 #pragma unroll
         for (int r = 0; r < 25; ++r) {
             const int dy = r % 5 - 2, dz = r / 5 - 2;
             const int R = Rh + dy + kSY * dz;
-            const float h2a = P.rl2_margin - (ay2[dy + 2] + az2[dz + 2]);
-            const float h2b = P.rl2_margin - (by2[dy + 2] + bz2[dz + 2]);
-            const bool oka = valid && h2a > 0.0f, okb = vb && h2b > 0.0f;
-            // approximate roots (relative error ~1e-6): the margin absorbs them
-            const float ha = fmaxf(h2a, 1e-20f), hbw = fmaxf(h2b, 1e-20f);
-            const float wa = ha * rsqrtf(ha) + P.eps, wb = hbw * rsqrtf(hbw) + P.eps;
-            const int b0a = __float2int_rd((mxa - wa) * P.inv_bin);
-            const int b1a = __float2int_rd((mxa + wa) * P.inv_bin) + 1;
-            const int b0b = __float2int_rd((mxb - wb) * P.inv_bin);
-            const int b1b = __float2int_rd((mxb + wb) * P.inv_bin) + 1;
-            int b0 = oka ? (okb ? min(b0a, b0b) : b0a) : b0b;
-            int b1 = oka ? (okb ? max(b1a, b1b) : b1a) : b1b;
-            b0 = min(max(b0, 0), nbins - 1);
-            b1 = min(max(b1, 0), nbins);
-            const bool ok = oka || okb;
+            const float h2 = P.rl2_margin - (py2[dy + 2] + pz2[dz + 2]);
+            const bool ok = valid && h2 > 0.0f;
+            // approximate root (relative error ~1e-6): the margin absorbs it
+            const float hc = fmaxf(h2, 1e-20f);
+            const float hw = hc * rsqrtf(hc) + P.eps;
+            const int b0 = min(max(__float2int_rd((mxr - hw) * P.inv_bin), 0), nbins - 1);
+            const int b1 = min(max(__float2int_rd((mxr + hw) * P.inv_bin) + 1, 0), nbins);
             const uint16_t *tb = sbin + R * kBinStride;
             const int lo = tb[b0], hi = tb[b1];
-            if (r == 12) {   // home row: around the atoms' own slots sa .. sb
-                const int e1 = min(hi, sa);
+            if (r == 12) {   // home row: around the atom's own slot
+                const int e1 = min(hi, slot);
                 const int n1 = ok ? e1 - lo : 0;
                 const int ng1 = n1 > 0 ? (n1 + 3) >> 2 : 0;
                 dsc[32 * nseg] = seg_pack((uint32_t)(e1 - 4 * ng1), (uint32_t)ng1, (uint32_t)R);
                 nseg += ng1 > 0 ? 1 : 0;
                 tot += ng1;
-                const int s1 = max(lo, sb + 1);
+                const int s1 = max(lo, slot + 1);
                 const int n2 = ok ? hi - s1 : 0;
                 const int ng2 = n2 > 0 ? (n2 + 3) >> 2 : 0;
                 dsc[32 * nseg] = seg_pack((uint32_t)s1, (uint32_t)ng2, (uint32_t)R);
@@ -792,35 +693,39 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         dsc[32 * nseg] = seg_pack(0u, 1u, 0u);   // end marker: the first gap, repeated
         const int G4 = (__reduce_max_sync(0xffffffffu, tot) + 3) & ~3;
 
-        // ---- the pair A-B itself (skipped by the home-row segments)
-        const int ida = __float_as_int(ma.w), idb = __float_as_int(mb.w);
-        LaneOut oa, ob;
-        oa.buf = oa.bp = hb;
-        ob.buf = ob.bp = hb + 4u * kBuf;
-        oa.gfl = ob.gfl = 0u;
-        oa.Kb = ob.Kb = 4u * (uint32_t)P.K;
-        oa.grow = reinterpret_cast<char *>(P.nbr + (int64_t)(valid ? ida : 0) * P.K);
-        ob.grow = reinterpret_cast<char *>(P.nbr + (int64_t)(vb ? idb : 0) * P.K);
-        if (vb) {
-            const float r2 = r2_of(__fsub_rn(mb.x, ma.x), __fsub_rn(mb.y, ma.y),
-                                   __fsub_rn(mb.z, ma.z));
-            if (r2 < rl2) {
-                sts_u32(oa.bp, (uint32_t)idb);
-                oa.bp += 4u;
-                sts_u32(ob.bp, (uint32_t)ida);
-                ob.bp += 4u;
-            }
-        }
-
         // ---- walk
-        const uint64_t mx = pack2(ma.x, mb.x), my = pack2(ma.y, mb.y), mz = pack2(ma.z, mb.z);
+        LaneOut o;
+        o.buf = hb;
+        o.bp = hb;
+        o.gfl = 0u;
+        o.Kb = 4u * (uint32_t)P.K;
+        const int myid = __float_as_int(me.w);
+        o.grow = reinterpret_cast<char *>(P.nbr + (int64_t)(valid ? myid : 0) * P.K);
         if (general)
-            walk_segments<true>(stage, dsc, nseg, G4, mx, my, mz, rl2, rinfo, g.Lx, oa, ob);
+            walk_segments<true>(stage, dsc, nseg, G4, me, rl2, rinfo, g.Lx, o);
         else
-            walk_segments<false>(stage, dsc, nseg, G4, mx, my, mz, rl2, rinfo, g.Lx, oa, ob);
+            walk_segments<false>(stage, dsc, nseg, G4, me, rl2, rinfo, g.Lx, o);
 
-        if (valid) finish_row(oa, negs_addr, P, ida);
-        if (vb) finish_row(ob, negs_addr, P, idb);
+        // ---- finish the row (the walk ends with a flush: at most 3 entries
+        //      pending): the partial vector completed with -1, then -1 from
+        //      the shared block up to the capacity
+        if (valid) {
+            const uint32_t u = o.bp - o.buf;
+            uint32_t pf = o.gfl;
+            if (u != 0u) {
+                uint4 v = lds_u4(o.buf);
+                if (u <= 4u) v.y = 0xffffffffu;
+                if (u <= 8u) v.z = 0xffffffffu;
+                v.w = 0xffffffffu;
+                if (o.gfl < o.Kb) stg_u4(o.grow + o.gfl, v);
+                pf += 16u;
+            }
+            if (pf < o.Kb) bulk_s2g(o.grow + pf, negs_addr, o.Kb - pf);
+            bulk_commit();
+            const int cnt = (int)((o.gfl + u) >> 2);
+            P.counts[myid] = cnt;
+            if (cnt > P.K) atomicOr(P.flags, kFlagOverflow);
+        }
     }
     bulk_wait_read<0>();   // the -1 block stays readable until the copies are done
 }
@@ -859,7 +764,7 @@ size_t tile_fixed_smem(int K)
 {
     return (size_t)kSRows * kRowTab + (size_t)kSRows * kBinStride * sizeof(uint16_t) +
            (size_t)kTileWarps * kSeg * 32 * sizeof(uint32_t) +
-           (size_t)kTileWarps * 32 * 2 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
+           (size_t)kTileWarps * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
 }  // namespace
