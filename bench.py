@@ -29,6 +29,25 @@ sys.path.insert(0, ROOT)
 METRIC = "neighbor-list build atoms/s and pairs/s at 1 B200; % of HBM roofline"
 NOMINAL_HBM_GBS = 8000.0
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# pair-search launch on the saltwater10m workload, from one ncu capture.  It
+# belongs to the kernel source it was taken on: with any other source of the
+# pair kernel the bench reports null.
+PAIR_TRAFFIC = {"workload": "saltwater10m",
+                "sha256": "d7ee0d83f3a952ef945acf42179f2a3eb3f45b958276172662972548b70a59af",
+                "bytes": 668699136 + 10583890176}
+
+
+def pair_traffic(workload: str):
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("nl_pairs.cu", "nl_internal.cuh"):
+        with open(os.path.join(ROOT, "neighbor_list_construction_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if workload == PAIR_TRAFFIC["workload"] and h.hexdigest() == PAIR_TRAFFIC["sha256"]:
+        return PAIR_TRAFFIC["bytes"]
+    return None
+
 
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -332,6 +351,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         bytes_per_atom = 16 + 4 * K + 4
         alg_bytes = n * bytes_per_atom
         achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
+        traffic = pair_traffic(args.workload) if dom == "pair_search" else None
         build_ms = sum(phases.get(p, (0.0, 0))[0] for p in
                        ("bin_count", "cell_scan", "bin_scatter", "cell_sort", "pair_search",
                         "pair_search_per_atom")) / args.steps
@@ -366,7 +386,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved,
                          "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": None,
+                         "traffic": traffic,
+                         "traffic_over_algorithmic": (traffic / alg_bytes) if traffic else None,
                          "bytes_per_atom": bytes_per_atom, "launch_ms": dom_ms},
             "phases_ms": {k: v[0] / args.steps for k, v in phases.items() if v[1]},
             "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "atoms/s",
