@@ -211,12 +211,15 @@ __device__ __forceinline__ void sort_large_cell(float4 *__restrict__ cell_pos, i
     if (lane < 16) tab[lane] = (uint8_t)below;
 }
 
-// Two cells per warp (one per half); a cell above 16 atoms is redone by the
-// whole warp, and one above kCellSortMax stays in scatter order and raises
-// `unsorted`.
+// Two cells per warp, one per half.  A cell of at most 16 atoms is sorted
+// here; a larger one (up to kCellSortMax) is listed for k_cell_sort_large,
+// and one above kCellSortMax stays in scatter order and raises `unsorted`.
+// Keeping the large path out of this kernel keeps its register count low, so
+// enough warps are resident to cover the two dependent global loads per cell.
 __global__ void __launch_bounds__(256)
 k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell,
-            int nx, float side_x, float inv_bin, uint8_t *__restrict__ cell_tab, uint32_t *unsorted)
+            int nx, float side_x, float inv_bin, uint8_t *__restrict__ cell_tab,
+            uint32_t *__restrict__ large_list, uint32_t *large_count, uint32_t *unsorted)
 {
     const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -228,27 +231,33 @@ k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_star
         const int m = have ? cell_start[c + 1] - s : 0;
         const float face = (float)(int)(c % nx) * side_x;
         const bool small = m <= 16;
-        if (__all_sync(0xffffffffu, small)) {
-            sort_small_cell(cell_pos, s, m, face, inv_bin, cell_tab + (have ? c : 0) * 16, hl, have);
-            continue;
+        sort_small_cell(cell_pos, s, small ? m : 0, face, inv_bin, cell_tab + (have ? c : 0) * 16,
+                        hl, have && small);
+        if (have && !small && hl == 0) {
+            if (m > kCellSortMax)
+                atomicOr(unsorted, 1u);
+            else
+                large_list[atomicAdd(large_count, 1u)] = (uint32_t)c;
         }
-        // at least one of the two cells is large: whole warp, one cell at a time
-        for (int h = 0; h < 2; ++h) {
-            const int64_t cc = c0 + h;
-            if (cc >= ncell) break;
-            const int32_t ss = cell_start[cc];
-            const int mm = cell_start[cc + 1] - ss;
-            const float ff = (float)(int)(cc % nx) * side_x;
-            if (mm > kCellSortMax) {
-                if (lane == 0) atomicOr(unsorted, 1u);
-            } else if (mm <= 16) {
-                // half 0 sorts; half 1 only pairs the shuffles
-                sort_small_cell(cell_pos, ss, half == 0 ? mm : 0, ff, inv_bin, cell_tab + cc * 16, hl,
-                                half == 0);
-            } else {
-                sort_large_cell(cell_pos, ss, mm, ff, inv_bin, cell_tab + cc * 16, lane);
-            }
-        }
+    }
+}
+
+// The listed cells of 17..kCellSortMax atoms, one warp per cell.
+__global__ void __launch_bounds__(256)
+k_cell_sort_large(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int nx,
+                  float side_x, float inv_bin, uint8_t *__restrict__ cell_tab,
+                  const uint32_t *__restrict__ large_list, const uint32_t *large_count)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const uint32_t nlisted = *large_count;
+    for (int64_t e = warp; e < (int64_t)nlisted; e += nwarps) {
+        const int64_t c = large_list[e];
+        const int32_t s = cell_start[c];
+        const int m = cell_start[c + 1] - s;
+        const float face = (float)(int)(c % nx) * side_x;
+        sort_large_cell(cell_pos, s, m, face, inv_bin, cell_tab + c * 16, lane);
     }
 }
 
@@ -294,11 +303,18 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
         NL_CUDA_TRY(cudaGetLastError());
     }
     {
+        // cells above 16 atoms are listed in fb_list (free until the pair
+        // search, which resets fb_count before it lists its own tiles)
         ProfScope ps(ctx, PH_CELL_SORT, s);
         const float side_x = g.Lx / (float)g.nx;
-        k_cell_sort<<<grid_for(g.ncell * 32, 256, cap), 256, 0, s>>>(
+        NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, sizeof(uint32_t), s));
+        k_cell_sort<<<grid_for(g.ncell * 16, 256, (int64_t)ctx->sm_count * 32), 256, 0, s>>>(
             ctx->cell_pos, ctx->cell_start, g.ncell, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
-            ctx->unsorted);
+            ctx->fb_list, ctx->fb_count, ctx->unsorted);
+        NL_CUDA_TRY(cudaGetLastError());
+        k_cell_sort_large<<<(unsigned)(ctx->sm_count * 2), 256, 0, s>>>(
+            ctx->cell_pos, ctx->cell_start, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
+            ctx->fb_list, ctx->fb_count);
         NL_CUDA_TRY(cudaGetLastError());
     }
     return cudaSuccess;

@@ -19,7 +19,7 @@ constexpr int kKeyPasses = 8;                 // 63-bit keys: 8 digits of 8 bits
 
 // Onesweep tile: 256 threads x 16 keys.
 constexpr int kSortThreads = 256;
-constexpr int kSortItems = 16;
+constexpr int kSortItems = 8;
 constexpr int kSortTile = kSortThreads * kSortItems;
 
 // Cell-count scan tile: 256 threads x 16 cells.

@@ -17,7 +17,7 @@ constexpr int kWarps = kSortThreads / 32;
 constexpr size_t kSortDynSmem = (size_t)kSortTile * (sizeof(uint64_t) + sizeof(uint32_t));
 
 template <bool WRITE_KEYS>
-__global__ void __launch_bounds__(kSortThreads)
+__global__ void __launch_bounds__(kSortThreads, 4)
 k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
            uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, int64_t n,
            int shift, const uint32_t *__restrict__ digit_start, uint32_t *status,
@@ -39,8 +39,9 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
     const uint32_t tile = s_tile;
     const int64_t base = (int64_t)tile * kSortTile;
 
-    // warp w owns elements [base + 512w, base + 512w + 512); item k of lane l
-    // is element base + 512w + 32k + l, so (k, lane) order is index order.
+    // warp w owns elements [base + Ew, base + Ew + E), E = 32 kSortItems; item
+    // k of lane l is element base + Ew + 32k + l, so (k, lane) order is index
+    // order.
     uint64_t key[kSortItems];
     uint32_t val[kSortItems];
     uint32_t rank[kSortItems];
