@@ -14,6 +14,7 @@ namespace nl {
 namespace {
 
 constexpr int kWarps = kSortThreads / 32;
+constexpr int kLookBack = 8;   // predecessor status words read per look-back round
 constexpr size_t kSortDynSmem = (size_t)kSortTile * (sizeof(uint64_t) + sizeof(uint32_t));
 
 template <bool WRITE_KEYS>
@@ -88,22 +89,38 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
         st_volatile_u32(st, kStPrefix | cnt);
     } else {
         st_volatile_u32(st, kStAggregate | cnt);
+        // look back kLookBack predecessors per round: their status words are
+        // read with independent loads, then taken in order until a prefix
+        // (done) or a word not yet published (poll again from there)
         int64_t j = (int64_t)tile - 1;
         uint32_t spins = 0u;
-        while (j >= 0) {
-            const uint32_t s = ld_volatile_u32(status + (size_t)j * kRadixBins + t);
-            const uint32_t f = s & ~kStValue;
-            if (f == 0u) {
+        bool done = false;
+        while (!done) {
+            uint32_t sw[kLookBack];
+#pragma unroll
+            for (int q = 0; q < kLookBack; ++q)
+                sw[q] = j - q >= 0 ? ld_volatile_u32(status + (size_t)(j - q) * kRadixBins + t)
+                                   : kStPrefix;
+            int q = 0;
+#pragma unroll
+            for (int qq = 0; qq < kLookBack; ++qq) {
+                if (q == qq && !done) {
+                    const uint32_t f = sw[qq] & ~kStValue;
+                    if (f != 0u) {
+                        excl += sw[qq] & kStValue;
+                        done = f == kStPrefix;
+                        ++q;
+                    }
+                }
+            }
+            j -= q;
+            if (!done && q < kLookBack) {   // word j not yet published
                 if (++spins >= kSpinLimit) {
                     atomicOr(flags, kFlagTimeout);
                     break;
                 }
                 if (spins > 64u) __nanosleep(64);
-                continue;
             }
-            excl += s & kStValue;
-            if (f == kStPrefix) break;
-            --j;
         }
         st_volatile_u32(st, kStPrefix | ((excl + cnt) & kStValue));
     }
