@@ -103,8 +103,7 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // conceptual cells cx0-1 .. cx0+Gx along x, with a periodic image cell at
 // either end of the box.  Every row is a contiguous range of the
 // cell-ordered array; one lane per row issues its cp.async.bulk copies into
-// shared memory, all completing on one mbarrier.  Rows are separated by
-// kGap slots of NaN (a NaN candidate never passes r2 < rl2).
+// shared memory, all completing on one mbarrier.
 //
 // A home atom meets 25 rows (dy, dz in -2..2).  Atoms of a row are sorted by
 // x, so its candidates in a row lie in the slot window of [x - h, x + h],
@@ -129,18 +128,9 @@ constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
 constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
 constexpr int kRowTab = kSCells * kBinsPerCell;
 constexpr int kBinStride = kRowTab + 2;     // slot-table entries per row (bins and the row end)
-constexpr int kGap = 4;                     // NaN slots before, between and after rows
-constexpr int kSeg = 27;                    // segment descriptors per lane (25 rows, self split, end)
 constexpr int kBuf = 20;                    // entries of a lane's hit buffer
 constexpr int kTileWarps = 5;
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
-
-// Segment descriptor: first slot (14 bits), groups of 4 slots (12 bits),
-// staged row (6 bits).
-__host__ __device__ constexpr uint32_t seg_pack(uint32_t slot, uint32_t ng, uint32_t row)
-{
-    return slot | (ng << 14) | (row << 26);
-}
 
 struct TileRows {
     int off[kSRows];                 // slot of the row's first atom
@@ -304,6 +294,69 @@ __device__ __forceinline__ void test_cand(const float4 c, const float4 me, float
               "f"(me.z), "f"(rl2));
 }
 
+// Four consecutive slots at shared address `addr` of which the first `act`
+// (0..4 or more) belong to this lane's range: the active ones are loaded
+// into c[0..3] (an inactive slot keeps a stale value), and each is tested as
+// in test_cand, a hit requiring the slot to be active.  GEN: x shifts
+// sx0..sx3 per slot and the row's y, z shifts.
+template <bool GEN>
+__device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], const float4 me,
+                                      float rl2, float sx0, float sx1, float sx2, float sx3,
+                                      float sy, float sz, uint32_t &bp)
+{
+#define NL_S4_HEAD                                                                      \
+    "{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3;\n\t"                      \
+    "setp.gt.s32 q0, %17, 0;\n\t"                                                       \
+    "setp.gt.s32 q1, %17, 1;\n\t"                                                       \
+    "setp.gt.s32 q2, %17, 2;\n\t"                                                       \
+    "setp.gt.s32 q3, %17, 3;\n\t"                                                       \
+    "@q0 ld.shared.v4.f32 {%1, %2, %3, %4}, [%18];\n\t"                                 \
+    "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%18+16];\n\t"                              \
+    "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%18+32];\n\t"                           \
+    "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%18+48];\n\t"
+#define NL_S4_TEST(q, X, Y, Z, W, SHIFT)                                                 \
+    "sub.rn.f32 dx, " X ", %19;\n\t"                                                    \
+    "sub.rn.f32 dy, " Y ", %20;\n\t"                                                    \
+    "sub.rn.f32 dz, " Z ", %21;\n\t" SHIFT                                             \
+    "mul.rn.f32 dx, dx, dx;\n\t"                                                        \
+    "mul.rn.f32 dy, dy, dy;\n\t"                                                        \
+    "mul.rn.f32 dz, dz, dz;\n\t"                                                        \
+    "add.rn.f32 dx, dx, dy;\n\t"                                                        \
+    "add.rn.f32 dx, dx, dz;\n\t"                                                        \
+    "setp.lt.and.f32 " q ", dx, %22, " q ";\n\t"                                        \
+    "@" q " st.shared.b32 [%0], " W ";\n\t"                                             \
+    "@" q " add.u32 %0, %0, 4;\n\t"
+#define NL_S4_SHIFT(SX)                                                                 \
+    "add.rn.f32 dx, dx, " SX ";\n\t"                                                    \
+    "add.rn.f32 dy, dy, %27;\n\t"                                                       \
+    "add.rn.f32 dz, dz, %28;\n\t"
+#define NL_S4_OUTS                                                                      \
+    "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x),      \
+        "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), \
+        "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
+    if (GEN)
+        asm volatile(NL_S4_HEAD
+                     NL_S4_TEST("q0", "%1", "%2", "%3", "%4", NL_S4_SHIFT("%23"))
+                     NL_S4_TEST("q1", "%5", "%6", "%7", "%8", NL_S4_SHIFT("%24"))
+                     NL_S4_TEST("q2", "%9", "%10", "%11", "%12", NL_S4_SHIFT("%25"))
+                     NL_S4_TEST("q3", "%13", "%14", "%15", "%16", NL_S4_SHIFT("%26")) "}"
+                     : NL_S4_OUTS
+                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(sx0),
+                       "f"(sx1), "f"(sx2), "f"(sx3), "f"(sy), "f"(sz));
+    else
+        asm volatile(NL_S4_HEAD
+                     NL_S4_TEST("q0", "%1", "%2", "%3", "%4", "")
+                     NL_S4_TEST("q1", "%5", "%6", "%7", "%8", "")
+                     NL_S4_TEST("q2", "%9", "%10", "%11", "%12", "")
+                     NL_S4_TEST("q3", "%13", "%14", "%15", "%16", "") "}"
+                     : NL_S4_OUTS
+                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2));
+#undef NL_S4_HEAD
+#undef NL_S4_TEST
+#undef NL_S4_SHIFT
+#undef NL_S4_OUTS
+}
+
 __device__ __forceinline__ void stg_u4(char *p, uint4 v)
 {
     asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
@@ -336,55 +389,89 @@ __device__ __forceinline__ void flush_check(LaneOut &o)
     }
 }
 
-// Walks this lane's segments (descriptors dsc[0], dsc[32], ...; entry nseg
-// is the end marker, a group of NaN slots that repeats) for G4 groups of 4
-// slots, G4 a multiple of 4.  GEN: periodic shifts per slot (x image cells
-// at the row ends) and per row (y, z), from rinfo.
+// Tests this lane's slots lo .. lo+len-1 of one staged row.  The warp runs
+// its longest range in groups of 4; a lane past its own range loads nothing
+// (a NaN candidate), so no shared-memory traffic is spent on it.  The lanes
+// are consecutive x-sorted home atoms and scan the same row at the same
+// step, so their 16-byte loads fall on nearly consecutive slots (few bank
+// conflicts).  Every 16 slots, counted across rows in gc, the lane's whole
+// hit vectors are flushed.  GEN: periodic shifts, per slot in x (slots below
+// ri.x are the low image cell, at or above ri.y the high one) and per row in
+// y, z (ri.z, ri.w).
 template <bool GEN>
-__device__ __forceinline__ void walk_segments(const float4 *__restrict__ stage,
-                                              const uint32_t *__restrict__ dsc, int nseg, int G4,
-                                              const float4 me, float rl2, const int4 *rinfo,
-                                              float Lx, LaneOut &o)
+__device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int lo, int len,
+                                           const float4 me, float rl2, int4 ri, float Lx, int &gc,
+                                           float4 (&c)[4], LaneOut &o)
 {
-    const uint32_t d0 = dsc[0];
-    int sl = (int)(d0 & 0x3FFFu);
-    int se = sl + 4 * (int)((d0 >> 14) & 0xFFFu);
-    int sidx = nseg < 1 ? nseg : 1;
-    uint32_t nd = dsc[sidx * 32];
-    int4 ri = make_int4(0, 0, 0, 0), nri = make_int4(0, 0, 0, 0);
-    if (GEN) {
-        ri = rinfo[d0 >> 26];
-        nri = rinfo[nd >> 26];
-    }
-    for (int g = 0; g < G4; g += 4) {
+    const int Lmax = __reduce_max_sync(0xffffffffu, len);
+    const float sy = __int_as_float(ri.z), sz = __int_as_float(ri.w);
+    const uint32_t a0 = smem_u32(stage) + 16u * (uint32_t)lo;
+#pragma unroll 1
+    for (int j = 0; j < Lmax; j += 4) {
+        float sxv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (GEN) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            float4 c[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) c[k] = stage[sl + k];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float sx = 0.0f, sy = 0.0f, sz = 0.0f;
-                if (GEN) {
-                    sx = sl + k < ri.x ? -Lx : (sl + k >= ri.y ? Lx : 0.0f);
-                    sy = __int_as_float(ri.z);
-                    sz = __int_as_float(ri.w);
-                }
-                test_cand<GEN>(c[k], me, sx, sy, sz, rl2, o.bp);
-            }
-            sl += 4;
-            const bool adv = sl == se;
-            const int nsl = (int)(nd & 0x3FFFu);
-            const int nse = nsl + 4 * (int)((nd >> 14) & 0xFFFu);
-            sl = adv ? nsl : sl;
-            se = adv ? nse : se;
-            if (GEN) ri = adv ? nri : ri;
-            sidx = adv ? (sidx + 1 < nseg ? sidx + 1 : nseg) : sidx;
-            nd = dsc[sidx * 32];
-            if (GEN) nri = rinfo[nd >> 26];
+            for (int u = 0; u < 4; ++u)
+                sxv[u] = lo + j + u < ri.x ? -Lx : (lo + j + u >= ri.y ? Lx : 0.0f);
         }
-        flush_check(o);
+        scan4<GEN>(a0 + 16u * (uint32_t)j, len - j, c, me, rl2, sxv[0], sxv[1], sxv[2], sxv[3],
+                   sy, sz, o.bp);
+        if (++gc == 4) {
+            gc = 0;
+            flush_check(o);
+        }
     }
+}
+
+// All 25 rows of one lane's atom: per row, the x half-width h of the window
+// from the squared distance (less the margin) between the atom and the row's
+// (y, z) cell column, its bins, and from the slot table its slots.  The home
+// row is scanned in two ranges around the atom's own slot, so self never
+// reaches the predicate.
+template <bool GEN>
+__device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
+                                          const uint16_t *__restrict__ sbin, const int4 *rinfo,
+                                          const TileParams &P, float rl2, float Lx, int nbins,
+                                          const float4 me, bool valid, int slot, int Rh,
+                                          float dy_lo, float dy_hi, float dz_lo, float dz_hi,
+                                          float mxr, LaneOut &o)
+{
+    int gc = 0;
+    // candidate registers, carried across groups (an inactive slot's stale
+    // value is never taken: its hit predicate is false)
+    float4 c[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) c[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 1
+    for (int r = 0; r < 25; ++r) {
+        const int dy = r % 5 - 2, dz = r / 5 - 2;
+        const int R = Rh + dy + kSY * dz;
+        float py = dy > 0 ? dy_hi + (float)(dy - 1) * P.side_y
+                          : (dy < 0 ? dy_lo + (float)(-dy - 1) * P.side_y : 0.0f);
+        float pz = dz > 0 ? dz_hi + (float)(dz - 1) * P.side_z
+                          : (dz < 0 ? dz_lo + (float)(-dz - 1) * P.side_z : 0.0f);
+        py = fmaxf(py - P.eps, 0.0f);
+        pz = fmaxf(pz - P.eps, 0.0f);
+        const float h2 = P.rl2_margin - (py * py + pz * pz);
+        const bool ok = valid && h2 > 0.0f;
+        // approximate root (relative error ~1e-6): the margin absorbs it
+        const float hc = fmaxf(h2, 1e-20f);
+        const float hw = hc * rsqrtf(hc) + P.eps;
+        const int b0 = min(max(__float2int_rd((mxr - hw) * P.inv_bin), 0), nbins - 1);
+        const int b1 = min(max(__float2int_rd((mxr + hw) * P.inv_bin) + 1, 0), nbins);
+        const uint16_t *tb = sbin + R * kBinStride;
+        const int lo = tb[b0], hi = tb[b1];
+        const int4 ri = GEN ? rinfo[R] : make_int4(0, 0, 0, 0);
+        if (r == 12) {
+            const int e1 = min(hi, slot);
+            scan_range<GEN>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, gc, c, o);
+            const int s1 = max(lo, slot + 1);
+            scan_range<GEN>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, gc, c, o);
+        } else {
+            scan_range<GEN>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, gc, c, o);
+        }
+    }
+    flush_check(o);
 }
 
 // Staged row R of a tile: conceptual cells cx0-1 .. cx0+Gx of the (y, z)
@@ -488,15 +575,14 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-__global__ void __launch_bounds__(kTileWarps * 32, 3)
+__global__ void __launch_bounds__(kTileWarps * 32, 4)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
     extern __shared__ __align__(16) unsigned char tile_smem[];
     float4 *stage = reinterpret_cast<float4 *>(tile_smem);
     uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
     uint16_t *sbin = reinterpret_cast<uint16_t *>(tabs + kSRows * kRowTab);   // [kSRows][kBinStride]
-    uint32_t *desc = reinterpret_cast<uint32_t *>(sbin + kSRows * kBinStride);   // [W][kSeg][32]
-    int32_t *hits = reinterpret_cast<int32_t *>(desc + kTileWarps * kSeg * 32);  // [W*32][kBuf]
+    int32_t *hits = reinterpret_cast<int32_t *>(sbin + kSRows * kBinStride);     // [W*32][kBuf]
     int32_t *negs = hits + kTileWarps * 32 * kBuf;                     // P.K entries of -1
     __shared__ TileRows tr;
     __shared__ int4 rinfo[kSRows];   // GEN: x image bounds (slots) and y, z shifts per row
@@ -523,8 +609,8 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         describe_row(g, P.cell_start, lane, cx0, cy0, cz0, Gx, Gy, Gz, ra, tr.cell[lane]);
         describe_row(g, P.cell_start, lane + 32, cx0, cy0, cz0, Gx, Gy, Gz, rb,
                      lane + 32 < kSRows ? tr.cell[lane + 32] : cell_scratch);
-        // offsets: kGap NaN slots before every row and after the last
-        const int va = ra.len + kGap, vb = lane + 32 < kSRows ? rb.len + kGap : 0;
+        // offsets: rows back to back in staged order
+        const int va = ra.len, vb = lane + 32 < kSRows ? rb.len : 0;
         int xa = va, xb = vb;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -537,9 +623,9 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         }
         const int suma = __shfl_sync(0xffffffffu, xa, 31);
         const int sumb = __shfl_sync(0xffffffffu, xb, 31);
-        const int offa = kGap + xa - va;
-        const int offb = kGap + suma + xb - vb;
-        const int total = kGap + suma + sumb;
+        const int offa = xa - va;
+        const int offb = suma + xb - vb;
+        const int total = suma + sumb;
         tr.off[lane] = offa;
         tr.len[lane] = ra.len;
         rinfo[lane] = make_int4(offa + ra.lend, offa + ra.rbeg, __float_as_int(ra.sy),
@@ -587,16 +673,6 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     }
     __syncthreads();
     if (tr.fallback) return;
-    // NaN in the gaps (disjoint from the copies still in flight)
-    {
-        const float qn = __int_as_float(0x7fc00000);
-        const float4 nan4 = make_float4(qn, qn, qn, qn);
-        for (int e = threadIdx.x; e < (kSRows + 1) * kGap; e += blockDim.x) {
-            const int q = e / kGap, j = e % kGap;
-            stage[(q < kSRows ? tr.off[q] : tr.total) - kGap + j] = nan4;
-        }
-    }
-    __syncthreads();
     {
         bool done = false;
         for (uint32_t spins = 0; spins < 4096u && !done; ++spins)   // ~4 s
@@ -620,7 +696,6 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
     const float rl2 = g.rl2;
     const int nhome = tr.home_pref[4];
-    uint32_t *dsc = desc + warp * kSeg * 32 + lane;   // this lane's descriptors, stride 32
     const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * kBuf * 4);
     const uint32_t negs_addr = smem_u32(negs);
 
@@ -638,62 +713,6 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
         const float dz_lo = me.z - zlo, dz_hi = zhi - me.z;
 
-        // ---- this lane's segments: for each of the 25 rows, squared distance
-        //      (less the margin) from the atom to the row's (y, z) cell column,
-        //      x half-width h of the window, its bins and slots
-        float py2[5], pz2[5];
-#pragma unroll
-        for (int d = -2; d <= 2; ++d) {
-            float py = d > 0 ? dy_hi + (float)(d - 1) * P.side_y
-                             : (d < 0 ? dy_lo + (float)(-d - 1) * P.side_y : 0.0f);
-            float pz = d > 0 ? dz_hi + (float)(d - 1) * P.side_z
-                             : (d < 0 ? dz_lo + (float)(-d - 1) * P.side_z : 0.0f);
-            py = fmaxf(py - P.eps, 0.0f);
-            pz = fmaxf(pz - P.eps, 0.0f);
-            py2[d + 2] = py * py;
-            pz2[d + 2] = pz * pz;
-        }
-        const float mxr = me.x - X0;
-        const int Rh = (hy + 2) + kSY * (hz + 2);
-        int nseg = 0, tot = 0;
-#pragma unroll
-        for (int r = 0; r < 25; ++r) {
-            const int dy = r % 5 - 2, dz = r / 5 - 2;
-            const int R = Rh + dy + kSY * dz;
-            const float h2 = P.rl2_margin - (py2[dy + 2] + pz2[dz + 2]);
-            const bool ok = valid && h2 > 0.0f;
-            // approximate root (relative error ~1e-6): the margin absorbs it
-            const float hc = fmaxf(h2, 1e-20f);
-            const float hw = hc * rsqrtf(hc) + P.eps;
-            const int b0 = min(max(__float2int_rd((mxr - hw) * P.inv_bin), 0), nbins - 1);
-            const int b1 = min(max(__float2int_rd((mxr + hw) * P.inv_bin) + 1, 0), nbins);
-            const uint16_t *tb = sbin + R * kBinStride;
-            const int lo = tb[b0], hi = tb[b1];
-            if (r == 12) {   // home row: around the atom's own slot
-                const int e1 = min(hi, slot);
-                const int n1 = ok ? e1 - lo : 0;
-                const int ng1 = n1 > 0 ? (n1 + 3) >> 2 : 0;
-                dsc[32 * nseg] = seg_pack((uint32_t)(e1 - 4 * ng1), (uint32_t)ng1, (uint32_t)R);
-                nseg += ng1 > 0 ? 1 : 0;
-                tot += ng1;
-                const int s1 = max(lo, slot + 1);
-                const int n2 = ok ? hi - s1 : 0;
-                const int ng2 = n2 > 0 ? (n2 + 3) >> 2 : 0;
-                dsc[32 * nseg] = seg_pack((uint32_t)s1, (uint32_t)ng2, (uint32_t)R);
-                nseg += ng2 > 0 ? 1 : 0;
-                tot += ng2;
-            } else {
-                const int n = ok ? hi - lo : 0;
-                const int ng = n > 0 ? (n + 3) >> 2 : 0;
-                dsc[32 * nseg] = seg_pack((uint32_t)lo, (uint32_t)ng, (uint32_t)R);
-                nseg += ng > 0 ? 1 : 0;
-                tot += ng;
-            }
-        }
-        dsc[32 * nseg] = seg_pack(0u, 1u, 0u);   // end marker: the first gap, repeated
-        const int G4 = (__reduce_max_sync(0xffffffffu, tot) + 3) & ~3;
-
-        // ---- walk
         LaneOut o;
         o.buf = hb;
         o.bp = hb;
@@ -701,12 +720,16 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         o.Kb = 4u * (uint32_t)P.K;
         const int myid = __float_as_int(me.w);
         o.grow = reinterpret_cast<char *>(P.nbr + (int64_t)(valid ? myid : 0) * P.K);
+        const float mxr = me.x - X0;
+        const int Rh = (hy + 2) + kSY * (hz + 2);
         if (general)
-            walk_segments<true>(stage, dsc, nseg, G4, me, rl2, rinfo, g.Lx, o);
+            scan_rows<true>(stage, sbin, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
+                            dy_hi, dz_lo, dz_hi, mxr, o);
         else
-            walk_segments<false>(stage, dsc, nseg, G4, me, rl2, rinfo, g.Lx, o);
+            scan_rows<false>(stage, sbin, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
+                             dy_hi, dz_lo, dz_hi, mxr, o);
 
-        // ---- finish the row (the walk ends with a flush: at most 3 entries
+        // ---- finish the row (the scan ends with a flush: at most 3 entries
         //      pending): the partial vector completed with -1, then -1 from
         //      the shared block up to the capacity
         if (valid) {
@@ -758,12 +781,11 @@ k_pairs_listed(const float4 *__restrict__ cell_pos, const int32_t *__restrict__ 
     }
 }
 
-constexpr int kSlotLimit = 16000;   // descriptor slot field is 14 bits
+constexpr int kSlotLimit = 65000;   // slot-table entries are 16 bits
 
 size_t tile_fixed_smem(int K)
 {
     return (size_t)kSRows * kRowTab + (size_t)kSRows * kBinStride * sizeof(uint16_t) +
-           (size_t)kTileWarps * kSeg * 32 * sizeof(uint32_t) +
            (size_t)kTileWarps * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
@@ -790,9 +812,9 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
     if (n <= 0) return cudaSuccess;
     // Staged kernel: column grid and rows of whole 16-byte vectors.  The
     // stage must hold a typical tile (36 rows x (kTX + 2) cells at the mean
-    // cell occupancy, plus the gaps) with 10 % to spare; take the largest
-    // number of CTAs per SM whose shared-memory share still does.  Denser
-    // tiles are listed and searched per atom.
+    // cell occupancy) with 10 % to spare; take the largest number of CTAs per
+    // SM (up to 4) whose shared-memory share still does.  Denser tiles are
+    // listed and searched per atom.
     int stage_max = 0;
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
         (reinterpret_cast<uintptr_t>(nbr) & 15u) == 0 && n < (int64_t(1) << 31)) {
@@ -806,9 +828,9 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         const size_t fixed = tile_fixed_smem(capacity);
         const double per_cell = (double)n / (double)g.ncell;
         const int want =
-            (int)(1.1 * per_cell * kSRows * kSCells) + (kSRows + 1) * kGap + 32;
+            (int)(1.1 * per_cell * kSRows * kSCells) + 32;
         const int need = want > kStageMin ? want : kStageMin;
-        for (int ctas = 3; ctas >= 1; --ctas) {
+        for (int ctas = 4; ctas >= 1; --ctas) {
             long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
             const long cap = (long)optin - (long)fa.sharedSizeBytes;
             if (budget > cap) budget = cap;
