@@ -127,8 +127,8 @@ constexpr int kSRows = kSY * kSZ;           // 36 staged rows
 constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
 constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
 constexpr int kRowTab = kSCells * kBinsPerCell;
-constexpr int kBinStride = kRowTab + 2;     // slot-table entries per row (bins and the row end)
-constexpr int kBuf = 20;                    // entries of a lane's hit buffer
+constexpr int kFlushGroups = 2;             // 4-slot groups between flushes of a lane's hits
+constexpr int kBuf = 4 + 4 * kFlushGroups;   // entries of a lane's hit buffer (3 pending + new)
 constexpr int kTileWarps = 5;
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
@@ -372,16 +372,17 @@ struct LaneOut {
     char *grow;
 };
 
-// Every 16 slots (at most 16 new hits, so at most 3 + 16 pending): store the
-// whole 16-byte vectors to the row (entries past the capacity are only
-// counted) and move the partial vector to the buffer's start.
+// Every kFlushGroups groups of 4 slots (at most 3 + 4 kFlushGroups entries
+// pending): store the whole 16-byte vectors to the row (entries past the
+// capacity are only counted) and move the partial vector to the buffer's
+// start.
 __device__ __forceinline__ void flush_check(LaneOut &o)
 {
     const uint32_t u = o.bp - o.buf;
     const uint32_t nv = u & ~15u;
     if (nv != 0u) {
 #pragma unroll
-        for (uint32_t b = 0; b < 64u; b += 16u)
+        for (uint32_t b = 0; b < 16u * (kBuf / 4 - 1); b += 16u)
             if (b < nv && o.gfl + b < o.Kb) stg_u4(o.grow + o.gfl + b, lds_u4(o.buf + b));
         sts_u4(o.buf, lds_u4(o.buf + nv));
         o.gfl += nv;
@@ -394,8 +395,8 @@ __device__ __forceinline__ void flush_check(LaneOut &o)
 // (a NaN candidate), so no shared-memory traffic is spent on it.  The lanes
 // are consecutive x-sorted home atoms and scan the same row at the same
 // step, so their 16-byte loads fall on nearly consecutive slots (few bank
-// conflicts).  Every 16 slots, counted across rows in gc, the lane's whole
-// hit vectors are flushed.  GEN: periodic shifts, per slot in x (slots below
+// conflicts).  Every kFlushGroups groups, counted across rows in gc, the
+// lane's whole hit vectors are flushed.  GEN: periodic shifts, per slot in x (slots below
 // ri.x are the low image cell, at or above ri.y the high one) and per row in
 // y, z (ri.z, ri.w).
 template <bool GEN>
@@ -416,7 +417,7 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
         }
         scan4<GEN>(a0 + 16u * (uint32_t)j, len - j, c, me, rl2, sxv[0], sxv[1], sxv[2], sxv[3],
                    sy, sz, o.bp);
-        if (++gc == 4) {
+        if (++gc == kFlushGroups) {
             gc = 0;
             flush_check(o);
         }
@@ -430,7 +431,8 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
 // reaches the predicate.
 template <bool GEN>
 __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
-                                          const uint16_t *__restrict__ sbin, const int4 *rinfo,
+                                          const uint8_t *__restrict__ tabs,
+                                          const TileRows &tr, const int4 *rinfo,
                                           const TileParams &P, float rl2, float Lx, int nbins,
                                           const float4 me, bool valid, int slot, int Rh,
                                           float dy_lo, float dy_hi, float dz_lo, float dz_hi,
@@ -459,8 +461,12 @@ __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
         const float hw = hc * rsqrtf(hc) + P.eps;
         const int b0 = min(max(__float2int_rd((mxr - hw) * P.inv_bin), 0), nbins - 1);
         const int b1 = min(max(__float2int_rd((mxr + hw) * P.inv_bin) + 1, 0), nbins);
-        const uint16_t *tb = sbin + R * kBinStride;
-        const int lo = tb[b0], hi = tb[b1];
+        // first staged slot at or above a bin: start of its cell + the cell's
+        // table entry; past the last bin, the row end
+        const uint8_t *tb = tabs + R * kRowTab;
+        const int off = tr.off[R];
+        const int lo = off + tr.cell[R][b0 >> 4] + tb[b0];
+        const int hi = off + (b1 < nbins ? tr.cell[R][b1 >> 4] + tb[b1] : tr.len[R]);
         const int4 ri = GEN ? rinfo[R] : make_int4(0, 0, 0, 0);
         if (r == 12) {
             const int e1 = min(hi, slot);
@@ -575,14 +581,13 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-__global__ void __launch_bounds__(kTileWarps * 32, 4)
+__global__ void __launch_bounds__(kTileWarps * 32, 5)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
     extern __shared__ __align__(16) unsigned char tile_smem[];
     float4 *stage = reinterpret_cast<float4 *>(tile_smem);
     uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
-    uint16_t *sbin = reinterpret_cast<uint16_t *>(tabs + kSRows * kRowTab);   // [kSRows][kBinStride]
-    int32_t *hits = reinterpret_cast<int32_t *>(sbin + kSRows * kBinStride);     // [W*32][kBuf]
+    int32_t *hits = reinterpret_cast<int32_t *>(tabs + kSRows * kRowTab);       // [W*32][kBuf]
     int32_t *negs = hits + kTileWarps * 32 * kBuf;                     // P.K entries of -1
     __shared__ TileRows tr;
     __shared__ int4 rinfo[kSRows];   // GEN: x image bounds (slots) and y, z shifts per row
@@ -683,16 +688,6 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         }
     }
     const int nbins = (Gx + 2) * kBinsPerCell;
-    // slot table: sbin[R][b] = first staged slot of row R at or above x bin
-    // b (start of b's cell + the cell's table entry); b >= nbins: row end
-    for (int e = threadIdx.x; e < kSRows * kBinStride; e += blockDim.x) {
-        const int R = e / kBinStride, b = e - R * kBinStride;
-        const int v = b < nbins ? tr.off[R] + tr.cell[R][b >> 4] + tabs[R * kRowTab + b]
-                                : tr.off[R] + tr.len[R];
-        sbin[e] = (uint16_t)v;
-    }
-    __syncthreads();
-
     const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
     const float rl2 = g.rl2;
     const int nhome = tr.home_pref[4];
@@ -723,10 +718,10 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         const float mxr = me.x - X0;
         const int Rh = (hy + 2) + kSY * (hz + 2);
         if (general)
-            scan_rows<true>(stage, sbin, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
+            scan_rows<true>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
                             dy_hi, dz_lo, dz_hi, mxr, o);
         else
-            scan_rows<false>(stage, sbin, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
+            scan_rows<false>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
                              dy_hi, dz_lo, dz_hi, mxr, o);
 
         // ---- finish the row (the scan ends with a flush: at most 3 entries
@@ -785,7 +780,7 @@ constexpr int kSlotLimit = 65000;   // slot-table entries are 16 bits
 
 size_t tile_fixed_smem(int K)
 {
-    return (size_t)kSRows * kRowTab + (size_t)kSRows * kBinStride * sizeof(uint16_t) +
+    return (size_t)kSRows * kRowTab +
            (size_t)kTileWarps * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
@@ -813,7 +808,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
     // Staged kernel: column grid and rows of whole 16-byte vectors.  The
     // stage must hold a typical tile (36 rows x (kTX + 2) cells at the mean
     // cell occupancy) with 10 % to spare; take the largest number of CTAs per
-    // SM (up to 4) whose shared-memory share still does.  Denser tiles are
+    // SM (up to 5) whose shared-memory share still does.  Denser tiles are
     // listed and searched per atom.
     int stage_max = 0;
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
@@ -830,7 +825,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         const int want =
             (int)(1.1 * per_cell * kSRows * kSCells) + 32;
         const int need = want > kStageMin ? want : kStageMin;
-        for (int ctas = 4; ctas >= 1; --ctas) {
+        for (int ctas = 5; ctas >= 1; --ctas) {
             long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
             const long cap = (long)optin - (long)fa.sharedSizeBytes;
             if (budget > cap) budget = cap;
