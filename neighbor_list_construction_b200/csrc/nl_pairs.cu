@@ -829,7 +829,16 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
             long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
             const long cap = (long)optin - (long)fa.sharedSizeBytes;
             if (budget > cap) budget = cap;
-            const long fit = budget > (long)fixed ? (budget - (long)fixed) / (long)sizeof(float4) : 0;
+            long fit = budget > (long)fixed ? (budget - (long)fixed) / (long)sizeof(float4) : 0;
+            // shared memory is handed out in granules: shrink the stage until
+            // `ctas` CTAs really fit on one SM
+            while (ctas > 1 && fit >= need) {
+                int nb = 0;
+                NL_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &nb, k_pairs_tiles, kTileWarps * 32, sizeof(float4) * (size_t)fit + fixed));
+                if (nb >= ctas) break;
+                fit -= 32;
+            }
             if (fit >= need || ctas == 1) {
                 stage_max = (int)(fit < kSlotLimit ? fit : kSlotLimit);
                 break;
