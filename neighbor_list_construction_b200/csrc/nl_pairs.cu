@@ -424,6 +424,25 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
     }
 }
 
+// A range of a tile that touches the periodic faces takes the shifted scan
+// only when some lane's range needs it: the row has a y or z shift, or the
+// range reaches one of the row's x image cells.  Otherwise every shift is 0
+// and the plain scan gives the same bits.
+template <bool GEN>
+__device__ __forceinline__ void scan_checked(const float4 *__restrict__ stage, int lo, int len,
+                                             const float4 me, float rl2, int4 ri, float Lx,
+                                             int &gc, float4 (&c)[4], LaneOut &o)
+{
+    if (GEN) {
+        const bool need = (ri.z != 0 || ri.w != 0 || lo < ri.x || lo + len > ri.y) && len > 0;
+        if (__any_sync(0xffffffffu, need)) {
+            scan_range<true>(stage, lo, len, me, rl2, ri, Lx, gc, c, o);
+            return;
+        }
+    }
+    scan_range<false>(stage, lo, len, me, rl2, ri, Lx, gc, c, o);
+}
+
 // All 25 rows of one lane's atom: per row, the x half-width h of the window
 // from the squared distance (less the margin) between the atom and the row's
 // (y, z) cell column, its bins, and from the slot table its slots.  The home
@@ -470,11 +489,11 @@ __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
         const int4 ri = GEN ? rinfo[R] : make_int4(0, 0, 0, 0);
         if (r == 12) {
             const int e1 = min(hi, slot);
-            scan_range<GEN>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, gc, c, o);
+            scan_checked<GEN>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, gc, c, o);
             const int s1 = max(lo, slot + 1);
-            scan_range<GEN>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, gc, c, o);
+            scan_checked<GEN>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, gc, c, o);
         } else {
-            scan_range<GEN>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, gc, c, o);
+            scan_checked<GEN>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, gc, c, o);
         }
     }
     flush_check(o);
