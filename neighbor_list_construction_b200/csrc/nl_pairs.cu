@@ -98,7 +98,7 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // Staged tile search (column grid only: cells >= rl wide in x, >= rl/2 in y
 // and z, so the stencil is +-1 cell in x and +-2 cells in y and z).
 //
-// A tile is kTX x kTY x kTZ home cells.  Its 36 staged rows (y and z from
+// A tile is kTX x kTY x kTZ home cells.  Its staged rows (y and z from
 // two cells below to two cells above the home block) each cover the
 // conceptual cells cx0-1 .. cx0+Gx along x, with a periodic image cell at
 // either end of the box.  Every row is a contiguous range of the
@@ -121,23 +121,24 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // partial vector to the buffer's start.  Rows are finished with one
 // cp.async.bulk copy from a shared block of -1.
 // ---------------------------------------------------------------------------
-constexpr int kTX = 4, kTY = 2, kTZ = 2;   // home cells per tile
+constexpr int kTX = 4, kTY = 2, kTZ = 3;   // home cells per tile
 constexpr int kSY = kTY + 4, kSZ = kTZ + 4;
-constexpr int kSRows = kSY * kSZ;           // 36 staged rows
+constexpr int kSRows = kSY * kSZ;           // staged rows (42)
+constexpr int kHome = kTY * kTZ;            // home rows
 constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
 constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
 constexpr int kRowTab = kSCells * kBinsPerCell;
 constexpr int kFlushGroups = 2;             // 4-slot groups between flushes of a lane's hits
 constexpr int kBuf = 4 + 4 * kFlushGroups;   // entries of a lane's hit buffer (3 pending + new)
-constexpr int kTileWarps = 5;
+constexpr int kTileWarps = 7;
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
 struct TileRows {
     int off[kSRows];                 // slot of the row's first atom
     int len[kSRows];
     int cell[kSRows][kSCells + 1];   // row-local start of conceptual cell k
-    int home_begin[4];               // slot of the first home atom of home row h
-    int home_pref[5];                // home atoms before home row h
+    int home_begin[kHome];           // slot of the first home atom of home row h
+    int home_pref[kHome + 1];        // home atoms before home row h
     int total;                       // staged slots, gaps included
     int fallback;
 };
@@ -600,7 +601,7 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-__global__ void __launch_bounds__(kTileWarps * 32, 5)
+__global__ void __launch_bounds__(kTileWarps * 32, 4)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
     extern __shared__ __align__(16) unsigned char tile_smem[];
@@ -660,24 +661,26 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
             rinfo[lane + 32] = make_int4(offb + rb.lend, offb + rb.rbeg, __float_as_int(rb.sy),
                                          __float_as_int(rb.sz));
         }
-        // home rows h = hy + 2 hz are staged rows (hy + 2) + kSY (hz + 2), all below 32
-        const int h = lane == 14 ? 0 : lane == 15 ? 1 : lane == 20 ? 2 : lane == 21 ? 3 : -1;
+        // home rows h = hy + kTY hz are staged rows (hy + 2) + kSY (hz + 2)
+        __syncwarp();
         int hcnt = 0;
-        if (h >= 0) {
-            const bool valid = (h & 1) < Gy && (h >> 1) < Gz;
-            tr.home_begin[h] = offa + tr.cell[lane][1];
-            hcnt = valid ? tr.cell[lane][Gx + 1] - tr.cell[lane][1] : 0;
+        if (lane < kHome) {
+            const int hy = lane % kTY, hz = lane / kTY;
+            const int R = (hy + 2) + kSY * (hz + 2);
+            tr.home_begin[lane] = tr.off[R] + tr.cell[R][1];
+            hcnt = hy < Gy && hz < Gz ? tr.cell[R][Gx + 1] - tr.cell[R][1] : 0;
         }
-        const int c0 = __shfl_sync(0xffffffffu, hcnt, 14), c1 = __shfl_sync(0xffffffffu, hcnt, 15);
-        const int c2 = __shfl_sync(0xffffffffu, hcnt, 20), c3 = __shfl_sync(0xffffffffu, hcnt, 21);
+        int hx = hcnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, hx, o);
+            if (lane >= o) hx += y;
+        }
+        if (lane < kHome) tr.home_pref[lane] = hx - hcnt;
+        if (lane == kHome - 1) tr.home_pref[kHome] = hx;
         const uint32_t bytes = __reduce_add_sync(0xffffffffu, row_bytes(ra) + row_bytes(rb));
         const int fb = (total > P.stage_max || *P.unsorted != 0u) ? 1 : 0;
         if (lane == 0) {
-            tr.home_pref[0] = 0;
-            tr.home_pref[1] = c0;
-            tr.home_pref[2] = c0 + c1;
-            tr.home_pref[3] = c0 + c1 + c2;
-            tr.home_pref[4] = c0 + c1 + c2 + c3;
             tr.total = total;
             tr.fallback = fb;
             if (fb) {
@@ -709,7 +712,7 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     const int nbins = (Gx + 2) * kBinsPerCell;
     const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
     const float rl2 = g.rl2;
-    const int nhome = tr.home_pref[4];
+    const int nhome = tr.home_pref[kHome];
     const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * kBuf * 4);
     const uint32_t negs_addr = smem_u32(negs);
 
@@ -717,11 +720,11 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         const int a = c * 32 + lane;
         const bool valid = a < nhome;
         int h = 0;
-        while (h < 3 && a >= tr.home_pref[h + 1]) ++h;
+        while (h < kHome - 1 && a >= tr.home_pref[h + 1]) ++h;
         const int slot = tr.home_begin[h] + (a - tr.home_pref[h]);
         const float qn = __int_as_float(0x7fc00000);
         const float4 me = valid ? stage[slot] : make_float4(qn, qn, qn, qn);
-        const int hy = h & 1, hz = h >> 1;
+        const int hy = h % kTY, hz = h / kTY;
         const float ylo = (float)(cy0 + hy) * P.side_y, yhi = (float)(cy0 + hy + 1) * P.side_y;
         const float zlo = (float)(cz0 + hz) * P.side_z, zhi = (float)(cz0 + hz + 1) * P.side_z;
         const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
@@ -827,7 +830,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
     // Staged kernel: column grid and rows of whole 16-byte vectors.  The
     // stage must hold a typical tile (36 rows x (kTX + 2) cells at the mean
     // cell occupancy) with 10 % to spare; take the largest number of CTAs per
-    // SM (up to 5) whose shared-memory share still does.  Denser tiles are
+    // SM (up to 4) whose shared-memory share still does.  Denser tiles are
     // listed and searched per atom.
     int stage_max = 0;
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
@@ -844,7 +847,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         const int want =
             (int)(1.1 * per_cell * kSRows * kSCells) + 32;
         const int need = want > kStageMin ? want : kStageMin;
-        for (int ctas = 5; ctas >= 1; --ctas) {
+        for (int ctas = 4; ctas >= 1; --ctas) {
             long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
             const long cap = (long)optin - (long)fa.sharedSizeBytes;
             if (budget > cap) budget = cap;
