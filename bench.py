@@ -34,8 +34,8 @@ NOMINAL_HBM_GBS = 8000.0
 # belongs to the kernel source it was taken on: with any other source of the
 # pair kernel the bench reports null.
 PAIR_TRAFFIC = {"workload": "saltwater10m",
-                "sha256": "d7ee0d83f3a952ef945acf42179f2a3eb3f45b958276172662972548b70a59af",
-                "bytes": 668699136 + 10583890176}
+                "sha256": "b9fdd6b53191ffd7e0d1ea8c434e93775ff78a93a5be1dabb0c25bb369ffb8e6",
+                "bytes": 796743424 + 10741738240}
 
 
 def pair_traffic(workload: str):

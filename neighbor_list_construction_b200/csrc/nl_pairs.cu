@@ -110,16 +110,16 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // h = sqrt(rl^2 - d_perp^2) from the atom's distance to the row's (y, z)
 // cell face plus a margin; the window ends come from per-cell tables of
 // first slots at 1/16-cell steps in x (conservative: no candidate is lost).
-// Each window becomes a segment of whole groups of 4 slots (extended into
-// the row or into the NaN gap; an extra tested atom is decided by the exact
-// predicate like any other).  The home row's window is split around the
-// atom's own slot, so self never reaches the predicate.  A lane walks the
-// concatenation of its segments; the warp runs for the largest lane total.
+// A warp scans one row for all its lanes at once: the lanes are consecutive
+// x-sorted home atoms, so at each step their windows sit on nearly
+// consecutive slots and the 16-byte loads rarely share a bank; a lane past
+// its own window loads nothing.  The home row is scanned in two ranges
+// around the atom's own slot, so self never reaches the predicate.
 //
-// Hits go to a small per-lane buffer in shared memory; every 16 slots a
-// lane stores its whole 16-byte vectors to its global row and moves the
-// partial vector to the buffer's start.  Rows are finished with one
-// cp.async.bulk copy from a shared block of -1.
+// Hits go to a small per-lane buffer in shared memory; every 8 slots a lane
+// stores its whole 16-byte vectors to its global row and moves the partial
+// vector to the buffer's start.  Rows are finished with one cp.async.bulk
+// copy from a shared block of -1.
 // ---------------------------------------------------------------------------
 constexpr int kTX = 4, kTY = 2, kTZ = 3;   // home cells per tile
 constexpr int kSY = kTY + 4, kSZ = kTZ + 4;
