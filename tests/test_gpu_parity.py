@@ -156,6 +156,24 @@ def test_overflow_status_and_rows(ctx, oracle):
     gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt, full_sets=sets)
 
 
+@pytest.mark.parametrize("K", [102, 104])
+def test_build_capacity_not_multiple_of_vector(ctx, oracle, K):
+    """A box large enough for the staged kernel, with a capacity that is
+    (104) or is not (102) a whole number of 16-byte row vectors: the second
+    goes to the per-atom kernel; both must equal the oracle, overflowing
+    rows included."""
+    rng = np.random.default_rng(23)
+    L = 40.0
+    n = 7000
+    pos = np.zeros((n, 4), np.float32)
+    pos[:, :3] = rng.random((n, 3)) * L
+    box = np.array([L, L, L], np.float32)
+    nbr, cnt, st = gpu_build(ctx, pos, box, 5.75, 1.0, K)
+    o_nbr, o_cnt, o_ov = oracle.build(pos, box, 5.75, 1.0, K)
+    assert st == (1 if o_ov else 0)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+
+
 def test_build_cutoff_shell_pairs(ctx, oracle):
     """Partners placed within a few ulps of the cutoff radius: every pair
     decision sits on the r2 < rl2 boundary, so any change in rounding (a
