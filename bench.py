@@ -285,8 +285,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     cnt_host = torch.empty(n, dtype=torch.int32).pin_memory()
     stream = torch.cuda.current_stream()
 
+    sort_fn = nl.nl_sort_morton if args.curve == "morton" else nl.nl_sort_hilbert
+
     def step(src):
-        nl.nl_sort_hilbert(h, src, box, perm, ps, None, stream)
+        sort_fn(h, src, box, perm, ps, None, stream)
         nl.nl_build(h, ps, box, w.cutoff, w.skin, K, nbr, cnt, stream)
         nl.nl_skin_check(h, ps, box, w.skin, rb, None, stream)
 
@@ -370,7 +372,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"{args.workload}: {w.description}", "atoms": n,
                        "cutoff": w.cutoff, "skin": w.skin, "capacity": K,
-                       "step": "nl_sort_hilbert + nl_build + nl_skin_check",
+                       "step": f"nl_sort_{args.curve} + nl_build + nl_skin_check",
                        "cells": info[:3], "staged_pair_kernel": bool(info[3]),
                        "l2": "inputs larger than L2 (positions 165 MB, rows "
                              f"{n * K * 4 / 1e9:.1f} GB per step)",
@@ -417,6 +419,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="saltwater10m")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--curve", default="hilbert", choices=["hilbert", "morton"],
+                    help="curve of the sort in the timed step (Morton: the pages' baseline order)")
     ap.add_argument("--extras", action="store_true",
                     help="also time the replayed skin-check interval (graph vs eager) "
                          "and nl_build after Hilbert vs Morton order")

@@ -145,6 +145,7 @@ struct TileRows {
 
 struct TileParams {
     const float4 *cell_pos;
+    const uint32_t *atom_cell;
     const int32_t *cell_start;
     const uint8_t *cell_tab;
     int32_t *nbr;
@@ -601,7 +602,12 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-__global__ void __launch_bounds__(kTileWarps * 32, 4)
+// LISTED = false: one tile per CTA (blockIdx), 4 CTAs per SM; a tile whose
+// rows exceed the stage is listed.  LISTED = true: persistent CTAs, one per
+// SM with a large stage, over the listed tiles; a tile that still does not
+// fit is searched per atom from global memory.
+template <bool LISTED>
+__global__ void __launch_bounds__(kTileWarps * 32, LISTED ? 1 : 4)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
     extern __shared__ __align__(16) unsigned char tile_smem[];
@@ -616,8 +622,24 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < P.K; e += blockDim.x) negs[e] = -1;
     fence_proxy_async_smem();   // -1 block is read by bulk copies of any thread
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    uint32_t phase = 0;   // parity of the mbarrier phase the next staging completes
 
-    int t = blockIdx.x;
+    for (int it = 0;; ++it) {
+    int t;
+    if (LISTED) {
+        const uint32_t e = blockIdx.x + (uint32_t)it * gridDim.x;
+        if (e >= *P.fb_count) break;
+        t = (int)P.fb_list[e];
+    } else {
+        if (it > 0) break;
+        t = blockIdx.x;
+    }
+    const int tile = t;
     const int tx = t % P.tiles_x;
     t /= P.tiles_x;
     const int ty = t % P.tiles_y, tz = t / P.tiles_y;
@@ -628,7 +650,6 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
                          cz0 < 2 || cz0 + Gz + 2 > g.nz;
 
     if (warp == 0) {
-        if (lane == 0) mbar_init(&bar, 1);
         RowSrc ra, rb;   // rows lane and lane + 32
         int cell_scratch[kSCells + 1];
         describe_row(g, P.cell_start, lane, cx0, cy0, cz0, Gx, Gy, Gz, ra, tr.cell[lane]);
@@ -684,10 +705,11 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
             tr.total = total;
             tr.fallback = fb;
             if (fb) {
-                const uint32_t slot = atomicAdd(P.fb_count, 1u);
-                P.fb_list[slot] = (uint32_t)blockIdx.x;
+                if (!LISTED) {
+                    const uint32_t slot = atomicAdd(P.fb_count, 1u);
+                    P.fb_list[slot] = (uint32_t)tile;
+                }
             } else {
-                asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
                 mbar_arrive_expect_tx(&bar, bytes);
             }
         }
@@ -699,15 +721,29 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         }
     }
     __syncthreads();
-    if (tr.fallback) return;
+    if (tr.fallback) {
+        if (LISTED) {   // per atom, straight from global memory
+            for (int hz = 0; hz < Gz; ++hz)
+                for (int hy = 0; hy < Gy; ++hy) {
+                    const int64_t rowc = ((int64_t)(cz0 + hz) * g.ny + (cy0 + hy)) * g.nx;
+                    const int32_t k0 = P.cell_start[rowc + cx0], k1 = P.cell_start[rowc + cx0 + Gx];
+                    for (int32_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
+                        pair_row_per_atom<false>(k, P.cell_pos, P.cell_start, P.atom_cell, g, P.K,
+                                                 P.nbr, P.counts, P.flags);
+                }
+        }
+        __syncthreads();
+        continue;
+    }
     {
         bool done = false;
         for (uint32_t spins = 0; spins < 4096u && !done; ++spins)   // ~4 s
-            done = mbar_try_wait(&bar, 0);
+            done = mbar_try_wait(&bar, phase);
         if (__syncthreads_or(!done)) {
             if (threadIdx.x == 0) atomicOr(P.flags, kFlagTimeout);
             return;
         }
+        phase ^= 1u;
     }
     const int nbins = (Gx + 2) * kBinsPerCell;
     const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
@@ -767,35 +803,9 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
             if (cnt > P.K) atomicOr(P.flags, kFlagOverflow);
         }
     }
-    bulk_wait_read<0>();   // the -1 block stays readable until the copies are done
-}
-
-// Home atoms of the tiles the staged kernel listed (stage too small or cells
-// unsorted): per-atom search straight from global memory.
-__global__ void __launch_bounds__(128)
-k_pairs_listed(const float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start,
-               const uint32_t *__restrict__ atom_cell, CellGrid g, int32_t K, int tiles_x,
-               int tiles_y, const uint32_t *__restrict__ fb_list,
-               const uint32_t *__restrict__ fb_count, int32_t *__restrict__ nbr,
-               int32_t *__restrict__ counts, uint32_t *flags)
-{
-    const uint32_t nlisted = *fb_count;
-    for (uint32_t e = blockIdx.x; e < nlisted; e += gridDim.x) {
-        int t = (int)fb_list[e];
-        const int tx = t % tiles_x;
-        t /= tiles_x;
-        const int ty = t % tiles_y, tz = t / tiles_y;
-        const int cx0 = tx * kTX, cy0 = ty * kTY, cz0 = tz * kTZ;
-        const int Gx = min(kTX, g.nx - cx0), Gy = min(kTY, g.ny - cy0), Gz = min(kTZ, g.nz - cz0);
-        for (int hz = 0; hz < Gz; ++hz)
-            for (int hy = 0; hy < Gy; ++hy) {
-                const int64_t rowc = ((int64_t)(cz0 + hz) * g.ny + (cy0 + hy)) * g.nx;
-                const int32_t k0 = cell_start[rowc + cx0], k1 = cell_start[rowc + cx0 + Gx];
-                for (int32_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
-                    pair_row_per_atom<false>(k, cell_pos, cell_start, atom_cell, g, K, nbr, counts,
-                                             flags);
-            }
+    __syncthreads();   // the tile's shared data is reused by the next one
     }
+    bulk_wait_read<0>();   // the -1 block stays readable until the copies are done
 }
 
 constexpr int kSlotLimit = 65000;   // slot-table entries are 16 bits
@@ -816,9 +826,14 @@ cudaError_t pairs_set_attributes()
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, k_pairs_tiles);
+    e = cudaFuncGetAttributes(&fa, k_pairs_tiles<false>);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_pairs_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_pairs_tiles<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)fa.sharedSizeBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncGetAttributes(&fa, k_pairs_tiles<true>);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_pairs_tiles<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 optin - (int)fa.sharedSizeBytes);
 }
 
@@ -841,7 +856,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         NL_CUDA_TRY(cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
         cudaFuncAttributes fa;
-        NL_CUDA_TRY(cudaFuncGetAttributes(&fa, k_pairs_tiles));
+        NL_CUDA_TRY(cudaFuncGetAttributes(&fa, k_pairs_tiles<false>));
         const size_t fixed = tile_fixed_smem(capacity);
         const double per_cell = (double)n / (double)g.ncell;
         const int want =
@@ -857,7 +872,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
             while (ctas > 1 && fit >= need) {
                 int nb = 0;
                 NL_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &nb, k_pairs_tiles, kTileWarps * 32, sizeof(float4) * (size_t)fit + fixed));
+                    &nb, k_pairs_tiles<false>, kTileWarps * 32, sizeof(float4) * (size_t)fit + fixed));
                 if (nb >= ctas) break;
                 fit -= 32;
             }
@@ -871,6 +886,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
     if (stage_max > 0) {
         TileParams P;
         P.cell_pos = ctx->cell_pos;
+        P.atom_cell = ctx->atom_cell;
         P.cell_start = ctx->cell_start;
         P.cell_tab = ctx->cell_tab;
         P.nbr = nbr;
@@ -897,14 +913,24 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, sizeof(uint32_t), s));
         {
             ProfScope ps(ctx, PH_PAIRS, s);
-            k_pairs_tiles<<<(unsigned)ntiles, kTileWarps * 32, smem, s>>>(g, P);
+            k_pairs_tiles<false><<<(unsigned)ntiles, kTileWarps * 32, smem, s>>>(g, P);
             NL_CUDA_TRY(cudaGetLastError());
         }
         *used_fast = 1;
+        // the listed tiles: one persistent CTA per SM with the largest stage
+        int dev = 0, optin = 0;
+        NL_CUDA_TRY(cudaGetDevice(&dev));
+        NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+        cudaFuncAttributes fl;
+        NL_CUDA_TRY(cudaFuncGetAttributes(&fl, k_pairs_tiles<true>));
+        const long big = ((long)optin - (long)fl.sharedSizeBytes - (long)tile_fixed_smem(capacity)) /
+                         (long)sizeof(float4);
+        TileParams PL = P;
+        PL.stage_max = (int)(big < kSlotLimit ? big : kSlotLimit);
         ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
-        k_pairs_listed<<<(unsigned)(ctx->sm_count * 4), 128, 0, s>>>(
-            ctx->cell_pos, ctx->cell_start, ctx->atom_cell, g, capacity, P.tiles_x, P.tiles_y,
-            ctx->fb_list, ctx->fb_count, nbr, counts, ctx->flags);
+        k_pairs_tiles<true><<<(unsigned)ctx->sm_count, kTileWarps * 32,
+                              sizeof(float4) * (size_t)PL.stage_max + tile_fixed_smem(capacity), s>>>(
+            g, PL);
         return cudaGetLastError();
     }
     ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
