@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
             "oracle_rows": (ctypes.c_int, [i64, vp, vp, f32, f32, i32, i64, vp, vp, vp]),
             "oracle_build": (ctypes.c_int, [i64, vp, vp, f32, f32, i32, vp, vp]),
             "oracle_skin_check": (f32, [i64, vp, vp, vp, f32, vp]),
+            "oracle_close_pairs": (ctypes.c_int, [i64, vp, vp, f32, f32, f32, vp, vp]),
             "oracle_displacement": (f32, [u64, i64, i64, ctypes.c_int, f32]),
             "oracle_displace": (None, [i64, vp, u64, i64, f32]),
             "oracle_md_decisions": (i64, [i64, vp, vp, vp, f32, u64, f32, i64, vp]),
@@ -199,6 +200,20 @@ def bruteforce(pos, box, cutoff: float, skin: float, capacity: int):
     if rc < 0:
         raise MemoryError("oracle_bruteforce failed")
     return nbr, cnt, bool(rc)
+
+
+def close_pairs(pos, box, cutoff: float, skin: float, close_d2: float):
+    """Smallest r2 over all directed neighbor pairs (inf if none) and the
+    number of directed neighbor pairs with r2 < close_d2."""
+    p = _pos4(pos)
+    bx = _box(box)
+    mn = np.zeros(1, np.float32)
+    nc = np.zeros(1, np.int64)
+    rc = lib().oracle_close_pairs(p.shape[0], _p(p), _p(bx), np.float32(cutoff),
+                                  np.float32(skin), np.float32(close_d2), _p(mn), _p(nc))
+    if rc < 0:
+        raise MemoryError("oracle_close_pairs failed")
+    return float(mn[0]), int(nc[0])
 
 
 def skin_check(pos, ref, box, skin: float):

@@ -399,6 +399,45 @@ int oracle_build(int64_t n, const float *pos4, const float box[3], float cutoff,
     return oracle_rows(n, pos4, box, cutoff, skin, K, n, NULL, nbr, counts);
 }
 
+/* Close-pair detector over the full neighbor sets (no capacity cut): the
+ * smallest r2 of any directed neighbor pair (i, j in N(i)), +inf when there
+ * is none, and the number of directed neighbor pairs with r2 < close_d2.
+ * Reading of the pages' "no anomalously close pairs" check (Tessera,
+ * abstract): a by-product of the same predicate and candidate set.
+ * Returns 0, or -1 when memory runs out. */
+int oracle_close_pairs(int64_t n, const float *pos4, const float box[3], float cutoff,
+                       float skin, float close_d2, float *min_d2, int64_t *n_close)
+{
+    int32_t *cnt = (int32_t *)malloc((size_t)(n > 0 ? n : 1) * sizeof(int32_t));
+    int32_t *one = (int32_t *)malloc((size_t)(n > 0 ? n : 1) * sizeof(int32_t));
+    int32_t *nbr = NULL, K = 1;
+    float *w = NULL, mn = INFINITY;
+    int64_t i, k, nc = 0;
+    if (!cnt || !one) goto fail;
+    if (oracle_rows(n, pos4, box, cutoff, skin, 1, n, NULL, one, cnt) < 0) goto fail;
+    for (i = 0; i < n; i++)
+        if (cnt[i] > K) K = cnt[i];
+    nbr = (int32_t *)malloc((size_t)(n > 0 ? n : 1) * (size_t)K * sizeof(int32_t));
+    if (!nbr) goto fail;
+    if (oracle_rows(n, pos4, box, cutoff, skin, K, n, NULL, nbr, cnt) < 0) goto fail;
+    w = or_wrap_all(n, pos4, box);
+    if (!w) goto fail;
+    for (i = 0; i < n; i++)
+        for (k = 0; k < cnt[i]; k++) {
+            int64_t j = nbr[i * (int64_t)K + k];
+            float r2 = oracle_r2(&w[3 * i], &w[3 * j], box);
+            if (r2 < mn) mn = r2;
+            if (r2 < close_d2) nc++;
+        }
+    *min_d2 = mn;
+    *n_close = nc;
+    free(cnt); free(one); free(nbr); free(w);
+    return 0;
+fail:
+    free(cnt); free(one); free(nbr); free(w);
+    return -1;
+}
+
 /* ----------------------------------------------------------- skin check */
 
 /* Largest squared minimum-image displacement since the reference positions,
