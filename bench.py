@@ -260,6 +260,38 @@ def curve_comparison(nl, torch, h, pos, w, K, reps: int = 5) -> dict:
     return res
 
 
+def close_pair_timing(nl, torch, h, ps, w, K, close_d2: float = 1.0, reps: int = 5) -> dict:
+    """nl_build_close (the list plus the close-pair detector) against
+    nl_build on the same sorted positions: device time per call, and the
+    detector's results (smallest pair r2, directed pairs with r2 < close_d2)."""
+    n = ps.shape[0]
+    stream = torch.cuda.current_stream()
+    nbr = torch.empty(n, K, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(n, dtype=torch.int32, device="cuda")
+    mn = torch.empty(1, dtype=torch.float32, device="cuda")
+    nc = torch.empty(1, dtype=torch.int64, device="cuda")
+    res = {"close_d2": close_d2}
+    for name in ("build", "build_close"):
+        def call():
+            if name == "build":
+                nl.nl_build(h, ps, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+            else:
+                nl.nl_build_close(h, ps, w.box, w.cutoff, w.skin, K, nbr, cnt, close_d2, mn, nc,
+                                  stream)
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res[f"{name}_ms"] = e0.elapsed_time(e1) / reps
+    res["min_d2"] = float(mn.item())
+    res["n_close"] = int(nc.item())
+    return res
+
+
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -449,6 +481,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         if args.extras and world == 1:
             line["interval"] = interval_timing(nl, torch, h, ps, w, K, w.steps or 200)
             line["curves"] = curve_comparison(nl, torch, h, pos, w, K)
+            line["close_pairs"] = close_pair_timing(nl, torch, h, ps, w, K)
         if world == 1 and not args.no_cpu_baseline:
             cb = oracle_sample(1)
             line["cpu_baseline"] = {"value": cb["value"], "unit": "atoms/s", "cores": cb["cores"],

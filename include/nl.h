@@ -103,6 +103,23 @@ nl_status nl_build(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
                    float cutoff, float skin, int32_t capacity,
                    int32_t *nbr_out, int32_t *counts_out, void *stream);
 
+/* nl_build with a close-pair detector as a by-product (Tessera abstract:
+ * the simulations show no anomalously close pairs; this reports them while
+ * the list is built).  Same arguments, results and status as nl_build, plus:
+ *   *min_d2_out  (device float[1], 4-byte aligned): the smallest r2 over all
+ *                directed neighbor pairs (i, j in N(i)), counted before the
+ *                capacity cut; +inf when there is no pair within rl;
+ *   *n_close_out (device int64[1], 8-byte aligned): the number of directed
+ *                neighbor pairs with r2 < close_d2 (strict), again over the
+ *                full neighbor sets.
+ * r2 is the same fp32 value that decides membership.  close_d2 must be
+ * finite and >= 0, and both pointers non-NULL, else NL_ERR_ARG.  Both
+ * outputs are written on `stream` (initialised there before the search). */
+nl_status nl_build_close(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                         float cutoff, float skin, int32_t capacity,
+                         int32_t *nbr_out, int32_t *counts_out, float close_d2,
+                         float *min_d2_out, int64_t *n_close_out, void *stream);
+
 /* Skin check (Tessera abstract: a conservative neighbor skin preserves the
  * topology across updates).  m = max over atoms of the squared minimum-image
  * displacement between `pos` and the positions of the last nl_build (raw,

@@ -174,12 +174,20 @@ nl_status build_checked(nl_ctx *ctx, int64_t n, const float *pos, const float *b
 }
 
 nl_status build_enqueue(nl_ctx *ctx, int64_t n, const float *pos, const CellGrid &g,
-                        int32_t capacity, int32_t *nbr, int32_t *counts, cudaStream_t s, int *fast)
+                        int32_t capacity, int32_t *nbr, int32_t *counts, cudaStream_t s, int *fast,
+                        const CloseOut *close = nullptr)
 {
     const float4 *p4 = reinterpret_cast<const float4 *>(pos);
     if (launch_binning(ctx, n, p4, g, s) != cudaSuccess) return NL_ERR_CUDA;
-    if (launch_pairs(ctx, n, g, capacity, nbr, counts, s, fast) != cudaSuccess) return NL_ERR_CUDA;
+    if (launch_pairs(ctx, n, g, capacity, nbr, counts, s, fast, close) != cudaSuccess)
+        return NL_ERR_CUDA;
     return NL_OK;
+}
+
+__global__ void k_close_init(float *min_d2, int64_t *n_close)
+{
+    *min_d2 = __int_as_float(0x7f800000);
+    *n_close = 0;
 }
 
 // ------------------------------------------------------------- replay
@@ -448,6 +456,29 @@ nl_status nl_build(nl_ctx *ctx, int64_t n, const float *pos, const float *box, f
     if (st != NL_OK) return st;
     int fast = 0;
     st = build_enqueue(ctx, n, pos, g, capacity, nbr_out, counts_out, S(stream), &fast);
+    if (st != NL_OK) return st;
+    ctx->last_n = n;
+    ctx->last_grid = g;
+    ctx->last_fast = fast;
+    return NL_OK;
+}
+
+nl_status nl_build_close(nl_ctx *ctx, int64_t n, const float *pos, const float *box, float cutoff,
+                         float skin, int32_t capacity, int32_t *nbr_out, int32_t *counts_out,
+                         float close_d2, float *min_d2_out, int64_t *n_close_out, void *stream)
+{
+    if (!min_d2_out || !n_close_out || !std::isfinite(close_d2) || close_d2 < 0.0f)
+        return NL_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(min_d2_out) & 3u) || (reinterpret_cast<uintptr_t>(n_close_out) & 7u))
+        return NL_ERR_ARG;
+    CellGrid g;
+    nl_status st = build_checked(ctx, n, pos, box, cutoff, skin, capacity, nbr_out, counts_out, &g);
+    if (st != NL_OK) return st;
+    k_close_init<<<1, 1, 0, S(stream)>>>(min_d2_out, n_close_out);
+    if (cudaGetLastError() != cudaSuccess) return NL_ERR_CUDA;
+    CloseOut close{close_d2, min_d2_out, n_close_out};
+    int fast = 0;
+    st = build_enqueue(ctx, n, pos, g, capacity, nbr_out, counts_out, S(stream), &fast, &close);
     if (st != NL_OK) return st;
     ctx->last_n = n;
     ctx->last_grid = g;

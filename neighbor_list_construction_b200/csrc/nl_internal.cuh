@@ -160,9 +160,17 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
                            cudaStream_t s);
 // One-time kernel attributes of the pair search (large dynamic shared memory).
 cudaError_t pairs_set_attributes();
-// Pair search over the binned atoms.
+// Close-pair outputs of a build (device pointers): smallest pair r2 and the
+// number of directed pairs with r2 < close_d2.
+struct CloseOut {
+    float close_d2;
+    float *min_d2;
+    int64_t *n_close;
+};
+// Pair search over the binned atoms; close may be NULL.
 cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
-                         int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast);
+                         int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast,
+                         const CloseOut *close);
 
 // Skin check.  decisions/step may be NULL; cond_handle 0 = none.
 cudaError_t launch_skin(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,

@@ -18,19 +18,41 @@
 namespace nl {
 namespace {
 
+// Close-pair accumulator of one thread: smallest r2 of its hits (+inf when
+// none) and the number of hits with r2 < close_d2.
+struct CloseAcc {
+    float mn;
+    uint32_t nc;
+};
+
+// Folds a warp's accumulators into the global minimum (r2 >= 0, so the
+// float bits order like unsigned integers) and count.
+__device__ __forceinline__ void close_publish(const CloseAcc &cl, uint32_t *min_bits,
+                                              unsigned long long *n_close)
+{
+    const uint32_t mb = __reduce_min_sync(0xffffffffu, __float_as_uint(cl.mn));
+    const uint32_t nc = __reduce_add_sync(0xffffffffu, cl.nc);
+    if ((threadIdx.x & 31) == 0) {
+        if (mb != 0x7f800000u) atomicMin(min_bits, mb);
+        if (nc) atomicAdd(n_close, (unsigned long long)nc);
+    }
+}
+
+
 // ---------------------------------------------------------------------------
 // Per-atom search: one thread per atom, the stencil cells straight from
 // global memory, hits stored directly into the atom's row.  Used for small
 // boxes (literal minimum image), for tiles the staged kernel cannot take,
 // and when the staged kernel's preconditions fail.
 // ---------------------------------------------------------------------------
-template <bool LITERAL>
+template <bool LITERAL, bool CLOSE>
 __device__ __forceinline__ void pair_row_per_atom(int64_t k, const float4 *__restrict__ cell_pos,
                                                   const int32_t *__restrict__ cell_start,
                                                   const uint32_t *__restrict__ atom_cell,
                                                   const CellGrid &g, int32_t K,
                                                   int32_t *__restrict__ nbr,
-                                                  int32_t *__restrict__ counts, uint32_t *flags)
+                                                  int32_t *__restrict__ counts, uint32_t *flags,
+                                                  float close_d2, CloseAcc &cl)
 {
     const float4 p = cell_pos[k];
     const int i = __float_as_int(p.w);
@@ -70,9 +92,14 @@ __device__ __forceinline__ void pair_row_per_atom(int64_t k, const float4 *__res
                         if (sy != 0.0f) dy = __fadd_rn(dy, sy);
                         if (sz != 0.0f) dz = __fadd_rn(dz, sz);
                     }
-                    if (r2_of(dx, dy, dz) < g.rl2) {
+                    const float r2 = r2_of(dx, dy, dz);
+                    if (r2 < g.rl2) {
                         if (cnt < K) row[cnt] = jid;
                         ++cnt;
+                        if (CLOSE) {
+                            cl.mn = fminf(cl.mn, r2);
+                            cl.nc += r2 < close_d2 ? 1u : 0u;
+                        }
                     }
                 }
             }
@@ -83,15 +110,19 @@ __device__ __forceinline__ void pair_row_per_atom(int64_t k, const float4 *__res
     if (cnt > K) atomicOr(flags, kFlagOverflow);
 }
 
-template <bool LITERAL>
+template <bool LITERAL, bool CLOSE>
 __global__ void __launch_bounds__(128)
 k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start,
                  const uint32_t *__restrict__ atom_cell, int64_t n, CellGrid g, int32_t K,
-                 int32_t *__restrict__ nbr, int32_t *__restrict__ counts, uint32_t *flags)
+                 int32_t *__restrict__ nbr, int32_t *__restrict__ counts, uint32_t *flags,
+                 float close_d2, uint32_t *min_bits, unsigned long long *n_close)
 {
+    CloseAcc cl{__int_as_float(0x7f800000), 0u};
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride)
-        pair_row_per_atom<LITERAL>(k, cell_pos, cell_start, atom_cell, g, K, nbr, counts, flags);
+        pair_row_per_atom<LITERAL, CLOSE>(k, cell_pos, cell_start, atom_cell, g, K, nbr, counts,
+                                          flags, close_d2, cl);
+    if (CLOSE) close_publish(cl, min_bits, n_close);
 }
 
 // ---------------------------------------------------------------------------
@@ -144,6 +175,9 @@ struct TileRows {
 };
 
 struct TileParams {
+    float close_d2;                 // close-pair threshold (CLOSE kernels)
+    uint32_t *min_bits;             // float bits of the smallest pair r2 (CLOSE)
+    unsigned long long *n_close;    // directed pairs with r2 < close_d2 (CLOSE)
     const float4 *cell_pos;
     const uint32_t *atom_cell;
     const int32_t *cell_start;
@@ -300,63 +334,298 @@ __device__ __forceinline__ void test_cand(const float4 c, const float4 me, float
 // (0..4 or more) belong to this lane's range: the active ones are loaded
 // into c[0..3] (an inactive slot keeps a stale value), and each is tested as
 // in test_cand, a hit requiring the slot to be active.  GEN: x shifts
-// sx0..sx3 per slot and the row's y, z shifts.
-template <bool GEN>
+// sx0..sx3 per slot and the row's y, z shifts.  CLOSE: each hit also lowers
+// cl.mn to its r2 and counts in cl.nc when r2 < close_d2.
+template <bool GEN, bool CLOSE>
 __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], const float4 me,
                                       float rl2, float sx0, float sx1, float sx2, float sx3,
-                                      float sy, float sz, uint32_t &bp)
+                                      float sy, float sz, float close_d2, CloseAcc &cl,
+                                      uint32_t &bp)
 {
-#define NL_S4_HEAD                                                                      \
-    "{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3;\n\t"                      \
-    "setp.gt.s32 q0, %17, 0;\n\t"                                                       \
-    "setp.gt.s32 q1, %17, 1;\n\t"                                                       \
-    "setp.gt.s32 q2, %17, 2;\n\t"                                                       \
-    "setp.gt.s32 q3, %17, 3;\n\t"                                                       \
-    "@q0 ld.shared.v4.f32 {%1, %2, %3, %4}, [%18];\n\t"                                 \
-    "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%18+16];\n\t"                              \
-    "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%18+32];\n\t"                           \
-    "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%18+48];\n\t"
-#define NL_S4_TEST(q, X, Y, Z, W, SHIFT)                                                 \
-    "sub.rn.f32 dx, " X ", %19;\n\t"                                                    \
-    "sub.rn.f32 dy, " Y ", %20;\n\t"                                                    \
-    "sub.rn.f32 dz, " Z ", %21;\n\t" SHIFT                                             \
-    "mul.rn.f32 dx, dx, dx;\n\t"                                                        \
-    "mul.rn.f32 dy, dy, dy;\n\t"                                                        \
-    "mul.rn.f32 dz, dz, dz;\n\t"                                                        \
-    "add.rn.f32 dx, dx, dy;\n\t"                                                        \
-    "add.rn.f32 dx, dx, dz;\n\t"                                                        \
-    "setp.lt.and.f32 " q ", dx, %22, " q ";\n\t"                                        \
-    "@" q " st.shared.b32 [%0], " W ";\n\t"                                             \
-    "@" q " add.u32 %0, %0, 4;\n\t"
-#define NL_S4_SHIFT(SX)                                                                 \
-    "add.rn.f32 dx, dx, " SX ";\n\t"                                                    \
-    "add.rn.f32 dy, dy, %27;\n\t"                                                       \
-    "add.rn.f32 dz, dz, %28;\n\t"
-#define NL_S4_OUTS                                                                      \
-    "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x),      \
-        "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), \
-        "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
-    if (GEN)
-        asm volatile(NL_S4_HEAD
-                     NL_S4_TEST("q0", "%1", "%2", "%3", "%4", NL_S4_SHIFT("%23"))
-                     NL_S4_TEST("q1", "%5", "%6", "%7", "%8", NL_S4_SHIFT("%24"))
-                     NL_S4_TEST("q2", "%9", "%10", "%11", "%12", NL_S4_SHIFT("%25"))
-                     NL_S4_TEST("q3", "%13", "%14", "%15", "%16", NL_S4_SHIFT("%26")) "}"
-                     : NL_S4_OUTS
-                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(sx0),
-                       "f"(sx1), "f"(sx2), "f"(sx3), "f"(sy), "f"(sz));
-    else
-        asm volatile(NL_S4_HEAD
-                     NL_S4_TEST("q0", "%1", "%2", "%3", "%4", "")
-                     NL_S4_TEST("q1", "%5", "%6", "%7", "%8", "")
-                     NL_S4_TEST("q2", "%9", "%10", "%11", "%12", "")
-                     NL_S4_TEST("q3", "%13", "%14", "%15", "%16", "") "}"
-                     : NL_S4_OUTS
+    if (GEN && CLOSE)
+        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3, qc;\n\t"
+                     "setp.gt.s32 q0, %19, 0;\n\t"
+                     "setp.gt.s32 q1, %19, 1;\n\t"
+                     "setp.gt.s32 q2, %19, 2;\n\t"
+                     "setp.gt.s32 q3, %19, 3;\n\t"
+                     "@q0 ld.shared.v4.f32 {%1, %2, %3, %4}, [%20];\n\t"
+                     "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%20+16];\n\t"
+                     "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%20+32];\n\t"
+                     "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%20+48];\n\t"
+                     "sub.rn.f32 dx, %1, %21;\n\t"
+                     "sub.rn.f32 dy, %2, %22;\n\t"
+                     "sub.rn.f32 dz, %3, %23;\n\t"
+                     "add.rn.f32 dx, dx, %26;\n\t"
+                     "add.rn.f32 dy, dy, %30;\n\t"
+                     "add.rn.f32 dz, dz, %31;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q0, dx, %24, q0;\n\t"
+                     "@q0 st.shared.b32 [%0], %4;\n\t"
+                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "@q0 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q0;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "sub.rn.f32 dx, %5, %21;\n\t"
+                     "sub.rn.f32 dy, %6, %22;\n\t"
+                     "sub.rn.f32 dz, %7, %23;\n\t"
+                     "add.rn.f32 dx, dx, %27;\n\t"
+                     "add.rn.f32 dy, dy, %30;\n\t"
+                     "add.rn.f32 dz, dz, %31;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q1, dx, %24, q1;\n\t"
+                     "@q1 st.shared.b32 [%0], %8;\n\t"
+                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "@q1 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q1;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "sub.rn.f32 dx, %9, %21;\n\t"
+                     "sub.rn.f32 dy, %10, %22;\n\t"
+                     "sub.rn.f32 dz, %11, %23;\n\t"
+                     "add.rn.f32 dx, dx, %28;\n\t"
+                     "add.rn.f32 dy, dy, %30;\n\t"
+                     "add.rn.f32 dz, dz, %31;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q2, dx, %24, q2;\n\t"
+                     "@q2 st.shared.b32 [%0], %12;\n\t"
+                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "@q2 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q2;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "sub.rn.f32 dx, %13, %21;\n\t"
+                     "sub.rn.f32 dy, %14, %22;\n\t"
+                     "sub.rn.f32 dz, %15, %23;\n\t"
+                     "add.rn.f32 dx, dx, %29;\n\t"
+                     "add.rn.f32 dy, dy, %30;\n\t"
+                     "add.rn.f32 dz, dz, %31;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q3, dx, %24, q3;\n\t"
+                     "@q3 st.shared.b32 [%0], %16;\n\t"
+                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "@q3 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q3;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "}"
+                     : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w), "+f"(cl.mn), "+r"(cl.nc)
+                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(close_d2), "f"(sx0), "f"(sx1), "f"(sx2), "f"(sx3), "f"(sy), "f"(sz));
+    if (GEN && !CLOSE)
+        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3;\n\t"
+                     "setp.gt.s32 q0, %17, 0;\n\t"
+                     "setp.gt.s32 q1, %17, 1;\n\t"
+                     "setp.gt.s32 q2, %17, 2;\n\t"
+                     "setp.gt.s32 q3, %17, 3;\n\t"
+                     "@q0 ld.shared.v4.f32 {%1, %2, %3, %4}, [%18];\n\t"
+                     "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%18+16];\n\t"
+                     "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%18+32];\n\t"
+                     "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%18+48];\n\t"
+                     "sub.rn.f32 dx, %1, %19;\n\t"
+                     "sub.rn.f32 dy, %2, %20;\n\t"
+                     "sub.rn.f32 dz, %3, %21;\n\t"
+                     "add.rn.f32 dx, dx, %23;\n\t"
+                     "add.rn.f32 dy, dy, %27;\n\t"
+                     "add.rn.f32 dz, dz, %28;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q0, dx, %22, q0;\n\t"
+                     "@q0 st.shared.b32 [%0], %4;\n\t"
+                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "sub.rn.f32 dx, %5, %19;\n\t"
+                     "sub.rn.f32 dy, %6, %20;\n\t"
+                     "sub.rn.f32 dz, %7, %21;\n\t"
+                     "add.rn.f32 dx, dx, %24;\n\t"
+                     "add.rn.f32 dy, dy, %27;\n\t"
+                     "add.rn.f32 dz, dz, %28;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q1, dx, %22, q1;\n\t"
+                     "@q1 st.shared.b32 [%0], %8;\n\t"
+                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "sub.rn.f32 dx, %9, %19;\n\t"
+                     "sub.rn.f32 dy, %10, %20;\n\t"
+                     "sub.rn.f32 dz, %11, %21;\n\t"
+                     "add.rn.f32 dx, dx, %25;\n\t"
+                     "add.rn.f32 dy, dy, %27;\n\t"
+                     "add.rn.f32 dz, dz, %28;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q2, dx, %22, q2;\n\t"
+                     "@q2 st.shared.b32 [%0], %12;\n\t"
+                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "sub.rn.f32 dx, %13, %19;\n\t"
+                     "sub.rn.f32 dy, %14, %20;\n\t"
+                     "sub.rn.f32 dz, %15, %21;\n\t"
+                     "add.rn.f32 dx, dx, %26;\n\t"
+                     "add.rn.f32 dy, dy, %27;\n\t"
+                     "add.rn.f32 dz, dz, %28;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q3, dx, %22, q3;\n\t"
+                     "@q3 st.shared.b32 [%0], %16;\n\t"
+                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "}"
+                     : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
+                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(sx0), "f"(sx1), "f"(sx2), "f"(sx3), "f"(sy), "f"(sz));
+    if (!GEN && CLOSE)
+        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3, qc;\n\t"
+                     "setp.gt.s32 q0, %19, 0;\n\t"
+                     "setp.gt.s32 q1, %19, 1;\n\t"
+                     "setp.gt.s32 q2, %19, 2;\n\t"
+                     "setp.gt.s32 q3, %19, 3;\n\t"
+                     "@q0 ld.shared.v4.f32 {%1, %2, %3, %4}, [%20];\n\t"
+                     "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%20+16];\n\t"
+                     "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%20+32];\n\t"
+                     "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%20+48];\n\t"
+                     "sub.rn.f32 dx, %1, %21;\n\t"
+                     "sub.rn.f32 dy, %2, %22;\n\t"
+                     "sub.rn.f32 dz, %3, %23;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q0, dx, %24, q0;\n\t"
+                     "@q0 st.shared.b32 [%0], %4;\n\t"
+                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "@q0 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q0;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "sub.rn.f32 dx, %5, %21;\n\t"
+                     "sub.rn.f32 dy, %6, %22;\n\t"
+                     "sub.rn.f32 dz, %7, %23;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q1, dx, %24, q1;\n\t"
+                     "@q1 st.shared.b32 [%0], %8;\n\t"
+                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "@q1 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q1;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "sub.rn.f32 dx, %9, %21;\n\t"
+                     "sub.rn.f32 dy, %10, %22;\n\t"
+                     "sub.rn.f32 dz, %11, %23;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q2, dx, %24, q2;\n\t"
+                     "@q2 st.shared.b32 [%0], %12;\n\t"
+                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "@q2 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q2;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "sub.rn.f32 dx, %13, %21;\n\t"
+                     "sub.rn.f32 dy, %14, %22;\n\t"
+                     "sub.rn.f32 dz, %15, %23;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q3, dx, %24, q3;\n\t"
+                     "@q3 st.shared.b32 [%0], %16;\n\t"
+                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "@q3 min.f32 %17, %17, dx;\n\t"
+                     "setp.lt.and.f32 qc, dx, %25, q3;\n\t"
+                     "@qc add.u32 %18, %18, 1;\n\t"
+                     "}"
+                     : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w), "+f"(cl.mn), "+r"(cl.nc)
+                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(close_d2));
+    if (!GEN && !CLOSE)
+        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3;\n\t"
+                     "setp.gt.s32 q0, %17, 0;\n\t"
+                     "setp.gt.s32 q1, %17, 1;\n\t"
+                     "setp.gt.s32 q2, %17, 2;\n\t"
+                     "setp.gt.s32 q3, %17, 3;\n\t"
+                     "@q0 ld.shared.v4.f32 {%1, %2, %3, %4}, [%18];\n\t"
+                     "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%18+16];\n\t"
+                     "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%18+32];\n\t"
+                     "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%18+48];\n\t"
+                     "sub.rn.f32 dx, %1, %19;\n\t"
+                     "sub.rn.f32 dy, %2, %20;\n\t"
+                     "sub.rn.f32 dz, %3, %21;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q0, dx, %22, q0;\n\t"
+                     "@q0 st.shared.b32 [%0], %4;\n\t"
+                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "sub.rn.f32 dx, %5, %19;\n\t"
+                     "sub.rn.f32 dy, %6, %20;\n\t"
+                     "sub.rn.f32 dz, %7, %21;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q1, dx, %22, q1;\n\t"
+                     "@q1 st.shared.b32 [%0], %8;\n\t"
+                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "sub.rn.f32 dx, %9, %19;\n\t"
+                     "sub.rn.f32 dy, %10, %20;\n\t"
+                     "sub.rn.f32 dz, %11, %21;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q2, dx, %22, q2;\n\t"
+                     "@q2 st.shared.b32 [%0], %12;\n\t"
+                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "sub.rn.f32 dx, %13, %19;\n\t"
+                     "sub.rn.f32 dy, %14, %20;\n\t"
+                     "sub.rn.f32 dz, %15, %21;\n\t"
+                     "mul.rn.f32 dx, dx, dx;\n\t"
+                     "mul.rn.f32 dy, dy, dy;\n\t"
+                     "mul.rn.f32 dz, dz, dz;\n\t"
+                     "add.rn.f32 dx, dx, dy;\n\t"
+                     "add.rn.f32 dx, dx, dz;\n\t"
+                     "setp.lt.and.f32 q3, dx, %22, q3;\n\t"
+                     "@q3 st.shared.b32 [%0], %16;\n\t"
+                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "}"
+                     : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
                      : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2));
-#undef NL_S4_HEAD
-#undef NL_S4_TEST
-#undef NL_S4_SHIFT
-#undef NL_S4_OUTS
+    (void)close_d2;
+    (void)cl;
+    (void)sx0;
+    (void)sx1;
+    (void)sx2;
+    (void)sx3;
+    (void)sy;
+    (void)sz;
 }
 
 __device__ __forceinline__ void stg_u4(char *p, uint4 v)
@@ -401,10 +670,11 @@ __device__ __forceinline__ void flush_check(LaneOut &o)
 // lane's whole hit vectors are flushed.  GEN: periodic shifts, per slot in x (slots below
 // ri.x are the low image cell, at or above ri.y the high one) and per row in
 // y, z (ri.z, ri.w).
-template <bool GEN>
+template <bool GEN, bool CLOSE>
 __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int lo, int len,
                                            const float4 me, float rl2, int4 ri, float Lx, int &gc,
-                                           float4 (&c)[4], LaneOut &o)
+                                           float4 (&c)[4], float close_d2, CloseAcc &cl,
+                                           LaneOut &o)
 {
     const int Lmax = __reduce_max_sync(0xffffffffu, len);
     const float sy = __int_as_float(ri.z), sz = __int_as_float(ri.w);
@@ -417,8 +687,8 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
             for (int u = 0; u < 4; ++u)
                 sxv[u] = lo + j + u < ri.x ? -Lx : (lo + j + u >= ri.y ? Lx : 0.0f);
         }
-        scan4<GEN>(a0 + 16u * (uint32_t)j, len - j, c, me, rl2, sxv[0], sxv[1], sxv[2], sxv[3],
-                   sy, sz, o.bp);
+        scan4<GEN, CLOSE>(a0 + 16u * (uint32_t)j, len - j, c, me, rl2, sxv[0], sxv[1], sxv[2],
+                          sxv[3], sy, sz, close_d2, cl, o.bp);
         if (++gc == kFlushGroups) {
             gc = 0;
             flush_check(o);
@@ -430,19 +700,20 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
 // only when some lane's range needs it: the row has a y or z shift, or the
 // range reaches one of the row's x image cells.  Otherwise every shift is 0
 // and the plain scan gives the same bits.
-template <bool GEN>
+template <bool GEN, bool CLOSE>
 __device__ __forceinline__ void scan_checked(const float4 *__restrict__ stage, int lo, int len,
                                              const float4 me, float rl2, int4 ri, float Lx,
-                                             int &gc, float4 (&c)[4], LaneOut &o)
+                                             int &gc, float4 (&c)[4], float close_d2,
+                                             CloseAcc &cl, LaneOut &o)
 {
     if (GEN) {
         const bool need = (ri.z != 0 || ri.w != 0 || lo < ri.x || lo + len > ri.y) && len > 0;
         if (__any_sync(0xffffffffu, need)) {
-            scan_range<true>(stage, lo, len, me, rl2, ri, Lx, gc, c, o);
+            scan_range<true, CLOSE>(stage, lo, len, me, rl2, ri, Lx, gc, c, close_d2, cl, o);
             return;
         }
     }
-    scan_range<false>(stage, lo, len, me, rl2, ri, Lx, gc, c, o);
+    scan_range<false, CLOSE>(stage, lo, len, me, rl2, ri, Lx, gc, c, close_d2, cl, o);
 }
 
 // All 25 rows of one lane's atom: per row, the x half-width h of the window
@@ -450,14 +721,14 @@ __device__ __forceinline__ void scan_checked(const float4 *__restrict__ stage, i
 // (y, z) cell column, its bins, and from the slot table its slots.  The home
 // row is scanned in two ranges around the atom's own slot, so self never
 // reaches the predicate.
-template <bool GEN>
+template <bool GEN, bool CLOSE>
 __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
                                           const uint8_t *__restrict__ tabs,
                                           const TileRows &tr, const int4 *rinfo,
                                           const TileParams &P, float rl2, float Lx, int nbins,
                                           const float4 me, bool valid, int slot, int Rh,
                                           float dy_lo, float dy_hi, float dz_lo, float dz_hi,
-                                          float mxr, LaneOut &o)
+                                          float mxr, float close_d2, CloseAcc &cl, LaneOut &o)
 {
     int gc = 0;
     // candidate registers, carried across groups (an inactive slot's stale
@@ -491,11 +762,14 @@ __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
         const int4 ri = GEN ? rinfo[R] : make_int4(0, 0, 0, 0);
         if (r == 12) {
             const int e1 = min(hi, slot);
-            scan_checked<GEN>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, gc, c, o);
+            scan_checked<GEN, CLOSE>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, gc, c,
+                                     close_d2, cl, o);
             const int s1 = max(lo, slot + 1);
-            scan_checked<GEN>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, gc, c, o);
+            scan_checked<GEN, CLOSE>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, gc, c,
+                                     close_d2, cl, o);
         } else {
-            scan_checked<GEN>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, gc, c, o);
+            scan_checked<GEN, CLOSE>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, gc, c,
+                                     close_d2, cl, o);
         }
     }
     flush_check(o);
@@ -606,7 +880,7 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
 // rows exceed the stage is listed.  LISTED = true: persistent CTAs, one per
 // SM with a large stage, over the listed tiles; a tile that still does not
 // fit is searched per atom from global memory.
-template <bool LISTED>
+template <bool LISTED, bool CLOSE>
 __global__ void __launch_bounds__(kTileWarps * 32, LISTED ? 1 : 4)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
@@ -628,6 +902,7 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     }
     __syncthreads();
     uint32_t phase = 0;   // parity of the mbarrier phase the next staging completes
+    CloseAcc cl{__int_as_float(0x7f800000), 0u};
 
     for (int it = 0;; ++it) {
     int t;
@@ -728,8 +1003,9 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
                     const int64_t rowc = ((int64_t)(cz0 + hz) * g.ny + (cy0 + hy)) * g.nx;
                     const int32_t k0 = P.cell_start[rowc + cx0], k1 = P.cell_start[rowc + cx0 + Gx];
                     for (int32_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
-                        pair_row_per_atom<false>(k, P.cell_pos, P.cell_start, P.atom_cell, g, P.K,
-                                                 P.nbr, P.counts, P.flags);
+                        pair_row_per_atom<false, CLOSE>(k, P.cell_pos, P.cell_start, P.atom_cell,
+                                                        g, P.K, P.nbr, P.counts, P.flags,
+                                                        P.close_d2, cl);
                 }
         }
         __syncthreads();
@@ -776,11 +1052,11 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         const float mxr = me.x - X0;
         const int Rh = (hy + 2) + kSY * (hz + 2);
         if (general)
-            scan_rows<true>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
-                            dy_hi, dz_lo, dz_hi, mxr, o);
+            scan_rows<true, CLOSE>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot,
+                                   Rh, dy_lo, dy_hi, dz_lo, dz_hi, mxr, P.close_d2, cl, o);
         else
-            scan_rows<false>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh, dy_lo,
-                             dy_hi, dz_lo, dz_hi, mxr, o);
+            scan_rows<false, CLOSE>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot,
+                                    Rh, dy_lo, dy_hi, dz_lo, dz_hi, mxr, P.close_d2, cl, o);
 
         // ---- finish the row (the scan ends with a flush: at most 3 entries
         //      pending): the partial vector completed with -1, then -1 from
@@ -805,6 +1081,7 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     }
     __syncthreads();   // the tile's shared data is reused by the next one
     }
+    if (CLOSE) close_publish(cl, P.min_bits, P.n_close);
     bulk_wait_read<0>();   // the -1 block stays readable until the copies are done
 }
 
@@ -816,6 +1093,18 @@ size_t tile_fixed_smem(int K)
            (size_t)kTileWarps * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
+
+template <bool LISTED, bool CLOSE>
+cudaError_t tiles_allow_smem(int optin)
+{
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, k_pairs_tiles<LISTED, CLOSE>);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_pairs_tiles<LISTED, CLOSE>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin - (int)fa.sharedSizeBytes);
+}
+
 }  // namespace
 
 cudaError_t pairs_set_attributes()
@@ -825,20 +1114,18 @@ cudaError_t pairs_set_attributes()
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, k_pairs_tiles<false>);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_pairs_tiles<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             optin - (int)fa.sharedSizeBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncGetAttributes(&fa, k_pairs_tiles<true>);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_pairs_tiles<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                optin - (int)fa.sharedSizeBytes);
+    if ((e = tiles_allow_smem<false, false>(optin)) != cudaSuccess) return e;
+    if ((e = tiles_allow_smem<true, false>(optin)) != cudaSuccess) return e;
+    if ((e = tiles_allow_smem<false, true>(optin)) != cudaSuccess) return e;
+    return tiles_allow_smem<true, true>(optin);
 }
 
-cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
-                         int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast)
+namespace {
+
+template <bool CLOSE>
+cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
+                           int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast,
+                           const CloseOut *close)
 {
     *used_fast = 0;
     if (n <= 0) return cudaSuccess;
@@ -856,7 +1143,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         NL_CUDA_TRY(cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
         cudaFuncAttributes fa;
-        NL_CUDA_TRY(cudaFuncGetAttributes(&fa, k_pairs_tiles<false>));
+        NL_CUDA_TRY(cudaFuncGetAttributes(&fa, k_pairs_tiles<false, CLOSE>));
         const size_t fixed = tile_fixed_smem(capacity);
         const double per_cell = (double)n / (double)g.ncell;
         const int want =
@@ -872,7 +1159,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
             while (ctas > 1 && fit >= need) {
                 int nb = 0;
                 NL_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &nb, k_pairs_tiles<false>, kTileWarps * 32, sizeof(float4) * (size_t)fit + fixed));
+                    &nb, k_pairs_tiles<false, CLOSE>, kTileWarps * 32, sizeof(float4) * (size_t)fit + fixed));
                 if (nb >= ctas) break;
                 fit -= 32;
             }
@@ -885,6 +1172,9 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
     }
     if (stage_max > 0) {
         TileParams P;
+        P.close_d2 = CLOSE ? close->close_d2 : 0.0f;
+        P.min_bits = CLOSE ? reinterpret_cast<uint32_t *>(close->min_d2) : nullptr;
+        P.n_close = CLOSE ? reinterpret_cast<unsigned long long *>(close->n_close) : nullptr;
         P.cell_pos = ctx->cell_pos;
         P.atom_cell = ctx->atom_cell;
         P.cell_start = ctx->cell_start;
@@ -913,7 +1203,7 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, sizeof(uint32_t), s));
         {
             ProfScope ps(ctx, PH_PAIRS, s);
-            k_pairs_tiles<false><<<(unsigned)ntiles, kTileWarps * 32, smem, s>>>(g, P);
+            k_pairs_tiles<false, CLOSE><<<(unsigned)ntiles, kTileWarps * 32, smem, s>>>(g, P);
             NL_CUDA_TRY(cudaGetLastError());
         }
         *used_fast = 1;
@@ -922,13 +1212,13 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
         NL_CUDA_TRY(cudaGetDevice(&dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
         cudaFuncAttributes fl;
-        NL_CUDA_TRY(cudaFuncGetAttributes(&fl, k_pairs_tiles<true>));
+        NL_CUDA_TRY(cudaFuncGetAttributes(&fl, k_pairs_tiles<true, CLOSE>));
         const long big = ((long)optin - (long)fl.sharedSizeBytes - (long)tile_fixed_smem(capacity)) /
                          (long)sizeof(float4);
         TileParams PL = P;
         PL.stage_max = (int)(big < kSlotLimit ? big : kSlotLimit);
         ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
-        k_pairs_tiles<true><<<(unsigned)ctx->sm_count, kTileWarps * 32,
+        k_pairs_tiles<true, CLOSE><<<(unsigned)ctx->sm_count, kTileWarps * 32,
                               sizeof(float4) * (size_t)PL.stage_max + tile_fixed_smem(capacity), s>>>(
             g, PL);
         return cudaGetLastError();
@@ -937,13 +1227,29 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
     int64_t blocks = (n + 127) / 128;
     const int64_t cap = (int64_t)ctx->sm_count * 16;
     if (blocks > cap) blocks = cap;
+    const float cd2 = CLOSE ? close->close_d2 : 0.0f;
+    uint32_t *mb = CLOSE ? reinterpret_cast<uint32_t *>(close->min_d2) : nullptr;
+    unsigned long long *nc = CLOSE ? reinterpret_cast<unsigned long long *>(close->n_close) : nullptr;
     if (g.literal)
-        k_pairs_per_atom<true><<<(unsigned)blocks, 128, 0, s>>>(
-            ctx->cell_pos, ctx->cell_start, ctx->atom_cell, n, g, capacity, nbr, counts, ctx->flags);
+        k_pairs_per_atom<true, CLOSE><<<(unsigned)blocks, 128, 0, s>>>(
+            ctx->cell_pos, ctx->cell_start, ctx->atom_cell, n, g, capacity, nbr, counts, ctx->flags,
+            cd2, mb, nc);
     else
-        k_pairs_per_atom<false><<<(unsigned)blocks, 128, 0, s>>>(
-            ctx->cell_pos, ctx->cell_start, ctx->atom_cell, n, g, capacity, nbr, counts, ctx->flags);
+        k_pairs_per_atom<false, CLOSE><<<(unsigned)blocks, 128, 0, s>>>(
+            ctx->cell_pos, ctx->cell_start, ctx->atom_cell, n, g, capacity, nbr, counts, ctx->flags,
+            cd2, mb, nc);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
+                         int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast,
+                         const CloseOut *close)
+{
+    if (close)
+        return launch_pairs_t<true>(ctx, n, g, capacity, nbr, counts, s, used_fast, close);
+    return launch_pairs_t<false>(ctx, n, g, capacity, nbr, counts, s, used_fast, nullptr);
 }
 
 }  // namespace nl

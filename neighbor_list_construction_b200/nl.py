@@ -32,6 +32,8 @@ _SIGS = {
     "nl_sort_hilbert": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_sort_morton": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_build": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
+    "nl_build_close": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _f32, _vp, _vp,
+                              _vp]),
     "nl_skin_check": (_i32, [_vp, _i64, _vp, _vp, _f32, _vp, _vp, _vp]),
     "nl_replay": (_i32, [_vp, _vp, _i32, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp, _vp]),
     "nl_step_counter": (_vp, [_vp]),
@@ -140,6 +142,15 @@ def nl_build(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, stream=
                                 _stream(stream)), "nl_build")
 
 
+def nl_build_close(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, close_d2,
+                   min_d2_out, n_close_out, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_build_close(ctx, pos.shape[0], _ptr(pos), _box(box), float(cutoff),
+                                      float(skin), int(capacity), _ptr(nbr_out),
+                                      _ptr(counts_out), float(close_d2), _ptr(min_d2_out),
+                                      _ptr(n_close_out), _stream(stream)), "nl_build_close")
+
+
 def nl_skin_check(ctx, pos, box, skin, rebuild_out, max_d2_out=None, stream=None) -> int:
     _pos(pos)
     return _check(_lib.nl_skin_check(ctx, pos.shape[0], _ptr(pos), _box(box), float(skin),
@@ -241,6 +252,17 @@ class Context:
             counts = torch.empty(n, dtype=torch.int32, device=pos.device)
         nl_build(self.handle, pos, box, cutoff, skin, capacity, nbr, counts, stream)
         return nbr, counts
+
+    def build_close(self, pos, box, cutoff, skin, capacity, close_d2, stream=None):
+        """nl_build plus the close-pair detector: (nbr, counts, min_d2[1], n_close[1])."""
+        n = pos.shape[0]
+        nbr = torch.empty(n, capacity, dtype=torch.int32, device=pos.device)
+        counts = torch.empty(n, dtype=torch.int32, device=pos.device)
+        mn = torch.empty(1, dtype=torch.float32, device=pos.device)
+        nc = torch.empty(1, dtype=torch.int64, device=pos.device)
+        nl_build_close(self.handle, pos, box, cutoff, skin, capacity, nbr, counts, close_d2, mn,
+                       nc, stream)
+        return nbr, counts, mn, nc
 
     def skin_check(self, pos, box, skin, stream=None):
         rb = torch.zeros(1, dtype=torch.int32, device=pos.device)
