@@ -181,7 +181,11 @@ cudaError_t launch_skin(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
 // ------------------------------------------------------- device helpers
 __device__ __forceinline__ float wrap_coord(float x, float L)
 {
-    // w = x - L*floor(x/L), one fold into [0, L), else 0
+    // w = x - L*floor(x/L), one fold into [0, L), else 0.
+    // For 0 < x <= fl_down(L*(1 - 2^-23)) the quotient x/L rounds to a float
+    // below 1, so t = 0 and w = fl(x - 0) = x: the same bits without the
+    // division (zeros take the full path, which maps -0 to +0).
+    if (x > 0.0f && x <= __fmul_rd(L, 0.99999988f)) return x;
     float t = floorf(__fdiv_rn(x, L));
     float w = __fsub_rn(x, __fmul_rn(L, t));
     if (w < 0.0f) w = __fadd_rn(w, L);
