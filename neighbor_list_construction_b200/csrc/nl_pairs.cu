@@ -159,8 +159,8 @@ constexpr int kHome = kTY * kTZ;            // home rows
 constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
 constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
 constexpr int kRowTab = kSCells * kBinsPerCell;
-constexpr int kFlushGroups = 2;             // 4-slot groups between flushes of a lane's hits
-constexpr int kBuf = 4 + 4 * kFlushGroups;   // entries of a lane's hit buffer (3 pending + new)
+constexpr int kFlushAt = 8;                 // pending hits that make the warp flush
+constexpr int kBuf = kFlushAt + 4;          // entries of a lane's hit buffer (7 pending + 4 new)
 constexpr int kTileWarps = 7;
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
@@ -643,10 +643,10 @@ struct LaneOut {
     char *grow;
 };
 
-// Every kFlushGroups groups of 4 slots (at most 3 + 4 kFlushGroups entries
-// pending): store the whole 16-byte vectors to the row (entries past the
+// Store the lane's whole 16-byte vectors to its row (entries past the
 // capacity are only counted) and move the partial vector to the buffer's
-// start.
+// start; called when some lane of the warp holds kFlushAt entries, so at
+// most kBuf - 1 are pending.
 __device__ __forceinline__ void flush_check(LaneOut &o)
 {
     const uint32_t u = o.bp - o.buf;
@@ -666,13 +666,13 @@ __device__ __forceinline__ void flush_check(LaneOut &o)
 // (a NaN candidate), so no shared-memory traffic is spent on it.  The lanes
 // are consecutive x-sorted home atoms and scan the same row at the same
 // step, so their 16-byte loads fall on nearly consecutive slots (few bank
-// conflicts).  Every kFlushGroups groups, counted across rows in gc, the
-// lane's whole hit vectors are flushed.  GEN: periodic shifts, per slot in x (slots below
+// conflicts).  When a lane of the warp holds kFlushAt pending hits, the
+// lanes' whole hit vectors are flushed.  GEN: periodic shifts, per slot in x (slots below
 // ri.x are the low image cell, at or above ri.y the high one) and per row in
 // y, z (ri.z, ri.w).
 template <bool GEN, bool CLOSE>
 __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int lo, int len,
-                                           const float4 me, float rl2, int4 ri, float Lx, int &gc,
+                                           const float4 me, float rl2, int4 ri, float Lx,
                                            float4 (&c)[4], float close_d2, CloseAcc &cl,
                                            LaneOut &o)
 {
@@ -689,10 +689,8 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
         }
         scan4<GEN, CLOSE>(a0 + 16u * (uint32_t)j, len - j, c, me, rl2, sxv[0], sxv[1], sxv[2],
                           sxv[3], sy, sz, close_d2, cl, o.bp);
-        if (++gc == kFlushGroups) {
-            gc = 0;
-            flush_check(o);
-        }
+        // flush when some lane holds kFlushAt entries (at most kFlushAt - 1 + 4 pending)
+        if (__any_sync(0xffffffffu, o.bp - o.buf >= 4u * kFlushAt)) flush_check(o);
     }
 }
 
@@ -703,17 +701,17 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
 template <bool GEN, bool CLOSE>
 __device__ __forceinline__ void scan_checked(const float4 *__restrict__ stage, int lo, int len,
                                              const float4 me, float rl2, int4 ri, float Lx,
-                                             int &gc, float4 (&c)[4], float close_d2,
+                                             float4 (&c)[4], float close_d2,
                                              CloseAcc &cl, LaneOut &o)
 {
     if (GEN) {
         const bool need = (ri.z != 0 || ri.w != 0 || lo < ri.x || lo + len > ri.y) && len > 0;
         if (__any_sync(0xffffffffu, need)) {
-            scan_range<true, CLOSE>(stage, lo, len, me, rl2, ri, Lx, gc, c, close_d2, cl, o);
+            scan_range<true, CLOSE>(stage, lo, len, me, rl2, ri, Lx, c, close_d2, cl, o);
             return;
         }
     }
-    scan_range<false, CLOSE>(stage, lo, len, me, rl2, ri, Lx, gc, c, close_d2, cl, o);
+    scan_range<false, CLOSE>(stage, lo, len, me, rl2, ri, Lx, c, close_d2, cl, o);
 }
 
 // All 25 rows of one lane's atom: per row, the x half-width h of the window
@@ -730,7 +728,6 @@ __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
                                           float dy_lo, float dy_hi, float dz_lo, float dz_hi,
                                           float mxr, float close_d2, CloseAcc &cl, LaneOut &o)
 {
-    int gc = 0;
     // candidate registers, carried across groups (an inactive slot's stale
     // value is never taken: its hit predicate is false)
     float4 c[4];
@@ -762,13 +759,13 @@ __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
         const int4 ri = GEN ? rinfo[R] : make_int4(0, 0, 0, 0);
         if (r == 12) {
             const int e1 = min(hi, slot);
-            scan_checked<GEN, CLOSE>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, gc, c,
+            scan_checked<GEN, CLOSE>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, c,
                                      close_d2, cl, o);
             const int s1 = max(lo, slot + 1);
-            scan_checked<GEN, CLOSE>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, gc, c,
+            scan_checked<GEN, CLOSE>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, c,
                                      close_d2, cl, o);
         } else {
-            scan_checked<GEN, CLOSE>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, gc, c,
+            scan_checked<GEN, CLOSE>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, c,
                                      close_d2, cl, o);
         }
     }
