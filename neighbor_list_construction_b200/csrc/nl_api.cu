@@ -150,7 +150,8 @@ nl_status sort_impl(nl_ctx *ctx, int64_t n, const float *pos, const float *box, 
     }
     {
         ProfScope ps(ctx, PH_SORT, s);
-        if (launch_radix_passes(ctx, n, keys_out, reinterpret_cast<uint32_t *>(perm), s) !=
+        const SortRecompute rk{p4, n, box[0], box[1], box[2], sx, sy, sz, curve};
+        if (launch_radix_passes(ctx, n, keys_out, reinterpret_cast<uint32_t *>(perm), s, rk) !=
             cudaSuccess)
             return NL_ERR_CUDA;
     }
@@ -393,8 +394,8 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
     ok &= alloc(&c->vals[0], N) == cudaSuccess;
     ok &= alloc(&c->vals[1], N) == cudaSuccess;
     ok &= alloc(&c->hist, kKeyPasses * kRadixBins) == cudaSuccess;
-    ok &= alloc(&c->sort_status, (size_t)kKeyPasses * c->max_sort_tiles * kRadixBins) == cudaSuccess;
-    ok &= alloc(&c->sort_ctr, kKeyPasses) == cudaSuccess;
+    ok &= alloc(&c->sort_status, (size_t)kStatusPasses * c->max_sort_tiles * kRadixBins) == cudaSuccess;
+    ok &= alloc(&c->sort_ctr, kStatusPasses) == cudaSuccess;
     ok &= alloc(&c->cell_count, c->max_cells) == cudaSuccess;
     ok &= alloc(&c->cell_start, c->max_cells + 1) == cudaSuccess;
     ok &= alloc(&c->scan_status, c->max_scan_tiles) == cudaSuccess;
@@ -413,6 +414,7 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
         c->rebuild_tmp = reinterpret_cast<int32_t *>(c->zero_block + 9);
         c->unsorted = c->zero_block + 12;
         c->fb_count = c->zero_block + 13;
+        c->sort_gate = c->zero_block + 14;
         ok &= pairs_set_attributes() == cudaSuccess;
         ok &= cudaMemset(c->zero_block, 0, 64 * sizeof(uint32_t)) == cudaSuccess;
         ok &= cudaDeviceSynchronize() == cudaSuccess;

@@ -16,6 +16,10 @@ constexpr uint32_t kQMax = (1u << kQBits) - 1u;
 constexpr int kRadixBits = 8;                 // LSD digit width
 constexpr int kRadixBins = 1 << kRadixBits;
 constexpr int kKeyPasses = 8;                 // 63-bit keys: 8 digits of 8 bits
+constexpr int kTopPasses = 3;                 // fast path: the top digits (bits 40..63)
+constexpr int kStatusPasses = kKeyPasses + kTopPasses;   // look-back status slots
+constexpr int kPrefixShift = 8 * (kKeyPasses - kTopPasses);  // key >> this = sorted prefix
+constexpr int kRunMax = 64;                   // longest prefix run one thread finishes
 
 // Onesweep tile: 256 threads x 16 keys.
 constexpr int kSortThreads = 256;
@@ -101,6 +105,7 @@ struct nl_ctx {
     int32_t *rebuild_tmp = nullptr;    // [1]
     uint32_t *unsorted = nullptr;      // [1] 1 if a cell was too large for the in-cell sort
     uint32_t *fb_count = nullptr;      // [1] tiles listed for the per-atom search
+    uint32_t *sort_gate = nullptr;     // [1] set when the sort needs its full path
     uint32_t *fb_list = nullptr;       // [max_cells] their ids
     uint32_t *zero_block = nullptr;    // one allocation holding the small state
 
@@ -144,14 +149,26 @@ struct ProfScope {
 // ------------------------------------------------------------- launchers
 // Curve keys of all atoms into ctx->keys[0]/vals[0] and the 8 digit
 // histograms into ctx->hist (which must be zero); curve 0 Hilbert, 1 Morton.
+// With a gate: only when *gate != 0, keys only (no histograms).
 cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
-                        float Lz, float Sx, float Sy, float Sz, int curve, cudaStream_t s);
+                        float Lz, float Sx, float Sy, float Sz, int curve, cudaStream_t s,
+                        const uint32_t *gate = nullptr);
 // Exclusive scan of the 8 histograms in place.
 cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s);
-// 8 onesweep passes; the last writes keys to keys_final (may be ctx->keys[0])
-// and indices to vals_final.
+// What the gated full sort needs to recompute the keys.
+struct SortRecompute {
+    const float4 *pos;
+    int64_t n;
+    float Lx, Ly, Lz, Sx, Sy, Sz;
+    int curve;
+};
+// The sort of ctx->keys[0]/vals[0] (keys, histograms scanned): onesweep
+// passes over the top kTopPasses digits and the prefix-run finish; behind
+// them a gated full sort (keys recomputed, 8 passes) that runs only when a
+// prefix run was longer than kRunMax.  Writes keys to keys_final (NULL: not
+// kept) and indices to vals_final.
 cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
-                                uint32_t *vals_final, cudaStream_t s);
+                                uint32_t *vals_final, cudaStream_t s, const SortRecompute &rk);
 cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, float4 *out,
                           cudaStream_t s);
 

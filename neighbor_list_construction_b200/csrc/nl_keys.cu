@@ -83,8 +83,13 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
                                               float Lx, float Ly, float Lz, float Sx,
                                               float Sy, float Sz, uint64_t *__restrict__ keys,
                                               uint32_t *__restrict__ vals,
-                                              uint32_t *__restrict__ hist)
+                                              uint32_t *__restrict__ hist,
+                                              const uint32_t *gate)
 {
+    // gated recompute (the full sort's keys): only when the gate is set, and
+    // without the histograms, which the first pass already made
+    const bool recompute = gate != nullptr;
+    if (recompute && ld_volatile_u32(gate) == 0u) return;
     __shared__ uint32_t sh[kKeyPasses * kRadixBins];
     for (int i = threadIdx.x; i < kKeyPasses * kRadixBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
@@ -97,11 +102,13 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
         const uint64_t k = CURVE == 0 ? hilbert_index(qx, qy, qz) : morton_index(qx, qy, qz);
         keys[i] = k;
         vals[i] = (uint32_t)i;
+        if (recompute) continue;
 #pragma unroll
         for (int d = 0; d < kKeyPasses; ++d)
             atomicAdd(&sh[d * kRadixBins + (uint32_t)((k >> (kRadixBits * d)) & 0xffu)], 1u);
     }
     __syncthreads();
+    if (recompute) return;
     for (int i = threadIdx.x; i < kKeyPasses * kRadixBins; i += blockDim.x) {
         const uint32_t v = sh[i];
         if (v) atomicAdd(&hist[i], v);
@@ -142,7 +149,8 @@ __global__ void k_gather(int64_t n, const float4 *__restrict__ pos, const int32_
 }  // namespace
 
 cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly, float Lz,
-                        float Sx, float Sy, float Sz, int curve, cudaStream_t s)
+                        float Sx, float Sy, float Sz, int curve, cudaStream_t s,
+                        const uint32_t *gate)
 {
     if (n <= 0) return cudaSuccess;
     int64_t blocks = (n + 255) / 256;
@@ -150,10 +158,10 @@ cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
     if (blocks > cap) blocks = cap;
     if (curve == 0)
         k_keys<0><<<(unsigned)blocks, 256, 0, s>>>(pos, n, Lx, Ly, Lz, Sx, Sy, Sz, ctx->keys[0],
-                                                    ctx->vals[0], ctx->hist);
+                                                    ctx->vals[0], ctx->hist, gate);
     else
         k_keys<1><<<(unsigned)blocks, 256, 0, s>>>(pos, n, Lx, Ly, Lz, Sx, Sy, Sz, ctx->keys[0],
-                                                    ctx->vals[0], ctx->hist);
+                                                    ctx->vals[0], ctx->hist, gate);
     return cudaGetLastError();
 }
 

@@ -36,10 +36,10 @@ constexpr size_t kOffVals0 = align256(kOffKeys1 + sizeof(uint64_t) * kNoallocMax
 constexpr size_t kOffVals1 = align256(kOffVals0 + sizeof(uint32_t) * kNoallocMaxAtoms);
 constexpr size_t kOffHist = align256(kOffVals1 + sizeof(uint32_t) * kNoallocMaxAtoms);
 constexpr size_t kOffStatus = align256(kOffHist + sizeof(uint32_t) * nl::kKeyPasses * nl::kRadixBins);
-constexpr size_t kOffCtr = align256(kOffStatus + sizeof(uint32_t) * nl::kKeyPasses * kNoallocTiles *
-                                                     nl::kRadixBins);
-constexpr size_t kOffFlags = align256(kOffCtr + sizeof(uint32_t) * nl::kKeyPasses);
-constexpr size_t kNoallocScratchBytes = align256(kOffFlags + sizeof(uint32_t));
+constexpr size_t kOffCtr = align256(kOffStatus + sizeof(uint32_t) * nl::kStatusPasses *
+                                                     kNoallocTiles * nl::kRadixBins);
+constexpr size_t kOffFlags = align256(kOffCtr + sizeof(uint32_t) * nl::kStatusPasses);
+constexpr size_t kNoallocScratchBytes = align256(kOffFlags + 2 * sizeof(uint32_t));   // flags, gate
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
@@ -99,10 +99,11 @@ extern "C" nl_status nl_sort_hilbert_noalloc(int64_t n, const float *pos, const 
     view.sort_status = reinterpret_cast<uint32_t *>(d.base + kOffStatus);
     view.sort_ctr = reinterpret_cast<uint32_t *>(d.base + kOffCtr);
     view.flags = reinterpret_cast<uint32_t *>(d.base + kOffFlags);
+    view.sort_gate = view.flags + 1;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the array keeps the previous call's contents: clear what must start at 0
-    if (cudaMemsetAsync(view.flags, 0, sizeof(uint32_t), s) != cudaSuccess) return NL_ERR_CUDA;
+    if (cudaMemsetAsync(view.flags, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return NL_ERR_CUDA;
     if (n > 0) {
         volatile float sx = 2097152.0f / box[0];
         volatile float sy = 2097152.0f / box[1];
@@ -114,8 +115,9 @@ extern "C" nl_status nl_sort_hilbert_noalloc(int64_t n, const float *pos, const 
         if (nl::launch_keys(&view, n, p4, box[0], box[1], box[2], sx, sy, sz, 0, s) != cudaSuccess)
             return NL_ERR_CUDA;
         if (nl::launch_hist_scan(&view, s) != cudaSuccess) return NL_ERR_CUDA;
-        if (nl::launch_radix_passes(&view, n, keys_out, reinterpret_cast<uint32_t *>(perm_out), s) !=
-            cudaSuccess)
+        const nl::SortRecompute rk{p4, n, box[0], box[1], box[2], sx, sy, sz, 0};
+        if (nl::launch_radix_passes(&view, n, keys_out, reinterpret_cast<uint32_t *>(perm_out), s,
+                                    rk) != cudaSuccess)
             return NL_ERR_CUDA;
         if (nl::launch_gather(n, p4, perm_out, reinterpret_cast<float4 *>(pos_sorted_out), s) !=
             cudaSuccess)

@@ -1,4 +1,16 @@
-// nl_sort.cu -- onesweep LSD radix sort of (63-bit key, 32-bit index) pairs.
+// nl_sort.cu -- sort of (63-bit key, 32-bit index) pairs: onesweep LSD radix
+// passes, and a prefix-run finish.
+//
+// Fast path: the three most significant 8-bit digits (bits 40..63) by
+// onesweep passes; the array is then ordered by its 24-bit key prefix, with
+// equal prefixes in index order.  A prefix is one cell of a 256^3 grid over
+// the box, so a run of equal prefixes holds about n / 2^24 keys (a handful
+// at most for atoms at liquid density); each run is finished by one thread
+// with an insertion sort on (key, index).  A run longer than kRunMax keys
+// (strongly clustered input) sets a gate word, and a gated copy of the full
+// eight-pass sort, already enqueued behind, then recomputes the keys and
+// redoes the whole order; when the gate is clear those launches return at
+// once.
 //
 // One kernel launch per 8-bit digit.  Each CTA takes the next tile from an
 // atomic ticket (so a tile only ever waits on tiles whose CTAs are already
@@ -22,8 +34,9 @@ __global__ void __launch_bounds__(kSortThreads, 4)
 k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
            uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, int64_t n,
            int shift, const uint32_t *__restrict__ digit_start, uint32_t *status,
-           uint32_t *ticket, uint32_t *flags)
+           uint32_t *ticket, uint32_t *flags, const uint32_t *gate)
 {
+    if (gate && ld_volatile_u32(gate) == 0u) return;   // gated pass not needed
     extern __shared__ __align__(16) unsigned char sort_smem[];
     uint64_t *s_keys = reinterpret_cast<uint64_t *>(sort_smem);
     uint32_t *s_vals = reinterpret_cast<uint32_t *>(sort_smem + sizeof(uint64_t) * kSortTile);
@@ -165,10 +178,50 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
     }
 }
 
+// Finishes the runs of equal 24-bit key prefix (the output of the passes
+// over bits 40..63): the thread at a run's first position sorts the run by
+// (key, index) and writes it to the final arrays.  A run of more than
+// kRunMax keys sets *gate instead (the full sort then redoes everything).
+__global__ void __launch_bounds__(256)
+k_run_sort(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ vals, int64_t n,
+           uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, uint32_t *gate)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const uint64_t pre = keys[i] >> kPrefixShift;
+        if (i > 0 && (keys[i - 1] >> kPrefixShift) == pre) continue;   // not a run head
+        int64_t e = i + 1;
+        while (e < n && e - i <= kRunMax && (keys[e] >> kPrefixShift) == pre) ++e;
+        if (e - i > kRunMax) {
+            atomicOr(gate, 1u);
+            continue;
+        }
+        const int m = (int)(e - i);
+        uint64_t k[kRunMax];
+        uint32_t v[kRunMax];
+        for (int a = 0; a < m; ++a) {
+            const uint64_t ka = keys[i + a];
+            const uint32_t va = vals[i + a];
+            int b = a;
+            while (b > 0 && (k[b - 1] > ka || (k[b - 1] == ka && v[b - 1] > va))) {
+                k[b] = k[b - 1];
+                v[b] = v[b - 1];
+                --b;
+            }
+            k[b] = ka;
+            v[b] = va;
+        }
+        for (int a = 0; a < m; ++a) {
+            if (keys_out) keys_out[i + a] = k[a];
+            vals_out[i + a] = v[a];
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
-                                uint32_t *vals_final, cudaStream_t s)
+                                uint32_t *vals_final, cudaStream_t s, const SortRecompute &rk)
 {
     if (n <= 0) return cudaSuccess;
     const int64_t tiles = (n + kSortTile - 1) / kSortTile;
@@ -183,9 +236,34 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
         attr_set = true;
     }
     NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_status, 0,
-                                sizeof(uint32_t) * kKeyPasses * tiles * kRadixBins, s));
-    NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_ctr, 0, sizeof(uint32_t) * kKeyPasses, s));
+                                sizeof(uint32_t) * kStatusPasses * tiles * kRadixBins, s));
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_ctr, 0, sizeof(uint32_t) * kStatusPasses, s));
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_gate, 0, sizeof(uint32_t), s));
+    // fast path: the top kTopPasses digits, then the prefix runs
     int src = 0;
+    for (int q = 0; q < kTopPasses; ++q) {
+        const int p = kKeyPasses - kTopPasses + q;   // digit
+        const int slot = kKeyPasses + q;             // status slot of the fast path
+        uint32_t *status = ctx->sort_status + (size_t)slot * tiles * kRadixBins;
+        k_onesweep<true><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
+            ctx->keys[src], ctx->vals[src], ctx->keys[1 - src], ctx->vals[1 - src], n,
+            kRadixBits * p, ctx->hist + p * kRadixBins, status, ctx->sort_ctr + slot, ctx->flags,
+            nullptr);
+        NL_CUDA_TRY(cudaGetLastError());
+        src = 1 - src;
+    }
+    {
+        int64_t blocks = (n + 255) / 256;
+        const int64_t cap = (int64_t)ctx->sm_count * 8;
+        if (blocks > cap) blocks = cap;
+        k_run_sort<<<(unsigned)blocks, 256, 0, s>>>(ctx->keys[src], ctx->vals[src], n, keys_final,
+                                                    vals_final, ctx->sort_gate);
+        NL_CUDA_TRY(cudaGetLastError());
+    }
+    // full sort, gated: runs only when a prefix run was too long
+    NL_CUDA_TRY(launch_keys(ctx, rk.n, rk.pos, rk.Lx, rk.Ly, rk.Lz, rk.Sx, rk.Sy, rk.Sz, rk.curve, s,
+                            ctx->sort_gate));
+    src = 0;
     for (int p = 0; p < kKeyPasses; ++p) {
         const bool last = p == kKeyPasses - 1;
         uint64_t *ko = last ? (keys_final ? keys_final : ctx->keys[1 - src]) : ctx->keys[1 - src];
@@ -194,11 +272,11 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
         if (last && !keys_final)
             k_onesweep<false><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
                 ctx->keys[src], ctx->vals[src], ko, vo, n, kRadixBits * p,
-                ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags);
+                ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags, ctx->sort_gate);
         else
             k_onesweep<true><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
                 ctx->keys[src], ctx->vals[src], ko, vo, n, kRadixBits * p,
-                ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags);
+                ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags, ctx->sort_gate);
         NL_CUDA_TRY(cudaGetLastError());
         src = 1 - src;
     }

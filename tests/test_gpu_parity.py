@@ -71,6 +71,35 @@ def test_sort_ragged_sizes(ctx, oracle, n):
     np.testing.assert_array_equal(perm, o_perm)
 
 
+# The sort finishes short runs of equal top-24-bit key prefixes in place and
+# falls back to all eight digit passes when a run is longer than 64 keys:
+# identical points give runs of exactly 64 and 65, a dense cluster gives runs
+# of thousands, and an all-equal input is one run of n.
+@pytest.mark.parametrize("case", ["run64", "run65", "cluster", "all_equal"])
+def test_sort_long_prefix_runs(ctx, oracle, case):
+    rng = np.random.default_rng(7)
+    box = np.array([40.0, 40.0, 40.0], np.float32)
+    n = 20000
+    pos = np.zeros((n, 4), np.float32)
+    pos[:, :3] = rng.uniform(0.0, 1.0, (n, 3)) * box
+    if case == "run64":
+        pos[100:164, :3] = pos[5000, :3]
+        pos[5000, :3] = pos[3000, :3]
+    elif case == "run65":
+        pos[100:165, :3] = pos[5000, :3]
+        pos[5000, :3] = pos[3000, :3]
+    elif case == "cluster":
+        c = rng.uniform(0.0, 1.0, 3).astype(np.float32) * box
+        pos[: n // 4, :3] = c + rng.uniform(0.0, 0.02, (n // 4, 3)).astype(np.float32)
+    else:
+        pos[:, :3] = box * np.float32(0.3)
+    perm, ps, ks = gpu_sort(ctx, pos, box)
+    o_perm, o_ks = oracle.sort(pos, box)
+    np.testing.assert_array_equal(ks, o_ks)
+    np.testing.assert_array_equal(perm, o_perm)
+    np.testing.assert_array_equal(ps[:, :3], pos[o_perm, :3])
+
+
 def test_sort_full_size_salt_solution(ctx, oracle):
     w = gu.workload("saltwater10m")
     perm, ps, ks = gpu_sort(ctx, w.pos, w.box)
