@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "oracle_build": (ctypes.c_int, [i64, vp, vp, f32, f32, i32, vp, vp]),
             "oracle_skin_check": (f32, [i64, vp, vp, vp, f32, vp]),
             "oracle_close_pairs": (ctypes.c_int, [i64, vp, vp, f32, f32, f32, vp, vp]),
+            "oracle_edge_features": (None, [i64, vp, vp, ctypes.c_int32, vp, vp, vp]),
             "oracle_displacement": (f32, [u64, i64, i64, ctypes.c_int, f32]),
             "oracle_displace": (None, [i64, vp, u64, i64, f32]),
             "oracle_md_decisions": (i64, [i64, vp, vp, vp, f32, u64, f32, i64, vp]),
@@ -214,6 +215,21 @@ def close_pairs(pos, box, cutoff: float, skin: float, close_d2: float):
     if rc < 0:
         raise MemoryError("oracle_close_pairs failed")
     return float(mn[0]), int(nc[0])
+
+
+def edge_features(pos, box, nbr, counts) -> np.ndarray:
+    """Per-slot (dx, dy, dz, r) of padded rows: n x K x 4 float32, the
+    minimum-image displacement from atom i to nbr[i][s] and its length for
+    s < min(counts[i], K), zeros elsewhere."""
+    p = _pos4(pos)
+    bx = _box(box)
+    nb = np.ascontiguousarray(nbr, dtype=np.int32)
+    ct = np.ascontiguousarray(counts, dtype=np.int32)
+    n, K = nb.shape
+    assert p.shape[0] == n and ct.shape == (n,)
+    out = np.zeros((n, K, 4), np.float32)
+    lib().oracle_edge_features(n, _p(p), _p(bx), K, _p(nb), _p(ct), _p(out))
+    return out
 
 
 def skin_check(pos, ref, box, skin: float):

@@ -438,6 +438,46 @@ fail:
     return -1;
 }
 
+/* --------------------------------------------------------- edge features */
+
+/* Per-slot edge features of padded rows (reading of the pages' padded,
+ * dense neighbor tensors that the message-passing layers consume; Tessera,
+ * abstract, and the page on batching and kernel fusion): for row i and slot
+ * s < min(counts[i], K), j = nbr[i][s] and
+ *     (dx, dy, dz) = minimum image of w_j - w_i, per axis as in oracle_r2,
+ *     r = sqrtf((dx*dx + dy*dy) + dz*dz)   (IEEE square root, one rounding),
+ * written as out[(i*K + s)*4 + 0..3]; every other slot is (0, 0, 0, 0).
+ * An index outside [0, n) also gives zeros.  The rows may come from any
+ * builder: the features depend only on (i, j). */
+void oracle_edge_features(int64_t n, const float *pos4, const float box[3], int32_t K,
+                          const int32_t *nbr, const int32_t *counts, float *out)
+{
+    int64_t i, s;
+    for (i = 0; i < n; i++) {
+        float wi[3], wj[3];
+        int32_t c = counts[i] < K ? counts[i] : K;
+        int a;
+        for (a = 0; a < 3; a++) wi[a] = oracle_wrap(pos4[4 * i + a], box[a]);
+        for (s = 0; s < K; s++) {
+            float *o = out + 4 * (i * (int64_t)K + s);
+            int64_t j = s < c ? nbr[i * (int64_t)K + s] : -1;
+            o[0] = o[1] = o[2] = o[3] = 0.0f;
+            if (j < 0 || j >= n) continue;
+            for (a = 0; a < 3; a++) wj[a] = oracle_wrap(pos4[4 * j + a], box[a]);
+            {
+                float dx = oracle_min_image(wj[0] - wi[0], box[0]);
+                float dy = oracle_min_image(wj[1] - wi[1], box[1]);
+                float dz = oracle_min_image(wj[2] - wi[2], box[2]);
+                float r2 = oracle_r2(wi, wj, box);
+                o[0] = dx;
+                o[1] = dy;
+                o[2] = dz;
+                o[3] = sqrtf(r2);
+            }
+        }
+    }
+}
+
 /* ----------------------------------------------------------- skin check */
 
 /* Largest squared minimum-image displacement since the reference positions,
