@@ -292,6 +292,37 @@ def close_pair_timing(nl, torch, h, ps, w, K, close_d2: float = 1.0, reps: int =
     return res
 
 
+def edge_feature_timing(nl, torch, h, ps, w, K, reps: int = 5) -> dict:
+    """nl_edge_features on the rows of one nl_build: device time per call and
+    its HBM roofline.  Algorithmic bytes: counts and positions of every row
+    (4 + 16 per atom), the index of every valid slot (4 per pair), and the
+    K float4 features of every row (16 K per atom); the gathered neighbor
+    positions are counted once, with the rows' own."""
+    n = ps.shape[0]
+    stream = torch.cuda.current_stream()
+    nbr = torch.empty(n, K, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(n, dtype=torch.int32, device="cuda")
+    nl.nl_build(h, ps, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+    out = torch.empty(n, K, 4, dtype=torch.float32, device="cuda")
+    nl.nl_edge_features(h, ps, w.box, nbr, cnt, out, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        nl.nl_edge_features(h, ps, w.box, nbr, cnt, out, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    slots = int(cnt.clamp(max=K).to(torch.int64).sum().item())
+    alg = n * (4 + 16 + 16 * K) + 4 * slots
+    peak = measured_peaks()
+    gbs = alg / (ms * 1e-3) / 1e9
+    del out
+    return {"ms": ms, "bytes": alg, "achieved_gbs": gbs, "peak_gbs": peak["hbm_gbs"],
+            "peak_source": peak["source"], "frac": gbs / peak["hbm_gbs"],
+            "layout": f"float32 [{n}, {K}, 4] (dx, dy, dz, r), zero padding"}
+
+
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -482,6 +513,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             line["interval"] = interval_timing(nl, torch, h, ps, w, K, w.steps or 200)
             line["curves"] = curve_comparison(nl, torch, h, pos, w, K)
             line["close_pairs"] = close_pair_timing(nl, torch, h, ps, w, K)
+            line["edge_features"] = edge_feature_timing(nl, torch, h, ps, w, K)
         if world == 1 and not args.no_cpu_baseline:
             cb = oracle_sample(1)
             line["cpu_baseline"] = {"value": cb["value"], "unit": "atoms/s", "cores": cb["cores"],

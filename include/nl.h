@@ -120,6 +120,27 @@ nl_status nl_build_close(nl_ctx *ctx, int64_t n, const float *pos, const float *
                          int32_t *nbr_out, int32_t *counts_out, float close_d2,
                          float *min_d2_out, int64_t *n_close_out, void *stream);
 
+/* Edge features of padded rows (Tessera abstract: the model consumes the
+ * neighbor topology as fixed-shape tensors; the page on batching and kernel
+ * fusion: padded, dense per-atom neighborhoods).  For row i and slot
+ * s < min(counts[i], capacity), with j = nbr[i][s]:
+ *     edges_out[i][s] = (dx, dy, dz, r),
+ * (dx, dy, dz) the minimum-image displacement from atom i to atom j (the
+ * same fp32 values as in nl_build's predicate: wrapped coordinates, per axis
+ * d - L*rintf(d/L) of d = w_j - w_i) and r = sqrt((dx*dx + dy*dy) + dz*dz),
+ * correctly rounded.  All other slots, and slots whose index lies outside
+ * [0, n), are (0, 0, 0, 0).
+ * Inputs (device): pos as for nl_build (n x 4 float, 16-byte aligned, the
+ * positions the rows were built from or any others), nbr n x capacity int32
+ * and counts int32[n] as nl_build writes them.
+ * Output (device): edges_out, n x capacity x 4 float32 row-major, 16-byte
+ * aligned, caller-owned.  Needs no scratch and does not touch the context's
+ * build state.  NULL pointers (n > 0), misalignment, n < 0 or n > 2^30,
+ * capacity < 1 or a bad box are NL_ERR_ARG. */
+nl_status nl_edge_features(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                           const int32_t *nbr, const int32_t *counts, int32_t capacity,
+                           float *edges_out, void *stream);
+
 /* Skin check (Tessera abstract: a conservative neighbor skin preserves the
  * topology across updates).  m = max over atoms of the squared minimum-image
  * displacement between `pos` and the positions of the last nl_build (raw,

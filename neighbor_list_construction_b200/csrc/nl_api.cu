@@ -503,6 +503,22 @@ nl_status nl_skin_check(nl_ctx *ctx, int64_t n, const float *pos, const float *b
     return NL_OK;
 }
 
+nl_status nl_edge_features(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                           const int32_t *nbr, const int32_t *counts, int32_t capacity,
+                           float *edges_out, void *stream)
+{
+    if (!ctx || n < 0 || n > ((int64_t)1 << 30) || capacity < 1 || check_box(box) != NL_OK)
+        return NL_ERR_ARG;
+    if (n > 0 && (!pos || !nbr || !counts || !edges_out || !aligned16(pos) ||
+                  !aligned16(edges_out)))
+        return NL_ERR_ARG;
+    if (launch_edge_features(ctx, n, reinterpret_cast<const float4 *>(pos), box[0], box[1], box[2],
+                             nbr, counts, capacity, reinterpret_cast<float4 *>(edges_out),
+                             S(stream)) != cudaSuccess)
+        return NL_ERR_CUDA;
+    return NL_OK;
+}
+
 nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, float *pos,
                     const float *box, float cutoff, float skin, int32_t capacity, int32_t *nbr,
                     int32_t *counts, int32_t *decisions_out, void *stream)
@@ -637,7 +653,7 @@ const char *nl_profile_phase_name(int32_t phase)
     static const char *names[PH_COUNT] = {"keys",        "key_scan",   "radix_sort", "gather",
                                           "bin_count",   "cell_scan",  "bin_scatter",
                                           "cell_sort",   "pair_search", "pair_search_per_atom",
-                                          "skin_check"};
+                                          "skin_check",  "edge_features"};
     if (phase < 0 || phase >= PH_COUNT) return "";
     return names[phase];
 }

@@ -54,6 +54,7 @@ enum Phase {
     PH_PAIRS,
     PH_PAIRS_FALLBACK,
     PH_SKIN,
+    PH_EDGES,
     PH_COUNT
 };
 
@@ -188,6 +189,11 @@ struct CloseOut {
 cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capacity,
                          int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast,
                          const CloseOut *close);
+
+// Edge features (dx, dy, dz, r) of padded rows into out[n][K].
+cudaError_t launch_edge_features(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
+                                 float Lz, const int32_t *nbr, const int32_t *counts, int32_t K,
+                                 float4 *out, cudaStream_t s);
 
 // Skin check.  decisions/step may be NULL; cond_handle 0 = none.
 cudaError_t launch_skin(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,

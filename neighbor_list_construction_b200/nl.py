@@ -35,6 +35,7 @@ _SIGS = {
     "nl_build_close": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _f32, _vp, _vp,
                               _vp]),
     "nl_skin_check": (_i32, [_vp, _i64, _vp, _vp, _f32, _vp, _vp, _vp]),
+    "nl_edge_features": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp, _vp]),
     "nl_replay": (_i32, [_vp, _vp, _i32, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp, _vp]),
     "nl_step_counter": (_vp, [_vp]),
     "nl_sync_status": (_i32, [_vp, _vp]),
@@ -158,6 +159,20 @@ def nl_skin_check(ctx, pos, box, skin, rebuild_out, max_d2_out=None, stream=None
                   "nl_skin_check")
 
 
+def nl_edge_features(ctx, pos, box, nbr, counts, edges_out, stream=None) -> int:
+    _pos(pos)
+    n = pos.shape[0]
+    if nbr.dtype != torch.int32 or nbr.dim() != 2 or nbr.shape[0] != n:
+        raise ValueError("nbr must be an int32 [n, K] CUDA tensor")
+    if counts.dtype != torch.int32 or tuple(counts.shape) != (n,):
+        raise ValueError("counts must be an int32 [n] CUDA tensor")
+    if edges_out.dtype != torch.float32 or tuple(edges_out.shape) != (n, nbr.shape[1], 4):
+        raise ValueError("edges_out must be a float32 [n, K, 4] CUDA tensor")
+    return _check(_lib.nl_edge_features(ctx, pos.shape[0], _ptr(pos), _box(box), _ptr(nbr),
+                                        _ptr(counts), int(nbr.shape[1]), _ptr(edges_out),
+                                        _stream(stream)), "nl_edge_features")
+
+
 def nl_replay(ctx, step_graph, n_steps, pos, box, cutoff, skin, capacity, nbr, counts,
               decisions_out, stream=None) -> int:
     _pos(pos)
@@ -263,6 +278,13 @@ class Context:
         nl_build_close(self.handle, pos, box, cutoff, skin, capacity, nbr, counts, close_d2, mn,
                        nc, stream)
         return nbr, counts, mn, nc
+
+    def edge_features(self, pos, box, nbr, counts, stream=None):
+        """Per-slot (dx, dy, dz, r) of the rows: float32 [n, K, 4]."""
+        n, K = nbr.shape
+        out = torch.empty(n, K, 4, dtype=torch.float32, device=pos.device)
+        nl_edge_features(self.handle, pos, box, nbr, counts, out, stream)
+        return out
 
     def skin_check(self, pos, box, skin, stream=None):
         rb = torch.zeros(1, dtype=torch.int32, device=pos.device)

@@ -12,6 +12,17 @@ def workload(name: str, seed: int | None = None):
     return workloads.make(name, seed=seed)
 
 
+@functools.lru_cache(maxsize=None)
+def oracle_sorted(name: str) -> np.ndarray:
+    """The workload's positions in the oracle's curve order (Hilbert), so that
+    tests run the GPU build in the benchmark's order on inputs that owe
+    nothing to the GPU path."""
+    import oracle
+    w = workload(name)
+    perm, _ = oracle.sort(w.pos, w.box)
+    return np.ascontiguousarray(w.pos[perm])
+
+
 def canonical(nbr: np.ndarray) -> np.ndarray:
     big = np.iinfo(np.int32).max
     out = np.sort(np.where(nbr < 0, big, nbr), axis=1)

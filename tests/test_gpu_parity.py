@@ -120,7 +120,7 @@ def test_build_uniform4k_equals_bruteforce(ctx, oracle):
 @pytest.mark.parametrize("name", ["lattice60k", "saltwater_n20", "uniform4k"])
 def test_build_matches_oracle_on_sorted_positions(ctx, oracle, name):
     w = gu.workload(name)
-    _, ps, _ = gpu_sort(ctx, w.pos, w.box)
+    ps = gu.oracle_sorted(name)
     nbr, cnt, st = gpu_build(ctx, ps, w.box, w.cutoff, w.skin, w.capacity)
     o_nbr, o_cnt, o_ov = oracle.build(ps, w.box, w.cutoff, w.skin, w.capacity)
     assert st == (1 if o_ov else 0)
@@ -255,7 +255,7 @@ def test_build_full_size_sampled(ctx, oracle, name):
     sampled rows against the oracle, symmetry of the sampled rows, and the
     global pair count parity."""
     w = gu.workload(name)
-    perm, ps, _ = gpu_sort(ctx, w.pos, w.box)
+    ps = gu.oracle_sorted(name)
     nbr_t, cnt_t = ctx.build(dev(ps), w.box, w.cutoff, w.skin, w.capacity)
     st = ctx.sync_status()
     assert st in (0, 1)
@@ -326,7 +326,7 @@ def test_displacement_stand_in_matches_oracle(ctx, nl, oracle):
 # ------------------------------------------------------------------ replay
 def _replay(ctx, nl, oracle, name, steps, seed=2024, check_lists=True):
     w = gu.workload(name)
-    _, ps, _ = gpu_sort(ctx, w.pos, w.box)
+    ps = gu.oracle_sorted(name)
     p = dev(ps)
     nbr, cnt = ctx.build(p, w.box, w.cutoff, w.skin, w.capacity)
     g = nl.nls_step_graph(p, seed, nl.nl_step_counter(ctx.handle), w.sigma_step)
