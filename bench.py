@@ -212,6 +212,28 @@ def interval_timing(nl, torch, h, ps_src, w, K, steps: int, seed: int = 2024) ->
         out["rebuilds"] = int(dec.sum().item())
     finally:
         nl.nls_graph_destroy(g)
+    # graph, re-sorting at each rebuild (ids follow the atoms)
+    p = ps_src.clone()
+    ids = torch.arange(n, dtype=torch.int32, device="cuda")
+    nl.nl_build(h, p, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+    g = nl.nls_step_graph_ids(p, ids, seed, nl.nl_step_counter(h), w.sigma_step)
+    try:
+        nl.nl_replay_resort(h, g, steps, p, ids, None, w.box, w.cutoff, w.skin, K, nbr, cnt, dec,
+                            stream)  # warm
+        p.copy_(ps_src)
+        ids.copy_(torch.arange(n, dtype=torch.int32, device="cuda"))
+        nl.nl_build(h, p, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        nl.nl_replay_resort(h, g, steps, p, ids, None, w.box, w.cutoff, w.skin, K, nbr, cnt, dec,
+                            stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out["graph_resort_ms_per_step"] = e0.elapsed_time(e1) / steps
+        out["resort_rebuilds"] = int(dec.sum().item())
+    finally:
+        nl.nls_graph_destroy(g)
     # eager
     p.copy_(ps_src)
     nl.nl_build(h, p, w.box, w.cutoff, w.skin, K, nbr, cnt, stream)

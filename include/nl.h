@@ -166,6 +166,22 @@ nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps,
                     int32_t capacity, int32_t *nbr, int32_t *counts,
                     int32_t *decisions_out, void *stream);
 
+/* nl_replay with a re-sort in every rebuild (Tessera abstract: atoms are
+ * kept in space-filling-curve order).  Each rebuild first permutes the atoms
+ * in place into the order nl_sort_hilbert gives for their current positions
+ * (stable: equal keys keep their slot order), then runs nl_build on the
+ * permuted `pos`.  The same permutation is applied to ids (device int32[n],
+ * e.g. initialised to 0..n-1 so that ids[k] names the atom now in slot k)
+ * and to aux (device n x 4 float, 16-byte aligned, per-atom state such as
+ * velocities) when they are not NULL.  nbr, counts and the skin-check
+ * reference then refer to the new slots.  Other arguments, results and
+ * errors as nl_replay; the step graph sees the permuted arrays at the same
+ * addresses. */
+nl_status nl_replay_resort(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n,
+                           float *pos, int32_t *ids, float *aux, const float *box,
+                           float cutoff, float skin, int32_t capacity, int32_t *nbr,
+                           int32_t *counts, int32_t *decisions_out, void *stream);
+
 /* Device pointer to the 0-based iteration index that nl_replay maintains
  * while its graph runs (int32[1], owned by the context). */
 const int32_t *nl_step_counter(nl_ctx *ctx);

@@ -10,7 +10,8 @@
  *   delta = fl(g * A),  A = fl(sigma * sqrt(3) / 65536)   (std. dev. sigma)
  *   x <- fl(x + delta)
  * (SplitMix64: Steele, Lea & Flood, OOPSLA 2014.)  `atom` is the index in
- * the array that is moved; step numbers start at 1.
+ * the array that is moved, or ids[index] when an id array is given (it
+ * follows the atoms through re-sorts); step numbers start at 1.
  */
 #ifndef NL_STANDIN_H
 #define NL_STANDIN_H
@@ -33,6 +34,11 @@ nl_status nls_displace(int64_t n, float *pos, uint64_t seed, int64_t step,
  * caller releases it with nls_graph_destroy. */
 nl_status nls_step_graph(void **graph_out, int64_t n, float *pos, uint64_t seed,
                          const int32_t *step_dev, float sigma);
+/* The same with atom = ids[slot] (device int32[n], read at each replay, so
+ * it may be the id array that nl_replay_resort permutes); ids NULL is
+ * nls_step_graph. */
+nl_status nls_step_graph_ids(void **graph_out, int64_t n, float *pos, const int32_t *ids,
+                             uint64_t seed, const int32_t *step_dev, float sigma);
 void nls_graph_destroy(void *graph);
 
 #ifdef __cplusplus

@@ -228,13 +228,20 @@ cudaError_t add_child_in_capture(cudaStream_t cs, cudaGraph_t child)
     return cudaStreamUpdateCaptureDependencies(cs, &node, 1, cudaStreamSetCaptureDependencies);
 }
 
+// What a rebuild re-sorts, when it does (nl_replay_resort).
+struct ResortArgs {
+    int32_t *ids;
+    float *aux;
+    float Sx, Sy, Sz;
+};
+
 // Builds the interval graph:
 //   init(step = 0) -> WHILE(loop) { [step graph] -> skin check (sets cond) ->
-//                                   IF(cond) { nl_build } -> advance(step++) }
+//                                   IF(cond) { [re-sort] -> nl_build } -> advance(step++) }
 cudaError_t make_replay_graph(nl_ctx *ctx, cudaGraph_t step_graph, int32_t n_steps, int64_t n,
                               float *pos, const CellGrid &g, float h2, int32_t capacity,
                               int32_t *nbr, int32_t *counts, int32_t *decisions,
-                              cudaGraph_t *out)
+                              const ResortArgs *rs, cudaGraph_t *out)
 {
     cudaStream_t cs;
     NL_CUDA_TRY(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
@@ -300,7 +307,12 @@ cudaError_t make_replay_graph(nl_ctx *ctx, cudaGraph_t step_graph, int32_t n_ste
         e = cudaStreamBeginCaptureToGraph(cs, ifbody, nullptr, nullptr, 0,
                                           cudaStreamCaptureModeRelaxed);
         if (e != cudaSuccess) break;
-        if (build_enqueue(ctx, n, pos, g, capacity, nbr, counts, cs, &fast) != NL_OK)
+        if (rs)
+            e = launch_resort(ctx, n, reinterpret_cast<float4 *>(pos), rs->ids,
+                              reinterpret_cast<float4 *>(rs->aux), g.Lx, g.Ly, g.Lz, rs->Sx, rs->Sy,
+                              rs->Sz, cs);
+        if (e == cudaSuccess &&
+            build_enqueue(ctx, n, pos, g, capacity, nbr, counts, cs, &fast) != NL_OK)
             e = cudaErrorUnknown;
         cudaGraph_t tmp2;
         cudaError_t e2 = cudaStreamEndCapture(cs, &tmp2);
@@ -519,9 +531,14 @@ nl_status nl_edge_features(nl_ctx *ctx, int64_t n, const float *pos, const float
     return NL_OK;
 }
 
-nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, float *pos,
-                    const float *box, float cutoff, float skin, int32_t capacity, int32_t *nbr,
-                    int32_t *counts, int32_t *decisions_out, void *stream)
+}  // extern "C"
+
+namespace {
+
+nl_status replay_impl(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, float *pos,
+                      const float *box, float cutoff, float skin, int32_t capacity, int32_t *nbr,
+                      int32_t *counts, int32_t *decisions_out, void *stream, bool resort,
+                      int32_t *ids, float *aux)
 {
     if (n_steps < 0 || (n_steps > 0 && !decisions_out)) return NL_ERR_ARG;
     CellGrid g;
@@ -549,14 +566,28 @@ nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, f
     put(&nbr, sizeof(nbr));
     put(&counts, sizeof(counts));
     put(&decisions_out, sizeof(decisions_out));
+    const unsigned char rflag = resort ? 1 : 0;
+    put(&rflag, 1);
+    put(&ids, sizeof(ids));
+    put(&aux, sizeof(aux));
     if (!ctx->replay_exec || ctx->replay_key_len != kl || memcmp(ctx->replay_key, key, kl) != 0) {
         if (ctx->replay_exec) cudaGraphExecDestroy(ctx->replay_exec);
         if (ctx->replay_graph) cudaGraphDestroy(ctx->replay_graph);
         ctx->replay_exec = nullptr;
         ctx->replay_graph = nullptr;
         cudaGraph_t gr = nullptr;
+        ResortArgs ra{ids, aux, 0.0f, 0.0f, 0.0f};
+        if (resort) {
+            volatile float sx = 2097152.0f / box[0];
+            volatile float sy = 2097152.0f / box[1];
+            volatile float sz = 2097152.0f / box[2];
+            ra.Sx = sx;
+            ra.Sy = sy;
+            ra.Sz = sz;
+        }
         cudaError_t e = make_replay_graph(ctx, reinterpret_cast<cudaGraph_t>(step_graph), n_steps,
-                                          n, pos, g, h2, capacity, nbr, counts, decisions_out, &gr);
+                                          n, pos, g, h2, capacity, nbr, counts, decisions_out,
+                                          resort ? &ra : nullptr, &gr);
         if (e != cudaSuccess || !gr) {
             fprintf(stderr, "nl_replay: graph construction failed: %s\n", cudaGetErrorString(e));
             return NL_ERR_CUDA;
@@ -577,6 +608,28 @@ nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, f
     if (cudaGraphLaunch(ctx->replay_exec, S(stream)) != cudaSuccess) return NL_ERR_CUDA;
     ctx->last_grid = g;
     return NL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, float *pos,
+                    const float *box, float cutoff, float skin, int32_t capacity, int32_t *nbr,
+                    int32_t *counts, int32_t *decisions_out, void *stream)
+{
+    return replay_impl(ctx, step_graph, n_steps, n, pos, box, cutoff, skin, capacity, nbr, counts,
+                       decisions_out, stream, false, nullptr, nullptr);
+}
+
+nl_status nl_replay_resort(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, float *pos,
+                           int32_t *ids, float *aux, const float *box, float cutoff, float skin,
+                           int32_t capacity, int32_t *nbr, int32_t *counts,
+                           int32_t *decisions_out, void *stream)
+{
+    if (aux && !aligned16(aux)) return NL_ERR_ARG;
+    return replay_impl(ctx, step_graph, n_steps, n, pos, box, cutoff, skin, capacity, nbr, counts,
+                       decisions_out, stream, true, ids, aux);
 }
 
 const int32_t *nl_step_counter(nl_ctx *ctx) { return ctx ? ctx->step : nullptr; }

@@ -190,6 +190,13 @@ cudaError_t launch_pairs(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t capa
                          int32_t *nbr, int32_t *counts, cudaStream_t s, int *used_fast,
                          const CloseOut *close);
 
+// Re-sort in place along the Hilbert curve of `pos` (S = fl(2^21 / L) per
+// axis): pos, and ids / aux when not NULL, are permuted by the stable
+// (key, slot) order.  Uses the sort scratch and the build's per-atom scratch.
+cudaError_t launch_resort(nl_ctx *ctx, int64_t n, float4 *pos, int32_t *ids, float4 *aux,
+                          float Lx, float Ly, float Lz, float Sx, float Sy, float Sz,
+                          cudaStream_t s);
+
 // Edge features (dx, dy, dz, r) of padded rows into out[n][K].
 cudaError_t launch_edge_features(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
                                  float Lz, const int32_t *nbr, const int32_t *counts, int32_t K,

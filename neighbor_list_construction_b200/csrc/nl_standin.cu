@@ -18,20 +18,24 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t x)
     return z ^ (z >> 31);
 }
 
-__global__ void k_displace(int64_t n, float *__restrict__ pos, uint64_t seed_mix, int64_t step,
-                           const int32_t *__restrict__ step_dev, float A)
+// The atom of slot k is ids[k] when ids is given (so that a re-sort does not
+// change which random stream moves which atom), else k.
+__global__ void k_displace(int64_t n, float *__restrict__ pos, const int32_t *__restrict__ ids,
+                           uint64_t seed_mix, int64_t step, const int32_t *__restrict__ step_dev,
+                           float A)
 {
     const int64_t t = step_dev ? (int64_t)(*step_dev) + 1 : step;
     const int64_t total = 3 * n;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
-        const int64_t atom = e / 3;
-        const int axis = (int)(e - atom * 3);
+        const int64_t slot = e / 3;
+        const int axis = (int)(e - slot * 3);
+        const int64_t atom = ids ? (int64_t)ids[slot] : slot;
         const uint64_t ctr = ((uint64_t)t << 42) | ((uint64_t)atom << 2) | (uint64_t)axis;
         const uint64_t u = splitmix64(seed_mix + ctr);
         const int32_t g = (int32_t)(u & 0xffffu) + (int32_t)((u >> 16) & 0xffffu) +
                           (int32_t)((u >> 32) & 0xffffu) + (int32_t)(u >> 48) - 131070;
-        float *x = pos + atom * 4 + axis;
+        float *x = pos + slot * 4 + axis;
         *x = __fadd_rn(*x, __fmul_rn((float)g, A));
     }
 }
@@ -63,20 +67,26 @@ nl_status nls_displace(int64_t n, float *pos, uint64_t seed, int64_t step,
     if (n == 0) return NL_OK;
     const float A = (float)((double)sigma * std::sqrt(3.0) / 65536.0);
     k_displace<<<blocks_for(n), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        n, pos, host_splitmix64(seed), step, step_dev, A);
+        n, pos, nullptr, host_splitmix64(seed), step, step_dev, A);
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
 }
 
 nl_status nls_step_graph(void **graph_out, int64_t n, float *pos, uint64_t seed,
                          const int32_t *step_dev, float sigma)
 {
+    return nls_step_graph_ids(graph_out, n, pos, nullptr, seed, step_dev, sigma);
+}
+
+nl_status nls_step_graph_ids(void **graph_out, int64_t n, float *pos, const int32_t *ids,
+                             uint64_t seed, const int32_t *step_dev, float sigma)
+{
     if (!graph_out || !step_dev || n <= 0 || !pos) return NL_ERR_ARG;
     *graph_out = nullptr;
     const float A = (float)((double)sigma * std::sqrt(3.0) / 65536.0);
     uint64_t mix = host_splitmix64(seed);
     int64_t step0 = 0;
-    void *args[] = {(void *)&n, (void *)&pos, (void *)&mix, (void *)&step0, (void *)&step_dev,
-                    (void *)&A};
+    void *args[] = {(void *)&n, (void *)&pos, (void *)&ids, (void *)&mix, (void *)&step0,
+                    (void *)&step_dev, (void *)&A};
     cudaGraph_t g = nullptr;
     if (cudaGraphCreate(&g, 0) != cudaSuccess) return NL_ERR_CUDA;
     cudaKernelNodeParams p = {};

@@ -37,6 +37,8 @@ _SIGS = {
     "nl_skin_check": (_i32, [_vp, _i64, _vp, _vp, _f32, _vp, _vp, _vp]),
     "nl_edge_features": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp, _vp]),
     "nl_replay": (_i32, [_vp, _vp, _i32, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp, _vp]),
+    "nl_replay_resort": (_i32, [_vp, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _f32, _f32, _i32, _vp,
+                                _vp, _vp, _vp]),
     "nl_step_counter": (_vp, [_vp]),
     "nl_sync_status": (_i32, [_vp, _vp]),
     "nl_status_string": (ctypes.c_char_p, [_i32]),
@@ -47,6 +49,7 @@ _SIGS = {
     "nl_sort_hilbert_noalloc": (_i32, [_i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nls_displace": (_i32, [_i64, _vp, _u64, _i64, _vp, _f32, _vp]),
     "nls_step_graph": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _u64, _vp, _f32]),
+    "nls_step_graph_ids": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _vp, _u64, _vp, _f32]),
     "nls_graph_destroy": (None, [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -181,6 +184,21 @@ def nl_replay(ctx, step_graph, n_steps, pos, box, cutoff, skin, capacity, nbr, c
                                  _ptr(counts), _ptr(decisions_out), _stream(stream)), "nl_replay")
 
 
+def nl_replay_resort(ctx, step_graph, n_steps, pos, ids, aux, box, cutoff, skin, capacity, nbr,
+                     counts, decisions_out, stream=None) -> int:
+    _pos(pos)
+    n = pos.shape[0]
+    if ids is not None and (ids.dtype != torch.int32 or tuple(ids.shape) != (n,)):
+        raise ValueError("ids must be an int32 [n] CUDA tensor")
+    if aux is not None and (aux.dtype != torch.float32 or tuple(aux.shape) != (n, 4)):
+        raise ValueError("aux must be a float32 [n, 4] CUDA tensor")
+    return _check(_lib.nl_replay_resort(ctx, step_graph, int(n_steps), n, _ptr(pos), _ptr(ids),
+                                        _ptr(aux), _box(box), float(cutoff), float(skin),
+                                        int(capacity), _ptr(nbr), _ptr(counts),
+                                        _ptr(decisions_out), _stream(stream)),
+                  "nl_replay_resort")
+
+
 def nl_step_counter(ctx) -> int:
     return _lib.nl_step_counter(ctx)
 
@@ -225,6 +243,15 @@ def nls_step_graph(pos, seed: int, step_dev: int, sigma: float) -> ctypes.c_void
     g = ctypes.c_void_p()
     _check(_lib.nls_step_graph(ctypes.byref(g), pos.shape[0], _ptr(pos), int(seed) & (2 ** 64 - 1),
                                ctypes.c_void_p(step_dev), float(sigma)), "nls_step_graph")
+    return g
+
+
+def nls_step_graph_ids(pos, ids, seed: int, step_dev: int, sigma: float) -> ctypes.c_void_p:
+    _pos(pos)
+    g = ctypes.c_void_p()
+    _check(_lib.nls_step_graph_ids(ctypes.byref(g), pos.shape[0], _ptr(pos), _ptr(ids),
+                                   int(seed) & (2 ** 64 - 1), ctypes.c_void_p(step_dev),
+                                   float(sigma)), "nls_step_graph_ids")
     return g
 
 

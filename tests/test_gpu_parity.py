@@ -361,6 +361,79 @@ def test_replay_salt_solution_200_steps(ctx, nl, oracle):
     assert 3 <= dec.sum() <= 40
 
 
+# ---------------------------------------------------------- replay, re-sorted
+def _replay_resort(ctx, nl, oracle, name, steps, start, seed=2024):
+    """nl_replay_resort against the oracle's plain interval: with the stand-in
+    keyed by atom id, re-sorting only permutes the trajectory, so decisions
+    are equal and every array is the oracle's, permuted by the final ids."""
+    w = gu.workload(name)
+    p0 = gu.oracle_sorted(name) if start == "curve" else w.pos
+    n = w.n
+    p = dev(p0)
+    ids = torch.arange(n, dtype=torch.int32, device="cuda")
+    aux0 = np.random.default_rng(1).random((n, 4)).astype(np.float32)
+    aux = dev(aux0)
+    nbr, cnt = ctx.build(p, w.box, w.cutoff, w.skin, w.capacity)
+    g = nl.nls_step_graph_ids(p, ids, seed, nl.nl_step_counter(ctx.handle), w.sigma_step)
+    dec = torch.full((steps,), -1, dtype=torch.int32, device="cuda")
+    try:
+        nl.nl_replay_resort(ctx.handle, g, steps, p, ids, aux, w.box, w.cutoff, w.skin,
+                            w.capacity, nbr, cnt, dec)
+        st = ctx.sync_status()
+    finally:
+        nl.nls_graph_destroy(g)
+    o_dec, o_final, o_ref = oracle.md_decisions(p0, w.box, w.skin, seed, w.sigma_step, steps)
+    np.testing.assert_array_equal(dec.cpu().numpy(), o_dec)
+    idh = ids.cpu().numpy()
+    np.testing.assert_array_equal(np.sort(idh), np.arange(n))
+    np.testing.assert_array_equal(p.cpu().numpy(), o_final[idh])
+    np.testing.assert_array_equal(aux.cpu().numpy(), aux0[idh])
+    if o_dec.any():
+        # the last rebuild put the atoms in curve order of their positions then
+        k = oracle.keys(o_ref[idh], w.box)
+        assert np.all(k[1:] >= k[:-1])
+    else:
+        np.testing.assert_array_equal(idh, np.arange(n))
+    o_nbr, o_cnt, o_ov = oracle.build(o_ref[idh], w.box, w.cutoff, w.skin, w.capacity)
+    assert st == (1 if o_ov else 0)
+    gu.assert_rows_match(nbr.cpu().numpy(), cnt.cpu().numpy(), o_nbr, o_cnt)
+    return o_dec, idh
+
+
+@pytest.mark.parametrize("name,steps,start", [("lattice60k", 50, "input"),
+                                              ("saltwater_n20", 120, "input"),
+                                              ("saltwater_n20", 120, "curve"),
+                                              ("uniform4k", 1, "input")])
+def test_replay_resort(ctx, nl, oracle, name, steps, start):
+    dec, ids = _replay_resort(ctx, nl, oracle, name, steps, start)
+    if steps > 1:
+        assert dec.sum() >= 1
+    if start == "input" and dec.any():
+        assert not np.array_equal(ids, np.arange(ids.size))
+
+
+def test_replay_resort_without_ids_or_aux(ctx, nl, oracle):
+    """ids and aux are optional; pos alone is permuted.  The stand-in is keyed
+    by slot here, so after the first re-sort the trajectory is no longer the
+    oracle's: decisions are compared up to and including the first rebuild."""
+    w = gu.workload("lattice60k")
+    p = dev(w.pos)
+    nbr, cnt = ctx.build(p, w.box, w.cutoff, w.skin, w.capacity)
+    g = nl.nls_step_graph(p, 11, nl.nl_step_counter(ctx.handle), w.sigma_step)
+    dec = torch.full((40,), -1, dtype=torch.int32, device="cuda")
+    try:
+        nl.nl_replay_resort(ctx.handle, g, 40, p, None, None, w.box, w.cutoff, w.skin,
+                            w.capacity, nbr, cnt, dec)
+        assert ctx.sync_status() == 0
+    finally:
+        nl.nls_graph_destroy(g)
+    d = dec.cpu().numpy()
+    o_dec, _, _ = oracle.md_decisions(w.pos, w.box, w.skin, 11, w.sigma_step, 40)
+    first = int(np.argmax(o_dec)) if o_dec.any() else 40
+    np.testing.assert_array_equal(d[: first + 1], o_dec[: first + 1])
+    assert set(np.unique(d)) <= {0, 1}
+
+
 # ------------------------------------------------------------------ errors
 def test_argument_errors(ctx, nl):
     p = dev(np.zeros((10, 4), np.float32))
