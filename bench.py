@@ -34,8 +34,8 @@ NOMINAL_HBM_GBS = 8000.0
 # belongs to the kernel source it was taken on: with any other source of the
 # pair kernel the bench reports null.
 PAIR_TRAFFIC = {"workload": "saltwater10m",
-                "sha256": "b9fdd6b53191ffd7e0d1ea8c434e93775ff78a93a5be1dabb0c25bb369ffb8e6",
-                "bytes": 796743424 + 10741738240}
+                "sha256": "510b0f106c3f422db82414975979ba45918643b569843b55655cc377f6f8a1b0",
+                "bytes": 793912832 + 10741550592}
 
 
 def pair_traffic(workload: str):
