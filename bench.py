@@ -489,7 +489,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                         "pair_search_per_atom")) / args.steps
         sort_ms = sum(phases.get(p, (0.0, 0))[0] for p in
                       ("keys", "key_scan", "radix_sort", "gather")) / args.steps
-        kernels_per_phase = {"radix_sort": 13, "cell_sort": 2}
+        kernels_per_phase = {"radix_sort": 14, "cell_sort": 2}
         launches_per_step = sum(v[1] * kernels_per_phase.get(k, 1)
                                 for k, v in phases.items()) / args.steps
         line = {

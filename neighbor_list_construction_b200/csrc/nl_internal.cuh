@@ -148,14 +148,16 @@ struct ProfScope {
 };
 
 // ------------------------------------------------------------- launchers
-// Curve keys of all atoms into ctx->keys[0]/vals[0] and the 8 digit
-// histograms into ctx->hist (which must be zero); curve 0 Hilbert, 1 Morton.
-// With a gate: only when *gate != 0, keys only (no histograms).
+// Curve keys of all atoms into ctx->keys[0]/vals[0] and the histograms of
+// the top kTopPasses digits into ctx->hist (which must be zero); curve 0
+// Hilbert, 1 Morton.  With a gate: only when *gate != 0, and the histograms
+// of the other digits.
 cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
                         float Lz, float Sx, float Sy, float Sz, int curve, cudaStream_t s,
                         const uint32_t *gate = nullptr);
-// Exclusive scan of the 8 histograms in place.
-cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s);
+// Exclusive scan of the 8 histograms in place; with a gate, only when
+// *gate != 0 and only the digits below the top kTopPasses.
+cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s, const uint32_t *gate = nullptr);
 // What the gated full sort needs to recompute the keys.
 struct SortRecompute {
     const float4 *pos;

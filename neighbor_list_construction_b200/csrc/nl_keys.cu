@@ -86,10 +86,14 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
                                               uint32_t *__restrict__ hist,
                                               const uint32_t *gate)
 {
-    // gated recompute (the full sort's keys): only when the gate is set, and
-    // without the histograms, which the first pass already made
+    // First pass: the histograms of the top kTopPasses digits, which the
+    // fast sort uses.  Gated recompute (the full sort's keys): only when the
+    // gate is set, with the histograms of the remaining low digits.
     const bool recompute = gate != nullptr;
     if (recompute && ld_volatile_u32(gate) == 0u) return;
+    constexpr int kLow = kKeyPasses - kTopPasses;
+    const int d0 = recompute ? 0 : kLow;
+    const int d1 = recompute ? kLow : kKeyPasses;
     __shared__ uint32_t sh[kKeyPasses * kRadixBins];
     for (int i = threadIdx.x; i < kKeyPasses * kRadixBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
@@ -102,22 +106,21 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
         const uint64_t k = CURVE == 0 ? hilbert_index(qx, qy, qz) : morton_index(qx, qy, qz);
         keys[i] = k;
         vals[i] = (uint32_t)i;
-        if (recompute) continue;
-#pragma unroll
-        for (int d = 0; d < kKeyPasses; ++d)
+        for (int d = d0; d < d1; ++d)
             atomicAdd(&sh[d * kRadixBins + (uint32_t)((k >> (kRadixBits * d)) & 0xffu)], 1u);
     }
     __syncthreads();
-    if (recompute) return;
-    for (int i = threadIdx.x; i < kKeyPasses * kRadixBins; i += blockDim.x) {
+    for (int i = d0 * kRadixBins + threadIdx.x; i < d1 * kRadixBins; i += blockDim.x) {
         const uint32_t v = sh[i];
         if (v) atomicAdd(&hist[i], v);
     }
 }
 
-// One block per digit position: exclusive scan of its 256 counts.
-__global__ void __launch_bounds__(256) k_hist_scan(uint32_t *hist)
+// One block per digit position: exclusive scan of its 256 counts.  With a
+// gate: only when the gate is set.
+__global__ void __launch_bounds__(256) k_hist_scan(uint32_t *hist, const uint32_t *gate)
 {
+    if (gate && ld_volatile_u32(gate) == 0u) return;
     __shared__ uint32_t warp_tot[8];
     uint32_t *h = hist + blockIdx.x * kRadixBins;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -154,7 +157,7 @@ cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
 {
     if (n <= 0) return cudaSuccess;
     int64_t blocks = (n + 255) / 256;
-    const int64_t cap = (int64_t)ctx->sm_count * 4;
+    const int64_t cap = (int64_t)ctx->sm_count * 8;
     if (blocks > cap) blocks = cap;
     if (curve == 0)
         k_keys<0><<<(unsigned)blocks, 256, 0, s>>>(pos, n, Lx, Ly, Lz, Sx, Sy, Sz, ctx->keys[0],
@@ -165,9 +168,11 @@ cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
     return cudaGetLastError();
 }
 
-cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s)
+cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s, const uint32_t *gate)
 {
-    k_hist_scan<<<kKeyPasses, kRadixBins, 0, s>>>(ctx->hist);
+    // ungated: all digits (the low ones are still zero); gated: the low ones
+    const int digits = gate ? kKeyPasses - kTopPasses : kKeyPasses;
+    k_hist_scan<<<digits, kRadixBins, 0, s>>>(ctx->hist, gate);
     return cudaGetLastError();
 }
 

@@ -5,8 +5,8 @@
 // onesweep passes; the array is then ordered by its 24-bit key prefix, with
 // equal prefixes in index order.  A prefix is one cell of a 256^3 grid over
 // the box, so a run of equal prefixes holds about n / 2^24 keys (a handful
-// at most for atoms at liquid density); each run is finished by one thread
-// with an insertion sort on (key, index).  A run longer than kRunMax keys
+// at most for atoms at liquid density); each element of a run is placed by
+// its rank in (key, index) within the run.  A run longer than kRunMax keys
 // (strongly clustered input) sets a gate word, and a gated copy of the full
 // eight-pass sort, already enqueued behind, then recomputes the keys and
 // redoes the whole order; when the gate is clear those launches return at
@@ -17,7 +17,8 @@
 // running), ranks its keys stably with warp match/popc, publishes its per-
 // digit counts, and finds the counts of all earlier tiles by decoupled
 // look-back over per-(tile, digit) status words.  The global digit starts
-// come from histograms computed once, in the key kernel.  Waits on a status
+// come from histograms made by the key kernel (those of the low digits only
+// by its gated recompute).  Waits on a status
 // word are bounded: past kSpinLimit polls the kernel records kFlagTimeout
 // and carries on, so a stuck predecessor cannot hang the device.
 #include "nl_internal.cuh"
@@ -179,43 +180,62 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
 }
 
 // Finishes the runs of equal 24-bit key prefix (the output of the passes
-// over bits 40..63): the thread at a run's first position sorts the run by
-// (key, index) and writes it to the final arrays.  A run of more than
-// kRunMax keys sets *gate instead (the full sort then redoes everything).
-__global__ void __launch_bounds__(256)
+// over bits 40..63).  Each thread takes one element p: it finds p's run
+// [h, e) and places p at h + (number of run members smaller in (key,
+// index)) -- a rank, so every element moves in parallel and no thread
+// sorts a whole run.  A CTA stages its tile of kRunTile keys plus kRunMax + 1
+// on either side in shared memory; a run that reaches the end of that window
+// is longer than kRunMax and sets *gate instead (the full sort then redoes
+// everything).
+constexpr int kRunThreads = 256;
+constexpr int kRunItems = 8;
+constexpr int kRunTile = kRunThreads * kRunItems;
+constexpr int kRunHalo = kRunMax + 1;
+
+__global__ void __launch_bounds__(kRunThreads)
 k_run_sort(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ vals, int64_t n,
            uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, uint32_t *gate)
 {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-        const uint64_t pre = keys[i] >> kPrefixShift;
-        if (i > 0 && (keys[i - 1] >> kPrefixShift) == pre) continue;   // not a run head
-        int64_t e = i + 1;
-        while (e < n && e - i <= kRunMax && (keys[e] >> kPrefixShift) == pre) ++e;
-        if (e - i > kRunMax) {
-            atomicOr(gate, 1u);
+    __shared__ uint64_t s_k[kRunTile + 2 * kRunHalo];
+    __shared__ uint32_t s_v[kRunTile + 2 * kRunHalo];
+    const int64_t t0 = (int64_t)blockIdx.x * kRunTile;
+    const int64_t lo = t0 - kRunHalo > 0 ? t0 - kRunHalo : 0;
+    const int64_t hi = t0 + kRunTile + kRunHalo < n ? t0 + kRunTile + kRunHalo : n;
+    const int w = (int)(hi - lo);
+    for (int q = threadIdx.x; q < w; q += kRunThreads) {
+        s_k[q] = keys[lo + q];
+        s_v[q] = vals[lo + q];
+    }
+    __syncthreads();
+    bool too_long = false;
+#pragma unroll 1
+    for (int u = 0; u < kRunItems; ++u) {
+        const int64_t p = t0 + threadIdx.x + (int64_t)kRunThreads * u;
+        if (p >= n) break;
+        const int a = (int)(p - lo);
+        const uint64_t kp = s_k[a];
+        const uint32_t vp = s_v[a];
+        const uint64_t pre = kp >> kPrefixShift;
+        int h = a;
+        while (h > 0 && (s_k[h - 1] >> kPrefixShift) == pre) --h;
+        int e = a + 1;
+        while (e < w && (s_k[e] >> kPrefixShift) == pre) ++e;
+        // a run cut by the window edge (h == 0 with lo > 0, or e == w with
+        // hi < n) is at least kRunMax + 2 long, so the length test covers it
+        if (e - h > kRunMax) {
+            too_long = true;
             continue;
         }
-        const int m = (int)(e - i);
-        uint64_t k[kRunMax];
-        uint32_t v[kRunMax];
-        for (int a = 0; a < m; ++a) {
-            const uint64_t ka = keys[i + a];
-            const uint32_t va = vals[i + a];
-            int b = a;
-            while (b > 0 && (k[b - 1] > ka || (k[b - 1] == ka && v[b - 1] > va))) {
-                k[b] = k[b - 1];
-                v[b] = v[b - 1];
-                --b;
-            }
-            k[b] = ka;
-            v[b] = va;
+        int rank = 0;
+        for (int q = h; q < e; ++q) {
+            const uint64_t kq = s_k[q];
+            rank += (kq < kp || (kq == kp && s_v[q] < vp)) ? 1 : 0;
         }
-        for (int a = 0; a < m; ++a) {
-            if (keys_out) keys_out[i + a] = k[a];
-            vals_out[i + a] = v[a];
-        }
+        const int64_t out = lo + h + rank;
+        if (keys_out) keys_out[out] = kp;
+        vals_out[out] = vp;
     }
+    if (__any_sync(0xffffffffu, too_long) && (threadIdx.x & 31) == 0) atomicOr(gate, 1u);
 }
 
 }  // namespace
@@ -253,16 +273,15 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
         src = 1 - src;
     }
     {
-        int64_t blocks = (n + 255) / 256;
-        const int64_t cap = (int64_t)ctx->sm_count * 8;
-        if (blocks > cap) blocks = cap;
-        k_run_sort<<<(unsigned)blocks, 256, 0, s>>>(ctx->keys[src], ctx->vals[src], n, keys_final,
-                                                    vals_final, ctx->sort_gate);
+        const int64_t blocks = (n + kRunTile - 1) / kRunTile;
+        k_run_sort<<<(unsigned)blocks, kRunThreads, 0, s>>>(ctx->keys[src], ctx->vals[src], n,
+                                                           keys_final, vals_final, ctx->sort_gate);
         NL_CUDA_TRY(cudaGetLastError());
     }
     // full sort, gated: runs only when a prefix run was too long
     NL_CUDA_TRY(launch_keys(ctx, rk.n, rk.pos, rk.Lx, rk.Ly, rk.Lz, rk.Sx, rk.Sy, rk.Sz, rk.curve, s,
                             ctx->sort_gate));
+    NL_CUDA_TRY(launch_hist_scan(ctx, s, ctx->sort_gate));
     src = 0;
     for (int p = 0; p < kKeyPasses; ++p) {
         const bool last = p == kKeyPasses - 1;
