@@ -103,6 +103,16 @@ nl_status nl_build(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
                    float cutoff, float skin, int32_t capacity,
                    int32_t *nbr_out, int32_t *counts_out, void *stream);
 
+/* nl_build that writes rows for the first n_rows atoms of `pos` only
+ * (0 <= n_rows <= n): their neighbors are searched among all n atoms, but
+ * the atoms at n_rows.. (a halo received from other GPUs, say) get no row.
+ * nbr_out is n_rows x capacity, counts_out int32[n_rows] (either may be NULL
+ * when n_rows == 0); everything else as nl_build, which is n_rows == n.
+ * n_rows outside [0, n] is NL_ERR_ARG. */
+nl_status nl_build_rows(nl_ctx *ctx, int64_t n, int64_t n_rows, const float *pos,
+                        const float *box, float cutoff, float skin, int32_t capacity,
+                        int32_t *nbr_out, int32_t *counts_out, void *stream);
+
 /* nl_build with a close-pair detector as a by-product (Tessera abstract:
  * the simulations show no anomalously close pairs; this reports them while
  * the list is built).  Same arguments, results and status as nl_build, plus:

@@ -66,6 +66,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // stencil.  Grids above the context's cell budget are coarsened.
 nl_status make_grid(nl_ctx *ctx, const float *box, float cutoff, float skin, CellGrid *g)
 {
+    g->n_rows = INT64_MAX;
     if (!std::isfinite(cutoff) || !std::isfinite(skin) || cutoff < 0.0f || skin < 0.0f)
         return NL_ERR_ARG;
     volatile float rl = cutoff + skin;
@@ -164,13 +165,15 @@ nl_status sort_impl(nl_ctx *ctx, int64_t n, const float *pos, const float *box, 
 }
 
 nl_status build_checked(nl_ctx *ctx, int64_t n, const float *pos, const float *box, float cutoff,
-                        float skin, int32_t capacity, int32_t *nbr, int32_t *counts, CellGrid *g)
+                        float skin, int32_t capacity, int32_t *nbr, int32_t *counts, CellGrid *g,
+                        bool need_rows = true)
 {
     if (!ctx || n < 0) return NL_ERR_ARG;
     if (n > ctx->max_atoms || capacity > ctx->max_capacity) return NL_ERR_CAPACITY;
     if (capacity < 1) return NL_ERR_ARG;
     if (check_box(box) != NL_OK) return NL_ERR_ARG;
-    if (n > 0 && (!pos || !nbr || !counts || !aligned16(pos))) return NL_ERR_ARG;
+    if (n > 0 && (!pos || !aligned16(pos))) return NL_ERR_ARG;
+    if (n > 0 && need_rows && (!nbr || !counts)) return NL_ERR_ARG;
     return make_grid(ctx, box, cutoff, skin, g);
 }
 
@@ -178,6 +181,7 @@ nl_status build_enqueue(nl_ctx *ctx, int64_t n, const float *pos, const CellGrid
                         int32_t capacity, int32_t *nbr, int32_t *counts, cudaStream_t s, int *fast,
                         const CloseOut *close = nullptr)
 {
+    // g.n_rows (INT64_MAX unless the caller set it) limits the rows written
     const float4 *p4 = reinterpret_cast<const float4 *>(pos);
     if (launch_binning(ctx, n, p4, g, s) != cudaSuccess) return NL_ERR_CUDA;
     if (launch_pairs(ctx, n, g, capacity, nbr, counts, s, fast, close) != cudaSuccess)
@@ -468,6 +472,25 @@ nl_status nl_build(nl_ctx *ctx, int64_t n, const float *pos, const float *box, f
     CellGrid g;
     nl_status st = build_checked(ctx, n, pos, box, cutoff, skin, capacity, nbr_out, counts_out, &g);
     if (st != NL_OK) return st;
+    int fast = 0;
+    st = build_enqueue(ctx, n, pos, g, capacity, nbr_out, counts_out, S(stream), &fast);
+    if (st != NL_OK) return st;
+    ctx->last_n = n;
+    ctx->last_grid = g;
+    ctx->last_fast = fast;
+    return NL_OK;
+}
+
+nl_status nl_build_rows(nl_ctx *ctx, int64_t n, int64_t n_rows, const float *pos,
+                        const float *box, float cutoff, float skin, int32_t capacity,
+                        int32_t *nbr_out, int32_t *counts_out, void *stream)
+{
+    if (n_rows < 0 || n_rows > n) return NL_ERR_ARG;
+    CellGrid g;
+    nl_status st = build_checked(ctx, n, pos, box, cutoff, skin, capacity, nbr_out, counts_out, &g,
+                                 n_rows > 0);
+    if (st != NL_OK) return st;
+    g.n_rows = n_rows;
     int fast = 0;
     st = build_enqueue(ctx, n, pos, g, capacity, nbr_out, counts_out, S(stream), &fast);
     if (st != NL_OK) return st;

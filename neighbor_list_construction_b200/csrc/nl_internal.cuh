@@ -67,6 +67,7 @@ struct CellGrid {
     int64_t ncell;
     int wy, wz;              // stencil half-width in y and z (x is always 1)
     int literal;             // 1: literal minimum image (small boxes)
+    int64_t n_rows;          // rows are written for atoms of index < n_rows only
 };
 
 }  // namespace nl

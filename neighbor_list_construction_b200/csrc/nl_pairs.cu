@@ -56,6 +56,7 @@ __device__ __forceinline__ void pair_row_per_atom(int64_t k, const float4 *__res
 {
     const float4 p = cell_pos[k];
     const int i = __float_as_int(p.w);
+    if (i >= g.n_rows) return;   // no row for this atom
     const uint32_t c = atom_cell[i];
     const int cx = (int)(c % (uint32_t)g.nx);
     const int cy = (int)((c / (uint32_t)g.nx) % (uint32_t)g.ny);
@@ -1027,12 +1028,14 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
 
     for (int c = warp; c * 32 < nhome; c += kTileWarps) {
         const int a = c * 32 + lane;
-        const bool valid = a < nhome;
         int h = 0;
         while (h < kHome - 1 && a >= tr.home_pref[h + 1]) ++h;
         const int slot = tr.home_begin[h] + (a - tr.home_pref[h]);
         const float qn = __int_as_float(0x7fc00000);
-        const float4 me = valid ? stage[slot] : make_float4(qn, qn, qn, qn);
+        float4 me = a < nhome ? stage[slot] : make_float4(qn, qn, qn, qn);
+        // a lane has a row to build when its atom exists and is below n_rows
+        const bool valid = a < nhome && __float_as_int(me.w) < g.n_rows;
+        if (!valid) me = make_float4(qn, qn, qn, qn);
         const int hy = h % kTY, hz = h / kTY;
         const float ylo = (float)(cy0 + hy) * P.side_y, yhi = (float)(cy0 + hy + 1) * P.side_y;
         const float zlo = (float)(cz0 + hz) * P.side_z, zhi = (float)(cz0 + hz + 1) * P.side_z;

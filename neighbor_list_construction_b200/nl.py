@@ -32,6 +32,7 @@ _SIGS = {
     "nl_sort_hilbert": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_sort_morton": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_build": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
+    "nl_build_rows": (_i32, [_vp, _i64, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
     "nl_build_close": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _f32, _vp, _vp,
                               _vp]),
     "nl_skin_check": (_i32, [_vp, _i64, _vp, _vp, _f32, _vp, _vp, _vp]),
@@ -47,6 +48,12 @@ _SIGS = {
     "nl_profile_read": (_i32, [_vp, _vp, _vp, _i32]),
     "nl_profile_phase_name": (ctypes.c_char_p, [_i32]),
     "nl_sort_hilbert_noalloc": (_i32, [_i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "nl_halo_grid": (_i32, [_vp, _f32, _f32, _vp]),
+    "nl_halo_mark": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _vp, _vp]),
+    "nl_halo_needed": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "nl_halo_count": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp]),
+    "nl_halo_fill": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "nl_map_ids": (_i32, [_vp, _i64, _i32, _vp, _i64, _vp, _vp]),
     "nls_displace": (_i32, [_i64, _vp, _u64, _i64, _vp, _f32, _vp]),
     "nls_step_graph": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _u64, _vp, _f32]),
     "nls_step_graph_ids": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _vp, _u64, _vp, _f32]),
@@ -146,6 +153,14 @@ def nl_build(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, stream=
                                 _stream(stream)), "nl_build")
 
 
+def nl_build_rows(ctx, pos, n_rows, box, cutoff, skin, capacity, nbr_out, counts_out,
+                  stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_build_rows(ctx, pos.shape[0], int(n_rows), _ptr(pos), _box(box),
+                                     float(cutoff), float(skin), int(capacity), _ptr(nbr_out),
+                                     _ptr(counts_out), _stream(stream)), "nl_build_rows")
+
+
 def nl_build_close(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, close_d2,
                    min_d2_out, n_close_out, stream=None) -> int:
     _pos(pos)
@@ -197,6 +212,51 @@ def nl_replay_resort(ctx, step_graph, n_steps, pos, ids, aux, box, cutoff, skin,
                                         int(capacity), _ptr(nbr), _ptr(counts),
                                         _ptr(decisions_out), _stream(stream)),
                   "nl_replay_resort")
+
+
+def _dims(dims):
+    d = (ctypes.c_int32 * 3)(*[int(x) for x in dims])
+    return d
+
+
+def nl_halo_grid(box, cutoff, skin):
+    """Coarse grid of the halo selection: a tuple of 3 ints."""
+    out = (ctypes.c_int32 * 3)()
+    _check(_lib.nl_halo_grid(_box(box), float(cutoff), float(skin), out), "nl_halo_grid")
+    return tuple(out)
+
+
+def nl_halo_mark(ctx, pos, box, dims, rank, occ_out, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_halo_mark(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
+                                    int(rank), _ptr(occ_out), _stream(stream)), "nl_halo_mark")
+
+
+def nl_halo_needed(ctx, box, dims, occ_all, need_out, stream=None) -> int:
+    return _check(_lib.nl_halo_needed(ctx, _box(box), _dims(dims), _ptr(occ_all), _ptr(need_out),
+                                      _stream(stream)), "nl_halo_needed")
+
+
+def nl_halo_count(ctx, pos, box, dims, need, rank, nranks, counts_out, stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_halo_count(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
+                                     _ptr(need), int(rank), int(nranks), _ptr(counts_out),
+                                     _stream(stream)), "nl_halo_count")
+
+
+def nl_halo_fill(ctx, pos, box, dims, need, rank, nranks, offsets, counts, cursor, send_out,
+                 stream=None) -> int:
+    _pos(pos)
+    return _check(_lib.nl_halo_fill(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
+                                    _ptr(need), int(rank), int(nranks), _ptr(offsets),
+                                    _ptr(counts), _ptr(cursor), _ptr(send_out), _stream(stream)),
+                  "nl_halo_fill")
+
+
+def nl_map_ids(ctx, nbr, pos_all, stream=None) -> int:
+    _pos(pos_all)
+    return _check(_lib.nl_map_ids(ctx, nbr.shape[0], int(nbr.shape[1]), _ptr(nbr),
+                                  pos_all.shape[0], _ptr(pos_all), _stream(stream)), "nl_map_ids")
 
 
 def nl_step_counter(ctx) -> int:
@@ -293,6 +353,14 @@ class Context:
         if counts is None:
             counts = torch.empty(n, dtype=torch.int32, device=pos.device)
         nl_build(self.handle, pos, box, cutoff, skin, capacity, nbr, counts, stream)
+        return nbr, counts
+
+    def build_rows(self, pos, n_rows, box, cutoff, skin, capacity, stream=None):
+        """Rows for the first n_rows atoms of pos, neighbors among all."""
+        nbr = torch.empty(n_rows, capacity, dtype=torch.int32, device=pos.device)
+        counts = torch.empty(n_rows, dtype=torch.int32, device=pos.device)
+        nl_build_rows(self.handle, pos, n_rows, box, cutoff, skin, capacity,
+                      nbr if n_rows else None, counts if n_rows else None, stream)
         return nbr, counts
 
     def build_close(self, pos, box, cutoff, skin, capacity, close_d2, stream=None):

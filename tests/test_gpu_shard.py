@@ -1,0 +1,111 @@
+"""The sharded build on one GPU (all shards in one process, collectives
+routed in memory): the rows of every shard's own atoms, as global ids, are
+the oracle's rows of the whole system."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    from neighbor_list_construction_b200 import nl
+    c = nl.Context(10_400_000, 320)
+    yield c
+    c.close()
+
+
+@pytest.fixture(scope="module")
+def shard():
+    from neighbor_list_construction_b200 import shard as _shard
+    return _shard
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def run_sharded(ctx, shard, pos, box, cutoff, skin, K, owner):
+    """owner[k] = shard of atom k (global id k); returns rows by global id."""
+    p = shard.with_ids(dev(pos), 0)
+    nranks = int(owner.max()) + 1
+    ids = [np.nonzero(owner == r)[0] for r in range(nranks)]
+    shards = [p[torch.from_numpy(i).cuda()] for i in ids]
+    res = shard.build_sharded_local(ctx, shards, box, cutoff, skin, K)
+    n = pos.shape[0]
+    nbr = np.full((n, K), -1, np.int32)
+    cnt = np.zeros(n, np.int32)
+    halos = []
+    for i, (nb, c, h) in zip(ids, res):
+        nbr[i] = nb.cpu().numpy()
+        cnt[i] = c.cpu().numpy()
+        halos.append(h)
+    return nbr, cnt, halos
+
+
+@pytest.mark.parametrize("name,nranks", [("uniform4k", 1), ("uniform4k", 3), ("lattice60k", 2),
+                                         ("lattice60k", 8), ("saltwater_n20", 4),
+                                         ("saltwater_n20", 7)])
+def test_equal_count_shards_match_the_oracle(ctx, shard, oracle, name, nranks):
+    w = gu.workload(name)
+    ps = gu.oracle_sorted(name)                 # global id = place on the curve
+    owner = np.zeros(w.n, np.int64)
+    for r, (s, e) in enumerate(shard.shard_bounds(w.n, nranks)):
+        owner[s:e] = r
+    nbr, cnt, halos = run_sharded(ctx, shard, ps, w.box, w.cutoff, w.skin, w.capacity, owner)
+    st = ctx.sync_status()
+    o_nbr, o_cnt, o_ov = oracle.build(ps, w.box, w.cutoff, w.skin, w.capacity)
+    assert st == (1 if o_ov else 0)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+    sizes = [e - s for s, e in shard.shard_bounds(w.n, nranks)]
+    for h, m in zip(halos, sizes):
+        assert h <= w.n - m                     # never more than all other atoms
+        assert (h > 0) == (nranks > 1)
+
+
+def test_scattered_shards_match_the_oracle(ctx, shard, oracle):
+    """Owners drawn at random: every shard's halo is nearly everything."""
+    w = gu.workload("lattice60k")
+    owner = np.random.default_rng(5).integers(0, 5, w.n)
+    nbr, cnt, halos = run_sharded(ctx, shard, w.pos, w.box, w.cutoff, w.skin, w.capacity, owner)
+    assert ctx.sync_status() == 0
+    o_nbr, o_cnt, _ = oracle.build(w.pos, w.box, w.cutoff, w.skin, w.capacity)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+    assert min(halos) > 0.5 * w.n
+
+
+def test_an_empty_shard(ctx, shard, oracle):
+    w = gu.workload("uniform4k")
+    owner = np.zeros(w.n, np.int64)
+    owner[w.n // 2:] = 2                        # shard 1 owns nothing
+    nbr, cnt, halos = run_sharded(ctx, shard, w.pos, w.box, w.cutoff, w.skin, w.capacity, owner)
+    o_nbr, o_cnt, _ = oracle.build(w.pos, w.box, w.cutoff, w.skin, w.capacity)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+    assert ctx.sync_status() == 0
+
+
+def test_full_size_eight_shards_sampled(ctx, shard, oracle):
+    """saltwater10m cut into 8 curve shards: sampled rows of every shard
+    against the oracle, and the directed pair total against the one-GPU
+    build."""
+    w = gu.workload("saltwater10m")
+    ps = gu.oracle_sorted("saltwater10m")
+    p = shard.with_ids(dev(ps), 0)
+    bounds = shard.shard_bounds(w.n, 8)
+    res = shard.build_sharded_local(ctx, [p[s:e] for s, e in bounds], w.box, w.cutoff, w.skin,
+                                    w.capacity)
+    assert ctx.sync_status() == 0
+    rng = np.random.default_rng(8)
+    total = 0
+    for (s, e), (nb, c, h) in zip(bounds, res):
+        total += int(c.to(torch.int64).sum().item())
+        loc = np.unique(np.concatenate([rng.choice(e - s, 300, replace=False), [0, e - s - 1]]))
+        o_nbr, o_cnt, _ = oracle.rows(ps, w.box, w.cutoff, w.skin, w.capacity, s + loc)
+        idx = torch.from_numpy(loc).cuda()
+        gu.assert_rows_match(nb[idx].cpu().numpy(), c[idx].cpu().numpy(), o_nbr, o_cnt)
+        assert 0 < h < (e - s)
+    _, cnt_full = ctx.build(dev(ps), w.box, w.cutoff, w.skin, w.capacity)
+    assert total == int(cnt_full.to(torch.int64).sum().item())
