@@ -34,8 +34,8 @@ NOMINAL_HBM_GBS = 8000.0
 # belongs to the kernel source it was taken on: with any other source of the
 # pair kernel the bench reports null.
 PAIR_TRAFFIC = {"workload": "saltwater10m",
-                "sha256": "510b0f106c3f422db82414975979ba45918643b569843b55655cc377f6f8a1b0",
-                "bytes": 793912832 + 10741550592}
+                "sha256": "8b521ca0a9d041126389ac23e1809be61d00c09a64c20dcb928406f92b2ff37e",
+                "bytes": 800189696 + 10744392960}
 
 
 def pair_traffic(workload: str):
@@ -345,6 +345,32 @@ def edge_feature_timing(nl, torch, h, ps, w, K, reps: int = 5) -> dict:
             "layout": f"float32 [{n}, {K}, 4] (dx, dy, dz, r), zero padding"}
 
 
+def sharded_timing(torch, ctx, ps, w, K, nranks: int = 8, reps: int = 2) -> dict:
+    """The curve-sharded build of the whole system with nranks equal-count
+    shards, all in this process on this GPU (collectives routed in memory):
+    halo sizes, and the time of the whole sharded build (all shards, their
+    host round trips included) against one nl_build of the whole system."""
+    from neighbor_list_construction_b200 import shard
+    n = ps.shape[0]
+    p = shard.with_ids(ps, 0)
+    bounds = shard.shard_bounds(n, nranks)
+    shards = [p[s:e] for s, e in bounds]
+    res = shard.build_sharded_local(ctx, shards, w.box, w.cutoff, w.skin, K)
+    halos = [r[2] for r in res]
+    del res
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        res = shard.build_sharded_local(ctx, shards, w.box, w.cutoff, w.skin, K)
+        del res
+    e1.record()
+    torch.cuda.synchronize()
+    return {"shards": nranks, "atoms_per_shard": [e - s for s, e in bounds],
+            "halo_atoms": halos, "halo_fraction": sum(halos) / n,
+            "ms_all_shards_one_gpu": e0.elapsed_time(e1) / reps}
+
+
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -536,6 +562,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
             line["curves"] = curve_comparison(nl, torch, h, pos, w, K)
             line["close_pairs"] = close_pair_timing(nl, torch, h, ps, w, K)
             line["edge_features"] = edge_feature_timing(nl, torch, h, ps, w, K)
+            line["sharded"] = sharded_timing(torch, ctx, ps, w, K)
         if world == 1 and not args.no_cpu_baseline:
             cb = oracle_sample(1)
             line["cpu_baseline"] = {"value": cb["value"], "unit": "atoms/s", "cores": cb["cores"],
