@@ -166,3 +166,67 @@ def test_edges_full_size_sampled(ctx, oracle):
                        kind="stable")
     g_sorted = np.take_along_axis(g_e, order[:, :, None], axis=1)
     np.testing.assert_array_equal(bits(g_sorted), bits(o_e))
+
+
+# -------------------------------------------- features of rows in every regime
+def check_rows_and_edges(ctx, oracle, pos, box, cutoff, skin, K):
+    """nl_build then nl_edge_features: slot by slot the oracle's feature of
+    the same (i, j), looked up in the oracle's complete rows; zeros in the
+    padding."""
+    p = dev(pos)
+    nbr, cnt = ctx.build(p, box, cutoff, skin, K)
+    st = ctx.sync_status()
+    e = ctx.edge_features(p, box, nbr, cnt)
+    assert ctx.sync_status() == 0
+    g_nbr, g_cnt, g_e = nbr.cpu().numpy(), cnt.cpu().numpy(), e.cpu().numpy()
+    o_nbr, o_cnt, o_e = full_features(pos, box, cutoff, skin, oracle)
+    np.testing.assert_array_equal(g_cnt, o_cnt)
+    for i in range(g_nbr.shape[0]):
+        c = min(int(g_cnt[i]), K)
+        t = np.searchsorted(o_nbr[i, : o_cnt[i]], g_nbr[i, :c])
+        np.testing.assert_array_equal(o_nbr[i, t], g_nbr[i, :c])
+        np.testing.assert_array_equal(bits(g_e[i, :c]), bits(o_e[i, t]))
+        np.testing.assert_array_equal(bits(g_e[i, c:]), 0)
+    return st
+
+
+@pytest.mark.parametrize("box", [[7.6, 7.6, 7.6], [13.0, 10.1, 7.6]])
+def test_edges_small_boxes(ctx, oracle, box):
+    """Rows from the per-atom kernel with the literal minimum image."""
+    rng = np.random.default_rng(9)
+    box = np.array(box, np.float32)
+    n = int(0.1 * np.prod(box)) + 7
+    pos = np.zeros((n, 4), np.float32)
+    pos[:, :3] = rng.random((n, 3)) * box
+    check_rows_and_edges(ctx, oracle, pos, box, 2.0, 0.5, 64)
+
+
+def test_edges_dense_slab(ctx, oracle):
+    """Rows from the listed (dense) tiles and the per-atom search next to a
+    sparse region; planted pairs across the periodic face."""
+    rng = np.random.default_rng(5)
+    box = np.array([25.0, 25.0, 25.0], np.float32)
+    sparse = rng.random((1600, 3)) * box
+    dense = rng.random((20000, 3)) * np.array([5.5, 25.0, 25.0])
+    pos = np.zeros((21604, 4), np.float32)
+    pos[:21600, :3] = np.concatenate([sparse, dense])
+    pos[21600:, :3] = [[15.0, 12.0, 12.0], [15.0625, 12.0, 12.0],
+                       [24.9375, 3.0, 3.0], [0.0, 3.0, 3.0]]
+    check_rows_and_edges(ctx, oracle, pos, box, 2.0, 0.5, 256)
+
+
+def test_edges_cutoff_shell(ctx, oracle):
+    """Partners within a few ulps of rl: lengths at the edge of the
+    membership test."""
+    rng = np.random.default_rng(17)
+    L, cutoff, skin = 48.0, 5.75, 1.0
+    rl = np.float64(np.float32(cutoff + skin))
+    nb = 4000
+    base = rng.random((nb, 3)) * L
+    u = rng.normal(size=(nb, 3))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    pos = np.zeros((2 * nb, 4), np.float32)
+    pos[:nb, :3] = base
+    pos[nb:, :3] = base + rl * (1.0 + rng.uniform(-3e-7, 3e-7, size=(nb, 1))) * u
+    box = np.array([L, L, L], np.float32)
+    check_rows_and_edges(ctx, oracle, pos, box, cutoff, skin, 256)
