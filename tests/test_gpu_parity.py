@@ -390,13 +390,19 @@ def _replay_resort(ctx, nl, oracle, name, steps, start, seed=2024):
     np.testing.assert_array_equal(aux.cpu().numpy(), aux0[idh])
     if o_dec.any():
         # the last rebuild put the atoms in curve order of their positions then
-        k = oracle.keys(o_ref[idh], w.box)
+        k = oracle.keys(o_ref, w.box)[idh]
         assert np.all(k[1:] >= k[:-1])
     else:
         np.testing.assert_array_equal(idh, np.arange(n))
-    o_nbr, o_cnt, o_ov = oracle.build(o_ref[idh], w.box, w.cutoff, w.skin, w.capacity)
+    # rows by atom id: slot k holds atom idh[k], its entries are slots too
+    g_nbr = nbr.cpu().numpy()
+    by_id = np.full_like(g_nbr, -1)
+    by_id[idh] = np.where(g_nbr >= 0, idh[np.maximum(g_nbr, 0)], -1)
+    by_cnt = np.zeros(n, np.int32)
+    by_cnt[idh] = cnt.cpu().numpy()
+    o_nbr, o_cnt, o_ov = oracle.build(o_ref, w.box, w.cutoff, w.skin, w.capacity)
     assert st == (1 if o_ov else 0)
-    gu.assert_rows_match(nbr.cpu().numpy(), cnt.cpu().numpy(), o_nbr, o_cnt)
+    gu.assert_rows_match(by_id, by_cnt, o_nbr, o_cnt)
     return o_dec, idh
 
 
