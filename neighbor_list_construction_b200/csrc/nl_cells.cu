@@ -158,7 +158,9 @@ __device__ __forceinline__ void sort_small_cell(float4 *__restrict__ cell_pos, i
     const int id = __float_as_int(v.w);
     const int bin = max(0, min(15, (int)floorf((v.x - face) * inv_bin)));
     int r = 0, below = 0;
-    for (int j = 0; j < 16; ++j) {
+    // both halves run to the larger of their two cells
+    const int mm = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
+    for (int j = 0; j < mm; ++j) {
         const float xj = __shfl_sync(0xffffffffu, v.x, j, 16);
         const int ij = __shfl_sync(0xffffffffu, id, j, 16);
         const int bj = __shfl_sync(0xffffffffu, bin, j, 16);
