@@ -109,3 +109,27 @@ def test_full_size_eight_shards_sampled(ctx, shard, oracle):
         assert 0 < h < (e - s)
     _, cnt_full = ctx.build(dev(ps), w.box, w.cutoff, w.skin, w.capacity)
     assert total == int(cnt_full.to(torch.int64).sum().item())
+
+
+@pytest.mark.parametrize("name", ["uniform4k", "saltwater_n20"])
+def test_build_rows_prefix(ctx, oracle, name):
+    """nl_build_rows: the rows of the first n_rows atoms are nl_build's rows
+    (the oracle's) whatever n_rows is; out-of-range n_rows is an error."""
+    from neighbor_list_construction_b200 import nl
+    w = gu.workload(name)
+    p = dev(w.pos)
+    o_nbr, o_cnt, o_ov = oracle.build(w.pos, w.box, w.cutoff, w.skin, w.capacity)
+    for n_rows in (0, 1, 777, w.n // 2, w.n):
+        nbr, cnt = ctx.build_rows(p, n_rows, w.box, w.cutoff, w.skin, w.capacity)
+        assert ctx.sync_status() == (1 if o_ov and o_cnt[:n_rows].max(initial=0) > w.capacity
+                                     else 0)
+        assert nbr.shape == (n_rows, w.capacity)
+        gu.assert_rows_match(nbr.cpu().numpy(), cnt.cpu().numpy(), o_nbr[:n_rows],
+                             o_cnt[:n_rows])
+    with pytest.raises(nl.NLError):
+        ctx.build_rows(p, w.n + 1, w.box, w.cutoff, w.skin, w.capacity)
+    nb = torch.empty(1, w.capacity, dtype=torch.int32, device="cuda")
+    c1 = torch.empty(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(nl.NLError):
+        nl.nl_build_rows(ctx.handle, p, -1, w.box, w.cutoff, w.skin, w.capacity, nb, c1)
+    assert ctx.sync_status() == 0
