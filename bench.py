@@ -31,17 +31,17 @@ NOMINAL_HBM_GBS = 8000.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
 # pair-search launch on the saltwater10m workload, from one ncu capture.  It
-# belongs to the kernel source it was taken on: with any other source of the
-# pair kernel the bench reports null.
+# belongs to the kernel source it was taken on (nl_pairs.cu and the device
+# header it includes): with any other source the bench reports null.
 PAIR_TRAFFIC = {"workload": "saltwater10m",
-                "sha256": "8b521ca0a9d041126389ac23e1809be61d00c09a64c20dcb928406f92b2ff37e",
-                "bytes": 800189696 + 10744392960}
+                "sha256": "05dcfffb7fc577ba2b99f9b61e3cce4d117adf88aa34f35fa88c8b2dce84fa15",
+                "bytes": 803095808 + 10746583296}
 
 
 def pair_traffic(workload: str):
     import hashlib
     h = hashlib.sha256()
-    for f in ("nl_pairs.cu", "nl_internal.cuh"):
+    for f in ("nl_pairs.cu", "nl_device.cuh"):
         with open(os.path.join(ROOT, "neighbor_list_construction_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     if workload == PAIR_TRAFFIC["workload"] and h.hexdigest() == PAIR_TRAFFIC["sha256"]:

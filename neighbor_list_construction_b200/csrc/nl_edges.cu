@@ -82,11 +82,12 @@ cudaError_t launch_edge_features(nl_ctx *ctx, int64_t n, const float4 *pos, floa
     if (n <= 0) return cudaSuccess;
     ProfScope ps(ctx, PH_EDGES, s);
     // one resident wave of CTAs; the warps stride over rows
-    static int per_sm = 0;
-    if (per_sm == 0) {
+    if (ctx->edge_blocks_per_sm == 0) {   // per context, so per device
+        int per_sm = 0;
         NL_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_edge_features, 128, 0));
-        if (per_sm < 1) per_sm = 1;
+        ctx->edge_blocks_per_sm = per_sm < 1 ? 1 : per_sm;
     }
+    const int per_sm = ctx->edge_blocks_per_sm;
     int64_t blocks = (n + 3) / 4;
     const int64_t cap = (int64_t)ctx->sm_count * per_sm;
     if (blocks > cap) blocks = cap;

@@ -7,75 +7,14 @@
 #include <stdint.h>
 
 #include "nl.h"
+#include "nl_device.cuh"
 
-namespace nl {
-
-// ----------------------------------------------------------------- constants
-constexpr int kQBits = 21;                    // bits per axis of the curve grid
-constexpr uint32_t kQMax = (1u << kQBits) - 1u;
-constexpr int kRadixBits = 8;                 // LSD digit width
-constexpr int kRadixBins = 1 << kRadixBits;
-constexpr int kKeyPasses = 8;                 // 63-bit keys: 8 digits of 8 bits
-constexpr int kTopPasses = 3;                 // fast path: the top digits (bits 40..63)
-constexpr int kStatusPasses = kKeyPasses + kTopPasses;   // look-back status slots
-constexpr int kPrefixShift = 8 * (kKeyPasses - kTopPasses);  // key >> this = sorted prefix
-constexpr int kRunMax = 64;                   // longest prefix run one thread finishes
-
-// Onesweep tile: 256 threads x 16 keys.
-constexpr int kSortThreads = 256;
-constexpr int kSortItems = 8;
-constexpr int kSortTile = kSortThreads * kSortItems;
-
-// Cell-count scan tile: 256 threads x 16 cells.
-constexpr int kScanThreads = 256;
-constexpr int kScanItems = 16;
-constexpr int kScanTile = kScanThreads * kScanItems;
-
-// Look-back status words: 2 flag bits over a 30-bit count.
-constexpr uint32_t kStAggregate = 1u << 30;
-constexpr uint32_t kStPrefix = 2u << 30;
-constexpr uint32_t kStValue = (1u << 30) - 1u;
-// Polls of one status word before a bounded wait gives up.
-constexpr uint32_t kSpinLimit = 1u << 22;
-
-// Device-detected conditions, accumulated in ctx->flags.
-constexpr uint32_t kFlagOverflow = 1u;
-constexpr uint32_t kFlagTimeout = 2u;
-
-enum Phase {
-    PH_KEYS = 0,
-    PH_KEY_SCAN,
-    PH_SORT,
-    PH_GATHER,
-    PH_BIN_COUNT,
-    PH_CELL_SCAN,
-    PH_BIN_SCATTER,
-    PH_CELL_SORT,
-    PH_PAIRS,
-    PH_PAIRS_FALLBACK,
-    PH_SKIN,
-    PH_EDGES,
-    PH_COUNT
-};
-
-// Cell grid of one build, all values computed on the host.
-struct CellGrid {
-    int nx, ny, nz;          // cells per axis
-    float Lx, Ly, Lz;        // box
-    float Tx, Ty, Tz;        // fl(n_a / L_a): cell coordinate = floor(w * T)
-    float rl2;               // fl(rl * rl)
-    int64_t ncell;
-    int wy, wz;              // stencil half-width in y and z (x is always 1)
-    int literal;             // 1: literal minimum image (small boxes)
-    int64_t n_rows;          // rows are written for atoms of index < n_rows only
-};
-
-}  // namespace nl
 
 // ------------------------------------------------------------------ context
 struct nl_ctx {
     int device = 0;
     int sm_count = 148;
+    int edge_blocks_per_sm = 0;   // resident CTAs of the edge-feature kernel (0: not asked yet)
     int64_t max_atoms = 0;
     int32_t max_capacity = 0;
     int64_t max_cells = 0;
@@ -210,58 +149,6 @@ cudaError_t launch_skin(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
                         float Lz, float h2, int32_t *rebuild_out, float *max_d2_out,
                         int32_t *decisions, const int32_t *step,
                         unsigned long long cond_handle, cudaStream_t s);
-
-// ------------------------------------------------------- device helpers
-__device__ __forceinline__ float wrap_coord(float x, float L)
-{
-    // w = x - L*floor(x/L), one fold into [0, L), else 0.
-    // For 0 < x <= fl_down(L*(1 - 2^-23)) the quotient x/L rounds to a float
-    // below 1, so t = 0 and w = fl(x - 0) = x: the same bits without the
-    // division (zeros take the full path, which maps -0 to +0).
-    if (x > 0.0f && x <= __fmul_rd(L, 0.99999988f)) return x;
-    float t = floorf(__fdiv_rn(x, L));
-    float w = __fsub_rn(x, __fmul_rn(L, t));
-    if (w < 0.0f) w = __fadd_rn(w, L);
-    if (w >= L) w = __fsub_rn(w, L);
-    if (!(w >= 0.0f && w < L)) w = 0.0f;
-    return w;
-}
-
-// Literal minimum image d - L*rintf(d/L).
-__device__ __forceinline__ float min_image_literal(float d, float L)
-{
-    float r = rintf(__fdiv_rn(d, L));
-    return __fsub_rn(d, __fmul_rn(L, r));
-}
-
-__device__ __forceinline__ float r2_of(float dx, float dy, float dz)
-{
-    return __fadd_rn(__fadd_rn(__fmul_rn(dx, dx), __fmul_rn(dy, dy)), __fmul_rn(dz, dz));
-}
-
-__device__ __forceinline__ int cell_coord(float w, float T, int n)
-{
-    float f = floorf(__fmul_rn(w, T));
-    int c = f >= 0.0f ? (int)f : 0;
-    return c < n ? c : n - 1;
-}
-
-__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t *p)
-{
-    return *(const volatile uint32_t *)p;
-}
-
-__device__ __forceinline__ void st_volatile_u32(uint32_t *p, uint32_t v)
-{
-    *(volatile uint32_t *)p = v;
-}
-
-__device__ __forceinline__ uint32_t lanemask_lt()
-{
-    uint32_t m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
 
 }  // namespace nl
 

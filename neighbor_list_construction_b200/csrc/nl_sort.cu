@@ -245,16 +245,9 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
 {
     if (n <= 0) return cudaSuccess;
     const int64_t tiles = (n + kSortTile - 1) / kSortTile;
-    static bool attr_set = false;
-    if (!attr_set) {
-        NL_CUDA_TRY(cudaFuncSetAttribute(k_onesweep<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSortDynSmem));
-        NL_CUDA_TRY(cudaFuncSetAttribute(k_onesweep<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSortDynSmem));
-        attr_set = true;
-    }
+    // kSortDynSmem (24 KB) is below the default dynamic shared-memory limit,
+    // so the passes need no per-device attribute
+    static_assert(kSortDynSmem <= 48 * 1024, "onesweep tile needs the opt-in shared memory");
     NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_status, 0,
                                 sizeof(uint32_t) * kStatusPasses * tiles * kRadixBins, s));
     NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_ctr, 0, sizeof(uint32_t) * kStatusPasses, s));
