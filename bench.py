@@ -137,13 +137,13 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(steps: int = 1) -> dict:
+def oracle_sample(steps: int = 1, nside: int = 60) -> dict:
     """The CPU oracle, as it stands, on a bounded sample of the salt-solution
-    recipe (60^3 sites, ~0.65M atoms): curve sort + neighbor list + skin
-    check per step, single-threaded."""
+    recipe (nside^3 sites: 60 -> ~0.65M atoms, 40 -> ~0.19M): curve sort +
+    neighbor list + skin check per step, single-threaded."""
     import oracle
     from neighbor_list_construction_b200 import workloads
-    w = workloads.make("saltwater_n60", seed=4)
+    w = workloads.make(f"saltwater_n{nside}", seed=4)
     oracle.lib()
     t0 = time.perf_counter()
     pairs = 0
@@ -155,25 +155,39 @@ def oracle_sample(steps: int = 1) -> dict:
         pairs += int(cnt.sum())
     dt = time.perf_counter() - t0
     return {"value": steps * w.n / dt, "unit": "atoms/s", "cores": 1, "kind": "oracle",
-            "sample": f"{w.n} atoms, salt-solution recipe on 60^3 sites (same density, "
+            "sample": f"{w.n} atoms, salt-solution recipe on {nside}^3 sites (same density, "
                       f"cutoff 5.75, skin 1.0, capacity 256), sort+build+skin x{steps}, "
                       f"{dt:.1f} s single-threaded",
             "pairs_per_s": pairs / dt, "seconds": dt}
 
 
+def arm_config(workload: str, world: int) -> dict:
+    """The config of the GPU arm's line, from the workload table."""
+    from neighbor_list_construction_b200 import workloads
+    n, cutoff, skin, K, desc = workloads.INFO[workload]
+    return {"workload": f"{workload}: {desc}", "atoms": n, "cutoff": cutoff, "skin": skin,
+            "capacity": K, "step": "nl_sort_hilbert + nl_build + nl_skin_check",
+            "parallelism": "replicas" if world > 1 else "single"}
+
+
 def run_reference(args, rank: int, world: int) -> None:
+    """The oracle on the host cores: K timed steps (after up to 3 warm-up
+    steps), each a ~0.19M-atom sample of the salt-solution recipe, so the
+    whole run takes about a minute."""
     if rank != 0:
         return
-    steps = max(1, min(args.steps, 3))
-    for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample(1)
-    r = oracle_sample(steps)
+    warm = max(0, min(args.warmup, 3))
+    if warm:
+        oracle_sample(warm, nside=40)
+    r = oracle_sample(args.steps, nside=40)
+    cfg = arm_config(args.workload, world)
+    cfg["sample"] = r["sample"]
     line = {
         "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "atoms/s",
-        "n_gpus": world, "steps": steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * r["seconds"] / steps, "higher_is_better": True,
+        "n_gpus": world, "steps": args.steps, "warmup": warm,
+        "ms_per_step": 1000.0 * r["seconds"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "saltwater10m recipe, bounded sample", "parallelism": "replicas"},
+        "config": cfg,
         "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
         "e2e": {"value": r["value"], "unit": "atoms/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},

@@ -186,3 +186,15 @@ def make(name: str, seed: int | None = None) -> Workload:
 
 
 NAMES = ("uniform4k", "lattice60k", "saltwater1m", "saltwater10m", "shell10m")
+
+# (atoms, cutoff, skin, capacity, description) of the named workloads, for
+# reports that name a workload without generating it
+INFO = {
+    "uniform4k": (4096, 5.75, 1.0, 256, "4,096 atoms uniform random at 0.1/A^3, cubic box 34.47 A"),
+    "lattice60k": (59319, 5.75, 1.0, 256, "59,319 atoms, 39^3 sc lattice at 0.1/A^3, jitter 0.3 A"),
+    "saltwater1m": (981975, 6.0, 1.5, 320, "981,975 atoms rigid water + 0.15 M NaCl, 69^3 sites"),
+    "saltwater10m": (10291605, 5.75, 1.0, 256,
+                     "10,291,605 atoms rigid water + 0.15 M NaCl, 151^3 sites"),
+    "shell10m": (10060000, 5.75, 1.0, 320,
+                 "10,060,000 atoms: 0.12/A^3 shell r 120-150 A in 0.1/A^3 fill"),
+}
