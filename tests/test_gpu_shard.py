@@ -133,3 +133,33 @@ def test_build_rows_prefix(ctx, oracle, name):
     with pytest.raises(nl.NLError):
         nl.nl_build_rows(ctx.handle, p, -1, w.box, w.cutoff, w.skin, w.capacity, nb, c1)
     assert ctx.sync_status() == 0
+
+
+def test_dist_driver_over_nccl_one_rank(ctx, shard, oracle):
+    """build_sharded through DistExchange on a one-rank NCCL group: the same
+    collective calls the multi-GPU run makes, on CUDA tensors."""
+    import os
+    import socket
+    import torch.distributed as dist
+    if dist.is_initialized():
+        pytest.skip("a process group already exists")
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = gu.workload("lattice60k")
+        ps = gu.oracle_sorted("lattice60k")
+        p = shard.with_ids(dev(ps), 0)
+        nbr, cnt, halo = shard.build_sharded(ctx, p, w.box, w.cutoff, w.skin, w.capacity,
+                                             shard.DistExchange())
+        assert halo == 0
+        assert ctx.sync_status() == 0
+        o_nbr, o_cnt, _ = oracle.build(ps, w.box, w.cutoff, w.skin, w.capacity)
+        gu.assert_rows_match(nbr.cpu().numpy(), cnt.cpu().numpy(), o_nbr, o_cnt)
+    finally:
+        dist.destroy_process_group()
