@@ -263,20 +263,11 @@ k_cell_sort_large(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cel
     }
 }
 
-unsigned grid_for(int64_t work, int threads, int64_t cap)
-{
-    int64_t b = (work + threads - 1) / threads;
-    if (b < 1) b = 1;
-    if (b > cap) b = cap;
-    return (unsigned)b;
-}
-
 }  // namespace
 
 cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const CellGrid &g,
                            cudaStream_t s)
 {
-    const int64_t cap = (int64_t)ctx->sm_count * 8;
     const int64_t scan_tiles = (g.ncell + kScanTile - 1) / kScanTile;
     NL_CUDA_TRY(cudaMemsetAsync(ctx->cell_count, 0, sizeof(int32_t) * g.ncell, s));
     NL_CUDA_TRY(cudaMemsetAsync(ctx->scan_status, 0, sizeof(uint32_t) * scan_tiles, s));
@@ -285,9 +276,8 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
     {
         ProfScope ps(ctx, PH_BIN_COUNT, s);
         if (n > 0)
-            k_bin_count<<<grid_for(n, 256, cap), 256, 0, s>>>(pos, n, g, ctx->atom_cell,
-                                                               ctx->atom_rank, ctx->cell_count,
-                                                               ctx->ref);
+            k_bin_count<<<resident_grid(ctx, k_bin_count, 256, 0, (n + 255) / 256), 256, 0, s>>>(
+                pos, n, g, ctx->atom_cell, ctx->atom_rank, ctx->cell_count, ctx->ref);
         NL_CUDA_TRY(cudaGetLastError());
     }
     {
@@ -299,7 +289,7 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
     if (n <= 0) return cudaSuccess;
     {
         ProfScope ps(ctx, PH_BIN_SCATTER, s);
-        k_bin_scatter<<<grid_for(n, 256, cap), 256, 0, s>>>(pos, n, g, ctx->atom_cell,
+        k_bin_scatter<<<resident_grid(ctx, k_bin_scatter, 256, 0, (n + 255) / 256), 256, 0, s>>>(pos, n, g, ctx->atom_cell,
                                                              ctx->atom_rank, ctx->cell_start,
                                                              ctx->cell_pos);
         NL_CUDA_TRY(cudaGetLastError());
@@ -310,7 +300,11 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
         ProfScope ps(ctx, PH_CELL_SORT, s);
         const float side_x = g.Lx / (float)g.nx;
         NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, sizeof(uint32_t), s));
-        k_cell_sort<<<grid_for(g.ncell * 16, 256, (int64_t)ctx->sm_count * 32), 256, 0, s>>>(
+        // several waves of CTAs over the cells: measured faster than one
+        // resident wave striding over them
+        int64_t sort_blocks = (g.ncell * 16 + 255) / 256;
+        if (sort_blocks > (int64_t)ctx->sm_count * 32) sort_blocks = (int64_t)ctx->sm_count * 32;
+        k_cell_sort<<<(unsigned)sort_blocks, 256, 0, s>>>(
             ctx->cell_pos, ctx->cell_start, g.ncell, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
             ctx->fb_list, ctx->fb_count, ctx->unsorted);
         NL_CUDA_TRY(cudaGetLastError());

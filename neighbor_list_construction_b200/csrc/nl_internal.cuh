@@ -152,6 +152,27 @@ cudaError_t launch_skin(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
 
 }  // namespace nl
 
+namespace nl {
+
+// Grid of a grid-stride kernel: `want` CTAs of `threads` threads, at most
+// one resident wave (the SMs times the CTAs per SM the kernel's registers
+// and shared memory allow), so no CTA waits for a second wave.
+template <class Kernel>
+inline unsigned resident_grid(const nl_ctx *ctx, Kernel kernel, int threads, size_t smem,
+                              int64_t want)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t cap = (int64_t)ctx->sm_count * per_sm;
+    if (want > cap) want = cap;
+    return (unsigned)(want < 1 ? 1 : want);
+}
+
+}  // namespace nl
+
 #define NL_CUDA_TRY(expr)                                   \
     do {                                                    \
         cudaError_t _e = (expr);                            \

@@ -156,9 +156,9 @@ cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
                         const uint32_t *gate)
 {
     if (n <= 0) return cudaSuccess;
-    int64_t blocks = (n + 255) / 256;
-    const int64_t cap = (int64_t)ctx->sm_count * 8;
-    if (blocks > cap) blocks = cap;
+    const int64_t want = (n + 255) / 256;
+    const unsigned blocks = curve == 0 ? resident_grid(ctx, k_keys<0>, 256, 0, want)
+                                       : resident_grid(ctx, k_keys<1>, 256, 0, want);
     if (curve == 0)
         k_keys<0><<<(unsigned)blocks, 256, 0, s>>>(pos, n, Lx, Ly, Lz, Sx, Sy, Sz, ctx->keys[0],
                                                     ctx->vals[0], ctx->hist, gate);

@@ -1224,9 +1224,9 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         return cudaGetLastError();
     }
     ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
-    int64_t blocks = (n + 127) / 128;
-    const int64_t cap = (int64_t)ctx->sm_count * 16;
-    if (blocks > cap) blocks = cap;
+    const unsigned blocks =
+        g.literal ? resident_grid(ctx, k_pairs_per_atom<true, CLOSE>, 128, 0, (n + 127) / 128)
+                  : resident_grid(ctx, k_pairs_per_atom<false, CLOSE>, 128, 0, (n + 127) / 128);
     const float cd2 = CLOSE ? close->close_d2 : 0.0f;
     uint32_t *mb = CLOSE ? reinterpret_cast<uint32_t *>(close->min_d2) : nullptr;
     unsigned long long *nc = CLOSE ? reinterpret_cast<unsigned long long *>(close->n_close) : nullptr;

@@ -68,9 +68,7 @@ cudaError_t launch_resort(nl_ctx *ctx, int64_t n, float4 *pos, int32_t *ids, flo
     }
     {
         ProfScope ps(ctx, PH_GATHER, s);
-        int64_t blocks = (n + 255) / 256;
-        const int64_t cap = (int64_t)ctx->sm_count * 8;
-        if (blocks > cap) blocks = cap;
+        const unsigned blocks = resident_grid(ctx, k_permute_gather, 256, 0, (n + 255) / 256);
         int32_t *ids_tmp = reinterpret_cast<int32_t *>(ctx->atom_cell);
         k_permute_gather<<<(unsigned)blocks, 256, 0, s>>>(n, perm, pos, ctx->cell_pos, ids, ids_tmp,
                                                           aux, ctx->ref);

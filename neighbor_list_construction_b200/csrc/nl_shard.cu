@@ -136,14 +136,6 @@ __global__ void k_map_ids(int64_t entries, int32_t *__restrict__ nbr, const floa
     }
 }
 
-unsigned blocks_for(int64_t work, int sm_count)
-{
-    int64_t b = (work + 255) / 256;
-    if (b < 1) b = 1;
-    const int64_t cap = (int64_t)sm_count * 8;
-    return (unsigned)(b > cap ? cap : b);
-}
-
 bool make_coarse(const float *box, const int32_t dims[3], Coarse *C)
 {
     if (!box || !dims) return false;
@@ -203,7 +195,7 @@ nl_status nl_halo_mark(nl_ctx *ctx, int64_t n, const float *pos, const float *bo
     const int64_t nc = (int64_t)C.nx * C.ny * C.nz;
     if (cudaMemsetAsync(occ_out, 0, sizeof(int32_t) * nc, s) != cudaSuccess) return NL_ERR_CUDA;
     if (n > 0)
-        k_halo_mark<<<blocks_for(n, ctx->sm_count), 256, 0, s>>>(
+        k_halo_mark<<<resident_grid(ctx, k_halo_mark, 256, 0, (n + 255) / 256), 256, 0, s>>>(
             reinterpret_cast<const float4 *>(pos), n, C, 1u << rank, occ_out);
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
 }
@@ -214,7 +206,8 @@ nl_status nl_halo_needed(nl_ctx *ctx, const float *box, const int32_t dims[3],
     Coarse C;
     if (!ctx || !occ_all || !need_out || !make_coarse(box, dims, &C)) return NL_ERR_ARG;
     const int64_t nc = (int64_t)C.nx * C.ny * C.nz;
-    k_halo_needed<<<blocks_for(nc, ctx->sm_count), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+    k_halo_needed<<<resident_grid(ctx, k_halo_needed, 256, 0, (nc + 255) / 256), 256, 0,
+                    reinterpret_cast<cudaStream_t>(stream)>>>(
         C, occ_all, need_out);
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
 }
@@ -232,7 +225,7 @@ nl_status nl_halo_count(nl_ctx *ctx, int64_t n, const float *pos, const float *b
     if (cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * nranks, s) != cudaSuccess)
         return NL_ERR_CUDA;
     if (n > 0)
-        k_halo_count<<<blocks_for(n, ctx->sm_count), 256, 0, s>>>(
+        k_halo_count<<<resident_grid(ctx, k_halo_count, 256, 0, (n + 255) / 256), 256, 0, s>>>(
             reinterpret_cast<const float4 *>(pos), n, C, need, rank, nranks, counts_out);
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
 }
@@ -251,7 +244,7 @@ nl_status nl_halo_fill(nl_ctx *ctx, int64_t n, const float *pos, const float *bo
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(cursor, 0, sizeof(int32_t) * nranks, s) != cudaSuccess) return NL_ERR_CUDA;
     if (n > 0 && send_out)
-        k_halo_fill<<<blocks_for(n, ctx->sm_count), 256, 0, s>>>(
+        k_halo_fill<<<resident_grid(ctx, k_halo_fill, 256, 0, (n + 255) / 256), 256, 0, s>>>(
             reinterpret_cast<const float4 *>(pos), n, C, need, rank, nranks, offsets, counts,
             cursor, reinterpret_cast<float4 *>(send_out));
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
@@ -264,7 +257,8 @@ nl_status nl_map_ids(nl_ctx *ctx, int64_t n_rows, int32_t capacity, int32_t *nbr
     if (n_rows == 0) return NL_OK;
     if (!nbr || !pos_all || (reinterpret_cast<uintptr_t>(pos_all) & 15u)) return NL_ERR_ARG;
     const int64_t entries = n_rows * (int64_t)capacity;
-    k_map_ids<<<blocks_for(entries, ctx->sm_count), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+    k_map_ids<<<resident_grid(ctx, k_map_ids, 256, 0, (entries + 255) / 256), 256, 0,
+                reinterpret_cast<cudaStream_t>(stream)>>>(
         entries, nbr, reinterpret_cast<const float4 *>(pos_all), n_all);
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
 }

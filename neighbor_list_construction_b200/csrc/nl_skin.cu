@@ -68,10 +68,7 @@ cudaError_t launch_skin(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
                         const int32_t *step, unsigned long long cond, cudaStream_t s)
 {
     ProfScope ps(ctx, PH_SKIN, s);
-    int64_t blocks = (n + 255) / 256;
-    const int64_t cap = (int64_t)ctx->sm_count * 8;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
+    const unsigned blocks = resident_grid(ctx, k_skin, 256, 0, (n + 255) / 256);
     k_skin<<<(unsigned)blocks, 256, 0, s>>>(pos, ctx->ref, n, Lx, Ly, Lz, h2, ctx->skin_acc,
                                             rebuild_out, max_d2_out, decisions, step, cond);
     return cudaGetLastError();
