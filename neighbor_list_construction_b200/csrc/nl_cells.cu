@@ -226,11 +226,23 @@ k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_star
     const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    // the next iteration's cell range is loaded one iteration ahead, so only
+    // the position load stays on each iteration's dependent chain
+    int32_t s_next = 0, e_next = 0;
+    if (2 * warp + half < ncell) {
+        s_next = cell_start[2 * warp + half];
+        e_next = cell_start[2 * warp + half + 1];
+    }
     for (int64_t c0 = 2 * warp; c0 < ncell; c0 += 2 * nwarps) {
         const int64_t c = c0 + half;
         const bool have = c < ncell;
-        const int32_t s = have ? cell_start[c] : 0;
-        const int m = have ? cell_start[c + 1] - s : 0;
+        const int32_t s = have ? s_next : 0;
+        const int m = have ? e_next - s_next : 0;
+        const int64_t cn = c + 2 * nwarps;
+        if (cn < ncell) {
+            s_next = cell_start[cn];
+            e_next = cell_start[cn + 1];
+        }
         const float face = (float)(int)(c % nx) * side_x;
         const bool small = m <= 16;
         sort_small_cell(cell_pos, s, small ? m : 0, face, inv_bin, cell_tab + (have ? c : 0) * 16,
