@@ -3,7 +3,8 @@
 // Tessera abstract: atoms are sorted along a space-filling curve (a Morton
 // order is the baseline it is compared against).  The curve here is the
 // 3-D Hilbert curve of J. Skilling, "Programming the Hilbert curve" (AIP
-// Conf. Proc. 707, 2004), on a 2^21 grid per axis, giving 63-bit keys.
+// Conf. Proc. 707, 2004), on a 2^21 grid per axis, giving 63-bit keys,
+// evaluated as a table-driven state machine built from that transform.
 #include "nl_internal.cuh"
 
 namespace nl {
@@ -21,47 +22,106 @@ __device__ __forceinline__ uint64_t spread3(uint32_t a)
     return x;
 }
 
-// Skilling's axes-to-transpose transform for three 21-bit axes, then the
-// transposed index read level by level (x first in each triple).
-__device__ __forceinline__ uint64_t hilbert_index(uint32_t x, uint32_t y, uint32_t z)
+// Skilling's transform as a state machine.  Going down the levels, the
+// axes-to-transpose step at a level only changes the bits below it (it
+// inverts the low bits of axis 0, or exchanges them with those of axis 1 or
+// 2, depending on the level's bits); so every lower level sees the same
+// signed permutation of the three axes, fixed by the levels above.  The Gray
+// code and its correction turn a level's three transposed bits into the
+// key's three bits, with one carried bit: the parity of the third Gray bit
+// over the levels above.  State = (signed permutation, parity): 48 are
+// reachable from the identity.  A step reads one level's octant (x bit, y
+// bit, z bit) and gives the key digit and the next state; the tables here
+// hold one step and two steps (12 bits: next state, two digits).
+struct HState {
+    int pi[3];   // transposed axis i reads input axis pi[i]
+    int f;       // bit i: transposed axis i is inverted
+    int p;       // parity carried by the Gray correction
+};
+
+constexpr bool hstate_eq(const HState &a, const HState &b)
 {
-#pragma unroll
-    for (int l = kQBits - 1; l >= 1; --l) {
-        const uint32_t Q = 1u << l;
-        const uint32_t P = Q - 1u;
-        // axis 0 against itself: the exchange is empty, only the inversion
-        x ^= (x & Q) ? P : 0u;
-        // axis 1: invert the low bits of x, or exchange them with y's
-        uint32_t t = (x ^ y) & P;
-        if (y & Q) {
-            x ^= P;
-        } else {
-            x ^= t;
-            y ^= t;
-        }
-        // axis 2
-        t = (x ^ z) & P;
-        if (z & Q) {
-            x ^= P;
-        } else {
-            x ^= t;
-            z ^= t;
-        }
+    return a.pi[0] == b.pi[0] && a.pi[1] == b.pi[1] && a.pi[2] == b.pi[2] && a.f == b.f &&
+           a.p == b.p;
+}
+
+constexpr HState hstep(const HState &s, int oct, int &digit)
+{
+    const int a[3] = {(oct >> 2) & 1, (oct >> 1) & 1, oct & 1};
+    const int v0 = a[s.pi[0]] ^ (s.f & 1);
+    const int v1 = a[s.pi[1]] ^ ((s.f >> 1) & 1);
+    const int v2 = a[s.pi[2]] ^ ((s.f >> 2) & 1);
+    const int g0 = v0, g1 = v0 ^ v1, g2 = v0 ^ v1 ^ v2;   // Gray code of the level
+    digit = ((g0 ^ s.p) << 2) | ((g1 ^ s.p) << 1) | (g2 ^ s.p);
+    int pi[3] = {s.pi[0], s.pi[1], s.pi[2]};
+    int f[3] = {s.f & 1, (s.f >> 1) & 1, (s.f >> 2) & 1};
+    // the level's operations on the lower bits, axis 0, 1, 2 in turn
+    if (v0) f[0] ^= 1;
+    if (v1) {
+        f[0] ^= 1;
+    } else {
+        const int tp = pi[0], tf = f[0];
+        pi[0] = pi[1]; f[0] = f[1];
+        pi[1] = tp; f[1] = tf;
     }
-    // Gray encode
-    y ^= x;
-    z ^= y;
-    // bit k of the correction = parity of z's bits at levels k+1 .. 20
-    uint32_t t = (z & ~1u) >> 1;
-    t ^= t >> 1;
-    t ^= t >> 2;
-    t ^= t >> 4;
-    t ^= t >> 8;
-    t ^= t >> 16;
-    x ^= t;
-    y ^= t;
-    z ^= t;
-    return (spread3(x) << 2) | (spread3(y) << 1) | spread3(z);
+    if (v2) {
+        f[0] ^= 1;
+    } else {
+        const int tp = pi[0], tf = f[0];
+        pi[0] = pi[2]; f[0] = f[2];
+        pi[2] = tp; f[2] = tf;
+    }
+    return HState{{pi[0], pi[1], pi[2]}, f[0] | (f[1] << 1) | (f[2] << 2), s.p ^ g2};
+}
+
+constexpr int kHStates = 48;
+
+struct HilbertTables {
+    uint16_t one[kHStates * 8];    // (next << 3) | digit
+    uint16_t two[kHStates * 64];   // (next << 6) | (digit of the upper level << 3) | digit
+};
+
+constexpr HilbertTables make_hilbert_tables()
+{
+    HilbertTables t{};
+    HState st[kHStates] = {};
+    int ns = 1;
+    st[0] = HState{{0, 1, 2}, 0, 0};
+    for (int i = 0; i < ns; ++i)
+        for (int o = 0; o < 8; ++o) {
+            int d = 0;
+            const HState n = hstep(st[i], o, d);
+            int j = 0;
+            while (j < ns && !hstate_eq(st[j], n)) ++j;
+            if (j == ns) st[ns++] = n;   // more than kHStates would not compile
+            t.one[i * 8 + o] = (uint16_t)((j << 3) | d);
+        }
+    for (int i = 0; i < kHStates; ++i)
+        for (int o = 0; o < 64; ++o) {
+            const int e1 = t.one[i * 8 + (o >> 3)];
+            const int e2 = t.one[(e1 >> 3) * 8 + (o & 7)];
+            t.two[i * 64 + o] = (uint16_t)(((e2 >> 3) << 6) | ((e1 & 7) << 3) | (e2 & 7));
+        }
+    return t;
+}
+
+__device__ const HilbertTables g_hilbert = make_hilbert_tables();
+
+// 63-bit Hilbert key of (x, y, z) from the octants of the Morton code m:
+// the top level by one step, the other 20 by two-level steps.
+__device__ __forceinline__ uint64_t hilbert_index(uint64_t m, const uint16_t *one,
+                                                  const uint16_t *two)
+{
+    uint32_t e = one[(uint32_t)(m >> 60) & 7u];   // from state 0
+    uint64_t k = e & 7u;
+    uint32_t s = e >> 3;
+#pragma unroll
+    for (int l = 19; l >= 1; l -= 2) {
+        e = two[s * 64u + ((uint32_t)(m >> (3 * (l - 1))) & 63u)];
+        k = (k << 6) | (e & 63u);
+        s = e >> 6;
+    }
+    return k;
 }
 
 __device__ __forceinline__ uint64_t morton_index(uint32_t x, uint32_t y, uint32_t z)
@@ -95,6 +155,12 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
     const int d0 = recompute ? 0 : kLow;
     const int d1 = recompute ? kLow : kKeyPasses;
     __shared__ uint32_t sh[kKeyPasses * kRadixBins];
+    __shared__ uint16_t s_one[kHStates * 8];
+    __shared__ uint16_t s_two[kHStates * 64];
+    if (CURVE == 0) {
+        for (int i = threadIdx.x; i < kHStates * 8; i += blockDim.x) s_one[i] = g_hilbert.one[i];
+        for (int i = threadIdx.x; i < kHStates * 64; i += blockDim.x) s_two[i] = g_hilbert.two[i];
+    }
     for (int i = threadIdx.x; i < kKeyPasses * kRadixBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -103,7 +169,8 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
         const uint32_t qx = quantize(wrap_coord(p.x, Lx), Sx);
         const uint32_t qy = quantize(wrap_coord(p.y, Ly), Sy);
         const uint32_t qz = quantize(wrap_coord(p.z, Lz), Sz);
-        const uint64_t k = CURVE == 0 ? hilbert_index(qx, qy, qz) : morton_index(qx, qy, qz);
+        const uint64_t m = morton_index(qx, qy, qz);
+        const uint64_t k = CURVE == 0 ? hilbert_index(m, s_one, s_two) : m;
         keys[i] = k;
         vals[i] = (uint32_t)i;
         for (int d = d0; d < d1; ++d)
