@@ -205,14 +205,30 @@ __global__ void __launch_bounds__(256) k_hist_scan(uint32_t *hist, const uint32_
     h[t] = before + x - v;
 }
 
-__global__ void k_gather(int64_t n, const float4 *__restrict__ pos, const int32_t *__restrict__ perm,
-                         float4 *__restrict__ out)
+// Each thread gathers kGatherItems elements of its CTA's block, issuing all
+// index loads and then all (random) position loads before any store, so a
+// warp keeps several gathers in flight.
+constexpr int kGatherItems = 4;
+
+__global__ void __launch_bounds__(256)
+k_gather(int64_t n, const float4 *__restrict__ pos, const int32_t *__restrict__ perm,
+         float4 *__restrict__ out)
 {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride) {
-        const int32_t i = perm[k];
-        const float4 p = pos[i];
-        out[k] = make_float4(p.x, p.y, p.z, __int_as_float(i));
+    const int64_t base = (int64_t)blockIdx.x * (256 * kGatherItems) + threadIdx.x;
+    int32_t i[kGatherItems];
+#pragma unroll
+    for (int u = 0; u < kGatherItems; ++u) {
+        const int64_t k = base + 256 * u;
+        i[u] = k < n ? perm[k] : -1;
+    }
+    float4 p[kGatherItems];
+#pragma unroll
+    for (int u = 0; u < kGatherItems; ++u)
+        if (i[u] >= 0) p[u] = pos[i[u]];
+#pragma unroll
+    for (int u = 0; u < kGatherItems; ++u) {
+        const int64_t k = base + 256 * u;
+        if (k < n) out[k] = make_float4(p[u].x, p[u].y, p[u].z, __int_as_float(i[u]));
     }
 }
 
@@ -247,8 +263,7 @@ cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, flo
                           cudaStream_t s)
 {
     if (n <= 0) return cudaSuccess;
-    int64_t blocks = (n + 255) / 256;
-    if (blocks > 65535 * 8) blocks = 65535 * 8;
+    const int64_t blocks = (n + 256 * kGatherItems - 1) / (256 * kGatherItems);
     k_gather<<<(unsigned)blocks, 256, 0, s>>>(n, pos, perm, out);
     return cudaGetLastError();
 }
