@@ -34,8 +34,8 @@ NOMINAL_HBM_GBS = 8000.0
 # belongs to the kernel source it was taken on (nl_pairs.cu and the device
 # header it includes): with any other source the bench reports null.
 PAIR_TRAFFIC = {"workload": "saltwater10m",
-                "sha256": "05dcfffb7fc577ba2b99f9b61e3cce4d117adf88aa34f35fa88c8b2dce84fa15",
-                "bytes": 803095808 + 10746583296}
+                "sha256": "20146b9e86ec65bcf0de0fc92b781b5d5053aeb8ae9436f50e1758f91501f971",
+                "bytes": 826731264 + 10761926400}
 
 
 def pair_traffic(workload: str):
