@@ -155,6 +155,49 @@ def test_build_small_boxes(ctx, oracle, box, cutoff, skin):
     gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
 
 
+@pytest.mark.parametrize("case", ["one_atom", "two_coincident", "all_coincident",
+                                  "on_the_faces", "far_outside", "cutoff_zero_skin"])
+def test_build_degenerate_inputs(ctx, oracle, case):
+    """Inputs at the edges of the definition: a single atom, coincident atoms
+    (r2 = 0 < rl2: neighbors of each other), every atom at one point (rows of
+    n - 1), atoms exactly on the box faces (x = 0 and x = L wrap together),
+    coordinates many boxes away, and rl = skin alone (cutoff 0)."""
+    rng = np.random.default_rng(31)
+    box = np.array([20.0, 22.0, 24.0], np.float32)
+    cutoff, skin, K = 2.5, 0.5, 64
+    if case == "one_atom":
+        pos = np.zeros((1, 4), np.float32)
+        pos[0, :3] = [3.0, 4.0, 5.0]
+    elif case == "two_coincident":
+        pos = np.zeros((2, 4), np.float32)
+        pos[:, :3] = [7.0, 7.0, 7.0]
+    elif case == "all_coincident":
+        pos = np.zeros((50, 4), np.float32)
+        pos[:, :3] = [1.0, 21.5, 0.0]
+    elif case == "on_the_faces":
+        n = 600
+        pos = np.zeros((n, 4), np.float32)
+        pos[:, :3] = rng.random((n, 3)) * box
+        face = rng.integers(0, 3, n)
+        side = rng.integers(0, 2, n).astype(np.float32)
+        pos[np.arange(n), face] = side * box[face]
+    elif case == "far_outside":
+        n = 800
+        pos = np.zeros((n, 4), np.float32)
+        pos[:, :3] = (rng.random((n, 3)) * 2.0 - 1.0) * box * 40.0
+    else:
+        cutoff, skin = 0.0, 3.0
+        n = 900
+        pos = np.zeros((n, 4), np.float32)
+        pos[:, :3] = rng.random((n, 3)) * box
+    nbr, cnt, st = gpu_build(ctx, pos, box, cutoff, skin, K)
+    o_nbr, o_cnt, o_ov = oracle.build(pos, box, cutoff, skin, K)
+    assert st == (1 if o_ov else 0)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+    if case == "all_coincident":
+        assert np.all(cnt == 49)
+
+
 def test_build_golden_fixtures(ctx):
     import glob
     import json
