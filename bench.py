@@ -586,6 +586,81 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     ctx.close()
 
 
+def run_sharded(args, rank: int, world: int, local_rank: int) -> None:
+    """The pages' multi-GPU design (opt-in, --sharded): the whole workload is
+    sorted along the curve and cut into `world` equal-count shards, one per
+    rank; a timed step is every rank's halo build (coarse-cell marks, an
+    all-reduce, counts and atoms by all-to-all, nl_build_rows over own + halo
+    atoms, global ids).  Total work is fixed: "scaling": "strong"."""
+    import torch
+    import torch.distributed as dist
+    from neighbor_list_construction_b200 import nl, shard, workloads
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    torch.cuda.set_device(local_rank)
+    w = workloads.make(args.workload)
+    n, K = w.n, w.capacity
+    bounds = shard.shard_bounds(n, world)
+    s0, s1 = bounds[rank]
+    ctx = nl.Context(n, K)
+    pos = torch.from_numpy(w.pos).cuda()
+    perm, ps, _ = ctx.sort(pos, w.box)
+    own = shard.with_ids(ps[s0:s1].contiguous(), s0)
+    del perm, ps, pos
+    comm = shard.DistExchange() if world > 1 else None
+
+    def step():
+        if comm is not None:
+            return shard.build_sharded(ctx, own, w.box, w.cutoff, w.skin, K, comm)
+        return shard.build_sharded_local(ctx, [own], w.box, w.cutoff, w.skin, K)[0]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        res = step()
+    halo = res[2]
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.monotonic()
+    e0.record()
+    for _ in range(args.steps):
+        res = step()
+    e1.record()
+    barrier()
+    clk = clocks.window(t_host0, time.monotonic())
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        h = torch.tensor([halo], dtype=torch.int64, device="cuda")
+        dist.all_reduce(h, op=dist.ReduceOp.SUM)
+        halo_total = int(h.item())
+    else:
+        halo_total = halo
+    st = ctx.sync_status()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": n / (ms * 1e-3), "unit": "atoms/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": dict(arm_config(args.workload, world),
+                           parallelism=f"curve shards x{world}, halo exchange",
+                           step="halo build: marks, all-reduce, all-to-all, nl_build_rows"),
+            "halo_atoms_total": halo_total, "halo_fraction": halo_total / n,
+            "clocks": clk, "status": nl.nl_status_string(st),
+        }
+        print(json.dumps(line), flush=True)
+    clocks.stop()
+    del own
+    ctx.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -596,6 +671,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--curve", default="hilbert", choices=["hilbert", "morton"],
                     help="curve of the sort in the timed step (Morton: the pages' baseline order)")
+    ap.add_argument("--sharded", action="store_true",
+                    help="time the pages' multi-GPU design instead of replicas: equal-count "
+                         "curve shards of the one workload, halo exchange over NCCL")
     ap.add_argument("--extras", action="store_true",
                     help="also time the replayed skin-check interval (graph vs eager) "
                          "and nl_build after Hilbert vs Morton order")
@@ -616,7 +694,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_gpu(args, rank, world, local_rank)
+        if args.sharded:
+            run_sharded(args, rank, world, local_rank)
+        else:
+            run_gpu(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -68,9 +68,11 @@ nl_status nl_halo_fill(nl_ctx *ctx, int64_t n, const float *pos, const float *bo
 
 /* In place: every entry j >= 0 of the n_rows x capacity rows nbr (indices
  * into pos_all, n_all atoms) becomes the global id in pos_all[j]'s fourth
- * float; -1 stays. */
+ * float; -1 stays.  counts (device int32[n_rows], the build's) may be NULL;
+ * given, only the first min(counts[i], capacity) entries of row i are read,
+ * which is all a build writes before its -1 padding. */
 nl_status nl_map_ids(nl_ctx *ctx, int64_t n_rows, int32_t capacity, int32_t *nbr,
-                     int64_t n_all, const float *pos_all, void *stream);
+                     const int32_t *counts, int64_t n_all, const float *pos_all, void *stream);
 
 #ifdef __cplusplus
 }

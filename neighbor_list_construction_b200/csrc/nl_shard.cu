@@ -125,7 +125,8 @@ __global__ void k_halo_fill(const float4 *__restrict__ pos, int64_t n, Coarse C,
 }
 
 // Row entries (indices into pos_all) replaced by the global ids in the
-// fourth lane of pos_all; -1 stays.
+// fourth lane of pos_all; -1 stays.  With counts, a warp takes a row and
+// maps its first min(count, K) entries only (the rest is -1).
 __global__ void k_map_ids(int64_t entries, int32_t *__restrict__ nbr, const float4 *__restrict__ pos_all,
                           int64_t n_all)
 {
@@ -133,6 +134,23 @@ __global__ void k_map_ids(int64_t entries, int32_t *__restrict__ nbr, const floa
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < entries; e += stride) {
         const int32_t j = nbr[e];
         if (j >= 0 && j < n_all) nbr[e] = __float_as_int(pos_all[j].w);
+    }
+}
+
+__global__ void k_map_ids_rows(int64_t n_rows, int32_t K, int32_t *__restrict__ nbr,
+                               const int32_t *__restrict__ counts,
+                               const float4 *__restrict__ pos_all, int64_t n_all)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n_rows; i += nw) {
+        int32_t c = counts[i];
+        c = c < K ? c : K;
+        int32_t *row = nbr + i * (int64_t)K;
+        for (int32_t s = lane; s < c; s += 32) {
+            const int32_t j = row[s];
+            if (j >= 0 && j < n_all) row[s] = __float_as_int(pos_all[j].w);
+        }
     }
 }
 
@@ -251,15 +269,21 @@ nl_status nl_halo_fill(nl_ctx *ctx, int64_t n, const float *pos, const float *bo
 }
 
 nl_status nl_map_ids(nl_ctx *ctx, int64_t n_rows, int32_t capacity, int32_t *nbr,
-                     int64_t n_all, const float *pos_all, void *stream)
+                     const int32_t *counts, int64_t n_all, const float *pos_all, void *stream)
 {
     if (!ctx || n_rows < 0 || capacity < 1 || n_all < 0) return NL_ERR_ARG;
     if (n_rows == 0) return NL_OK;
     if (!nbr || !pos_all || (reinterpret_cast<uintptr_t>(pos_all) & 15u)) return NL_ERR_ARG;
-    const int64_t entries = n_rows * (int64_t)capacity;
-    k_map_ids<<<resident_grid(ctx, k_map_ids, 256, 0, (entries + 255) / 256), 256, 0,
-                reinterpret_cast<cudaStream_t>(stream)>>>(
-        entries, nbr, reinterpret_cast<const float4 *>(pos_all), n_all);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const float4 *p4 = reinterpret_cast<const float4 *>(pos_all);
+    if (counts) {
+        k_map_ids_rows<<<resident_grid(ctx, k_map_ids_rows, 256, 0, (n_rows + 7) / 8), 256, 0, s>>>(
+            n_rows, capacity, nbr, counts, p4, n_all);
+    } else {
+        const int64_t entries = n_rows * (int64_t)capacity;
+        k_map_ids<<<resident_grid(ctx, k_map_ids, 256, 0, (entries + 255) / 256), 256, 0, s>>>(
+            entries, nbr, p4, n_all);
+    }
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
 }
 

@@ -53,7 +53,7 @@ _SIGS = {
     "nl_halo_needed": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_halo_count": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp]),
     "nl_halo_fill": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
-    "nl_map_ids": (_i32, [_vp, _i64, _i32, _vp, _i64, _vp, _vp]),
+    "nl_map_ids": (_i32, [_vp, _i64, _i32, _vp, _vp, _i64, _vp, _vp]),
     "nls_displace": (_i32, [_i64, _vp, _u64, _i64, _vp, _f32, _vp]),
     "nls_step_graph": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _u64, _vp, _f32]),
     "nls_step_graph_ids": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _vp, _u64, _vp, _f32]),
@@ -253,9 +253,9 @@ def nl_halo_fill(ctx, pos, box, dims, need, rank, nranks, offsets, counts, curso
                   "nl_halo_fill")
 
 
-def nl_map_ids(ctx, nbr, pos_all, stream=None) -> int:
+def nl_map_ids(ctx, nbr, pos_all, counts=None, stream=None) -> int:
     _pos(pos_all)
-    return _check(_lib.nl_map_ids(ctx, nbr.shape[0], int(nbr.shape[1]), _ptr(nbr),
+    return _check(_lib.nl_map_ids(ctx, nbr.shape[0], int(nbr.shape[1]), _ptr(nbr), _ptr(counts),
                                   pos_all.shape[0], _ptr(pos_all), _stream(stream)), "nl_map_ids")
 
 

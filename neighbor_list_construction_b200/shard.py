@@ -83,7 +83,7 @@ def _steps(ctx, pos_own, box, cutoff, skin, capacity, rank, nranks):
     pos_all = torch.cat([pos_own, halo]) if halo.shape[0] else pos_own
     nbr, cnt = ctx.build_rows(pos_all, n_own, box, cutoff, skin, capacity)
     if n_own:
-        nl.nl_map_ids(ctx.handle, nbr, pos_all)
+        nl.nl_map_ids(ctx.handle, nbr, pos_all, cnt)
     return nbr, cnt, int(halo.shape[0])
 
 
