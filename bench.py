@@ -354,9 +354,31 @@ def edge_feature_timing(nl, torch, h, ps, w, K, reps: int = 5) -> dict:
     peak = measured_peaks()
     gbs = alg / (ms * 1e-3) / 1e9
     del out
+    # the CSR form with features: offsets, entries and (dx, dy, dz, r) per
+    # entry, no padding.  Algorithmic bytes: counts, positions and offsets
+    # (4 + 16 + 8 per atom), index in and index + feature out (4 + 20 per entry)
+    row_ptr = torch.empty(n + 1, dtype=torch.int64, device="cuda")
+    nl.nl_csr_offsets(h, cnt, K, row_ptr, stream)
+    E = int(row_ptr[n].item())
+    col = torch.empty(E, dtype=torch.int32, device="cuda")
+    feat = torch.empty(E, 4, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        nl.nl_csr_offsets(h, cnt, K, row_ptr, stream)
+        nl.nl_csr_fill(h, nbr, cnt, row_ptr, col, ps, w.box, feat, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    csr_ms = e0.elapsed_time(e1) / reps
+    csr_alg = n * (4 + 16 + 8) + E * (4 + 4 + 16)
+    csr_gbs = csr_alg / (csr_ms * 1e-3) / 1e9
+    del col, feat, row_ptr
     return {"ms": ms, "bytes": alg, "achieved_gbs": gbs, "peak_gbs": peak["hbm_gbs"],
             "peak_source": peak["source"], "frac": gbs / peak["hbm_gbs"],
-            "layout": f"float32 [{n}, {K}, 4] (dx, dy, dz, r), zero padding"}
+            "layout": f"float32 [{n}, {K}, 4] (dx, dy, dz, r), zero padding",
+            "csr": {"ms": csr_ms, "entries": E, "bytes": csr_alg, "achieved_gbs": csr_gbs,
+                    "frac": csr_gbs / peak["hbm_gbs"],
+                    "layout": f"int64 row_ptr [{n + 1}], int32 col [{E}], float32 [{E}, 4]"}}
 
 
 def sharded_timing(torch, ctx, ps, w, K, nranks: int = 8, reps: int = 2) -> dict:

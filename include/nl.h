@@ -151,6 +151,26 @@ nl_status nl_edge_features(nl_ctx *ctx, int64_t n, const float *pos, const float
                            const int32_t *nbr, const int32_t *counts, int32_t capacity,
                            float *edges_out, void *stream);
 
+/* Compressed-sparse-row form of padded rows, in two calls (the number of
+ * entries is known on the device only after the first):
+ *   nl_csr_offsets: row_ptr_out (device int64[n + 1]) = 0 followed by the
+ *     running sum of v_i = min(max(counts[i], 0), capacity), the valid
+ *     entries of row i; row_ptr_out[n] = E, all valid entries.
+ *   nl_csr_fill: col_out (device int32[E]) gets the first v_i entries of
+ *     row i at row_ptr[i] ..; when edges_out is not NULL (device float32
+ *     [E][4], 16-byte aligned) each entry also gets its edge feature, the
+ *     value nl_edge_features writes for its slot (pos and box as there).
+ * nbr, counts, capacity as nl_build writes them (any rows of that shape are
+ * accepted).  n > max_atoms of the context is NL_ERR_CAPACITY; NULL
+ * pointers (where needed), misalignment or a bad box are NL_ERR_ARG.  The
+ * offsets use the context's sort scratch, so they must not run concurrently
+ * with a sort of the same context. */
+nl_status nl_csr_offsets(nl_ctx *ctx, int64_t n, const int32_t *counts, int32_t capacity,
+                         int64_t *row_ptr_out, void *stream);
+nl_status nl_csr_fill(nl_ctx *ctx, int64_t n, const int32_t *nbr, const int32_t *counts,
+                      int32_t capacity, const int64_t *row_ptr, int32_t *col_out,
+                      const float *pos, const float *box, float *edges_out, void *stream);
+
 /* Skin check (Tessera abstract: a conservative neighbor skin preserves the
  * topology across updates).  m = max over atoms of the squared minimum-image
  * displacement between `pos` and the positions of the last nl_build (raw,

@@ -637,6 +637,37 @@ nl_status replay_impl(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n,
 
 extern "C" {
 
+nl_status nl_csr_offsets(nl_ctx *ctx, int64_t n, const int32_t *counts, int32_t capacity,
+                         int64_t *row_ptr_out, void *stream)
+{
+    if (!ctx || n < 0 || capacity < 1 || !row_ptr_out || (n > 0 && !counts)) return NL_ERR_ARG;
+    if (n > ctx->max_atoms) return NL_ERR_CAPACITY;
+    // the sort's look-back words serve as the scan's block sums (int64)
+    static_assert(sizeof(int64_t) == 2 * sizeof(uint32_t), "int64 block sums");
+    if (launch_csr_offsets(ctx, n, counts, capacity, row_ptr_out,
+                           reinterpret_cast<int64_t *>(ctx->sort_status), S(stream)) != cudaSuccess)
+        return NL_ERR_CUDA;
+    return NL_OK;
+}
+
+nl_status nl_csr_fill(nl_ctx *ctx, int64_t n, const int32_t *nbr, const int32_t *counts,
+                      int32_t capacity, const int64_t *row_ptr, int32_t *col_out,
+                      const float *pos, const float *box, float *edges_out, void *stream)
+{
+    if (!ctx || n < 0 || capacity < 1) return NL_ERR_ARG;
+    if (n > 0 && (!nbr || !counts || !row_ptr || !col_out)) return NL_ERR_ARG;
+    if (edges_out && (check_box(box) != NL_OK || (n > 0 && (!pos || !aligned16(pos))) ||
+                      !aligned16(edges_out)))
+        return NL_ERR_ARG;
+    const float Lx = edges_out ? box[0] : 1.0f, Ly = edges_out ? box[1] : 1.0f,
+                Lz = edges_out ? box[2] : 1.0f;
+    if (launch_csr_fill(ctx, n, nbr, counts, capacity, row_ptr, col_out,
+                        reinterpret_cast<const float4 *>(pos), Lx, Ly, Lz,
+                        reinterpret_cast<float4 *>(edges_out), S(stream)) != cudaSuccess)
+        return NL_ERR_CUDA;
+    return NL_OK;
+}
+
 nl_status nl_replay(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n, float *pos,
                     const float *box, float cutoff, float skin, int32_t capacity, int32_t *nbr,
                     int32_t *counts, int32_t *decisions_out, void *stream)

@@ -139,6 +139,16 @@ cudaError_t launch_resort(nl_ctx *ctx, int64_t n, float4 *pos, int32_t *ids, flo
                           float Lx, float Ly, float Lz, float Sx, float Sy, float Sz,
                           cudaStream_t s);
 
+// CSR form of padded rows: offsets (int64 row_ptr[n + 1]; block_sums is
+// scratch of csr_block_count(n) int64), then entries and, with edges, their
+// features.
+cudaError_t launch_csr_offsets(nl_ctx *ctx, int64_t n, const int32_t *counts, int32_t K,
+                               int64_t *row_ptr, int64_t *block_sums, cudaStream_t s);
+int64_t csr_block_count(int64_t n);
+cudaError_t launch_csr_fill(nl_ctx *ctx, int64_t n, const int32_t *nbr, const int32_t *counts,
+                            int32_t K, const int64_t *row_ptr, int32_t *col, const float4 *pos,
+                            float Lx, float Ly, float Lz, float4 *edges, cudaStream_t s);
+
 // Edge features (dx, dy, dz, r) of padded rows into out[n][K].
 cudaError_t launch_edge_features(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
                                  float Lz, const int32_t *nbr, const int32_t *counts, int32_t K,

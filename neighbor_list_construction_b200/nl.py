@@ -36,6 +36,8 @@ _SIGS = {
     "nl_build_close": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _f32, _vp, _vp,
                               _vp]),
     "nl_skin_check": (_i32, [_vp, _i64, _vp, _vp, _f32, _vp, _vp, _vp]),
+    "nl_csr_offsets": (_i32, [_vp, _i64, _vp, _i32, _vp, _vp]),
+    "nl_csr_fill": (_i32, [_vp, _i64, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_edge_features": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp, _vp]),
     "nl_replay": (_i32, [_vp, _vp, _i32, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp, _vp]),
     "nl_replay_resort": (_i32, [_vp, _vp, _i32, _i64, _vp, _vp, _vp, _vp, _f32, _f32, _i32, _vp,
@@ -175,6 +177,33 @@ def nl_skin_check(ctx, pos, box, skin, rebuild_out, max_d2_out=None, stream=None
     return _check(_lib.nl_skin_check(ctx, pos.shape[0], _ptr(pos), _box(box), float(skin),
                                      _ptr(rebuild_out), _ptr(max_d2_out), _stream(stream)),
                   "nl_skin_check")
+
+
+def nl_csr_offsets(ctx, counts, capacity, row_ptr_out, stream=None) -> int:
+    if counts.dtype != torch.int32 or counts.dim() != 1:
+        raise ValueError("counts must be an int32 [n] CUDA tensor")
+    n = counts.shape[0]
+    if row_ptr_out.dtype != torch.int64 or tuple(row_ptr_out.shape) != (n + 1,):
+        raise ValueError("row_ptr_out must be an int64 [n + 1] CUDA tensor")
+    return _check(_lib.nl_csr_offsets(ctx, n, _ptr(counts), int(capacity), _ptr(row_ptr_out),
+                                      _stream(stream)), "nl_csr_offsets")
+
+
+def nl_csr_fill(ctx, nbr, counts, row_ptr, col_out, pos=None, box=None, edges_out=None,
+                stream=None) -> int:
+    n, K = nbr.shape
+    if nbr.dtype != torch.int32 or counts.dtype != torch.int32 or tuple(counts.shape) != (n,):
+        raise ValueError("nbr must be int32 [n, K] and counts int32 [n]")
+    if col_out.dtype != torch.int32 or row_ptr.dtype != torch.int64:
+        raise ValueError("col_out must be int32 and row_ptr int64")
+    if edges_out is not None:
+        _pos(pos)
+        if edges_out.dtype != torch.float32 or edges_out.dim() != 2 or edges_out.shape[1] != 4:
+            raise ValueError("edges_out must be a float32 [E, 4] CUDA tensor")
+    bx = _box(box) if box is not None else None
+    return _check(_lib.nl_csr_fill(ctx, n, _ptr(nbr), _ptr(counts), int(K), _ptr(row_ptr),
+                                   _ptr(col_out), _ptr(pos), bx, _ptr(edges_out),
+                                   _stream(stream)), "nl_csr_fill")
 
 
 def nl_edge_features(ctx, pos, box, nbr, counts, edges_out, stream=None) -> int:
@@ -373,6 +402,22 @@ class Context:
         nl_build_close(self.handle, pos, box, cutoff, skin, capacity, nbr, counts, close_d2, mn,
                        nc, stream)
         return nbr, counts, mn, nc
+
+    def to_csr(self, nbr, counts, pos=None, box=None, stream=None):
+        """CSR form of the rows: (row_ptr int64 [n + 1], col int32 [E]) and,
+        with pos and box, the entries' edge features float32 [E, 4]."""
+        n, K = nbr.shape
+        row_ptr = torch.empty(n + 1, dtype=torch.int64, device=nbr.device)
+        nl_csr_offsets(self.handle, counts, K, row_ptr, stream)
+        E = int(row_ptr[n].item())
+        # at least one element, so the buffers have an address when E = 0
+        col = torch.empty(max(E, 1), dtype=torch.int32, device=nbr.device)
+        edges = None
+        if pos is not None:
+            edges = torch.empty(max(E, 1), 4, dtype=torch.float32, device=nbr.device)
+        nl_csr_fill(self.handle, nbr, counts, row_ptr, col, pos, box, edges, stream)
+        col = col[:E]
+        return (row_ptr, col) if edges is None else (row_ptr, col, edges[:E])
 
     def edge_features(self, pos, box, nbr, counts, stream=None):
         """Per-slot (dx, dy, dz, r) of the rows: float32 [n, K, 4]."""

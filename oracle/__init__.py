@@ -232,6 +232,19 @@ def edge_features(pos, box, nbr, counts) -> np.ndarray:
     return out
 
 
+def csr(nbr, counts):
+    """Compressed-sparse-row form of padded rows: row_ptr (int64 [n + 1]) =
+    0 and the running sum of v_i = min(max(counts[i], 0), K); col = the first
+    v_i entries of each row, row after row."""
+    nb = np.ascontiguousarray(nbr, dtype=np.int32)
+    n, K = nb.shape
+    v = np.clip(np.asarray(counts, np.int64), 0, K)
+    row_ptr = np.zeros(n + 1, np.int64)
+    np.cumsum(v, out=row_ptr[1:])
+    keep = np.arange(K)[None, :] < v[:, None]
+    return row_ptr, nb[keep]
+
+
 def skin_check(pos, ref, box, skin: float):
     """Returns (max squared displacement, rebuild flag)."""
     p = _pos4(pos)

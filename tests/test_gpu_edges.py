@@ -230,3 +230,52 @@ def test_edges_cutoff_shell(ctx, oracle):
     pos[nb:, :3] = base + rl * (1.0 + rng.uniform(-3e-7, 3e-7, size=(nb, 1))) * u
     box = np.array([L, L, L], np.float32)
     check_rows_and_edges(ctx, oracle, pos, box, cutoff, skin, 256)
+
+
+# ----------------------------------------------------------------- CSR form
+@pytest.mark.parametrize("K", [1, 33, 100])
+def test_csr_of_arbitrary_rows(ctx, oracle, K):
+    """to_csr on synthetic rows (indices -1 and n, counts above K, zero and
+    negative): offsets and entries equal the oracle's CSR form, and each
+    entry's feature equals the oracle's feature of its slot."""
+    rng = np.random.default_rng(100 + K)
+    n = 2501
+    box = np.array([31.0, 17.5, 23.25], np.float32)
+    pos = np.zeros((n, 4), np.float32)
+    pos[:, :3] = (rng.random((n, 3)) * 2.2 - 0.6) * box
+    nbr = rng.integers(0, n, (n, K)).astype(np.int32)
+    nbr[rng.random((n, K)) < 0.05] = -1
+    nbr[rng.random((n, K)) < 0.02] = n
+    cnt = rng.integers(-3, K + 5, n).astype(np.int32)
+    row_ptr, col, e = ctx.to_csr(dev(nbr), dev(cnt), dev(pos), box)
+    assert ctx.sync_status() == 0
+    o_ptr, o_col = oracle.csr(nbr, cnt)
+    np.testing.assert_array_equal(row_ptr.cpu().numpy(), o_ptr)
+    np.testing.assert_array_equal(col.cpu().numpy(), o_col)
+    keep = np.arange(K)[None, :] < np.clip(cnt, 0, K)[:, None]
+    o_e = oracle.edge_features(pos, box, nbr, cnt)[keep]
+    np.testing.assert_array_equal(bits(e.cpu().numpy()), bits(o_e))
+    r2, c2 = ctx.to_csr(dev(nbr), dev(cnt))          # entries only
+    assert torch.equal(r2, row_ptr) and torch.equal(c2, col)
+
+
+def test_csr_empty(ctx):
+    nbr = torch.zeros(0, 8, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(0, dtype=torch.int32, device="cuda")
+    row_ptr, col = ctx.to_csr(nbr, cnt)
+    assert row_ptr.tolist() == [0] and col.numel() == 0
+
+
+def test_csr_full_size(ctx):
+    """saltwater10m rows (1.29 G entries, past 2^30: the offsets are int64):
+    the CSR form equals the rows' valid prefixes, row after row."""
+    w = gu.workload("saltwater10m")
+    p = dev(gu.oracle_sorted("saltwater10m"))
+    nbr, cnt = ctx.build(p, w.box, w.cutoff, w.skin, w.capacity)
+    row_ptr, col = ctx.to_csr(nbr, cnt)
+    assert ctx.sync_status() == 0
+    v = cnt.clamp(min=0, max=w.capacity).to(torch.int64)
+    assert int(row_ptr[-1].item()) == int(v.sum().item()) > 2 ** 30
+    assert torch.equal(row_ptr[1:], torch.cumsum(v, 0))
+    keep = torch.arange(w.capacity, device="cuda")[None, :] < v[:, None]
+    assert torch.equal(col, nbr[keep])

@@ -141,3 +141,38 @@ def test_edges_padding_overflow_and_bad_indices():
     e2 = oracle.edge_features(pos, box, bad, np.maximum(cnt, 1))
     np.testing.assert_array_equal(e2[0, 0], 0.0)
     np.testing.assert_array_equal(e2[1, 0], 0.0)
+
+
+def test_csr_matches_a_loop_over_rows():
+    """The oracle's CSR form against a plain loop: offsets are the running
+    sum of the valid entries, entries are the rows' valid prefixes."""
+    rng = np.random.default_rng(12)
+    for n, K in [(0, 4), (1, 1), (37, 5), (300, 16)]:
+        nbr = rng.integers(-1, 1000, (n, K)).astype(np.int32)
+        cnt = rng.integers(-2, K + 4, n).astype(np.int32)
+        row_ptr, col = oracle.csr(nbr, cnt)
+        want_ptr, want_col = [0], []
+        for i in range(n):
+            v = min(max(int(cnt[i]), 0), K)
+            want_col.extend(int(x) for x in nbr[i, :v])
+            want_ptr.append(want_ptr[-1] + v)
+        assert row_ptr.dtype == np.int64 and col.dtype == np.int32
+        np.testing.assert_array_equal(row_ptr, want_ptr)
+        np.testing.assert_array_equal(col, np.array(want_col, np.int32))
+
+
+def test_csr_of_built_rows_round_trips():
+    """Rows rebuilt from the CSR form of an oracle build, padded with -1,
+    are the build's rows."""
+    rng = np.random.default_rng(13)
+    box = np.array([9.0, 9.0, 9.0], np.float32)
+    pos = np.zeros((200, 4), np.float32)
+    pos[:, :3] = rng.random((200, 3)) * box
+    for K in (8, 64):
+        nbr, cnt, _ = oracle.build(pos, box, 2.0, 0.5, K)
+        row_ptr, col = oracle.csr(nbr, cnt)
+        back = np.full_like(nbr, -1)
+        for i in range(nbr.shape[0]):
+            seg = col[row_ptr[i]:row_ptr[i + 1]]
+            back[i, :seg.size] = seg
+        np.testing.assert_array_equal(back, nbr)
