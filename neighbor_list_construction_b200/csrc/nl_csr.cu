@@ -108,8 +108,12 @@ __device__ __forceinline__ float3 wrap3(const float4 p, float Lx, float Ly, floa
 }
 
 // One warp per row: the row's valid entries to col[row_ptr[i] ...] and,
-// when edges is set, their features (as the edge-feature kernel).
-__global__ void __launch_bounds__(256)
+// when edges is set, their features (as the edge-feature kernel).  Each lane
+// issues the index loads and position gathers of kFillUnroll entries before
+// it uses any.
+constexpr int kFillUnroll = 8;
+
+__global__ void __launch_bounds__(128)
 k_csr_fill(int64_t n, const int32_t *__restrict__ nbr, const int32_t *__restrict__ counts,
            int32_t K, const int64_t *__restrict__ row_ptr, int32_t *__restrict__ col,
            const float4 *__restrict__ pos, float Lx, float Ly, float Lz, float4 *__restrict__ edges)
@@ -122,19 +126,35 @@ k_csr_fill(int64_t n, const int32_t *__restrict__ nbr, const int32_t *__restrict
         const int32_t *row = nbr + i * (int64_t)K;
         float3 wi = make_float3(0.0f, 0.0f, 0.0f);
         if (edges) wi = wrap3(__ldg(pos + i), Lx, Ly, Lz);
-        for (int32_t s = lane; s < c; s += 32) {
-            const int32_t j = __ldcs(row + s);
-            col[base + s] = j;
-            if (edges) {
-                float4 e = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                if ((uint64_t)(int64_t)j < (uint64_t)n) {
-                    const float3 wj = wrap3(__ldg(pos + j), Lx, Ly, Lz);
-                    const float dx = min_image_literal(__fsub_rn(wj.x, wi.x), Lx);
-                    const float dy = min_image_literal(__fsub_rn(wj.y, wi.y), Ly);
-                    const float dz = min_image_literal(__fsub_rn(wj.z, wi.z), Lz);
-                    e = make_float4(dx, dy, dz, __fsqrt_rn(r2_of(dx, dy, dz)));
+        for (int32_t s0 = 0; s0 < c; s0 += 32 * kFillUnroll) {
+            int32_t j[kFillUnroll];
+#pragma unroll
+            for (int u = 0; u < kFillUnroll; ++u) {
+                const int32_t s = s0 + lane + 32 * u;
+                j[u] = s < c ? __ldcs(row + s) : -1;
+            }
+            float4 q[kFillUnroll];
+#pragma unroll
+            for (int u = 0; u < kFillUnroll; ++u) {
+                q[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (edges && (uint64_t)(int64_t)j[u] < (uint64_t)n) q[u] = __ldg(pos + j[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < kFillUnroll; ++u) {
+                const int32_t s = s0 + lane + 32 * u;
+                if (s >= c) break;
+                col[base + s] = j[u];
+                if (edges) {
+                    float4 e = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if ((uint64_t)(int64_t)j[u] < (uint64_t)n) {
+                        const float3 wj = wrap3(q[u], Lx, Ly, Lz);
+                        const float dx = min_image_literal(__fsub_rn(wj.x, wi.x), Lx);
+                        const float dy = min_image_literal(__fsub_rn(wj.y, wi.y), Ly);
+                        const float dz = min_image_literal(__fsub_rn(wj.z, wi.z), Lz);
+                        e = make_float4(dx, dy, dz, __fsqrt_rn(r2_of(dx, dy, dz)));
+                    }
+                    __stcs(edges + base + s, e);
                 }
-                __stcs(edges + base + s, e);
             }
         }
     }
@@ -162,7 +182,7 @@ cudaError_t launch_csr_fill(nl_ctx *ctx, int64_t n, const int32_t *nbr, const in
                             float Lx, float Ly, float Lz, float4 *edges, cudaStream_t s)
 {
     if (n <= 0) return cudaSuccess;
-    k_csr_fill<<<resident_grid(ctx, k_csr_fill, 256, 0, (n + 7) / 8), 256, 0, s>>>(
+    k_csr_fill<<<resident_grid(ctx, k_csr_fill, 128, 0, (n + 3) / 4), 128, 0, s>>>(
         n, nbr, counts, K, row_ptr, col, pos, Lx, Ly, Lz, edges);
     return cudaGetLastError();
 }
