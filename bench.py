@@ -34,8 +34,8 @@ NOMINAL_HBM_GBS = 8000.0
 # belongs to the kernel source it was taken on (nl_pairs.cu and the device
 # header it includes): with any other source the bench reports null.
 PAIR_TRAFFIC = {"workload": "saltwater10m",
-                "sha256": "20146b9e86ec65bcf0de0fc92b781b5d5053aeb8ae9436f50e1758f91501f971",
-                "bytes": 826731264 + 10761926400}
+                "sha256": "aa437c68fed606436a320d88b280b473a0133a8df8e6d2867e79c6ade6283bb0",
+                "bytes": 767519232 + 10722416384}
 
 
 def pair_traffic(workload: str):

@@ -153,7 +153,7 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // vector to the buffer's start.  Rows are finished with one cp.async.bulk
 // copy from a shared block of -1.
 // ---------------------------------------------------------------------------
-constexpr int kTX = 4, kTY = 2, kTZ = 3;   // home cells per tile
+constexpr int kTX = 3, kTY = 2, kTZ = 3;   // home cells per tile
 constexpr int kSY = kTY + 4, kSZ = kTZ + 4;
 constexpr int kSRows = kSY * kSZ;           // staged rows (42)
 constexpr int kHome = kTY * kTZ;            // home rows
@@ -162,7 +162,8 @@ constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built
 constexpr int kRowTab = kSCells * kBinsPerCell;
 constexpr int kFlushAt = 8;                 // pending hits that make the warp flush
 constexpr int kBuf = kFlushAt + 4;          // entries of a lane's hit buffer (7 pending + 4 new)
-constexpr int kTileWarps = 7;
+constexpr int kTileWarps = 5;               // ~140 home atoms: 4-5 chunks of 32
+constexpr int kTileCtas = 5;                // CTAs per SM the stage is sized for
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
 struct TileRows {
@@ -874,12 +875,12 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-// LISTED = false: one tile per CTA (blockIdx), 4 CTAs per SM; a tile whose
+// LISTED = false: one tile per CTA (blockIdx), kTileCtas CTAs per SM; a tile whose
 // rows exceed the stage is listed.  LISTED = true: persistent CTAs, one per
 // SM with a large stage, over the listed tiles; a tile that still does not
 // fit is searched per atom from global memory.
 template <bool LISTED, bool CLOSE>
-__global__ void __launch_bounds__(kTileWarps * 32, LISTED ? 1 : 4)
+__global__ void __launch_bounds__(kTileWarps * 32, LISTED ? 1 : kTileCtas)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
     extern __shared__ __align__(16) unsigned char tile_smem[];
@@ -1130,10 +1131,10 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
     *used_fast = 0;
     if (n <= 0) return cudaSuccess;
     // Staged kernel: column grid and rows of whole 16-byte vectors.  The
-    // stage must hold a typical tile (36 rows x (kTX + 2) cells at the mean
-    // cell occupancy) with 10 % to spare; take the largest number of CTAs per
-    // SM (up to 4) whose shared-memory share still does.  Denser tiles are
-    // listed and searched per atom.
+    // stage must hold a typical tile (kSRows rows x (kTX + 2) cells at the
+    // mean cell occupancy) with 10 % to spare; take the largest number of
+    // CTAs per SM (up to kTileCtas) whose shared-memory share still does.
+    // Denser tiles are listed and searched per atom.
     int stage_max = 0;
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
         (reinterpret_cast<uintptr_t>(nbr) & 15u) == 0 && n < (int64_t(1) << 31)) {
@@ -1149,7 +1150,7 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         const int want =
             (int)(1.1 * per_cell * kSRows * kSCells) + 32;
         const int need = want > kStageMin ? want : kStageMin;
-        for (int ctas = 4; ctas >= 1; --ctas) {
+        for (int ctas = kTileCtas; ctas >= 1; --ctas) {
             long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
             const long cap = (long)optin - (long)fa.sharedSizeBytes;
             if (budget > cap) budget = cap;
