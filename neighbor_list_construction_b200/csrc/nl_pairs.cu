@@ -164,6 +164,7 @@ constexpr int kFlushAt = 8;                 // pending hits that make the warp f
 constexpr int kBuf = kFlushAt + 4;          // entries of a lane's hit buffer (7 pending + 4 new)
 constexpr int kTileWarps = 5;               // ~140 home atoms: 4-5 chunks of 32
 constexpr int kTileCtas = 5;                // CTAs per SM the stage is sized for
+constexpr int kListedCtas = 3;              // CTAs per SM the listed-tile launch may use
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
 struct TileRows {
@@ -1136,9 +1137,10 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
     // CTAs per SM (up to kTileCtas) whose shared-memory share still does.
     // Denser tiles are listed and searched per atom.
     int stage_max = 0;
+    int need = 0, per_sm = 0, reserved = 0;   // typical tile's slots; SM shared memory
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
         (reinterpret_cast<uintptr_t>(nbr) & 15u) == 0 && n < (int64_t(1) << 31)) {
-        int dev = 0, per_sm = 0, reserved = 0, optin = 0;
+        int dev = 0, optin = 0;
         NL_CUDA_TRY(cudaGetDevice(&dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev));
@@ -1149,7 +1151,7 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         const double per_cell = (double)n / (double)g.ncell;
         const int want =
             (int)(1.1 * per_cell * kSRows * kSCells) + 32;
-        const int need = want > kStageMin ? want : kStageMin;
+        need = want > kStageMin ? want : kStageMin;
         for (int ctas = kTileCtas; ctas >= 1; --ctas) {
             long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
             const long cap = (long)optin - (long)fa.sharedSizeBytes;
@@ -1208,19 +1210,42 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
             NL_CUDA_TRY(cudaGetLastError());
         }
         *used_fast = 1;
-        // the listed tiles: one persistent CTA per SM with the largest stage
+        // the listed tiles: persistent CTAs over the list, as many per SM (up
+        // to kListedCtas) as still give each a stage of twice a typical tile;
+        // one CTA with the largest stage when none does.  A tile beyond its
+        // stage is searched per atom from global memory in the same kernel.
         int dev = 0, optin = 0;
         NL_CUDA_TRY(cudaGetDevice(&dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
         cudaFuncAttributes fl;
         NL_CUDA_TRY(cudaFuncGetAttributes(&fl, k_pairs_tiles<true, CLOSE>));
-        const long big = ((long)optin - (long)fl.sharedSizeBytes - (long)tile_fixed_smem(capacity)) /
-                         (long)sizeof(float4);
+        const long lfixed = (long)tile_fixed_smem(capacity);
+        const long big = ((long)optin - (long)fl.sharedSizeBytes - lfixed) / (long)sizeof(float4);
+        long lfit = big;
+        int lctas = 1;
+        for (int c = kListedCtas; c >= 2; --c) {
+            const long b = (long)per_sm / c - reserved - (long)fl.sharedSizeBytes;
+            long f = b > lfixed ? (b - lfixed) / (long)sizeof(float4) : 0;
+            if (f > big) f = big;
+            while (f >= 2L * need) {
+                int nb = 0;
+                NL_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &nb, k_pairs_tiles<true, CLOSE>, kTileWarps * 32,
+                    sizeof(float4) * (size_t)f + (size_t)lfixed));
+                if (nb >= c) break;
+                f -= 32;
+            }
+            if (f >= 2L * need) {
+                lfit = f;
+                lctas = c;
+                break;
+            }
+        }
         TileParams PL = P;
-        PL.stage_max = (int)(big < kSlotLimit ? big : kSlotLimit);
+        PL.stage_max = (int)(lfit < kSlotLimit ? lfit : kSlotLimit);
         ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
-        k_pairs_tiles<true, CLOSE><<<(unsigned)ctx->sm_count, kTileWarps * 32,
-                              sizeof(float4) * (size_t)PL.stage_max + tile_fixed_smem(capacity), s>>>(
+        k_pairs_tiles<true, CLOSE><<<(unsigned)(ctx->sm_count * lctas), kTileWarps * 32,
+                                     sizeof(float4) * (size_t)PL.stage_max + (size_t)lfixed, s>>>(
             g, PL);
         return cudaGetLastError();
     }
