@@ -176,3 +176,23 @@ def test_csr_of_built_rows_round_trips():
             seg = col[row_ptr[i]:row_ptr[i + 1]]
             back[i, :seg.size] = seg
         np.testing.assert_array_equal(back, nbr)
+
+
+def test_edges_ignore_entries_past_the_count():
+    """Slots at or past min(counts[i], K) are padding whatever they hold: stale
+    valid indices there give zeros, as -1 does."""
+    rng = np.random.default_rng(21)
+    box = np.array([9.0, 9.0, 9.0], np.float32)
+    n = 150
+    pos = np.zeros((n, 4), np.float32)
+    pos[:, :3] = rng.random((n, 3)) * box
+    nbr, cnt = rows(pos, box, 2.0, 0.5)
+    K = nbr.shape[1]
+    stale = nbr.copy()
+    pad = np.arange(K)[None, :] >= cnt[:, None]
+    stale[pad] = rng.integers(0, n, int(pad.sum()))
+    e = oracle.edge_features(pos, box, nbr, cnt)
+    e_stale = oracle.edge_features(pos, box, stale, cnt)
+    assert pad.sum() > 100
+    np.testing.assert_array_equal(e_stale, e)
+    np.testing.assert_array_equal(e_stale[pad], 0.0)

@@ -36,6 +36,23 @@ MUTANTS = {
                         [("test_oracle_skin", "test_exactly_half_skin_is_not_a_rebuild")]),
     "cell_stencil_too_small": ("for (ox = -1; ox <= 1; ox++)", "for (ox = 0; ox <= 1; ox++)",
                                [("test_oracle_geometry", "test_cell_list_equals_bruteforce_water")]),
+    "edge_direction_reversed": ("float dx = oracle_min_image(wj[0] - wi[0], box[0]);",
+                                "float dx = oracle_min_image(wi[0] - wj[0], box[0]);",
+                                [("test_oracle_edges", "test_edges_planted_across_the_face", (0,))]),
+    "edge_length_squared": ("o[3] = sqrtf(r2);", "o[3] = r2;",
+                            [("test_oracle_edges", "test_edges_exact_pythagorean_length", ())]),
+    "edge_reads_past_count": ("int64_t j = s < c ? nbr[i * (int64_t)K + s] : -1;",
+                              "int64_t j = nbr[i * (int64_t)K + s];",
+                              [("test_oracle_edges", "test_edges_ignore_entries_past_the_count",
+                                ())]),
+    "close_not_strict": ("if (r2 < close_d2) nc++;", "if (r2 <= close_d2) nc++;",
+                         [("test_oracle_close", "test_planted_pairs_exact", ())]),
+    "close_half_pairs": ("            float r2 = oracle_r2(&w[3 * i], &w[3 * j], box);\n"
+                         "            if (r2 < mn) mn = r2;",
+                         "            float r2 = oracle_r2(&w[3 * i], &w[3 * j], box);\n"
+                         "            if (j < i) continue;\n"
+                         "            if (r2 < mn) mn = r2;",
+                         [("test_oracle_close", "test_planted_pairs_exact", ())]),
 }
 
 
@@ -55,11 +72,13 @@ def test_planted_mistake_is_caught(name, monkeypatch):
         monkeypatch.setattr(oracle_pkg, "compile_library", lambda force=False: so)
         oracle_pkg.lib()
         caught = False
-        for mod_name, fn_name in checks:
-            mod = importlib.import_module(mod_name)
-            fn = getattr(mod, fn_name)
+        for check in checks:
+            mod = importlib.import_module(check[0])
+            fn = getattr(mod, check[1])
             try:
-                if fn_name == "test_oracle_reproduces_golden":
+                if len(check) > 2:        # a pin with its own arguments
+                    fn(*check[2])
+                elif check[1] == "test_oracle_reproduces_golden":
                     for p in mod.GOLDEN:
                         fn(oracle_pkg, p)
                 else:
@@ -70,3 +89,27 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     finally:
         monkeypatch.setattr(oracle_pkg, "_lib", None)
         shutil.rmtree(d, ignore_errors=True)
+
+
+# The CSR form is numpy code in the oracle package: its mistakes are planted
+# in a copy of the function's source.
+CSR_MUTANTS = {
+    "csr_counts_not_clipped": ("v = np.clip(np.asarray(counts, np.int64), 0, K)",
+                               "v = np.asarray(counts, np.int64)"),
+    "csr_offsets_shifted": ("np.cumsum(v, out=row_ptr[1:])", "np.cumsum(v, out=row_ptr[:-1])"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CSR_MUTANTS))
+def test_planted_csr_mistake_is_caught(name, monkeypatch):
+    import inspect
+    import textwrap
+    old, new = CSR_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(oracle_pkg.csr))
+    assert src.count(old) == 1, f"mutation anchor for {name} not found"
+    ns = dict(vars(oracle_pkg))
+    exec(compile(src.replace(old, new), "<csr mutant>", "exec"), ns)
+    monkeypatch.setattr(oracle_pkg, "csr", ns["csr"])
+    mod = importlib.import_module("test_oracle_edges")
+    with pytest.raises(AssertionError):
+        mod.test_csr_matches_a_loop_over_rows()
