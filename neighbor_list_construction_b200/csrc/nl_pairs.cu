@@ -877,8 +877,8 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
 }
 
 // LISTED = false: one tile per CTA (blockIdx), kTileCtas CTAs per SM; a tile whose
-// rows exceed the stage is listed.  LISTED = true: persistent CTAs, one per
-// SM with a large stage, over the listed tiles; a tile that still does not
+// rows exceed the stage is listed.  LISTED = true: persistent CTAs (up to
+// kListedCtas per SM, larger stages) over the listed tiles; a tile that still does not
 // fit is searched per atom from global memory.
 template <bool LISTED, bool CLOSE>
 __global__ void __launch_bounds__(kTileWarps * 32, LISTED ? 1 : kTileCtas)
@@ -1135,7 +1135,7 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
     // stage must hold a typical tile (kSRows rows x (kTX + 2) cells at the
     // mean cell occupancy) with 10 % to spare; take the largest number of
     // CTAs per SM (up to kTileCtas) whose shared-memory share still does.
-    // Denser tiles are listed and searched per atom.
+    // Denser tiles are listed for a second launch with larger stages.
     int stage_max = 0;
     int need = 0, per_sm = 0, reserved = 0;   // typical tile's slots; SM shared memory
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
