@@ -9,6 +9,7 @@ no fallback path.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -95,6 +96,23 @@ def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+_I32, _I64, _F32 = (torch.int32,), (torch.int64,), (torch.float32,)
+_U64 = (torch.int64, torch.uint64)   # 64-bit keys: either view of the bits
+
+
+def _buf(t: torch.Tensor | None, name: str, dtypes, numel: int | None = None):
+    """Pointer of a buffer the library reads or writes through a raw pointer:
+    a contiguous CUDA tensor of one of `dtypes` holding at least `numel`
+    elements, so that no launch can run past its end.  None stays None."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or t.dtype not in dtypes:
+        raise ValueError(f"{name} must be a CUDA tensor of dtype {' or '.join(map(str, dtypes))}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; at least {numel} are needed")
+    return _ptr(t)
+
+
 def _box(box) -> ctypes.Array:
     b = [float(v) for v in (box.tolist() if hasattr(box, "tolist") else box)]
     if len(b) != 3:
@@ -125,57 +143,76 @@ def nl_destroy(ctx) -> None:
     _lib.nl_destroy(ctx)
 
 
+def _sort_outs(n, perm_out, pos_sorted_out, keys_out):
+    return (_buf(perm_out, "perm_out", _I32, n), _buf(pos_sorted_out, "pos_sorted_out", _F32, 4 * n),
+            _buf(keys_out, "keys_out", _U64, n))
+
+
+def _rows_outs(n_rows, capacity, nbr_out, counts_out):
+    return (_buf(nbr_out, "nbr_out", _I32, int(n_rows) * max(int(capacity), 0)),
+            _buf(counts_out, "counts_out", _I32, int(n_rows)))
+
+
 def nl_sort_hilbert(ctx, pos, box, perm_out, pos_sorted_out, keys_out=None, stream=None) -> int:
     _pos(pos)
-    return _check(_lib.nl_sort_hilbert(ctx, pos.shape[0], _ptr(pos), _box(box), _ptr(perm_out),
-                                       _ptr(pos_sorted_out), _ptr(keys_out), _stream(stream)),
-                  "nl_sort_hilbert")
+    n = pos.shape[0]
+    return _check(_lib.nl_sort_hilbert(ctx, n, _ptr(pos), _box(box),
+                                       *_sort_outs(n, perm_out, pos_sorted_out, keys_out),
+                                       _stream(stream)), "nl_sort_hilbert")
 
 
 def nl_sort_morton(ctx, pos, box, perm_out, pos_sorted_out, keys_out=None, stream=None) -> int:
     _pos(pos)
-    return _check(_lib.nl_sort_morton(ctx, pos.shape[0], _ptr(pos), _box(box), _ptr(perm_out),
-                                      _ptr(pos_sorted_out), _ptr(keys_out), _stream(stream)),
-                  "nl_sort_morton")
+    n = pos.shape[0]
+    return _check(_lib.nl_sort_morton(ctx, n, _ptr(pos), _box(box),
+                                      *_sort_outs(n, perm_out, pos_sorted_out, keys_out),
+                                      _stream(stream)), "nl_sort_morton")
 
 
 def nl_sort_hilbert_noalloc(pos, box, perm_out, pos_sorted_out, keys_out=None, status_out=None,
                             stream=None) -> int:
     _pos(pos)
-    return _check(_lib.nl_sort_hilbert_noalloc(pos.shape[0], _ptr(pos), _box(box), _ptr(perm_out),
-                                               _ptr(pos_sorted_out), _ptr(keys_out),
-                                               _ptr(status_out), _stream(stream)),
-                  "nl_sort_hilbert_noalloc")
+    n = pos.shape[0]
+    return _check(_lib.nl_sort_hilbert_noalloc(n, _ptr(pos), _box(box),
+                                               *_sort_outs(n, perm_out, pos_sorted_out, keys_out),
+                                               _buf(status_out, "status_out", _I32, 1),
+                                               _stream(stream)), "nl_sort_hilbert_noalloc")
 
 
 def nl_build(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, stream=None) -> int:
     _pos(pos)
-    return _check(_lib.nl_build(ctx, pos.shape[0], _ptr(pos), _box(box), float(cutoff),
-                                float(skin), int(capacity), _ptr(nbr_out), _ptr(counts_out),
+    n = pos.shape[0]
+    return _check(_lib.nl_build(ctx, n, _ptr(pos), _box(box), float(cutoff), float(skin),
+                                int(capacity), *_rows_outs(n, capacity, nbr_out, counts_out),
                                 _stream(stream)), "nl_build")
 
 
 def nl_build_rows(ctx, pos, n_rows, box, cutoff, skin, capacity, nbr_out, counts_out,
                   stream=None) -> int:
     _pos(pos)
+    rows = min(max(int(n_rows), 0), pos.shape[0])
     return _check(_lib.nl_build_rows(ctx, pos.shape[0], int(n_rows), _ptr(pos), _box(box),
-                                     float(cutoff), float(skin), int(capacity), _ptr(nbr_out),
-                                     _ptr(counts_out), _stream(stream)), "nl_build_rows")
+                                     float(cutoff), float(skin), int(capacity),
+                                     *_rows_outs(rows, capacity, nbr_out, counts_out),
+                                     _stream(stream)), "nl_build_rows")
 
 
 def nl_build_close(ctx, pos, box, cutoff, skin, capacity, nbr_out, counts_out, close_d2,
                    min_d2_out, n_close_out, stream=None) -> int:
     _pos(pos)
-    return _check(_lib.nl_build_close(ctx, pos.shape[0], _ptr(pos), _box(box), float(cutoff),
-                                      float(skin), int(capacity), _ptr(nbr_out),
-                                      _ptr(counts_out), float(close_d2), _ptr(min_d2_out),
-                                      _ptr(n_close_out), _stream(stream)), "nl_build_close")
+    n = pos.shape[0]
+    return _check(_lib.nl_build_close(ctx, n, _ptr(pos), _box(box), float(cutoff), float(skin),
+                                      int(capacity), *_rows_outs(n, capacity, nbr_out, counts_out),
+                                      float(close_d2), _buf(min_d2_out, "min_d2_out", _F32, 1),
+                                      _buf(n_close_out, "n_close_out", _I64, 1),
+                                      _stream(stream)), "nl_build_close")
 
 
 def nl_skin_check(ctx, pos, box, skin, rebuild_out, max_d2_out=None, stream=None) -> int:
     _pos(pos)
     return _check(_lib.nl_skin_check(ctx, pos.shape[0], _ptr(pos), _box(box), float(skin),
-                                     _ptr(rebuild_out), _ptr(max_d2_out), _stream(stream)),
+                                     _buf(rebuild_out, "rebuild_out", _I32, 1),
+                                     _buf(max_d2_out, "max_d2_out", _F32, 1), _stream(stream)),
                   "nl_skin_check")
 
 
@@ -201,7 +238,8 @@ def nl_csr_fill(ctx, nbr, counts, row_ptr, col_out, pos=None, box=None, edges_ou
         if edges_out.dtype != torch.float32 or edges_out.dim() != 2 or edges_out.shape[1] != 4:
             raise ValueError("edges_out must be a float32 [E, 4] CUDA tensor")
     bx = _box(box) if box is not None else None
-    return _check(_lib.nl_csr_fill(ctx, n, _ptr(nbr), _ptr(counts), int(K), _ptr(row_ptr),
+    return _check(_lib.nl_csr_fill(ctx, n, _ptr(nbr), _ptr(counts), int(K),
+                                   _buf(row_ptr, "row_ptr", _I64, n + 1),
                                    _ptr(col_out), _ptr(pos), bx, _ptr(edges_out),
                                    _stream(stream)), "nl_csr_fill")
 
@@ -223,9 +261,12 @@ def nl_edge_features(ctx, pos, box, nbr, counts, edges_out, stream=None) -> int:
 def nl_replay(ctx, step_graph, n_steps, pos, box, cutoff, skin, capacity, nbr, counts,
               decisions_out, stream=None) -> int:
     _pos(pos)
-    return _check(_lib.nl_replay(ctx, step_graph, int(n_steps), pos.shape[0], _ptr(pos),
-                                 _box(box), float(cutoff), float(skin), int(capacity), _ptr(nbr),
-                                 _ptr(counts), _ptr(decisions_out), _stream(stream)), "nl_replay")
+    n = pos.shape[0]
+    return _check(_lib.nl_replay(ctx, step_graph, int(n_steps), n, _ptr(pos), _box(box),
+                                 float(cutoff), float(skin), int(capacity),
+                                 *_rows_outs(n, capacity, nbr, counts),
+                                 _buf(decisions_out, "decisions_out", _I32, max(int(n_steps), 0)),
+                                 _stream(stream)), "nl_replay")
 
 
 def nl_replay_resort(ctx, step_graph, n_steps, pos, ids, aux, box, cutoff, skin, capacity, nbr,
@@ -238,9 +279,14 @@ def nl_replay_resort(ctx, step_graph, n_steps, pos, ids, aux, box, cutoff, skin,
         raise ValueError("aux must be a float32 [n, 4] CUDA tensor")
     return _check(_lib.nl_replay_resort(ctx, step_graph, int(n_steps), n, _ptr(pos), _ptr(ids),
                                         _ptr(aux), _box(box), float(cutoff), float(skin),
-                                        int(capacity), _ptr(nbr), _ptr(counts),
-                                        _ptr(decisions_out), _stream(stream)),
-                  "nl_replay_resort")
+                                        int(capacity), *_rows_outs(n, capacity, nbr, counts),
+                                        _buf(decisions_out, "decisions_out", _I32,
+                                             max(int(n_steps), 0)),
+                                        _stream(stream)), "nl_replay_resort")
+
+
+def _cells(dims) -> int:
+    return math.prod(max(int(x), 0) for x in dims) if len(dims) == 3 else 0
 
 
 def _dims(dims):
@@ -258,33 +304,44 @@ def nl_halo_grid(box, cutoff, skin):
 def nl_halo_mark(ctx, pos, box, dims, rank, occ_out, stream=None) -> int:
     _pos(pos)
     return _check(_lib.nl_halo_mark(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
-                                    int(rank), _ptr(occ_out), _stream(stream)), "nl_halo_mark")
+                                    int(rank), _buf(occ_out, "occ_out", _I32, _cells(dims)),
+                                    _stream(stream)), "nl_halo_mark")
 
 
 def nl_halo_needed(ctx, box, dims, occ_all, need_out, stream=None) -> int:
-    return _check(_lib.nl_halo_needed(ctx, _box(box), _dims(dims), _ptr(occ_all), _ptr(need_out),
-                                      _stream(stream)), "nl_halo_needed")
+    c = _cells(dims)
+    return _check(_lib.nl_halo_needed(ctx, _box(box), _dims(dims),
+                                      _buf(occ_all, "occ_all", _I32, c),
+                                      _buf(need_out, "need_out", _I32, c), _stream(stream)),
+                  "nl_halo_needed")
 
 
 def nl_halo_count(ctx, pos, box, dims, need, rank, nranks, counts_out, stream=None) -> int:
     _pos(pos)
     return _check(_lib.nl_halo_count(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
-                                     _ptr(need), int(rank), int(nranks), _ptr(counts_out),
+                                     _buf(need, "need", _I32, _cells(dims)), int(rank),
+                                     int(nranks), _buf(counts_out, "counts_out", _I32, int(nranks)),
                                      _stream(stream)), "nl_halo_count")
 
 
 def nl_halo_fill(ctx, pos, box, dims, need, rank, nranks, offsets, counts, cursor, send_out,
                  stream=None) -> int:
     _pos(pos)
+    q = int(nranks)
+    # send_out must hold sum(counts) x 4 floats; the counts live on the device
     return _check(_lib.nl_halo_fill(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
-                                    _ptr(need), int(rank), int(nranks), _ptr(offsets),
-                                    _ptr(counts), _ptr(cursor), _ptr(send_out), _stream(stream)),
-                  "nl_halo_fill")
+                                    _buf(need, "need", _I32, _cells(dims)), int(rank), q,
+                                    _buf(offsets, "offsets", _I32, q), _buf(counts, "counts", _I32, q),
+                                    _buf(cursor, "cursor", _I32, q), _buf(send_out, "send_out", _F32),
+                                    _stream(stream)), "nl_halo_fill")
 
 
 def nl_map_ids(ctx, nbr, pos_all, counts=None, stream=None) -> int:
     _pos(pos_all)
-    return _check(_lib.nl_map_ids(ctx, nbr.shape[0], int(nbr.shape[1]), _ptr(nbr), _ptr(counts),
+    if nbr.dtype != torch.int32 or nbr.dim() != 2:
+        raise ValueError("nbr must be an int32 [n_rows, K] CUDA tensor")
+    return _check(_lib.nl_map_ids(ctx, nbr.shape[0], int(nbr.shape[1]), _ptr(nbr),
+                                  _buf(counts, "counts", _I32, nbr.shape[0]),
                                   pos_all.shape[0], _ptr(pos_all), _stream(stream)), "nl_map_ids")
 
 
