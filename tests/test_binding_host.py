@@ -140,3 +140,24 @@ def test_buffer_check_on_real_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         nl._buf(torch.zeros(4, dtype=torch.int32), "x", nl._I32, 4)
     assert nl._buf(None, "x", nl._I32, 4) is None
+
+
+def test_context_methods_allocate_what_the_calls_need(fake):
+    """The Context helpers allocate buffers that pass the checks, including
+    the empty row range (no buffers at all)."""
+    ctx = nl.Context(N, K)
+    b = bufs()
+    perm, ps, ks = ctx.sort(b["pos"], BOX, keys=True)
+    assert perm.shape == (N,) and ps.shape == (N, 4) and ks.shape == (N,)
+    ctx.sort(b["pos"], BOX, curve="morton")
+    nbr, cnt = ctx.build(b["pos"], BOX, 2.0, 0.5, K)
+    assert nbr.shape == (N, K) and cnt.shape == (N,)
+    for rows in (0, 5, N):
+        nbr_r, cnt_r = ctx.build_rows(b["pos"], rows, BOX, 2.0, 0.5, K)
+        assert nbr_r.shape == (rows, K)
+    ctx.build_close(b["pos"], BOX, 2.0, 0.5, K, 1.0)
+    assert ctx.edge_features(b["pos"], BOX, nbr, cnt).shape == (N, K, 4)
+    ctx.skin_check(b["pos"], BOX, 0.5)
+    assert fake.calls == ["nl_create", "nl_sort_hilbert", "nl_sort_morton", "nl_build",
+                          "nl_build_rows", "nl_build_rows", "nl_build_rows", "nl_build_close",
+                          "nl_edge_features", "nl_skin_check"]
