@@ -137,10 +137,11 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(steps: int = 1, nside: int = 60) -> dict:
+def oracle_sample(steps: int = 1, nside: int = 66) -> dict:
     """The CPU oracle, as it stands, on a bounded sample of the salt-solution
-    recipe (nside^3 sites: 60 -> ~0.65M atoms, 40 -> ~0.19M): curve sort +
-    neighbor list + skin check per step, single-threaded."""
+    recipe (nside^3 sites: 66 -> ~0.86M atoms, about 11 s of one host core;
+    40 -> ~0.19M): curve sort + neighbor list + skin check per step,
+    single-threaded."""
     import oracle
     from neighbor_list_construction_b200 import workloads
     w = workloads.make(f"saltwater_n{nside}", seed=4)
