@@ -67,3 +67,24 @@ def test_sources_do_not_reference_the_oracle():
         if f.endswith((".cu", ".cuh", ".py", ".h")):
             text = open(f).read()
             assert "import oracle" not in text and "nl_oracle" not in text, f
+
+
+def test_every_declaration_is_documented():
+    """Each entry point in include/*.h has a comment block directly above it,
+    or follows, with no blank line, a declaration of the same documented
+    group: walking up over contiguous non-blank lines reaches a comment end."""
+    undocumented = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        lines = text.split("\n")
+        for m in DECL.finditer(text):
+            j = text.count("\n", 0, m.start()) - 1
+            ok = False
+            while j >= 0 and lines[j].strip():
+                if lines[j].rstrip().endswith("*/"):
+                    ok = True
+                    break
+                j -= 1
+            if not ok:
+                undocumented.append(m.group(1))
+    assert not undocumented, undocumented
