@@ -221,6 +221,18 @@ const int32_t *nl_step_counter(nl_ctx *ctx);
  * clears it. */
 nl_status nl_sync_status(nl_ctx *ctx, void *stream);
 
+/* Failure-path self-test of the bounded device waits.  Every spin-wait of
+ * the path (the look-back scans of the sort and the cell binning, the
+ * stage barrier of the pair search) gives up after a bounded number of
+ * polls and records NL_ERR_TIMEOUT in the context's status word instead of
+ * hanging.  This call enqueues on `stream` one device thread that polls a
+ * context word which nothing writes, under the look-back rule (a 64 ns
+ * sleep between polls after the first 64), and gives up after max_polls
+ * polls, recording the timeout the same way.  nl_sync_status then returns
+ * NL_ERR_TIMEOUT and clears it.  Nothing else is written, so the context
+ * stays usable.  max_polls outside [1, 2^22] is NL_ERR_ARG. */
+nl_status nl_wait_selftest(nl_ctx *ctx, int32_t max_polls, void *stream);
+
 /* Static, human-readable name of a status code. */
 const char *nl_status_string(nl_status s);
 

@@ -431,6 +431,7 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
         c->unsorted = c->zero_block + 12;
         c->fb_count = c->zero_block + 13;
         c->sort_gate = c->zero_block + 14;
+        c->probe_word = c->zero_block + 15;
         ok &= pairs_set_attributes() == cudaSuccess;
         ok &= cudaMemset(c->zero_block, 0, 64 * sizeof(uint32_t)) == cudaSuccess;
         ok &= cudaDeviceSynchronize() == cudaSuccess;
@@ -633,6 +634,21 @@ nl_status replay_impl(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64_t n,
     return NL_OK;
 }
 
+// One thread polls a word that nothing writes, under the rule of the
+// look-back waits (a 64 ns sleep between polls after the first 64), and
+// records the timeout in the status word as a look-back that gives up does.
+__global__ void k_wait_selftest(const uint32_t *word, uint32_t max_polls, uint32_t *flags)
+{
+    if (threadIdx.x != 0) return;
+    for (uint32_t spins = 0u; ld_volatile_u32(word) == 0u;) {
+        if (++spins >= max_polls) {
+            atomicOr(flags, kFlagTimeout);
+            return;
+        }
+        if (spins > 64u) __nanosleep(64);
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -687,6 +703,13 @@ nl_status nl_replay_resort(nl_ctx *ctx, void *step_graph, int32_t n_steps, int64
 }
 
 const int32_t *nl_step_counter(nl_ctx *ctx) { return ctx ? ctx->step : nullptr; }
+
+nl_status nl_wait_selftest(nl_ctx *ctx, int32_t max_polls, void *stream)
+{
+    if (!ctx || max_polls < 1 || (uint32_t)max_polls > kSpinLimit) return NL_ERR_ARG;
+    k_wait_selftest<<<1, 32, 0, S(stream)>>>(ctx->probe_word, (uint32_t)max_polls, ctx->flags);
+    return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
+}
 
 nl_status nl_sync_status(nl_ctx *ctx, void *stream)
 {

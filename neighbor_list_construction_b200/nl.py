@@ -45,6 +45,7 @@ _SIGS = {
                                 _vp, _vp, _vp]),
     "nl_step_counter": (_vp, [_vp]),
     "nl_sync_status": (_i32, [_vp, _vp]),
+    "nl_wait_selftest": (_i32, [_vp, _i32, _vp]),
     "nl_status_string": (ctypes.c_char_p, [_i32]),
     "nl_last_build_info": (_i32, [_vp, _vp]),
     "nl_profile_enable": (_i32, [_vp, ctypes.c_int]),
@@ -347,6 +348,10 @@ def nl_map_ids(ctx, nbr, pos_all, counts=None, stream=None) -> int:
 
 def nl_step_counter(ctx) -> int:
     return _lib.nl_step_counter(ctx)
+
+
+def nl_wait_selftest(ctx, max_polls: int, stream=None) -> int:
+    return _check(_lib.nl_wait_selftest(ctx, int(max_polls), _stream(stream)), "nl_wait_selftest")
 
 
 def nl_sync_status(ctx, stream=None) -> int:

@@ -84,6 +84,7 @@ def calls(b):
         "nl_halo_fill": lambda: nl.nl_halo_fill(ctx, b["pos"], BOX, DIMS, b["need"], 0, 2,
                                                 b["offs"], b["cnt2"], b["cursor"], b["send"]),
         "nl_map_ids": lambda: nl.nl_map_ids(ctx, b["nbr"], b["pos"], b["cnt"]),
+        "nl_wait_selftest": lambda: nl.nl_wait_selftest(ctx, 1000),
     }
 
 
