@@ -34,7 +34,7 @@ NOMINAL_HBM_GBS = 8000.0
 # belongs to the kernel source it was taken on (nl_pairs.cu and the device
 # header it includes): with any other source the bench reports null.
 PAIR_TRAFFIC = {"workload": "saltwater10m",
-                "sha256": "0405443e261ce63b5298391262b917319575c4d724aa55f96d3e309384d525b1",
+                "sha256": "fe3d0ce2455a16c8bbb475c2c2b18c52f615fc3f0f99d7204de5b111f6a063c7",
                 "bytes": 767583232 + 10721888256}
 
 

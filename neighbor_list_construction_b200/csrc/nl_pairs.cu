@@ -162,7 +162,7 @@ constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built
 constexpr int kRowTab = kSCells * kBinsPerCell;
 constexpr int kFlushAt = 8;                 // pending hits that make the warp flush
 constexpr int kBuf = kFlushAt + 4;          // entries of a lane's hit buffer (7 pending + 4 new)
-constexpr int kTileWarps = 5;               // ~140 home atoms: 4-5 chunks of 32
+constexpr int kTileWarps = 5;               // ~140 home atoms: mostly 4-6 chunks of 32
 constexpr int kTileCtas = 5;                // CTAs per SM the stage is sized for
 constexpr int kListedCtas = 3;              // CTAs per SM the listed-tile launch may use
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
