@@ -88,3 +88,60 @@ def test_every_declaration_is_documented():
             if not ok:
                 undocumented.append(m.group(1))
     assert not undocumented, undocumented
+
+
+NULL_CTX_PROBE = r'''
+import ctypes, sys
+sys.path.insert(0, sys.argv[1])
+from neighbor_list_construction_b200 import nl
+L = nl._lib
+box = (ctypes.c_float * 3)(10, 10, 10)
+dims = (ctypes.c_int32 * 3)(2, 2, 2)
+calls = [
+    L.nl_sort_hilbert(None, 10, None, box, None, None, None, None),
+    L.nl_sort_morton(None, 10, None, box, None, None, None, None),
+    L.nl_build(None, 10, None, box, 2.0, 0.5, 8, None, None, None),
+    L.nl_build_rows(None, 10, 5, None, box, 2.0, 0.5, 8, None, None, None),
+    L.nl_build_close(None, 10, None, box, 2.0, 0.5, 8, None, None, 1.0, None, None, None),
+    L.nl_edge_features(None, 10, None, box, None, None, 8, None, None),
+    L.nl_csr_offsets(None, 10, None, 8, None, None),
+    L.nl_csr_fill(None, 10, None, None, 8, None, None, None, box, None, None),
+    L.nl_skin_check(None, 10, None, box, 0.5, None, None, None),
+    L.nl_replay(None, None, 4, 10, None, box, 2.0, 0.5, 8, None, None, None, None),
+    L.nl_replay_resort(None, None, 4, 10, None, None, None, box, 2.0, 0.5, 8, None, None, None, None),
+    L.nl_sync_status(None, None),
+    L.nl_last_build_info(None, None),
+    L.nl_profile_enable(None, 1),
+    L.nl_profile_read(None, None, None, 4),
+    L.nl_halo_mark(None, 10, None, box, dims, 0, None, None),
+    L.nl_halo_needed(None, box, dims, None, None, None),
+    L.nl_halo_count(None, 10, None, box, dims, None, 0, 2, None, None),
+    L.nl_halo_fill(None, 10, None, box, dims, None, 0, 2, None, None, None, None, None),
+    L.nl_map_ids(None, 10, 8, None, None, 10, None, None),
+    L.nl_wait_selftest(None, 10, None),
+]
+h = ctypes.c_void_p()
+bad_create = [L.nl_create(ctypes.byref(h), 10, 0), L.nl_create(ctypes.byref(h), -1, 8),
+              L.nl_create(None, 10, 8)]
+L.nl_destroy(None)
+import json
+print("NULLCTX" + json.dumps({"calls": calls, "bad_create": bad_create,
+                              "counter": L.nl_step_counter(None)}))
+'''
+
+
+def test_null_context_and_bad_create_are_refused_without_a_gpu():
+    """Every entry point refuses a NULL context with NL_ERR_ARG before any
+    CUDA call (run in a child process, so a crash fails this test only);
+    nl_create refuses bad sizes and a NULL handle; nl_destroy(NULL) is a
+    no-op."""
+    import sys
+    out = subprocess.run([sys.executable, "-c", NULL_CTX_PROBE, ROOT], capture_output=True,
+                         text=True, timeout=120)
+    assert out.returncode == 0, out.stderr[-2000:]
+    import json
+    line = [ln for ln in out.stdout.splitlines() if ln.startswith("NULLCTX")][0]
+    got = json.loads(line[len("NULLCTX"):])
+    assert got["calls"] == [-1] * 21          # NL_ERR_ARG
+    assert got["bad_create"] == [-1] * 3
+    assert got["counter"] is None
