@@ -1,7 +1,8 @@
 """CPU oracle for the periodic neighbor-list build -- TEST INFRASTRUCTURE ONLY.
 
-A plain, slow restatement (``nl_oracle.c``, single-threaded C, fp32 without
-fused multiply-add) of what the GPU hot path computes: Hilbert-curve order,
+A plain, slow restatement (``nl_oracle.c``, plain C, fp32 without fused
+multiply-add; its per-atom and per-row loops may run on OpenMP threads, which
+changes no result) of what the GPU hot path computes: Hilbert-curve order,
 fixed-capacity padded neighbor rows, and the skin check.  Only ``tests/``,
 ``__graft_entry__.smoke()`` and the CPU legs of ``bench.py`` may import this
 package; the product library never does, and shares no code with it.
@@ -27,7 +28,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "nl_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
           "-fPIC", "-shared"]
 
 
@@ -71,6 +72,7 @@ def lib() -> ctypes.CDLL:
             "oracle_displacement": (f32, [u64, i64, i64, ctypes.c_int, f32]),
             "oracle_displace": (None, [i64, vp, u64, i64, f32]),
             "oracle_md_decisions": (i64, [i64, vp, vp, vp, f32, u64, f32, i64, vp]),
+            "oracle_set_threads": (ctypes.c_int, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -96,6 +98,12 @@ def _pos4(pos) -> np.ndarray:
 def _box(box) -> np.ndarray:
     b = np.ascontiguousarray(np.asarray(box, dtype=np.float32).reshape(3))
     return b
+
+
+def set_threads(n: int) -> int:
+    """Threads the oracle's per-atom and per-row loops may use (1 = plain
+    single-threaded).  Returns the previous setting."""
+    return int(lib().oracle_set_threads(int(n)))
 
 
 # ----------------------------------------------------------------- scalars

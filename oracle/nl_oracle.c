@@ -1,11 +1,11 @@
 /*
  * nl_oracle.c -- CPU oracle for the periodic neighbor-list build.
  *
- * TEST INFRASTRUCTURE ONLY.  This file is a plain, slow, single-threaded
- * restatement of what the neighbor-list hot path computes.  Only the test
- * suite, the smoke check and the benchmark's CPU-baseline / reference leg may
- * load it.  The product library never calls, links or includes it, and the
- * two share no code, headers or constants.
+ * TEST INFRASTRUCTURE ONLY.  This file is a plain, slow restatement of what
+ * the neighbor-list hot path computes.  Only the test suite, the smoke
+ * check and the benchmark's CPU-baseline / reference leg may load it.  The
+ * product library never calls, links or includes it, and the two share no
+ * code, headers or constants.
  *
  * Source of the method: "Ab Initio Accuracy Beyond the Cutoff: Distributed
  * Message-Passing Equivariant Attention at Tens-of-Millions-of-Atom Scale"
@@ -30,12 +30,20 @@
  * Every function below computes its definition directly; the cell list only
  * enumerates candidates, the predicate decides.
  *
- * Build: gcc -O2 -ffp-contract=off -fno-fast-math (x86-64 SSE arithmetic).
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -fopenmp (x86-64 SSE
+ * arithmetic).  Three loops run on OpenMP threads, each over independent
+ * elements: the keys of the atoms, their wrapped coordinates, and the rows
+ * of oracle_rows (each row computed and sorted by one thread).  No result
+ * depends on the thread count; oracle_set_threads(1) makes the oracle
+ * single-threaded.
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define OR_QBITS 21
 #define OR_QMAX ((1u << OR_QBITS) - 1u)
@@ -175,6 +183,7 @@ void oracle_keys(int64_t n, const float *pos4, const float box[3], int curve,
     int64_t i;
     int a;
     for (a = 0; a < 3; a++) S[a] = oracle_quant_scale(box[a]);
+#pragma omp parallel for private(a) schedule(static)
     for (i = 0; i < n; i++) {
         uint32_t q[3];
         for (a = 0; a < 3; a++)
@@ -284,6 +293,7 @@ static float *or_wrap_all(int64_t n, const float *pos4, const float box[3])
     int64_t i;
     int a;
     if (!w) return NULL;
+#pragma omp parallel for private(a) schedule(static)
     for (i = 0; i < n; i++)
         for (a = 0; a < 3; a++) w[3 * i + a] = oracle_wrap(pos4[4 * i + a], box[a]);
     return w;
@@ -328,10 +338,10 @@ int oracle_rows(int64_t n, const float *pos4, const float box[3], float cutoff,
     float rl = cutoff + skin;
     float rl2 = rl * rl;
     int m[3], a, over = 0, brute = 0;
-    int64_t ncell = 1, r, i, j;
+    volatile int failed = 0;
+    int64_t ncell = 1, r, i;
     int64_t *head = NULL, *next = NULL, *cellof = NULL;
     float *w;
-    or_vec hits = {0, 0, 0};
 
     w = or_wrap_all(n, pos4, box);
     if (!w) return -1;
@@ -364,33 +374,54 @@ int oracle_rows(int64_t n, const float *pos4, const float box[3], float cutoff,
             head[id] = i;
         }
     }
-    for (r = 0; r < nrows; r++) {
-        i = rows ? rows[r] : r;
-        hits.n = 0;
-        if (brute) {
-            for (j = 0; j < n; j++)
-                if (j != i && oracle_r2(&w[3 * i], &w[3 * j], box) < rl2)
-                    if (or_push(&hits, (int32_t)j)) goto fail;
-        } else {
-            int ox, oy, oz;
-            for (oz = -1; oz <= 1; oz++)
-                for (oy = -1; oy <= 1; oy++)
-                    for (ox = -1; ox <= 1; ox++) {
-                        int64_t cx = (cellof[3 * i + 0] + ox + m[0]) % m[0];
-                        int64_t cy = (cellof[3 * i + 1] + oy + m[1]) % m[1];
-                        int64_t cz = (cellof[3 * i + 2] + oz + m[2]) % m[2];
-                        for (j = head[(cz * m[1] + cy) * m[0] + cx]; j >= 0; j = next[j])
-                            if (j != i && oracle_r2(&w[3 * i], &w[3 * j], box) < rl2)
-                                if (or_push(&hits, (int32_t)j)) goto fail;
-                    }
+    /* Rows are independent and each is sorted before it is written, so the
+     * result does not depend on how the rows are shared out among threads. */
+#pragma omp parallel reduction(| : over)
+    {
+        or_vec hits = {0, 0, 0};
+        int64_t rr;
+#pragma omp for schedule(dynamic, 256)
+        for (rr = 0; rr < nrows; rr++) {
+            int64_t ii = rows ? rows[rr] : rr, jj;
+            if (failed) continue;
+            hits.n = 0;
+            if (brute) {
+                for (jj = 0; jj < n; jj++)
+                    if (jj != ii && oracle_r2(&w[3 * ii], &w[3 * jj], box) < rl2)
+                        if (or_push(&hits, (int32_t)jj)) { failed = 1; break; }
+            } else {
+                int ox, oy, oz;
+                for (oz = -1; oz <= 1; oz++)
+                    for (oy = -1; oy <= 1; oy++)
+                        for (ox = -1; ox <= 1; ox++) {
+                            int64_t cx = (cellof[3 * ii + 0] + ox + m[0]) % m[0];
+                            int64_t cy = (cellof[3 * ii + 1] + oy + m[1]) % m[1];
+                            int64_t cz = (cellof[3 * ii + 2] + oz + m[2]) % m[2];
+                            for (jj = head[(cz * m[1] + cy) * m[0] + cx]; jj >= 0; jj = next[jj])
+                                if (jj != ii && oracle_r2(&w[3 * ii], &w[3 * jj], box) < rl2)
+                                    if (or_push(&hits, (int32_t)jj)) failed = 1;
+                        }
+            }
+            if (!failed) over |= or_emit_row(&hits, K, nbr + rr * (int64_t)K, counts + rr);
         }
-        over |= or_emit_row(&hits, K, nbr + r * (int64_t)K, counts + r);
+        free(hits.v);
     }
-    free(w); free(head); free(next); free(cellof); free(hits.v);
-    return over;
-fail:
-    free(w); free(head); free(next); free(cellof); free(hits.v);
-    return -1;
+    free(w); free(head); free(next); free(cellof);
+    return failed ? -1 : over;
+}
+
+/* Number of threads the row loops of the oracle may use (OpenMP); 1 gives
+ * the plain single-threaded oracle.  Returns the previous setting. */
+int oracle_set_threads(int nthreads)
+{
+#ifdef _OPENMP
+    int old = omp_get_max_threads();
+    if (nthreads >= 1) omp_set_num_threads(nthreads);
+    return old;
+#else
+    (void)nthreads;
+    return 1;
+#endif
 }
 
 int oracle_build(int64_t n, const float *pos4, const float box[3], float cutoff,

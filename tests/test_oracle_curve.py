@@ -126,3 +126,140 @@ def test_hilbert_order_is_local(oracle):
     d_curve = np.linalg.norm(np.diff(p, axis=0), axis=1).mean()
     d_rand = np.linalg.norm(np.diff(w.pos[:, :3].astype(np.float64), axis=0), axis=1).mean()
     assert d_curve < 0.25 * d_rand
+
+
+# ---------------------------------------------------------------------------
+# The key of an atom is the curve index of its grid cell, and the grid cell is
+# fixed by the mathematics alone: per axis a, q_a = floor(frac(x_a / L_a) * 2^21)
+# for the real-valued coordinate.  The oracle computes it in fp32 (wrap, then
+# scale by fl(2^21 / L_a)), which agrees with the exact value except within a
+# few fp32 roundings of a cell face.  The pins below take the exact value from
+# rational arithmetic, skip only points that close to a face, and check the
+# whole composition (wrap of each axis by its own side, quantization with that
+# axis's own scale, the key of the three grid coordinates) on orthorhombic
+# boxes with coordinates far outside [0, L).
+# ---------------------------------------------------------------------------
+from fractions import Fraction
+
+_BOXES = [(30.5, 47.25, 91.75), (91.75, 30.5, 47.25), (47.25, 91.75, 30.5),
+          (468.88, 214.256, 84.023)]
+
+
+def _exact_cell(x: float, L: float):
+    """(q, distance to the nearest cell face in units of a cell) from exact
+    rationals: q = floor(frac(x / L) * 2^21)."""
+    fx, fl_ = Fraction(float(np.float32(x))), Fraction(float(np.float32(L)))
+    u = (fx / fl_) % 1 * 2 ** 21          # exact grid coordinate in [0, 2^21)
+    q = int(u)                            # floor (u >= 0)
+    frac = u - q
+    return q, float(min(frac, 1 - frac))
+
+
+def _coords(rng, L, n):
+    """Coordinates inside the box and up to five box lengths either side."""
+    span = rng.integers(-5, 6, size=n).astype(np.float64)
+    return (rng.random(n) * L + span * L).astype(np.float32)
+
+
+def _cells_of_keys(oracle, keys, curve):
+    """Grid cells of keys: the oracle's inverse Hilbert transform (pinned by
+    the curve tests above) or Morton de-interleaving (closed form)."""
+    out = []
+    for k in keys:
+        k = int(k)
+        if curve == "hilbert":
+            out.append(oracle.hilbert_axes(k, 21))
+        else:
+            q = [0, 0, 0]
+            for l in range(21):
+                q[0] |= ((k >> (3 * l + 2)) & 1) << l
+                q[1] |= ((k >> (3 * l + 1)) & 1) << l
+                q[2] |= ((k >> (3 * l)) & 1) << l
+            out.append(tuple(q))
+    return np.array(out, np.int64)
+
+
+@pytest.mark.parametrize("curve", ["hilbert", "morton"])
+@pytest.mark.parametrize("box", _BOXES)
+def test_keys_compose_wrap_quantize_per_axis(oracle, curve, box):
+    """Per axis, the key's grid coordinate is floor(frac(x/L_a) * 2^21) of
+    that axis's own side.  Error bound of the fp32 steps, in cells: the wrap
+    L*floor(x/L) rounds by at most 2^-24 |x| + 2^-24 L (|x| <= 6 L here, so
+    <= 7/8 cell), the scale fl(2^21/L) and the product by at most 1/4 cell:
+    at most 2 cells apart anywhere (cyclically: a point just below a
+    multiple of L may wrap to cell 0), and equal for in-box points more than
+    0.4 cell from a face, where the wrap is exact."""
+    rng = np.random.default_rng(11)
+    n = 3000
+    pos = np.zeros((n, 4), np.float32)
+    for a in range(3):
+        pos[:, a] = _coords(rng, box[a], n)
+    pos[:300, :3] = (rng.random((300, 3)) * np.asarray(box)).astype(np.float32)  # in-box
+    got = _cells_of_keys(oracle, oracle.keys(pos, box, curve), curve)
+    exact_in = 0
+    for i in range(n):
+        for a in range(3):
+            q, margin = _exact_cell(float(pos[i, a]), box[a])
+            d = abs(int(got[i, a]) - q)
+            d = min(d, 2 ** 21 - d)
+            assert d <= 2, (i, a, float(pos[i, a]), q, int(got[i, a]))
+            L = np.float32(box[a])
+            if np.float32(0) <= pos[i, a] < L and margin > 0.4:
+                assert int(got[i, a]) == q, (i, a, float(pos[i, a]))
+                exact_in += 1
+    assert exact_in > 100
+
+
+def _interior(L):
+    """The first float at or above 0.3 L whose exact grid coordinate is more
+    than 0.4 cell from a face."""
+    x = np.float32(L) * np.float32(0.3)
+    while _exact_cell(float(x), L)[1] <= 0.4:
+        x = np.nextafter(x, np.float32(np.inf))
+    return x
+
+
+@pytest.mark.parametrize("curve", ["hilbert", "morton"])
+def test_keys_special_coordinates(oracle, curve):
+    """-0, 0, L, multiples of L and the last float below L, on each axis of an
+    orthorhombic box, with the other axes held at an interior cell."""
+    box = (30.5, 47.25, 91.75)
+    keyfn = oracle.hilbert_key if curve == "hilbert" else oracle.morton_key
+    top = 2 ** 21 - 1
+    for a in range(3):
+        L = np.float32(box[a])
+        cases = {0.0: 0, -0.0: 0, float(L): 0, float(2 * L): 0, float(-L): 0,
+                 float(-3 * L): 0, float(np.nextafter(L, np.float32(0))): top}
+        for x, qa in cases.items():
+            pos = np.zeros((1, 4), np.float32)
+            base = []
+            for b in range(3):
+                # an interior coordinate far from any cell face
+                pos[0, b] = _interior(box[b])
+                base.append(_exact_cell(float(pos[0, b]), box[b])[0])
+            pos[0, a] = np.float32(x)
+            base[a] = qa
+            k = int(oracle.keys(pos, box, curve)[0])
+            assert k == keyfn(*base), (a, x)
+
+
+def test_sort_is_keys_then_index_on_orthorhombic_box(oracle):
+    """oracle.sort orders by the composed keys of an orthorhombic box with
+    out-of-box coordinates, ties by index (numpy lexsort as the textbook
+    routine)."""
+    box = (30.5, 47.25, 91.75)
+    rng = np.random.default_rng(12)
+    n = 5000
+    pos = np.zeros((n, 4), np.float32)
+    for a in range(3):
+        pos[:, a] = _coords(rng, box[a], n)
+    pos[n // 2:n // 2 + 50, :3] = pos[7, :3]       # a run of equal keys
+    for curve in ("hilbert", "morton"):
+        keyfn = oracle.hilbert_key if curve == "hilbert" else oracle.morton_key
+        perm, ks = oracle.sort(pos, box, curve)
+        # the sorted keys are the keys pinned above, taken along perm
+        np.testing.assert_array_equal(ks, oracle.keys(pos, box, curve)[perm])
+        assert sorted(perm.tolist()) == list(range(n))
+        kk = ks.astype(object)
+        for k in range(n - 1):
+            assert kk[k] < kk[k + 1] or (kk[k] == kk[k + 1] and perm[k] < perm[k + 1])

@@ -220,3 +220,25 @@ def test_rows_subset_matches_full(oracle):
     np.testing.assert_array_equal(cnt, fcnt[which])
     np.testing.assert_array_equal(nbr, full[which])
     assert 60 < fcnt.mean() < 200
+
+
+def test_threaded_oracle_equals_single_threaded(oracle):
+    """The OpenMP loops (keys, wrap, rows) give the same result on 1 and on
+    many threads: rows are independent and each is sorted before it is
+    written."""
+    from neighbor_list_construction_b200 import workloads
+    w = workloads.make("saltwater_n20")
+    old = oracle.set_threads(1)
+    try:
+        one = oracle.build(w.pos, w.box, w.cutoff, w.skin, w.capacity)
+        k1 = oracle.sort(w.pos, w.box)
+        oracle.set_threads(max(4, old))
+        many = oracle.build(w.pos, w.box, w.cutoff, w.skin, w.capacity)
+        km = oracle.sort(w.pos, w.box)
+    finally:
+        oracle.set_threads(old)
+    np.testing.assert_array_equal(one[0], many[0])
+    np.testing.assert_array_equal(one[1], many[1])
+    assert one[2] == many[2]
+    np.testing.assert_array_equal(k1[0], km[0])
+    np.testing.assert_array_equal(k1[1], km[1])

@@ -32,6 +32,17 @@ MUTANTS = {
                               [("test_oracle_curve", "test_hilbert_first_order_exhaustive")]),
     "wrap_no_second_fold": ("if (w >= L) w = w - L;", "",
                             [("test_oracle_geometry", "test_wrap_special_cases")]),
+    "keys_quantize_unwrapped": ("q[a] = oracle_quantize(oracle_wrap(pos4[4 * i + a], box[a]), S[a]);",
+                                "q[a] = oracle_quantize(pos4[4 * i + a], S[a]);",
+                                [("test_oracle_curve", "test_keys_compose_wrap_quantize_per_axis",
+                                  (oracle_pkg, "hilbert", (30.5, 47.25, 91.75)))]),
+    "keys_scale_of_axis0": ("q[a] = oracle_quantize(oracle_wrap(pos4[4 * i + a], box[a]), S[a]);",
+                            "q[a] = oracle_quantize(oracle_wrap(pos4[4 * i + a], box[a]), S[0]);",
+                            [("test_oracle_curve", "test_keys_compose_wrap_quantize_per_axis",
+                              (oracle_pkg, "hilbert", (30.5, 47.25, 91.75)))]),
+    "keys_wrap_by_axis0": ("q[a] = oracle_quantize(oracle_wrap(pos4[4 * i + a], box[a]), S[a]);",
+                           "q[a] = oracle_quantize(oracle_wrap(pos4[4 * i + a], box[0]), S[a]);",
+                           [("test_oracle_curve", "test_keys_special_coordinates", (oracle_pkg, "morton"))]),
     "skin_not_strict": ("*rebuild = m > h2 ? 1 : 0;", "*rebuild = m >= h2 ? 1 : 0;",
                         [("test_oracle_skin", "test_exactly_half_skin_is_not_a_rebuild")]),
     "cell_stencil_too_small": ("for (ox = -1; ox <= 1; ox++)", "for (ox = 0; ox <= 1; ox++)",
