@@ -158,7 +158,8 @@ nl_status sort_impl(nl_ctx *ctx, int64_t n, const float *pos, const float *box, 
     }
     {
         ProfScope ps(ctx, PH_GATHER, s);
-        if (launch_gather(n, p4, perm, reinterpret_cast<float4 *>(pos_sorted), s) != cudaSuccess)
+        if (launch_gather(n, p4, perm, reinterpret_cast<float4 *>(pos_sorted), ctx->flags, s) !=
+            cudaSuccess)
             return NL_ERR_CUDA;
     }
     return NL_OK;

@@ -126,8 +126,10 @@ k_cell_scan(const int32_t *__restrict__ count, int32_t *__restrict__ start, int6
 __global__ void __launch_bounds__(256)
 k_bin_scatter(const float4 *__restrict__ pos, int64_t n, CellGrid g,
               const uint32_t *__restrict__ atom_cell, const uint32_t *__restrict__ atom_rank,
-              const int32_t *__restrict__ cell_start, float4 *__restrict__ cell_pos)
+              const int32_t *__restrict__ cell_start, float4 *__restrict__ cell_pos,
+              const uint32_t *flags)
 {
+    if (timed_out(flags)) return;   // cell starts may not be monotonic
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const float4 p = pos[i];
@@ -221,8 +223,10 @@ __device__ __forceinline__ void sort_large_cell(float4 *__restrict__ cell_pos, i
 __global__ void __launch_bounds__(256)
 k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell,
             int nx, float side_x, float inv_bin, uint8_t *__restrict__ cell_tab,
-            uint32_t *__restrict__ large_list, uint32_t *large_count, uint32_t *unsorted)
+            uint32_t *__restrict__ large_list, uint32_t *large_count, uint32_t *unsorted,
+            const uint32_t *flags)
 {
+    if (timed_out(flags)) return;
     const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -260,8 +264,10 @@ k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_star
 __global__ void __launch_bounds__(256)
 k_cell_sort_large(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int nx,
                   float side_x, float inv_bin, uint8_t *__restrict__ cell_tab,
-                  const uint32_t *__restrict__ large_list, const uint32_t *large_count)
+                  const uint32_t *__restrict__ large_list, const uint32_t *large_count,
+                  const uint32_t *flags)
 {
+    if (timed_out(flags)) return;
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -303,7 +309,7 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
         ProfScope ps(ctx, PH_BIN_SCATTER, s);
         k_bin_scatter<<<resident_grid(ctx, k_bin_scatter, 256, 0, (n + 255) / 256), 256, 0, s>>>(pos, n, g, ctx->atom_cell,
                                                              ctx->atom_rank, ctx->cell_start,
-                                                             ctx->cell_pos);
+                                                             ctx->cell_pos, ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
     }
     {
@@ -318,11 +324,11 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
         if (sort_blocks > (int64_t)ctx->sm_count * 32) sort_blocks = (int64_t)ctx->sm_count * 32;
         k_cell_sort<<<(unsigned)sort_blocks, 256, 0, s>>>(
             ctx->cell_pos, ctx->cell_start, g.ncell, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
-            ctx->fb_list, ctx->fb_count, ctx->unsorted);
+            ctx->fb_list, ctx->fb_count, ctx->unsorted, ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
         k_cell_sort_large<<<(unsigned)(ctx->sm_count * 2), 256, 0, s>>>(
             ctx->cell_pos, ctx->cell_start, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
-            ctx->fb_list, ctx->fb_count);
+            ctx->fb_list, ctx->fb_count, ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
     }
     return cudaSuccess;

@@ -115,6 +115,17 @@ __device__ __forceinline__ void st_volatile_u32(uint32_t *p, uint32_t v)
     *(volatile uint32_t *)p = v;
 }
 
+// True once a bounded wait has given up (kFlagTimeout in the status word).
+// A look-back pass that gives up goes on with a partial prefix, so its output
+// is not a permutation (sort) or its cell starts are not monotonic (binning).
+// Every kernel that consumes such output checks this at entry and returns,
+// so a partial prefix never becomes an index, an address or a copy size.
+// The bit stays set until nl_sync_status reads and clears it.
+__device__ __forceinline__ bool timed_out(const uint32_t *flags)
+{
+    return (ld_volatile_u32(flags) & kFlagTimeout) != 0u;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt()
 {
     uint32_t m;

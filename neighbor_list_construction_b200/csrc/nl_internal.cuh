@@ -113,8 +113,9 @@ struct SortRecompute {
 // kept) and indices to vals_final.
 cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
                                 uint32_t *vals_final, cudaStream_t s, const SortRecompute &rk);
+// Returns at once when `flags` holds kFlagTimeout (perm may then be stale).
 cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, float4 *out,
-                          cudaStream_t s);
+                          const uint32_t *flags, cudaStream_t s);
 
 // Cell binning of `pos` into ctx->cell_pos (cell order, x-sorted in cells).
 cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const CellGrid &g,

@@ -15,8 +15,8 @@
 // Host code cannot use the array's name as a device address (in host code it
 // names a host-side shadow), so the first call on each device asks the
 // runtime for the device address with cudaGetSymbolAddress, with that device
-// current, and keeps it.  That first call should come before any stream
-// capture.  Every call shares the one array: calls whose work overlaps on the
+// current, and keeps it; a lookup that fails is not kept, and the next call
+// tries again.  That first call should come before any stream capture.  Every call shares the one array: calls whose work overlaps on the
 // GPU (different streams, or several host threads) race and must be ordered
 // by the caller.
 #include <cmath>
@@ -43,14 +43,37 @@ constexpr size_t kNoallocScratchBytes = align256(kOffFlags + 2 * sizeof(uint32_t
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
+// Device address of the array and SM count, per device, filled in by the
+// first call on that device that succeeds in looking them up.  A failed
+// lookup stores nothing, so the next call tries again.
 struct DeviceScratch {
-    std::once_flag once;
-    cudaError_t err = cudaSuccess;
     unsigned char *base = nullptr;
     int sm_count = 0;
 };
 constexpr int kMaxDevices = 64;
 DeviceScratch g_devices[kMaxDevices];
+std::mutex g_devices_mu;
+
+// The array's address on the current device `dev` (looked up on first use).
+cudaError_t device_scratch(int dev, DeviceScratch *out)
+{
+    std::lock_guard<std::mutex> lock(g_devices_mu);
+    DeviceScratch &d = g_devices[dev];
+    if (!d.base) {
+        void *p = nullptr;
+        int sms = 0;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess || !p) {
+            (void)cudaGetLastError();   // leave no stale error for the caller's next check
+            return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+        }
+        d.sm_count = sms;
+        d.base = static_cast<unsigned char *>(p);
+    }
+    *out = d;
+    return cudaSuccess;
+}
 
 __global__ void k_noalloc_status(const uint32_t *flags, int32_t *status_out)
 {
@@ -75,15 +98,8 @@ extern "C" nl_status nl_sort_hilbert_noalloc(int64_t n, const float *pos, const 
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NL_ERR_CUDA;
-    DeviceScratch &d = g_devices[dev];
-    std::call_once(d.once, [&d, dev]() {
-        void *p = nullptr;
-        d.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (d.err == cudaSuccess)
-            d.err = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
-        d.base = static_cast<unsigned char *>(p);
-    });
-    if (d.err != cudaSuccess || !d.base) return NL_ERR_CUDA;
+    DeviceScratch d;
+    if (device_scratch(dev, &d) != cudaSuccess) return NL_ERR_CUDA;
 
     // A context view over the static array; nothing here allocates.
     nl_ctx view;
@@ -119,7 +135,8 @@ extern "C" nl_status nl_sort_hilbert_noalloc(int64_t n, const float *pos, const 
         if (nl::launch_radix_passes(&view, n, keys_out, reinterpret_cast<uint32_t *>(perm_out), s,
                                     rk) != cudaSuccess)
             return NL_ERR_CUDA;
-        if (nl::launch_gather(n, p4, perm_out, reinterpret_cast<float4 *>(pos_sorted_out), s) !=
+        if (nl::launch_gather(n, p4, perm_out, reinterpret_cast<float4 *>(pos_sorted_out),
+                              view.flags, s) !=
             cudaSuccess)
             return NL_ERR_CUDA;
     }

@@ -118,6 +118,7 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
                  int32_t *__restrict__ nbr, int32_t *__restrict__ counts, uint32_t *flags,
                  float close_d2, uint32_t *min_bits, unsigned long long *n_close)
 {
+    if (timed_out(flags)) return;   // cell starts may not be monotonic
     CloseAcc cl{__int_as_float(0x7f800000), 0u};
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride)
@@ -884,6 +885,7 @@ template <bool LISTED, bool CLOSE>
 __global__ void __launch_bounds__(kTileWarps * 32, LISTED ? 1 : kTileCtas)
 k_pairs_tiles(const CellGrid g, const TileParams P)
 {
+    if (timed_out(P.flags)) return;   // cell starts may not be monotonic
     extern __shared__ __align__(16) unsigned char tile_smem[];
     float4 *stage = reinterpret_cast<float4 *>(tile_smem);
     uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
@@ -1016,7 +1018,15 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
         for (uint32_t spins = 0; spins < 4096u && !done; ++spins)   // ~4 s
             done = mbar_try_wait(&bar, phase);
         if (__syncthreads_or(!done)) {
+            // Entry already returned if a look-back gave up, so the cell starts
+            // are monotonic and the announced byte count is exactly what the
+            // row copies carry: the phase completes when they land.  A CTA
+            // that left now could leave copies writing into shared memory given
+            // to the next CTA, so it records the timeout and waits once more
+            // (bounded) before it returns.
             if (threadIdx.x == 0) atomicOr(P.flags, kFlagTimeout);
+            for (uint32_t spins = 0; spins < 4096u && !done; ++spins)
+                done = mbar_try_wait(&bar, phase);
             return;
         }
         phase ^= 1u;

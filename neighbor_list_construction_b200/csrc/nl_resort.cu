@@ -17,8 +17,10 @@ namespace {
 __global__ void k_permute_gather(int64_t n, const uint32_t *__restrict__ perm,
                                  const float4 *__restrict__ pos, float4 *__restrict__ pos_tmp,
                                  const int32_t *__restrict__ ids, int32_t *__restrict__ ids_tmp,
-                                 const float4 *__restrict__ aux, float4 *__restrict__ aux_tmp)
+                                 const float4 *__restrict__ aux, float4 *__restrict__ aux_tmp,
+                                 const uint32_t *flags)
 {
+    if (timed_out(flags)) return;   // perm may not be a permutation
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride) {
         const uint32_t i = perm[k];
@@ -32,8 +34,9 @@ __global__ void k_permute_gather(int64_t n, const uint32_t *__restrict__ perm,
 __global__ void k_permute_back(int64_t n, float4 *__restrict__ pos,
                                const float4 *__restrict__ pos_tmp, int32_t *__restrict__ ids,
                                const int32_t *__restrict__ ids_tmp, float4 *__restrict__ aux,
-                               const float4 *__restrict__ aux_tmp)
+                               const float4 *__restrict__ aux_tmp, const uint32_t *flags)
 {
+    if (timed_out(flags)) return;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride) {
         pos[k] = pos_tmp[k];
@@ -71,10 +74,10 @@ cudaError_t launch_resort(nl_ctx *ctx, int64_t n, float4 *pos, int32_t *ids, flo
         const unsigned blocks = resident_grid(ctx, k_permute_gather, 256, 0, (n + 255) / 256);
         int32_t *ids_tmp = reinterpret_cast<int32_t *>(ctx->atom_cell);
         k_permute_gather<<<(unsigned)blocks, 256, 0, s>>>(n, perm, pos, ctx->cell_pos, ids, ids_tmp,
-                                                          aux, ctx->ref);
+                                                          aux, ctx->ref, ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
         k_permute_back<<<(unsigned)blocks, 256, 0, s>>>(n, pos, ctx->cell_pos, ids, ids_tmp, aux,
-                                                        ctx->ref);
+                                                        ctx->ref, ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
     }
     return cudaSuccess;

@@ -20,7 +20,8 @@
 // come from histograms made by the key kernel (those of the low digits only
 // by its gated recompute).  Waits on a status
 // word are bounded: past kSpinLimit polls the kernel records kFlagTimeout
-// and carries on, so a stuck predecessor cannot hang the device.
+// and carries on, so a stuck predecessor cannot hang the device; every later
+// pass, the run finish and the gather then return at entry (timed_out).
 #include "nl_internal.cuh"
 
 namespace nl {
@@ -38,6 +39,7 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
            uint32_t *ticket, uint32_t *flags, const uint32_t *gate)
 {
     if (gate && ld_volatile_u32(gate) == 0u) return;   // gated pass not needed
+    if (timed_out(flags)) return;                       // an earlier wait gave up
     extern __shared__ __align__(16) unsigned char sort_smem[];
     uint64_t *s_keys = reinterpret_cast<uint64_t *>(sort_smem);
     uint32_t *s_vals = reinterpret_cast<uint32_t *>(sort_smem + sizeof(uint64_t) * kSortTile);
@@ -194,8 +196,10 @@ constexpr int kRunHalo = kRunMax + 1;
 
 __global__ void __launch_bounds__(kRunThreads)
 k_run_sort(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ vals, int64_t n,
-           uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, uint32_t *gate)
+           uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, uint32_t *gate,
+           const uint32_t *flags)
 {
+    if (timed_out(flags)) return;
     __shared__ uint64_t s_k[kRunTile + 2 * kRunHalo];
     __shared__ uint32_t s_v[kRunTile + 2 * kRunHalo];
     const int64_t t0 = (int64_t)blockIdx.x * kRunTile;
@@ -268,7 +272,8 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
     {
         const int64_t blocks = (n + kRunTile - 1) / kRunTile;
         k_run_sort<<<(unsigned)blocks, kRunThreads, 0, s>>>(ctx->keys[src], ctx->vals[src], n,
-                                                           keys_final, vals_final, ctx->sort_gate);
+                                                           keys_final, vals_final, ctx->sort_gate,
+                                                           ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
     }
     // full sort, gated: runs only when a prefix run was too long

@@ -46,3 +46,39 @@ def assert_rows_match(g_nbr, g_cnt, o_nbr, o_cnt, full_sets=None):
         assert np.all(row >= 0) and np.unique(row).size == K
         if full_sets is not None:
             assert set(row.tolist()) <= full_sets[r]
+
+
+def assert_all_rows_match(oracle, nbr_t, cnt_t, pos, box, cutoff, skin, K, chunk=1 << 21):
+    """Every row and count of a GPU build (device tensors, any slot order)
+    against the oracle, element by element, in chunks of rows.
+
+    The GPU rows are put in canonical order (ascending, -1 padding last) with
+    torch.sort on the device; the oracle's rows come from oracle.rows on the
+    same positions.  Rows whose count passes K must hold K distinct members of
+    the atom's full neighbor set.  Returns True when any row overflowed."""
+    import torch
+    n = pos.shape[0]
+    cnt = cnt_t.cpu().numpy()
+    big = torch.iinfo(torch.int32).max
+    overflow = False
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        which = np.arange(s, e, dtype=np.int64)
+        o_nbr, o_cnt, o_ov = oracle.rows(pos, box, cutoff, skin, K, which)
+        np.testing.assert_array_equal(cnt[s:e], o_cnt)
+        g = nbr_t[s:e]
+        g = torch.sort(torch.where(g < 0, big, g), dim=1).values
+        g = torch.where(g == big, -1, g).cpu().numpy()
+        ok = o_cnt <= K
+        bad = np.nonzero(np.any(g[ok] != o_nbr[ok], axis=1))[0]
+        assert bad.size == 0, f"{bad.size} rows differ, first {s + np.nonzero(ok)[0][bad[:5]]}"
+        over = np.nonzero(~ok)[0]
+        if over.size:
+            overflow = True
+            K2 = int(o_cnt[over].max())
+            f_nbr, f_cnt, _ = oracle.rows(pos, box, cutoff, skin, K2, which[over])
+            raw = nbr_t[s:e][torch.from_numpy(over).to(nbr_t.device)].cpu().numpy()
+            for r, row in enumerate(raw):
+                assert np.all(row >= 0) and np.unique(row).size == K
+                assert set(row.tolist()) <= set(f_nbr[r, :f_cnt[r]].tolist())
+    return overflow

@@ -1,9 +1,8 @@
 """GPU path vs the CPU oracle, through the C ABI (bit-exact).
 
 Curve order: the permutation (ties by index) and keys equal the oracle's at
-every size.  Neighbor lists: canonicalised rows and counts equal the
-oracle's; at the 1M and 10M workloads on sampled rows plus size-independent
-properties.  All inputs are the seeded workloads of
+every size, the 1M and 10M workloads included.  Neighbor lists: every
+canonicalised row and count equals the oracle's, at full size too.  All inputs are the seeded workloads of
 neighbor_list_construction_b200.workloads.
 """
 import numpy as np
@@ -100,12 +99,17 @@ def test_sort_long_prefix_runs(ctx, oracle, case):
     np.testing.assert_array_equal(ps[:, :3], pos[o_perm, :3])
 
 
-def test_sort_full_size_salt_solution(ctx, oracle):
-    w = gu.workload("saltwater10m")
-    perm, ps, ks = gpu_sort(ctx, w.pos, w.box)
-    o_perm, o_ks = oracle.sort(w.pos, w.box)
+@pytest.mark.parametrize("name", ["saltwater1m", "saltwater10m", "shell10m"])
+@pytest.mark.parametrize("curve", ["hilbert", "morton"])
+def test_sort_full_size(ctx, oracle, name, curve):
+    """The whole permutation, sorted keys and sorted positions of the 1M and
+    10M workloads, both curves."""
+    w = gu.workload(name)
+    perm, ps, ks = gpu_sort(ctx, w.pos, w.box, curve)
+    o_perm, o_ks = oracle.sort(w.pos, w.box, curve)
     np.testing.assert_array_equal(ks, o_ks)
     np.testing.assert_array_equal(perm, o_perm)
+    np.testing.assert_array_equal(ps[:, :3], w.pos[o_perm, :3])
 
 
 # --------------------------------------------------------------- neighbor lists
@@ -293,33 +297,28 @@ def test_build_mixed_density_uses_both_paths(ctx, nl, oracle):
 
 
 @pytest.mark.parametrize("name", ["saltwater1m", "saltwater10m", "shell10m"])
-def test_build_full_size_sampled(ctx, oracle, name):
-    """Full-size workloads, in the order the benchmark uses (curve-sorted):
-    sampled rows against the oracle, symmetry of the sampled rows, and the
-    global pair count parity."""
+def test_build_full_size(ctx, oracle, name):
+    """Full-size workloads in the order the benchmark uses (curve-sorted):
+    every row and count against the oracle, and the overflow status."""
     w = gu.workload(name)
     ps = gu.oracle_sorted(name)
     nbr_t, cnt_t = ctx.build(dev(ps), w.box, w.cutoff, w.skin, w.capacity)
     st = ctx.sync_status()
-    assert st in (0, 1)
-    cnt = cnt_t.cpu().numpy()
-    rng = np.random.default_rng(123)
-    n = w.n
-    sample = np.unique(np.concatenate([rng.choice(n, 3000, replace=False),
-                                       np.arange(0, 64), np.arange(n - 64, n)]))
-    nbr_s = nbr_t[torch.from_numpy(sample).cuda()].cpu().numpy()
-    o_nbr, o_cnt, o_ov = oracle.rows(ps, w.box, w.cutoff, w.skin, w.capacity, sample)
-    gu.assert_rows_match(nbr_s, cnt[sample], o_nbr, o_cnt)
-    assert (st == 1) == bool((cnt > w.capacity).any())
-    # every directed pair has its reverse: total is even, and sampled rows
-    # appear in their neighbors' rows
-    assert int(cnt.astype(np.int64).sum()) % 2 == 0
-    sub = sample[:200]
-    rows = nbr_t[torch.from_numpy(sub).cuda()].cpu().numpy()
-    for i, row in zip(sub, rows):
-        js = row[row >= 0]
-        back = nbr_t[torch.from_numpy(js.astype(np.int64)).cuda()].cpu().numpy()
-        assert np.all((back == i).sum(axis=1) == 1)
+    over = gu.assert_all_rows_match(oracle, nbr_t, cnt_t, ps, w.box, w.cutoff, w.skin,
+                                    w.capacity)
+    assert st == (1 if over else 0)
+
+
+@pytest.mark.parametrize("name", ["saltwater10m", "shell10m"])
+def test_build_full_size_unsorted_input(ctx, oracle, name):
+    """The same workloads in their shuffled input order (no curve sort): the
+    cell binning alone decides the staging, every row is compared."""
+    w = gu.workload(name)
+    nbr_t, cnt_t = ctx.build(dev(w.pos), w.box, w.cutoff, w.skin, w.capacity)
+    st = ctx.sync_status()
+    over = gu.assert_all_rows_match(oracle, nbr_t, cnt_t, w.pos, w.box, w.cutoff, w.skin,
+                                    w.capacity)
+    assert st == (1 if over else 0)
 
 
 # ------------------------------------------------------------------ skin check
@@ -368,6 +367,8 @@ def test_displacement_stand_in_matches_oracle(ctx, nl, oracle):
 
 # ------------------------------------------------------------------ replay
 def _replay(ctx, nl, oracle, name, steps, seed=2024, check_lists=True):
+    """nl_replay of `steps` steps against the oracle's loop: the decisions, the
+    final positions and every row of the lists of the last rebuild."""
     w = gu.workload(name)
     ps = gu.oracle_sorted(name)
     p = dev(ps)
@@ -383,9 +384,10 @@ def _replay(ctx, nl, oracle, name, steps, seed=2024, check_lists=True):
     np.testing.assert_array_equal(dec.cpu().numpy(), o_dec)
     np.testing.assert_array_equal(p.cpu().numpy()[:, :3], o_final[:, :3])
     if check_lists:
-        o_nbr, o_cnt, o_ov = oracle.build(o_ref, w.box, w.cutoff, w.skin, w.capacity)
-        assert st == (1 if o_ov else 0)
-        gu.assert_rows_match(nbr.cpu().numpy(), cnt.cpu().numpy(), o_nbr, o_cnt)
+        # the lists of the last rebuild: built on the positions of that step
+        over = gu.assert_all_rows_match(oracle, nbr, cnt, o_ref, w.box, w.cutoff, w.skin,
+                                        w.capacity)
+        assert st == (1 if over else 0)
     return o_dec
 
 
@@ -400,7 +402,7 @@ def test_replay_twice_reuses_graph(ctx, nl, oracle):
 
 
 def test_replay_salt_solution_200_steps(ctx, nl, oracle):
-    dec = _replay(ctx, nl, oracle, "saltwater10m", 200, check_lists=False)
+    dec = _replay(ctx, nl, oracle, "saltwater10m", 200)
     assert 3 <= dec.sum() <= 40
 
 
