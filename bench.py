@@ -137,29 +137,63 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(steps: int = 1, nside: int = 66) -> dict:
-    """The CPU oracle, as it stands, on a bounded sample of the salt-solution
-    recipe (nside^3 sites: 66 -> ~0.86M atoms, about 11 s of one host core;
-    40 -> ~0.19M): curve sort + neighbor list + skin check per step,
-    single-threaded."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_step(w, threads: int, steps: int = 1) -> dict:
+    """The CPU oracle, as it stands, on workload `w`: curve sort + neighbor
+    list + skin check per step, its per-atom and per-row loops on `threads`
+    OpenMP threads (1 = the plain single-threaded oracle)."""
     import oracle
-    from neighbor_list_construction_b200 import workloads
-    w = workloads.make(f"saltwater_n{nside}", seed=4)
     oracle.lib()
-    t0 = time.perf_counter()
-    pairs = 0
-    for _ in range(steps):
-        perm, _ = oracle.sort(w.pos, w.box)
-        ps = w.pos[perm]
-        nbr, cnt, _ = oracle.build(ps, w.box, w.cutoff, w.skin, w.capacity)
-        oracle.skin_check(ps, ps, w.box, w.skin)
-        pairs += int(cnt.sum())
-    dt = time.perf_counter() - t0
-    return {"value": steps * w.n / dt, "unit": "atoms/s", "cores": 1, "kind": "oracle",
-            "sample": f"{w.n} atoms, salt-solution recipe on {nside}^3 sites (same density, "
-                      f"cutoff 5.75, skin 1.0, capacity 256), sort+build+skin x{steps}, "
-                      f"{dt:.1f} s single-threaded",
-            "pairs_per_s": pairs / dt, "seconds": dt}
+    old = oracle.set_threads(threads)
+    try:
+        t0 = time.perf_counter()
+        pairs = 0
+        for _ in range(steps):
+            perm, _ = oracle.sort(w.pos, w.box)
+            ps = w.pos[perm]
+            nbr, cnt, _ = oracle.build(ps, w.box, w.cutoff, w.skin, w.capacity)
+            oracle.skin_check(ps, ps, w.box, w.skin)
+            pairs += int(cnt.sum())
+            del nbr
+        dt = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(old)
+    return {"value": steps * w.n / dt, "unit": "atoms/s", "cores": threads, "kind": "oracle",
+            "pairs_per_s": pairs / dt, "seconds": dt, "steps": steps}
+
+
+def sample_workload(nside: int = 66):
+    """A smaller instance of the salt-solution recipe (nside^3 sites; 66 ->
+    859,376 atoms, 1/12 of saltwater10m): same density, cutoff 5.75, skin 1.0,
+    capacity 256."""
+    from neighbor_list_construction_b200 import workloads
+    return workloads.make(f"saltwater_n{nside}", seed=4)
+
+
+def cpu_baseline(workload: str, w) -> dict:
+    """The oracle on the benchmark workload itself, all host cores (one step),
+    and single-threaded on the 66^3-site instance of the same recipe."""
+    cores = cpu_cores()
+    full = oracle_step(w, cores)
+    small = sample_workload()
+    one = oracle_step(small, 1)
+    return {"value": full["value"], "unit": "atoms/s", "cores": cores, "kind": "oracle",
+            "sample": f"{workload} itself ({w.n} atoms): sort+build+skin x1 on {cores} host "
+                      f"cores ({cpu_model()}), {full['seconds']:.1f} s",
+            "pairs_per_s": full["pairs_per_s"],
+            "single_core": {"value": one["value"], "unit": "atoms/s", "cores": 1,
+                            "sample": f"{small.n} atoms, salt-solution recipe on 66^3 sites, "
+                                      f"sort+build+skin x1, {one['seconds']:.1f} s"}}
 
 
 def arm_config(workload: str, world: int) -> dict:
@@ -172,24 +206,31 @@ def arm_config(workload: str, world: int) -> dict:
 
 
 def run_reference(args, rank: int, world: int) -> None:
-    """The oracle on the host cores: K timed steps (after up to 3 warm-up
-    steps), each a ~0.19M-atom sample of the salt-solution recipe, so the
-    whole run takes about a minute."""
+    """The oracle, as it stands, on all host cores: K timed steps (after up to
+    3 warm-up steps), each one curve sort + neighbor list + skin check of the
+    66^3-site instance of the benchmark's salt-solution recipe (859,376 atoms,
+    a twelfth of saltwater10m), so a 20-step run takes about a minute."""
     if rank != 0:
         return
+    cores = cpu_cores()
+    small = sample_workload()
     warm = max(0, min(args.warmup, 3))
     if warm:
-        oracle_sample(warm, nside=40)
-    r = oracle_sample(args.steps, nside=40)
+        oracle_step(small, cores, warm)
+    r = oracle_step(small, cores, args.steps)
     cfg = arm_config(args.workload, world)
-    cfg["sample"] = r["sample"]
+    sample = (f"{small.n} atoms, salt-solution recipe on 66^3 sites (same density, cutoff "
+              f"5.75, skin 1.0, capacity 256), sort+build+skin x{args.steps} on {cores} host "
+              f"cores ({cpu_model()}), {r['seconds']:.1f} s")
+    cfg["sample"] = sample
     line = {
         "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "atoms/s",
         "n_gpus": world, "steps": args.steps, "warmup": warm,
         "ms_per_step": 1000.0 * r["seconds"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": cfg,
-        "cpu_baseline": {k: r[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "cpu_baseline": {"value": r["value"], "unit": "atoms/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": r["value"], "unit": "atoms/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "pairs_per_s": r["pairs_per_s"],
@@ -408,6 +449,36 @@ def sharded_timing(torch, ctx, ps, w, K, nranks: int = 8, reps: int = 2) -> dict
             "ms_all_shards_one_gpu": e0.elapsed_time(e1) / reps}
 
 
+def run_extras(nl, torch, ctx, ps, pos, w, K, workload: str) -> dict:
+    """The rows of the scope table beyond the timed step, each timed on the
+    device after the step (outside its timed region): the replayed skin-check
+    interval against host-driven steps, nl_build after Hilbert vs Morton
+    order (this workload and shell10m, the non-uniform one), the close-pair
+    detector, edge features and their CSR form, and the curve-sharded build
+    (8 shards on this GPU)."""
+    h = ctx.handle
+    out = {"interval": interval_timing(nl, torch, h, ps, w, K, w.steps or 200),
+           "curves": curve_comparison(nl, torch, h, pos, w, K),
+           "close_pairs": close_pair_timing(nl, torch, h, ps, w, K),
+           "edge_features": edge_feature_timing(nl, torch, h, ps, w, K),
+           "sharded": sharded_timing(torch, ctx, ps, w, K)}
+    torch.cuda.empty_cache()
+    if workload != "shell10m":
+        from neighbor_list_construction_b200 import workloads
+        sw = workloads.make("shell10m")
+        sctx = nl.Context(sw.n, sw.capacity)
+        try:
+            spos = torch.from_numpy(sw.pos).cuda()
+            c = curve_comparison(nl, torch, sctx.handle, spos, sw, sw.capacity)
+            c["workload"] = "shell10m"
+            out["curves_shell10m"] = c
+            del spos
+        finally:
+            sctx.close()
+            torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     import torch
     import torch.distributed as dist
@@ -479,62 +550,79 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     ms_max = max_over_ranks(ms)
 
     # ---- end to end through the public API with host buffers.  Every step
-    # copies its positions from pinned host memory and its counts back.
-    # Serial: copy in, step, copy out on one stream.  Pipelined (the reported
-    # e2e): positions and counts double-buffered on the device, the copies on
-    # one stream per direction, so step i's kernels overlap the upload for
-    # step i+1 and the download of step i-1.
-    barrier()
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        pos.copy_(pos_host, non_blocking=True)
-        step(pos)
-        cnt_host.copy_(cnt, non_blocking=True)
-    f1.record(stream)
-    barrier()
-    e2e_serial_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps)
-
+    # copies its positions in from pinned host memory and its result back to
+    # pinned host memory: the padded rows and counts (the reported e2e), or,
+    # for comparison, the counts alone.  Pipelined: positions and results
+    # double-buffered on the device, one copy stream per direction, so step
+    # i's kernels overlap the upload for step i+1 and the download of step
+    # i-1.  Serial: copy in, step, copy out on one stream.
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    nbr_host = torch.empty(n, K, dtype=torch.int32).pin_memory()
     pos_buf = [pos, torch.empty_like(pos)]
     cnt_buf = [cnt, torch.empty_like(cnt)]
-    computed = [torch.cuda.Event(), torch.cuda.Event()]   # step done with pos_buf/cnt_buf[b]
-    uploaded = [torch.cuda.Event(), torch.cuda.Event()]
-    downloaded = [torch.cuda.Event(), torch.cuda.Event()]
+    nbr_buf = [nbr, torch.empty_like(nbr)]
 
-    def step_into(src, counts):
+    def step_into(src, counts, rows):
         sort_fn(h, src, box, perm, ps, None, stream)
-        nl.nl_build(h, ps, box, w.cutoff, w.skin, K, nbr, counts, stream)
+        nl.nl_build(h, ps, box, w.cutoff, w.skin, K, rows, counts, stream)
         nl.nl_skin_check(h, ps, box, w.skin, rb, None, stream)
 
-    barrier()
-    g0 = torch.cuda.Event(enable_timing=True)
-    g1 = torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    up.wait_event(g0)
-    down.wait_event(g0)
-    for i in range(args.steps):
-        b = i & 1
-        with torch.cuda.stream(up):
+    def e2e_serial(rows: bool) -> float:
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            pos.copy_(pos_host, non_blocking=True)
+            step_into(pos, cnt, nbr)
+            cnt_host.copy_(cnt, non_blocking=True)
+            if rows:
+                nbr_host.copy_(nbr, non_blocking=True)
+        f1.record(stream)
+        barrier()
+        return max_over_ranks(f0.elapsed_time(f1) / args.steps)
+
+    def e2e_pipelined(rows: bool) -> float:
+        computed = [torch.cuda.Event(), torch.cuda.Event()]   # step done with buffers b
+        uploaded = [torch.cuda.Event(), torch.cuda.Event()]
+        downloaded = [torch.cuda.Event(), torch.cuda.Event()]
+        barrier()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        up.wait_event(g0)
+        down.wait_event(g0)
+        for i in range(args.steps):
+            b = i & 1
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(computed[b])
+                pos_buf[b].copy_(pos_host, non_blocking=True)
+                uploaded[b].record(up)
+            stream.wait_event(uploaded[b])
             if i >= 2:
-                up.wait_event(computed[b])
-            pos_buf[b].copy_(pos_host, non_blocking=True)
-            uploaded[b].record(up)
-        stream.wait_event(uploaded[b])
-        if i >= 2:
-            stream.wait_event(downloaded[b])
-        step_into(pos_buf[b], cnt_buf[b])
-        computed[b].record(stream)
-        with torch.cuda.stream(down):
-            down.wait_event(computed[b])
-            cnt_host.copy_(cnt_buf[b], non_blocking=True)
-            downloaded[b].record(down)
-    stream.wait_stream(up)
-    stream.wait_stream(down)
-    g1.record(stream)
-    barrier()
-    e2e_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+                stream.wait_event(downloaded[b])
+            step_into(pos_buf[b], cnt_buf[b], nbr_buf[b])
+            computed[b].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                cnt_host.copy_(cnt_buf[b], non_blocking=True)
+                if rows:
+                    nbr_host.copy_(nbr_buf[b], non_blocking=True)
+                downloaded[b].record(down)
+        stream.wait_stream(up)
+        stream.wait_stream(down)
+        g1.record(stream)
+        barrier()
+        return max_over_ranks(g0.elapsed_time(g1) / args.steps)
+
+    e2e_ms = e2e_pipelined(True)
+    e2e_serial_ms = e2e_serial(True)
+    # the host rows are a bit-for-bit copy of the last step's device rows
+    rows_ok = bool(torch.equal(nbr_host[:4096], nbr[:4096].cpu()))
+    e2e_counts_ms = e2e_pipelined(False)
+    e2e_counts_serial_ms = e2e_serial(False)
+    del nbr_buf[1], cnt_buf[1], pos_buf[1]
     st = ctx.sync_status()
 
     if rank == 0:
@@ -586,24 +674,27 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                          "bytes_per_atom": bytes_per_atom, "launch_ms": dom_ms},
             "phases_ms": {k: v[0] / args.steps for k, v in phases.items() if v[1]},
             "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "atoms/s",
-                    "h2d_bytes_per_step": n * 16, "d2h_bytes_per_step": n * 4,
+                    "h2d_bytes_per_step": n * 16, "d2h_bytes_per_step": n * 4 * (K + 1),
+                    "result": "padded rows int32[n, K] and counts int32[n] to pinned host "
+                              "memory every step",
                     "ms_per_step": e2e_ms, "pipelined": True,
                     "serial_value": world * n / (e2e_serial_ms * 1e-3),
-                    "serial_ms_per_step": e2e_serial_ms},
+                    "serial_ms_per_step": e2e_serial_ms, "rows_copied_ok": rows_ok,
+                    "counts_only": {"value": world * n / (e2e_counts_ms * 1e-3),
+                                    "unit": "atoms/s", "h2d_bytes_per_step": n * 16,
+                                    "d2h_bytes_per_step": n * 4, "ms_per_step": e2e_counts_ms,
+                                    "serial_ms_per_step": e2e_counts_serial_ms,
+                                    "result": "counts int32[n] only; the rows stay on the "
+                                              "device"}},
             "clocks": clk,
             "gpu_launches": int(round(launches_per_step * args.steps)),
             "status": nl.nl_status_string(st),
         }
-        if args.extras and world == 1:
-            line["interval"] = interval_timing(nl, torch, h, ps, w, K, w.steps or 200)
-            line["curves"] = curve_comparison(nl, torch, h, pos, w, K)
-            line["close_pairs"] = close_pair_timing(nl, torch, h, ps, w, K)
-            line["edge_features"] = edge_feature_timing(nl, torch, h, ps, w, K)
-            line["sharded"] = sharded_timing(torch, ctx, ps, w, K)
+        if not args.no_extras and world == 1:
+            del nbr_host
+            line["extras"] = run_extras(nl, torch, ctx, ps, pos, w, K, args.workload)
         if world == 1 and not args.no_cpu_baseline:
-            cb = oracle_sample(1)
-            line["cpu_baseline"] = {"value": cb["value"], "unit": "atoms/s", "cores": cb["cores"],
-                                    "kind": "oracle", "sample": cb["sample"]}
+            line["cpu_baseline"] = cpu_baseline(args.workload, w)
         print(json.dumps(line), flush=True)
     clocks.stop()
     ctx.close()
@@ -697,9 +788,9 @@ def main():
     ap.add_argument("--sharded", action="store_true",
                     help="time the pages' multi-GPU design instead of replicas: equal-count "
                          "curve shards of the one workload, halo exchange over NCCL")
-    ap.add_argument("--extras", action="store_true",
-                    help="also time the replayed skin-check interval (graph vs eager) "
-                         "and nl_build after Hilbert vs Morton order")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the rows timed after the step (replayed interval vs eager, "
+                         "Hilbert vs Morton, close pairs, edge features and CSR, 8 shards)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
