@@ -431,8 +431,9 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
         c->rebuild_tmp = reinterpret_cast<int32_t *>(c->zero_block + 9);
         c->unsorted = c->zero_block + 12;
         c->fb_count = c->zero_block + 13;
-        c->sort_gate = c->zero_block + 14;
-        c->probe_word = c->zero_block + 15;
+        c->tile_ctr = c->zero_block + 14;
+        c->sort_gate = c->zero_block + 15;
+        c->probe_word = c->zero_block + 16;
         ok &= pairs_set_attributes() == cudaSuccess;
         ok &= cudaMemset(c->zero_block, 0, 64 * sizeof(uint32_t)) == cudaSuccess;
         ok &= cudaDeviceSynchronize() == cudaSuccess;

@@ -136,7 +136,7 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // conceptual cells cx0-1 .. cx0+Gx along x, with a periodic image cell at
 // either end of the box.  Every row is a contiguous range of the
 // cell-ordered array; one lane per row issues its cp.async.bulk copies into
-// shared memory, all completing on one mbarrier.
+// shared memory, all completing on the stage's mbarrier.
 //
 // A home atom meets 25 rows (dy, dz in -2..2).  Atoms of a row are sorted by
 // x, so its candidates in a row lie in the slot window of [x - h, x + h],
@@ -145,26 +145,37 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
 // first slots at 1/16-cell steps in x (conservative: no candidate is lost).
 // A warp scans one row for all its lanes at once: the lanes are consecutive
 // x-sorted home atoms, so at each step their windows sit on nearly
-// consecutive slots and the 16-byte loads rarely share a bank; a lane past
-// its own window loads nothing.  The home row is scanned in two ranges
-// around the atom's own slot, so self never reaches the predicate.
+// consecutive slots; a lane past its own window loads nothing.  The home row
+// is scanned in two ranges around the atom's own slot, so self never reaches
+// the predicate.
 //
-// Hits go to a small per-lane buffer in shared memory; every 8 slots a lane
-// stores its whole 16-byte vectors to its global row and moves the partial
-// vector to the buffer's start.  Rows are finished with one cp.async.bulk
-// copy from a shared block of -1.
+// Hits go to a small per-lane buffer in shared memory, interleaved across
+// the warp's lanes so that each per-slot store falls in the lane's own bank;
+// when a lane holds kFlushAt entries the warp stores its whole 16-byte
+// vectors to the rows.  Rows are finished with one cp.async.bulk copy from a
+// shared block of -1.
 // ---------------------------------------------------------------------------
-constexpr int kTX = 3, kTY = 2, kTZ = 3;   // home cells per tile
+constexpr int kTX = 3, kTY = 4, kTZ = 4;   // home cells per tile
 constexpr int kSY = kTY + 4, kSZ = kTZ + 4;
-constexpr int kSRows = kSY * kSZ;           // staged rows (42)
-constexpr int kHome = kTY * kTZ;            // home rows
+constexpr int kSRows = kSY * kSZ;           // staged rows (64)
+static_assert(kSRows <= 64, "a tile's rows are described two per lane of one warp");
+constexpr int kHome = kTY * kTZ;            // home rows (16)
+static_assert(kHome <= 32, "home rows are counted one per lane");
 constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
 constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
 constexpr int kRowTab = kSCells * kBinsPerCell;
 constexpr int kFlushAt = 8;                 // pending hits that make the warp flush
 constexpr int kBuf = kFlushAt + 4;          // entries of a lane's hit buffer (7 pending + 4 new)
-constexpr int kTileWarps = 5;               // ~140 home atoms: mostly 4-6 chunks of 32
-constexpr int kTileCtas = 5;                // CTAs per SM the stage is sized for
+constexpr uint32_t kHitStride = 128;        // bytes between a lane's buffer entries (32 lanes x 4)
+constexpr int kPipeStages = 3;              // staged tiles per CTA of the persistent launch
+constexpr int kPipeMeta = kPipeStages + 1;  // tile descriptions: one ahead of the stages
+constexpr int kPipeConsumers = 24;          // searching warps per CTA (plus one staging warp)
+constexpr int kPipeThreads = 32 * (1 + kPipeConsumers);
+constexpr int kQueue = 512;                 // chunk-queue entries
+constexpr uint32_t kQueueEnd = 0xffffffffu;
+constexpr uint32_t kEmptyCount = 1u << 16;  // arrivals that free a stage: the staging warp's
+                                            // (kEmptyCount - chunks) plus one per chunk
+constexpr int kListedWarps = 5;             // warps of a listed-tile CTA
 constexpr int kListedCtas = 3;              // CTAs per SM the listed-tile launch may use
 constexpr int kStageMin = 1024;             // fewest staged slots worth a launch
 
@@ -176,6 +187,13 @@ struct TileRows {
     int home_pref[kHome + 1];        // home atoms before home row h
     int total;                       // staged slots, gaps included
     int fallback;
+};
+
+// Where a staged tile sits in the grid.
+struct TileMeta {
+    int cx0, cy0, cz0;     // first home cell
+    int Gx, Gy, Gz;        // home cells (fewer at the high faces)
+    int general;           // touches a periodic face: shifted scans where needed
 };
 
 struct TileParams {
@@ -192,7 +210,9 @@ struct TileParams {
     const uint32_t *unsorted;
     uint32_t *fb_list;
     uint32_t *fb_count;
+    uint32_t *tile_ctr;             // next tile of the persistent launch
     int tiles_x, tiles_y;
+    int ntiles;
     int K;
     int stage_max;      // staged slots per tile, gaps included
     float side_x, side_y, side_z;
@@ -216,6 +236,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                  "r"(bytes)
+                 : "memory");
+}
+
+// Arrival of this thread (release: its earlier shared-memory reads and
+// writes are ordered before the phase completes), counting `count` arrivals.
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(count)
                  : "memory");
 }
 
@@ -270,74 +299,14 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ uint4 lds_u4(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v)
-{
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-
-
-// One candidate: three fp32 differences (each followed by its periodic
-// shift when GEN), three products, two sums, all round-to-nearest with no
-// contraction; on r2 < rl2 the candidate's atom index is appended at bp.
-template <bool GEN>
-__device__ __forceinline__ void test_cand(const float4 c, const float4 me, float sx, float sy,
-                                          float sz, float rl2, uint32_t &bp)
-{
-    if (GEN)
-        asm volatile(
-            "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
-            "sub.rn.f32 dx, %1, %5;\n\t"
-            "sub.rn.f32 dy, %2, %6;\n\t"
-            "sub.rn.f32 dz, %3, %7;\n\t"
-            "add.rn.f32 dx, dx, %9;\n\t"
-            "add.rn.f32 dy, dy, %10;\n\t"
-            "add.rn.f32 dz, dz, %11;\n\t"
-            "mul.rn.f32 dx, dx, dx;\n\t"
-            "mul.rn.f32 dy, dy, dy;\n\t"
-            "mul.rn.f32 dz, dz, dz;\n\t"
-            "add.rn.f32 s, dx, dy;\n\t"
-            "add.rn.f32 s, s, dz;\n\t"
-            "setp.lt.f32 p, s, %8;\n\t"
-            "@p st.shared.b32 [%0], %4;\n\t"
-            "@p add.u32 %0, %0, 4;\n\t}"
-            : "+r"(bp)
-            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "f"(me.x), "f"(me.y),
-              "f"(me.z), "f"(rl2), "f"(sx), "f"(sy), "f"(sz));
-    else
-        asm volatile(
-            "{\n\t.reg .f32 dx, dy, dz, s;\n\t.reg .pred p;\n\t"
-            "sub.rn.f32 dx, %1, %5;\n\t"
-            "sub.rn.f32 dy, %2, %6;\n\t"
-            "sub.rn.f32 dz, %3, %7;\n\t"
-            "mul.rn.f32 dx, dx, dx;\n\t"
-            "mul.rn.f32 dy, dy, dy;\n\t"
-            "mul.rn.f32 dz, dz, dz;\n\t"
-            "add.rn.f32 s, dx, dy;\n\t"
-            "add.rn.f32 s, s, dz;\n\t"
-            "setp.lt.f32 p, s, %8;\n\t"
-            "@p st.shared.b32 [%0], %4;\n\t"
-            "@p add.u32 %0, %0, 4;\n\t}"
-            : "+r"(bp)
-            : "f"(c.x), "f"(c.y), "f"(c.z), "r"(__float_as_uint(c.w)), "f"(me.x), "f"(me.y),
-              "f"(me.z), "f"(rl2));
-}
-
 // Four consecutive slots at shared address `addr` of which the first `act`
 // (0..4 or more) belong to this lane's range: the active ones are loaded
-// into c[0..3] (an inactive slot keeps a stale value), and each is tested as
-// in test_cand, a hit requiring the slot to be active.  GEN: x shifts
+// into c[0..3] (an inactive slot keeps a stale value), and each is tested:
+// three fp32 differences (each followed by its periodic shift when GEN),
+// three products and two sums, round-to-nearest with no contraction --
+// (dx*dx + dy*dy) + dz*dz -- a hit requiring r2 < rl2 and the slot to be
+// active.  A hit stores the candidate's index at bp and moves bp to the
+// lane's next buffer entry, 128 bytes on (kHitStride).  GEN: x shifts
 // sx0..sx3 per slot and the row's y, z shifts.  CLOSE: each hit also lowers
 // cl.mn to its r2 and counts in cl.nc when r2 < close_d2.
 template <bool GEN, bool CLOSE>
@@ -369,7 +338,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q0, dx, %24, q0;\n\t"
                      "@q0 st.shared.b32 [%0], %4;\n\t"
-                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "@q0 add.u32 %0, %0, 128;\n\t"
                      "@q0 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q0;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -386,7 +355,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q1, dx, %24, q1;\n\t"
                      "@q1 st.shared.b32 [%0], %8;\n\t"
-                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "@q1 add.u32 %0, %0, 128;\n\t"
                      "@q1 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q1;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -403,7 +372,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q2, dx, %24, q2;\n\t"
                      "@q2 st.shared.b32 [%0], %12;\n\t"
-                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "@q2 add.u32 %0, %0, 128;\n\t"
                      "@q2 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q2;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -420,7 +389,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q3, dx, %24, q3;\n\t"
                      "@q3 st.shared.b32 [%0], %16;\n\t"
-                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "@q3 add.u32 %0, %0, 128;\n\t"
                      "@q3 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q3;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -450,7 +419,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q0, dx, %22, q0;\n\t"
                      "@q0 st.shared.b32 [%0], %4;\n\t"
-                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "@q0 add.u32 %0, %0, 128;\n\t"
                      "sub.rn.f32 dx, %5, %19;\n\t"
                      "sub.rn.f32 dy, %6, %20;\n\t"
                      "sub.rn.f32 dz, %7, %21;\n\t"
@@ -464,7 +433,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q1, dx, %22, q1;\n\t"
                      "@q1 st.shared.b32 [%0], %8;\n\t"
-                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "@q1 add.u32 %0, %0, 128;\n\t"
                      "sub.rn.f32 dx, %9, %19;\n\t"
                      "sub.rn.f32 dy, %10, %20;\n\t"
                      "sub.rn.f32 dz, %11, %21;\n\t"
@@ -478,7 +447,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q2, dx, %22, q2;\n\t"
                      "@q2 st.shared.b32 [%0], %12;\n\t"
-                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "@q2 add.u32 %0, %0, 128;\n\t"
                      "sub.rn.f32 dx, %13, %19;\n\t"
                      "sub.rn.f32 dy, %14, %20;\n\t"
                      "sub.rn.f32 dz, %15, %21;\n\t"
@@ -492,7 +461,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q3, dx, %22, q3;\n\t"
                      "@q3 st.shared.b32 [%0], %16;\n\t"
-                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "@q3 add.u32 %0, %0, 128;\n\t"
                      "}"
                      : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
                      : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(sx0), "f"(sx1), "f"(sx2), "f"(sx3), "f"(sy), "f"(sz));
@@ -516,7 +485,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q0, dx, %24, q0;\n\t"
                      "@q0 st.shared.b32 [%0], %4;\n\t"
-                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "@q0 add.u32 %0, %0, 128;\n\t"
                      "@q0 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q0;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -530,7 +499,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q1, dx, %24, q1;\n\t"
                      "@q1 st.shared.b32 [%0], %8;\n\t"
-                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "@q1 add.u32 %0, %0, 128;\n\t"
                      "@q1 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q1;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -544,7 +513,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q2, dx, %24, q2;\n\t"
                      "@q2 st.shared.b32 [%0], %12;\n\t"
-                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "@q2 add.u32 %0, %0, 128;\n\t"
                      "@q2 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q2;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -558,7 +527,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q3, dx, %24, q3;\n\t"
                      "@q3 st.shared.b32 [%0], %16;\n\t"
-                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "@q3 add.u32 %0, %0, 128;\n\t"
                      "@q3 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q3;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
@@ -585,7 +554,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q0, dx, %22, q0;\n\t"
                      "@q0 st.shared.b32 [%0], %4;\n\t"
-                     "@q0 add.u32 %0, %0, 4;\n\t"
+                     "@q0 add.u32 %0, %0, 128;\n\t"
                      "sub.rn.f32 dx, %5, %19;\n\t"
                      "sub.rn.f32 dy, %6, %20;\n\t"
                      "sub.rn.f32 dz, %7, %21;\n\t"
@@ -596,7 +565,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q1, dx, %22, q1;\n\t"
                      "@q1 st.shared.b32 [%0], %8;\n\t"
-                     "@q1 add.u32 %0, %0, 4;\n\t"
+                     "@q1 add.u32 %0, %0, 128;\n\t"
                      "sub.rn.f32 dx, %9, %19;\n\t"
                      "sub.rn.f32 dy, %10, %20;\n\t"
                      "sub.rn.f32 dz, %11, %21;\n\t"
@@ -607,7 +576,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q2, dx, %22, q2;\n\t"
                      "@q2 st.shared.b32 [%0], %12;\n\t"
-                     "@q2 add.u32 %0, %0, 4;\n\t"
+                     "@q2 add.u32 %0, %0, 128;\n\t"
                      "sub.rn.f32 dx, %13, %19;\n\t"
                      "sub.rn.f32 dy, %14, %20;\n\t"
                      "sub.rn.f32 dz, %15, %21;\n\t"
@@ -618,7 +587,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q3, dx, %22, q3;\n\t"
                      "@q3 st.shared.b32 [%0], %16;\n\t"
-                     "@q3 add.u32 %0, %0, 4;\n\t"
+                     "@q3 add.u32 %0, %0, 128;\n\t"
                      "}"
                      : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
                      : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2));
@@ -639,41 +608,63 @@ __device__ __forceinline__ void stg_u4(char *p, uint4 v)
                  : "memory");
 }
 
-// Output state of one lane: hits are appended at bp in the lane's buffer
-// (shared memory from `buf`); the first gfl bytes of the atom's row are
-// stored; Kb = capacity in bytes.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Output state of one lane.  Its hit buffer is interleaved with the other
+// lanes of the warp: entry e sits at base + e * kHitStride (base = the
+// warp's buffer + 4 * lane), so the per-slot hit stores of a warp always fall
+// in 32 different banks.  bp = the next free entry; the first gfl bytes of
+// the atom's row are stored; Kb = capacity in bytes.
 struct LaneOut {
-    uint32_t bp, buf, gfl, Kb;
+    uint32_t bp, base, gfl, Kb;
     char *grow;
 };
 
-// Store the lane's whole 16-byte vectors to its row (entries past the
-// capacity are only counted) and move the partial vector to the buffer's
-// start; called when some lane of the warp holds kFlushAt entries, so at
-// most kBuf - 1 are pending.
+__device__ __forceinline__ uint4 buffer_vector(uint32_t base, uint32_t e)
+{
+    return make_uint4(lds_u32(base + (e + 0u) * kHitStride), lds_u32(base + (e + 1u) * kHitStride),
+                      lds_u32(base + (e + 2u) * kHitStride), lds_u32(base + (e + 3u) * kHitStride));
+}
+
+// Store the lane's whole 16-byte vectors (4 entries each) to its row
+// (entries past the capacity are only counted) and move the remaining
+// entries (at most 3) to the buffer's start; called when some lane of the
+// warp holds kFlushAt entries, so at most kBuf - 1 are pending.
 __device__ __forceinline__ void flush_check(LaneOut &o)
 {
-    const uint32_t u = o.bp - o.buf;
-    const uint32_t nv = u & ~15u;
+    const uint32_t u = (o.bp - o.base) / kHitStride;
+    const uint32_t nv = u & ~3u;
     if (nv != 0u) {
 #pragma unroll
-        for (uint32_t b = 0; b < 16u * (kBuf / 4 - 1); b += 16u)
-            if (b < nv && o.gfl + b < o.Kb) stg_u4(o.grow + o.gfl + b, lds_u4(o.buf + b));
-        sts_u4(o.buf, lds_u4(o.buf + nv));
-        o.gfl += nv;
-        o.bp -= nv;
+        for (uint32_t v = 0; v < (uint32_t)(kBuf / 4 - 1); ++v)
+            if (4u * v < nv && o.gfl + 16u * v < o.Kb)
+                stg_u4(o.grow + o.gfl + 16u * v, buffer_vector(o.base, 4u * v));
+#pragma unroll
+        for (uint32_t k = 0; k < 3u; ++k)
+            if (nv + k < u) sts_u32(o.base + k * kHitStride, lds_u32(o.base + (nv + k) * kHitStride));
+        o.gfl += 4u * nv;
+        o.bp -= nv * kHitStride;
     }
 }
 
 // Tests this lane's slots lo .. lo+len-1 of one staged row.  The warp runs
-// its longest range in groups of 4; a lane past its own range loads nothing
-// (a NaN candidate), so no shared-memory traffic is spent on it.  The lanes
-// are consecutive x-sorted home atoms and scan the same row at the same
-// step, so their 16-byte loads fall on nearly consecutive slots (few bank
-// conflicts).  When a lane of the warp holds kFlushAt pending hits, the
-// lanes' whole hit vectors are flushed.  GEN: periodic shifts, per slot in x (slots below
-// ri.x are the low image cell, at or above ri.y the high one) and per row in
-// y, z (ri.z, ri.w).
+// its longest range in groups of 4; a lane past its own range loads nothing,
+// so no shared-memory traffic is spent on it.  The lanes are consecutive
+// x-sorted home atoms and scan the same row at the same step, so their
+// 16-byte loads fall on nearly consecutive slots.  When a lane of the warp
+// holds kFlushAt pending hits, the lanes' whole hit vectors are flushed.
+// GEN: periodic shifts, per slot in x (slots below ri.x are the low image
+// cell, at or above ri.y the high one) and per row in y, z (ri.z, ri.w).
 template <bool GEN, bool CLOSE>
 __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int lo, int len,
                                            const float4 me, float rl2, int4 ri, float Lx,
@@ -694,7 +685,7 @@ __device__ __forceinline__ void scan_range(const float4 *__restrict__ stage, int
         scan4<GEN, CLOSE>(a0 + 16u * (uint32_t)j, len - j, c, me, rl2, sxv[0], sxv[1], sxv[2],
                           sxv[3], sy, sz, close_d2, cl, o.bp);
         // flush when some lane holds kFlushAt entries (at most kFlushAt - 1 + 4 pending)
-        if (__any_sync(0xffffffffu, o.bp - o.buf >= 4u * kFlushAt)) flush_check(o);
+        if (__any_sync(0xffffffffu, o.bp - o.base >= kHitStride * kFlushAt)) flush_check(o);
     }
 }
 
@@ -877,27 +868,349 @@ __device__ __forceinline__ uint32_t row_bytes(const RowSrc &rs)
            (uint32_t)kBinsPerCell * (uint32_t)(rs.has_lo + rs.mid_cells + rs.has_hi);
 }
 
-// LISTED = false: one tile per CTA (blockIdx), kTileCtas CTAs per SM; a tile whose
-// rows exceed the stage is listed.  LISTED = true: persistent CTAs (up to
-// kListedCtas per SM, larger stages) over the listed tiles; a tile that still does not
-// fit is searched per atom from global memory.
-template <bool LISTED, bool CLOSE>
-__global__ void __launch_bounds__(kTileWarps * 32, LISTED ? 1 : kTileCtas)
-k_pairs_tiles(const CellGrid g, const TileParams P)
+// Describes tile `t` (rows, their offsets in the stage, home rows) into `tr`
+// and `m` with the 32 lanes of one warp.  Returns, in every lane, the bytes
+// the row copies will carry; tr.fallback is set when the rows do not fit a
+// stage of P.stage_max slots (or the cells are not x-sorted).  ra, rb: the
+// lane's two rows (lane and lane + 32).
+__device__ __forceinline__ uint32_t describe_tile(int t, const CellGrid &g, const TileParams &P,
+                                                  TileRows &tr, int4 *rinfo, TileMeta &m,
+                                                  RowSrc &ra, RowSrc &rb)
 {
-    if (timed_out(P.flags)) return;   // cell starts may not be monotonic
-    extern __shared__ __align__(16) unsigned char tile_smem[];
-    float4 *stage = reinterpret_cast<float4 *>(tile_smem);
-    uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;         // [kSRows][kRowTab]
-    int32_t *hits = reinterpret_cast<int32_t *>(tabs + kSRows * kRowTab);       // [W*32][kBuf]
-    int32_t *negs = hits + kTileWarps * 32 * kBuf;                     // P.K entries of -1
-    __shared__ TileRows tr;
-    __shared__ int4 rinfo[kSRows];   // GEN: x image bounds (slots) and y, z shifts per row
-    __shared__ __align__(8) uint64_t bar;
+    const int lane = threadIdx.x & 31;
+    const int tx = t % P.tiles_x;
+    t /= P.tiles_x;
+    const int ty = t % P.tiles_y, tz = t / P.tiles_y;
+    const int cx0 = tx * kTX, cy0 = ty * kTY, cz0 = tz * kTZ;
+    const int Gx = min(kTX, g.nx - cx0), Gy = min(kTY, g.ny - cy0), Gz = min(kTZ, g.nz - cz0);
+    int cell_scratch[kSCells + 1];
+    describe_row(g, P.cell_start, lane, cx0, cy0, cz0, Gx, Gy, Gz, ra, tr.cell[lane]);
+    describe_row(g, P.cell_start, lane + 32, cx0, cy0, cz0, Gx, Gy, Gz, rb,
+                 lane + 32 < kSRows ? tr.cell[lane + 32] : cell_scratch);
+    // offsets: rows back to back in staged order
+    const int va = ra.len, vb = lane + 32 < kSRows ? rb.len : 0;
+    int xa = va, xb = vb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, xa, o);
+        const int yb = __shfl_up_sync(0xffffffffu, xb, o);
+        if (lane >= o) {
+            xa += ya;
+            xb += yb;
+        }
+    }
+    const int suma = __shfl_sync(0xffffffffu, xa, 31);
+    const int sumb = __shfl_sync(0xffffffffu, xb, 31);
+    const int offa = xa - va;
+    const int offb = suma + xb - vb;
+    const int total = suma + sumb;
+    tr.off[lane] = offa;
+    tr.len[lane] = ra.len;
+    rinfo[lane] = make_int4(offa + ra.lend, offa + ra.rbeg, __float_as_int(ra.sy),
+                            __float_as_int(ra.sz));
+    if (lane + 32 < kSRows) {
+        tr.off[lane + 32] = offb;
+        tr.len[lane + 32] = rb.len;
+        rinfo[lane + 32] = make_int4(offb + rb.lend, offb + rb.rbeg, __float_as_int(rb.sy),
+                                     __float_as_int(rb.sz));
+    }
+    // home rows h = hy + kTY hz are staged rows (hy + 2) + kSY (hz + 2)
+    __syncwarp();
+    int hcnt = 0;
+    if (lane < kHome) {
+        const int hy = lane % kTY, hz = lane / kTY;
+        const int R = (hy + 2) + kSY * (hz + 2);
+        tr.home_begin[lane] = tr.off[R] + tr.cell[R][1];
+        hcnt = hy < Gy && hz < Gz ? tr.cell[R][Gx + 1] - tr.cell[R][1] : 0;
+    }
+    int hx = hcnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, hx, o);
+        if (lane >= o) hx += y;
+    }
+    if (lane < kHome) tr.home_pref[lane] = hx - hcnt;
+    if (lane == kHome - 1) tr.home_pref[kHome] = hx;
+    const uint32_t bytes = __reduce_add_sync(0xffffffffu, row_bytes(ra) + row_bytes(rb));
+    if (lane == 0) {
+        tr.total = total;
+        tr.fallback = (total > P.stage_max || *P.unsorted != 0u) ? 1 : 0;
+        m.cx0 = cx0;
+        m.cy0 = cy0;
+        m.cz0 = cz0;
+        m.Gx = Gx;
+        m.Gy = Gy;
+        m.Gz = Gz;
+        m.general = cx0 == 0 || cx0 + Gx == g.nx || cy0 < 2 || cy0 + Gy + 2 > g.ny || cz0 < 2 ||
+                    cz0 + Gz + 2 > g.nz;
+    }
+    __syncwarp();
+    return bytes;
+}
+
+// Chunk c (home atoms 32c .. 32c + 31 in home-row order) of a staged tile:
+// each lane searches the 25 rows of its atom and writes the atom's row and
+// count.  hb: the warp's interleaved hit buffer; negs_addr: a shared block of
+// -1.
+template <bool CLOSE>
+__device__ __forceinline__ void search_chunk(int c, const float4 *__restrict__ stage,
+                                             const uint8_t *__restrict__ tabs,
+                                             const TileRows &tr, const int4 *rinfo,
+                                             const TileMeta &m, const CellGrid &g,
+                                             const TileParams &P, uint32_t hb,
+                                             uint32_t negs_addr, CloseAcc &cl)
+{
+    const int lane = threadIdx.x & 31;
+    const int nbins = (m.Gx + 2) * kBinsPerCell;
+    const float X0 = (float)(m.cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
+    const float rl2 = g.rl2;
+    const int nhome = tr.home_pref[kHome];
+    const int a = c * 32 + lane;
+    int h = 0;
+    while (h < kHome - 1 && a >= tr.home_pref[h + 1]) ++h;
+    const int slot = tr.home_begin[h] + (a - tr.home_pref[h]);
+    const float qn = __int_as_float(0x7fc00000);
+    float4 me = a < nhome ? stage[slot] : make_float4(qn, qn, qn, qn);
+    // a lane has a row to build when its atom exists and is below n_rows
+    const bool valid = a < nhome && __float_as_int(me.w) < g.n_rows;
+    if (!valid) me = make_float4(qn, qn, qn, qn);
+    const int hy = h % kTY, hz = h / kTY;
+    const float ylo = (float)(m.cy0 + hy) * P.side_y, yhi = (float)(m.cy0 + hy + 1) * P.side_y;
+    const float zlo = (float)(m.cz0 + hz) * P.side_z, zhi = (float)(m.cz0 + hz + 1) * P.side_z;
+    const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
+    const float dz_lo = me.z - zlo, dz_hi = zhi - me.z;
+
+    LaneOut o;
+    o.base = hb + 4u * (uint32_t)lane;
+    o.bp = o.base;
+    o.gfl = 0u;
+    o.Kb = 4u * (uint32_t)P.K;
+    const int myid = __float_as_int(me.w);
+    o.grow = reinterpret_cast<char *>(P.nbr + (int64_t)(valid ? myid : 0) * P.K);
+    const float mxr = me.x - X0;
+    const int Rh = (hy + 2) + kSY * (hz + 2);
+    if (m.general)
+        scan_rows<true, CLOSE>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh,
+                               dy_lo, dy_hi, dz_lo, dz_hi, mxr, P.close_d2, cl, o);
+    else
+        scan_rows<false, CLOSE>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot, Rh,
+                                dy_lo, dy_hi, dz_lo, dz_hi, mxr, P.close_d2, cl, o);
+
+    // ---- finish the row (the scan ends with a flush: at most 3 entries
+    //      pending): the partial vector completed with -1, then -1 from the
+    //      shared block up to the capacity
+    if (valid) {
+        const uint32_t u = (o.bp - o.base) / kHitStride;
+        uint32_t pf = o.gfl;
+        if (u != 0u) {
+            uint4 v;
+            v.x = lds_u32(o.base);
+            v.y = u > 1u ? lds_u32(o.base + kHitStride) : 0xffffffffu;
+            v.z = u > 2u ? lds_u32(o.base + 2u * kHitStride) : 0xffffffffu;
+            v.w = 0xffffffffu;
+            if (o.gfl < o.Kb) stg_u4(o.grow + o.gfl, v);
+            pf += 16u;
+        }
+        if (pf < o.Kb) bulk_s2g(o.grow + pf, negs_addr, o.Kb - pf);
+        bulk_commit();
+        const int cnt = (int)((o.gfl >> 2) + u);
+        P.counts[myid] = cnt;
+        if (cnt > P.K) atomicOr(P.flags, kFlagOverflow);
+    }
+}
+
+// Shared state of the persistent launch (static part).
+struct PipeShared {
+    uint64_t full[kPipeStages];      // a stage's rows have landed (tx-count phase)
+    uint64_t empty[kPipeStages];     // every chunk of a stage's tile is done
+    uint32_t queue[kQueue];          // chunks, in the order the staging warp filled them
+    uint32_t q_tail;                 // entries published
+    uint32_t q_head;                 // entries taken
+    TileRows tr[kPipeMeta];
+    int4 rinfo[kPipeMeta][kSRows];   // x image bounds (slots) and y, z shifts per row
+    TileMeta meta[kPipeMeta];
+};
+
+// Persistent pair search, one CTA per SM.  Warp 0 stages: it takes tiles from
+// a global counter, describes each (ahead of time, into one of kPipeMeta
+// description slots), waits for one of kPipeStages shared-memory stages to be
+// free, issues the rows' cp.async.bulk copies against the stage's `full`
+// barrier, and publishes the tile's chunks (32 home atoms each) on a queue.
+// Warps 1..kPipeConsumers each take the next chunk from the queue, wait for
+// its stage's rows, search it, and arrive on the stage's `empty` barrier; the
+// staging warp's own arrival at fill time counts kEmptyCount - chunks, so the
+// stage frees when its last chunk is done.  No warp waits for another at a
+// CTA barrier: a warp that finishes a chunk moves to the next one, in this
+// tile or the next, while warp 0 stages ahead.  A tile whose rows exceed a
+// stage is listed for k_pairs_listed.  Every wait is bounded: one that gives
+// up records kFlagTimeout and the warp leaves (the staging warp first
+// publishes an end entry per searching warp).
+template <bool CLOSE>
+__global__ void __launch_bounds__(kPipeThreads, 1)
+k_pairs_pipe(const CellGrid g, const TileParams P)
+{
+    // cell starts may not be monotonic; one decision for the whole CTA
+    if (__syncthreads_or(timed_out(P.flags))) return;
+    extern __shared__ __align__(16) unsigned char pipe_smem[];
+    __shared__ PipeShared sh;
+    float4 *stages = reinterpret_cast<float4 *>(pipe_smem);                       // [S][stage_max]
+    uint8_t *tabs = pipe_smem + sizeof(float4) * (size_t)kPipeStages * P.stage_max;   // [S][kSRows][kRowTab]
+    int32_t *hits = reinterpret_cast<int32_t *>(tabs + kPipeStages * kSRows * kRowTab);
+    int32_t *negs = hits + kPipeConsumers * 32 * kBuf;                           // P.K entries of -1
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < P.K; e += blockDim.x) negs[e] = -1;
     fence_proxy_async_smem();   // -1 block is read by bulk copies of any thread
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kPipeStages; ++st) {
+            mbar_init(&sh.full[st], 1);
+            mbar_init(&sh.empty[st], kEmptyCount);
+        }
+        sh.q_tail = 0u;
+        sh.q_head = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------ staging warp
+        uint32_t fpar = 0u, used = 0u;   // per stage: parity of its next fill, filled before
+        uint32_t tail = 0u;
+        int k = 0, mi = 0;               // fills issued; description slot of the next fill
+        bool gave_up = false;
+        int t = lane == 0 ? (int)atomicAdd(P.tile_ctr, 1u) : 0;
+        t = __shfl_sync(0xffffffffu, t, 0);
+        while (t < P.ntiles) {
+            RowSrc ra, rb;
+            const uint32_t bytes = describe_tile(t, g, P, sh.tr[mi], sh.rinfo[mi], sh.meta[mi], ra, rb);
+            const int tile = t;
+            t = lane == 0 ? (int)atomicAdd(P.tile_ctr, 1u) : 0;
+            t = __shfl_sync(0xffffffffu, t, 0);
+            const int nhome = sh.tr[mi].home_pref[kHome];
+            if (sh.tr[mi].fallback) {
+                if (lane == 0) P.fb_list[atomicAdd(P.fb_count, 1u)] = (uint32_t)tile;
+                continue;
+            }
+            if (nhome == 0) continue;
+            const int st = k % kPipeStages;
+            if (used >> st & 1u) {   // the stage's previous tile must be searched out
+                bool done = false;
+                for (uint32_t spins = 0; spins < 4096u && !done; ++spins)
+                    done = mbar_try_wait(&sh.empty[st], ((fpar >> st) & 1u) ^ 1u);
+                if (!done) {
+                    gave_up = true;
+                    break;
+                }
+            }
+            const uint32_t stage_base = smem_u32(stages + (size_t)st * P.stage_max);
+            const uint32_t tab_base = smem_u32(tabs + st * kSRows * kRowTab);
+            if (lane == 0) mbar_arrive_expect_tx(&sh.full[st], bytes);
+            __syncwarp();
+            copy_row(ra, P, g, stage_base, sh.tr[mi].off[lane], tab_base + (uint32_t)(lane * kRowTab),
+                     &sh.full[st]);
+            if (lane + 32 < kSRows)
+                copy_row(rb, P, g, stage_base, sh.tr[mi].off[lane + 32],
+                         tab_base + (uint32_t)((lane + 32) * kRowTab), &sh.full[st]);
+            const uint32_t nchunks = (uint32_t)(nhome + 31) >> 5;
+            if (lane == 0) {
+                mbar_arrive_cnt(&sh.empty[st], kEmptyCount - nchunks);
+                const uint32_t head = (uint32_t)st | ((uint32_t)mi << 2) |
+                                      (((fpar >> st) & 1u) << 5);
+                for (uint32_t c = 0; c < nchunks; ++c)
+                    sh.queue[(tail + c) % kQueue] = head | (c << 8);
+                __threadfence_block();
+                st_volatile_u32(&sh.q_tail, tail + nchunks);
+            }
+            tail += nchunks;
+            fpar ^= 1u << st;
+            used |= 1u << st;
+            ++k;
+            mi = (mi + 1) % kPipeMeta;
+        }
+        if (lane == 0) {
+            if (gave_up) atomicOr(P.flags, kFlagTimeout);
+            for (uint32_t c = 0; c < (uint32_t)kPipeConsumers; ++c)
+                sh.queue[(tail + c) % kQueue] = kQueueEnd;
+            __threadfence_block();
+            st_volatile_u32(&sh.q_tail, tail + (uint32_t)kPipeConsumers);
+        }
+        return;
+    }
+
+    // --------------------------------------------------------- searching warps
+    CloseAcc cl{__int_as_float(0x7f800000), 0u};
+    const uint32_t hb = smem_u32(hits) + (uint32_t)((warp - 1) * 32 * kBuf * 4);   // the warp's buffer
+    const uint32_t negs_addr = smem_u32(negs);
+    for (;;) {
+        uint32_t e = kQueueEnd;
+        if (lane == 0) {
+            const uint32_t tk = atomicAdd(&sh.q_head, 1u);
+            uint32_t spins = 0u;
+            bool ok = true;
+            while (ld_volatile_u32(&sh.q_tail) <= tk) {
+                if (++spins >= kSpinLimit) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(128);
+            }
+            if (ok) {
+                __threadfence_block();
+                e = ld_volatile_u32(&sh.queue[tk % kQueue]);
+            } else {
+                atomicOr(P.flags, kFlagTimeout);
+            }
+        }
+        e = __shfl_sync(0xffffffffu, e, 0);
+        if (e == kQueueEnd) break;
+        const int st = (int)(e & 3u), mslot = (int)((e >> 2) & 7u);
+        const uint32_t par = (e >> 5) & 1u;
+        const int c = (int)(e >> 8);
+        bool done = false;
+        for (uint32_t spins = 0; spins < 4096u && !done; ++spins)   // ~4 s
+            done = mbar_try_wait(&sh.full[st], par);
+        if (!__all_sync(0xffffffffu, done)) {
+            // the stage's copies carry exactly the announced bytes, so the
+            // phase completes when they land: record the timeout, wait once
+            // more (bounded) so no copy is left writing into shared memory,
+            // and leave
+            if (lane == 0) atomicOr(P.flags, kFlagTimeout);
+            for (uint32_t spins = 0; spins < 4096u && !done; ++spins)
+                done = mbar_try_wait(&sh.full[st], par);
+            break;
+        }
+        search_chunk<CLOSE>(c, stages + (size_t)st * P.stage_max, tabs + st * kSRows * kRowTab,
+                            sh.tr[mslot], sh.rinfo[mslot], sh.meta[mslot], g, P, hb, negs_addr, cl);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cnt(&sh.empty[st], 1u);
+    }
+    if (CLOSE) close_publish(cl, P.min_bits, P.n_close);
+    bulk_wait_read<0>();   // the -1 block stays readable until the copies are done
+}
+
+// The listed tiles (rows beyond the persistent launch's stages): persistent
+// CTAs over the list, up to kListedCtas per SM with larger stages, one tile
+// at a time.  A tile that still does not fit is searched per atom from
+// global memory.
+template <bool CLOSE>
+__global__ void __launch_bounds__(kListedWarps * 32, 1)
+k_pairs_listed(const CellGrid g, const TileParams P)
+{
+    // cell starts may not be monotonic; one decision for the whole CTA
+    if (__syncthreads_or(timed_out(P.flags))) return;
+    extern __shared__ __align__(16) unsigned char tile_smem[];
+    float4 *stage = reinterpret_cast<float4 *>(tile_smem);
+    uint8_t *tabs = tile_smem + sizeof(float4) * P.stage_max;                   // [kSRows][kRowTab]
+    int32_t *hits = reinterpret_cast<int32_t *>(tabs + kSRows * kRowTab);       // [W][kBuf][32]
+    int32_t *negs = hits + kListedWarps * 32 * kBuf;                           // P.K entries of -1
+    __shared__ TileRows tr;
+    __shared__ int4 rinfo[kSRows];
+    __shared__ TileMeta meta;
+    __shared__ __align__(8) uint64_t bar;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < P.K; e += blockDim.x) negs[e] = -1;
+    fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -905,193 +1218,57 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
     __syncthreads();
     uint32_t phase = 0;   // parity of the mbarrier phase the next staging completes
     CloseAcc cl{__int_as_float(0x7f800000), 0u};
+    const uint32_t hb = smem_u32(hits) + (uint32_t)(warp * 32 * kBuf * 4);   // the warp's buffer
+    const uint32_t negs_addr = smem_u32(negs);
 
-    for (int it = 0;; ++it) {
-    int t;
-    if (LISTED) {
-        const uint32_t e = blockIdx.x + (uint32_t)it * gridDim.x;
-        if (e >= *P.fb_count) break;
-        t = (int)P.fb_list[e];
-    } else {
-        if (it > 0) break;
-        t = blockIdx.x;
-    }
-    const int tile = t;
-    const int tx = t % P.tiles_x;
-    t /= P.tiles_x;
-    const int ty = t % P.tiles_y, tz = t / P.tiles_y;
-    const int cx0 = tx * kTX, cy0 = ty * kTY, cz0 = tz * kTZ;
-    const int Gx = min(kTX, g.nx - cx0), Gy = min(kTY, g.ny - cy0), Gz = min(kTZ, g.nz - cz0);
-    const uint32_t stage_base = smem_u32(stage);
-    const bool general = cx0 == 0 || cx0 + Gx == g.nx || cy0 < 2 || cy0 + Gy + 2 > g.ny ||
-                         cz0 < 2 || cz0 + Gz + 2 > g.nz;
-
-    if (warp == 0) {
-        RowSrc ra, rb;   // rows lane and lane + 32
-        int cell_scratch[kSCells + 1];
-        describe_row(g, P.cell_start, lane, cx0, cy0, cz0, Gx, Gy, Gz, ra, tr.cell[lane]);
-        describe_row(g, P.cell_start, lane + 32, cx0, cy0, cz0, Gx, Gy, Gz, rb,
-                     lane + 32 < kSRows ? tr.cell[lane + 32] : cell_scratch);
-        // offsets: rows back to back in staged order
-        const int va = ra.len, vb = lane + 32 < kSRows ? rb.len : 0;
-        int xa = va, xb = vb;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int ya = __shfl_up_sync(0xffffffffu, xa, o);
-            const int yb = __shfl_up_sync(0xffffffffu, xb, o);
-            if (lane >= o) {
-                xa += ya;
-                xb += yb;
+    for (uint32_t e = blockIdx.x; e < *P.fb_count; e += gridDim.x) {
+        const int t = (int)P.fb_list[e];
+        if (warp == 0) {
+            RowSrc ra, rb;
+            const uint32_t bytes = describe_tile(t, g, P, tr, rinfo, meta, ra, rb);
+            if (!tr.fallback) {
+                if (lane == 0) mbar_arrive_expect_tx(&bar, bytes);
+                __syncwarp();
+                const uint32_t stage_base = smem_u32(stage);
+                copy_row(ra, P, g, stage_base, tr.off[lane], smem_u32(tabs) + (uint32_t)(lane * kRowTab),
+                         &bar);
+                if (lane + 32 < kSRows)
+                    copy_row(rb, P, g, stage_base, tr.off[lane + 32],
+                             smem_u32(tabs) + (uint32_t)((lane + 32) * kRowTab), &bar);
             }
         }
-        const int suma = __shfl_sync(0xffffffffu, xa, 31);
-        const int sumb = __shfl_sync(0xffffffffu, xb, 31);
-        const int offa = xa - va;
-        const int offb = suma + xb - vb;
-        const int total = suma + sumb;
-        tr.off[lane] = offa;
-        tr.len[lane] = ra.len;
-        rinfo[lane] = make_int4(offa + ra.lend, offa + ra.rbeg, __float_as_int(ra.sy),
-                                __float_as_int(ra.sz));
-        if (lane + 32 < kSRows) {
-            tr.off[lane + 32] = offb;
-            tr.len[lane + 32] = rb.len;
-            rinfo[lane + 32] = make_int4(offb + rb.lend, offb + rb.rbeg, __float_as_int(rb.sy),
-                                         __float_as_int(rb.sz));
-        }
-        // home rows h = hy + kTY hz are staged rows (hy + 2) + kSY (hz + 2)
-        __syncwarp();
-        int hcnt = 0;
-        if (lane < kHome) {
-            const int hy = lane % kTY, hz = lane / kTY;
-            const int R = (hy + 2) + kSY * (hz + 2);
-            tr.home_begin[lane] = tr.off[R] + tr.cell[R][1];
-            hcnt = hy < Gy && hz < Gz ? tr.cell[R][Gx + 1] - tr.cell[R][1] : 0;
-        }
-        int hx = hcnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, hx, o);
-            if (lane >= o) hx += y;
-        }
-        if (lane < kHome) tr.home_pref[lane] = hx - hcnt;
-        if (lane == kHome - 1) tr.home_pref[kHome] = hx;
-        const uint32_t bytes = __reduce_add_sync(0xffffffffu, row_bytes(ra) + row_bytes(rb));
-        const int fb = (total > P.stage_max || *P.unsorted != 0u) ? 1 : 0;
-        if (lane == 0) {
-            tr.total = total;
-            tr.fallback = fb;
-            if (fb) {
-                if (!LISTED) {
-                    const uint32_t slot = atomicAdd(P.fb_count, 1u);
-                    P.fb_list[slot] = (uint32_t)tile;
-                }
-            } else {
-                mbar_arrive_expect_tx(&bar, bytes);
-            }
-        }
-        __syncwarp();
-        if (!fb) {
-            copy_row(ra, P, g, stage_base, offa, smem_u32(tabs) + (uint32_t)(lane * kRowTab), &bar);
-            copy_row(rb, P, g, stage_base, offb, smem_u32(tabs) + (uint32_t)((lane + 32) * kRowTab),
-                     &bar);
-        }
-    }
-    __syncthreads();
-    if (tr.fallback) {
-        if (LISTED) {   // per atom, straight from global memory
-            for (int hz = 0; hz < Gz; ++hz)
-                for (int hy = 0; hy < Gy; ++hy) {
-                    const int64_t rowc = ((int64_t)(cz0 + hz) * g.ny + (cy0 + hy)) * g.nx;
-                    const int32_t k0 = P.cell_start[rowc + cx0], k1 = P.cell_start[rowc + cx0 + Gx];
+        __syncthreads();
+        if (tr.fallback) {   // per atom, straight from global memory
+            for (int hz = 0; hz < meta.Gz; ++hz)
+                for (int hy = 0; hy < meta.Gy; ++hy) {
+                    const int64_t rowc = ((int64_t)(meta.cz0 + hz) * g.ny + (meta.cy0 + hy)) * g.nx;
+                    const int32_t k0 = P.cell_start[rowc + meta.cx0];
+                    const int32_t k1 = P.cell_start[rowc + meta.cx0 + meta.Gx];
                     for (int32_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
                         pair_row_per_atom<false, CLOSE>(k, P.cell_pos, P.cell_start, P.atom_cell,
                                                         g, P.K, P.nbr, P.counts, P.flags,
                                                         P.close_d2, cl);
                 }
+            __syncthreads();
+            continue;
         }
-        __syncthreads();
-        continue;
-    }
-    {
-        bool done = false;
-        for (uint32_t spins = 0; spins < 4096u && !done; ++spins)   // ~4 s
-            done = mbar_try_wait(&bar, phase);
-        if (__syncthreads_or(!done)) {
-            // Entry already returned if a look-back gave up, so the cell starts
-            // are monotonic and the announced byte count is exactly what the
-            // row copies carry: the phase completes when they land.  A CTA
-            // that left now could leave copies writing into shared memory given
-            // to the next CTA, so it records the timeout and waits once more
-            // (bounded) before it returns.
-            if (threadIdx.x == 0) atomicOr(P.flags, kFlagTimeout);
-            for (uint32_t spins = 0; spins < 4096u && !done; ++spins)
+        {
+            bool done = false;
+            for (uint32_t spins = 0; spins < 4096u && !done; ++spins)   // ~4 s
                 done = mbar_try_wait(&bar, phase);
-            return;
-        }
-        phase ^= 1u;
-    }
-    const int nbins = (Gx + 2) * kBinsPerCell;
-    const float X0 = (float)(cx0 - 1) * P.side_x;   // low x face of conceptual cell 0
-    const float rl2 = g.rl2;
-    const int nhome = tr.home_pref[kHome];
-    const uint32_t hb = smem_u32(hits) + (uint32_t)((warp * 32 + lane) * kBuf * 4);
-    const uint32_t negs_addr = smem_u32(negs);
-
-    for (int c = warp; c * 32 < nhome; c += kTileWarps) {
-        const int a = c * 32 + lane;
-        int h = 0;
-        while (h < kHome - 1 && a >= tr.home_pref[h + 1]) ++h;
-        const int slot = tr.home_begin[h] + (a - tr.home_pref[h]);
-        const float qn = __int_as_float(0x7fc00000);
-        float4 me = a < nhome ? stage[slot] : make_float4(qn, qn, qn, qn);
-        // a lane has a row to build when its atom exists and is below n_rows
-        const bool valid = a < nhome && __float_as_int(me.w) < g.n_rows;
-        if (!valid) me = make_float4(qn, qn, qn, qn);
-        const int hy = h % kTY, hz = h / kTY;
-        const float ylo = (float)(cy0 + hy) * P.side_y, yhi = (float)(cy0 + hy + 1) * P.side_y;
-        const float zlo = (float)(cz0 + hz) * P.side_z, zhi = (float)(cz0 + hz + 1) * P.side_z;
-        const float dy_lo = me.y - ylo, dy_hi = yhi - me.y;
-        const float dz_lo = me.z - zlo, dz_hi = zhi - me.z;
-
-        LaneOut o;
-        o.buf = hb;
-        o.bp = hb;
-        o.gfl = 0u;
-        o.Kb = 4u * (uint32_t)P.K;
-        const int myid = __float_as_int(me.w);
-        o.grow = reinterpret_cast<char *>(P.nbr + (int64_t)(valid ? myid : 0) * P.K);
-        const float mxr = me.x - X0;
-        const int Rh = (hy + 2) + kSY * (hz + 2);
-        if (general)
-            scan_rows<true, CLOSE>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot,
-                                   Rh, dy_lo, dy_hi, dz_lo, dz_hi, mxr, P.close_d2, cl, o);
-        else
-            scan_rows<false, CLOSE>(stage, tabs, tr, rinfo, P, rl2, g.Lx, nbins, me, valid, slot,
-                                    Rh, dy_lo, dy_hi, dz_lo, dz_hi, mxr, P.close_d2, cl, o);
-
-        // ---- finish the row (the scan ends with a flush: at most 3 entries
-        //      pending): the partial vector completed with -1, then -1 from
-        //      the shared block up to the capacity
-        if (valid) {
-            const uint32_t u = o.bp - o.buf;
-            uint32_t pf = o.gfl;
-            if (u != 0u) {
-                uint4 v = lds_u4(o.buf);
-                if (u <= 4u) v.y = 0xffffffffu;
-                if (u <= 8u) v.z = 0xffffffffu;
-                v.w = 0xffffffffu;
-                if (o.gfl < o.Kb) stg_u4(o.grow + o.gfl, v);
-                pf += 16u;
+            if (__syncthreads_or(!done)) {
+                // see k_pairs_pipe: record, wait once more (bounded), leave
+                if (threadIdx.x == 0) atomicOr(P.flags, kFlagTimeout);
+                for (uint32_t spins = 0; spins < 4096u && !done; ++spins)
+                    done = mbar_try_wait(&bar, phase);
+                break;
             }
-            if (pf < o.Kb) bulk_s2g(o.grow + pf, negs_addr, o.Kb - pf);
-            bulk_commit();
-            const int cnt = (int)((o.gfl + u) >> 2);
-            P.counts[myid] = cnt;
-            if (cnt > P.K) atomicOr(P.flags, kFlagOverflow);
+            phase ^= 1u;
         }
-    }
-    __syncthreads();   // the tile's shared data is reused by the next one
+        const int nhome = tr.home_pref[kHome];
+        for (int c = warp; c * 32 < nhome; c += kListedWarps)
+            search_chunk<CLOSE>(c, stage, tabs, tr, rinfo, meta, g, P, hb, negs_addr, cl);
+        __syncthreads();   // the tile's shared data is reused by the next one
     }
     if (CLOSE) close_publish(cl, P.min_bits, P.n_close);
     bulk_wait_read<0>();   // the -1 block stays readable until the copies are done
@@ -1099,21 +1276,26 @@ k_pairs_tiles(const CellGrid g, const TileParams P)
 
 constexpr int kSlotLimit = 65000;   // slot-table entries are 16 bits
 
-size_t tile_fixed_smem(int K)
+// Dynamic shared memory of the two launches besides their stages.
+size_t pipe_fixed_smem(int K)
 {
-    return (size_t)kSRows * kRowTab +
-           (size_t)kTileWarps * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
+    return (size_t)kPipeStages * kSRows * kRowTab +
+           (size_t)kPipeConsumers * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
 }
 
+size_t listed_fixed_smem(int K)
+{
+    return (size_t)kSRows * kRowTab + (size_t)kListedWarps * 32 * kBuf * sizeof(int32_t) +
+           (size_t)K * sizeof(int32_t);
+}
 
-template <bool LISTED, bool CLOSE>
-cudaError_t tiles_allow_smem(int optin)
+template <class Kernel>
+cudaError_t allow_smem(Kernel kernel, int optin)
 {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, k_pairs_tiles<LISTED, CLOSE>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_pairs_tiles<LISTED, CLOSE>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 optin - (int)fa.sharedSizeBytes);
 }
 
@@ -1126,10 +1308,10 @@ cudaError_t pairs_set_attributes()
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
-    if ((e = tiles_allow_smem<false, false>(optin)) != cudaSuccess) return e;
-    if ((e = tiles_allow_smem<true, false>(optin)) != cudaSuccess) return e;
-    if ((e = tiles_allow_smem<false, true>(optin)) != cudaSuccess) return e;
-    return tiles_allow_smem<true, true>(optin);
+    if ((e = allow_smem(k_pairs_pipe<false>, optin)) != cudaSuccess) return e;
+    if ((e = allow_smem(k_pairs_pipe<true>, optin)) != cudaSuccess) return e;
+    if ((e = allow_smem(k_pairs_listed<false>, optin)) != cudaSuccess) return e;
+    return allow_smem(k_pairs_listed<true>, optin);
 }
 
 namespace {
@@ -1141,47 +1323,32 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
 {
     *used_fast = 0;
     if (n <= 0) return cudaSuccess;
-    // Staged kernel: column grid and rows of whole 16-byte vectors.  The
-    // stage must hold a typical tile (kSRows rows x (kTX + 2) cells at the
-    // mean cell occupancy) with 10 % to spare; take the largest number of
-    // CTAs per SM (up to kTileCtas) whose shared-memory share still does.
-    // Denser tiles are listed for a second launch with larger stages.
+    // Persistent staged kernel: column grid and rows of whole 16-byte
+    // vectors.  Its kPipeStages stages share what is left of the SM's
+    // shared memory; a stage should hold a typical tile (kSRows rows x
+    // (kTX + 2) cells at the mean cell occupancy) with 10 % to spare.  Denser
+    // tiles are listed for a second launch with larger stages.
     int stage_max = 0;
-    int need = 0, per_sm = 0, reserved = 0;   // typical tile's slots; SM shared memory
+    int need = 0, per_sm = 0, reserved = 0, optin = 0;
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
         (reinterpret_cast<uintptr_t>(nbr) & 15u) == 0 && n < (int64_t(1) << 31)) {
-        int dev = 0, optin = 0;
+        int dev = 0;
         NL_CUDA_TRY(cudaGetDevice(&dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev));
         NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
         cudaFuncAttributes fa;
-        NL_CUDA_TRY(cudaFuncGetAttributes(&fa, k_pairs_tiles<false, CLOSE>));
-        const size_t fixed = tile_fixed_smem(capacity);
+        NL_CUDA_TRY(cudaFuncGetAttributes(&fa, k_pairs_pipe<CLOSE>));
         const double per_cell = (double)n / (double)g.ncell;
-        const int want =
-            (int)(1.1 * per_cell * kSRows * kSCells) + 32;
+        const int want = (int)(1.1 * per_cell * kSRows * kSCells) + 32;
         need = want > kStageMin ? want : kStageMin;
-        for (int ctas = kTileCtas; ctas >= 1; --ctas) {
-            long budget = (long)per_sm / ctas - reserved - (long)fa.sharedSizeBytes;
-            const long cap = (long)optin - (long)fa.sharedSizeBytes;
-            if (budget > cap) budget = cap;
-            long fit = budget > (long)fixed ? (budget - (long)fixed) / (long)sizeof(float4) : 0;
-            // shared memory is handed out in granules: shrink the stage until
-            // `ctas` CTAs really fit on one SM
-            while (ctas > 1 && fit >= need) {
-                int nb = 0;
-                NL_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &nb, k_pairs_tiles<false, CLOSE>, kTileWarps * 32, sizeof(float4) * (size_t)fit + fixed));
-                if (nb >= ctas) break;
-                fit -= 32;
-            }
-            if (fit >= need || ctas == 1) {
-                stage_max = (int)(fit < kSlotLimit ? fit : kSlotLimit);
-                break;
-            }
-        }
-        if (stage_max < 256) stage_max = 0;
+        const long budget = (long)optin - (long)fa.sharedSizeBytes - (long)pipe_fixed_smem(capacity);
+        long fit = budget > 0 ? budget / ((long)sizeof(float4) * kPipeStages) : 0;
+        // the chunk queue holds every chunk of kPipeStages tiles plus the end entries
+        const long qcap = (long)(kQueue - kPipeConsumers - 8) / kPipeStages * 32;
+        if (fit > qcap) fit = qcap;
+        if (fit > kSlotLimit) fit = kSlotLimit;
+        stage_max = fit >= 256 ? (int)(fit & ~31L) : 0;
     }
     if (stage_max > 0) {
         TileParams P;
@@ -1198,9 +1365,11 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         P.unsorted = ctx->unsorted;
         P.fb_list = ctx->fb_list;
         P.fb_count = ctx->fb_count;
+        P.tile_ctr = ctx->tile_ctr;
         P.tiles_x = (g.nx + kTX - 1) / kTX;
         P.tiles_y = (g.ny + kTY - 1) / kTY;
         const int tiles_z = (g.nz + kTZ - 1) / kTZ;
+        P.ntiles = P.tiles_x * P.tiles_y * tiles_z;
         P.K = capacity;
         P.stage_max = stage_max;
         P.side_x = g.Lx / (float)g.nx;
@@ -1211,25 +1380,21 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         const float Lmax = fmaxf(g.Lx, fmaxf(g.Ly, g.Lz));
         P.eps = 1e-3f * rl + 4e-6f * Lmax;
         P.rl2_margin = g.rl2 * (1.0f + 1e-4f);
-        const int64_t ntiles = (int64_t)P.tiles_x * P.tiles_y * tiles_z;
-        const size_t smem = sizeof(float4) * (size_t)stage_max + tile_fixed_smem(capacity);
-        NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, sizeof(uint32_t), s));
+        const size_t smem = sizeof(float4) * (size_t)kPipeStages * stage_max + pipe_fixed_smem(capacity);
+        NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, 2 * sizeof(uint32_t), s));   // and tile_ctr
         {
             ProfScope ps(ctx, PH_PAIRS, s);
-            k_pairs_tiles<false, CLOSE><<<(unsigned)ntiles, kTileWarps * 32, smem, s>>>(g, P);
+            k_pairs_pipe<CLOSE><<<(unsigned)ctx->sm_count, kPipeThreads, smem, s>>>(g, P);
             NL_CUDA_TRY(cudaGetLastError());
         }
         *used_fast = 1;
-        // the listed tiles: persistent CTAs over the list, as many per SM (up
-        // to kListedCtas) as still give each a stage of twice a typical tile;
-        // one CTA with the largest stage when none does.  A tile beyond its
-        // stage is searched per atom from global memory in the same kernel.
-        int dev = 0, optin = 0;
-        NL_CUDA_TRY(cudaGetDevice(&dev));
-        NL_CUDA_TRY(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+        // the listed tiles: as many CTAs per SM (up to kListedCtas) as still
+        // give each a stage of twice a typical tile; one CTA with the
+        // largest stage when none does.  A tile beyond its stage is searched
+        // per atom from global memory in the same kernel.
         cudaFuncAttributes fl;
-        NL_CUDA_TRY(cudaFuncGetAttributes(&fl, k_pairs_tiles<true, CLOSE>));
-        const long lfixed = (long)tile_fixed_smem(capacity);
+        NL_CUDA_TRY(cudaFuncGetAttributes(&fl, k_pairs_listed<CLOSE>));
+        const long lfixed = (long)listed_fixed_smem(capacity);
         const long big = ((long)optin - (long)fl.sharedSizeBytes - lfixed) / (long)sizeof(float4);
         long lfit = big;
         int lctas = 1;
@@ -1240,7 +1405,7 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
             while (f >= 2L * need) {
                 int nb = 0;
                 NL_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &nb, k_pairs_tiles<true, CLOSE>, kTileWarps * 32,
+                    &nb, k_pairs_listed<CLOSE>, kListedWarps * 32,
                     sizeof(float4) * (size_t)f + (size_t)lfixed));
                 if (nb >= c) break;
                 f -= 32;
@@ -1254,9 +1419,8 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         TileParams PL = P;
         PL.stage_max = (int)(lfit < kSlotLimit ? lfit : kSlotLimit);
         ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
-        k_pairs_tiles<true, CLOSE><<<(unsigned)(ctx->sm_count * lctas), kTileWarps * 32,
-                                     sizeof(float4) * (size_t)PL.stage_max + (size_t)lfixed, s>>>(
-            g, PL);
+        k_pairs_listed<CLOSE><<<(unsigned)(ctx->sm_count * lctas), kListedWarps * 32,
+                                sizeof(float4) * (size_t)PL.stage_max + (size_t)lfixed, s>>>(g, PL);
         return cudaGetLastError();
     }
     ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);

@@ -39,7 +39,9 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
            uint32_t *ticket, uint32_t *flags, const uint32_t *gate)
 {
     if (gate && ld_volatile_u32(gate) == 0u) return;   // gated pass not needed
-    if (timed_out(flags)) return;                       // an earlier wait gave up
+    // an earlier wait gave up (a CTA of this pass may set the bit while
+    // others start: one decision per CTA)
+    if (__syncthreads_or(timed_out(flags))) return;
     extern __shared__ __align__(16) unsigned char sort_smem[];
     uint64_t *s_keys = reinterpret_cast<uint64_t *>(sort_smem);
     uint32_t *s_vals = reinterpret_cast<uint32_t *>(sort_smem + sizeof(uint64_t) * kSortTile);
