@@ -640,7 +640,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
                         "pair_search_per_atom")) / args.steps
         sort_ms = sum(phases.get(p, (0.0, 0))[0] for p in
                       ("keys", "key_scan", "radix_sort", "gather")) / args.steps
-        kernels_per_phase = {"radix_sort": 14, "cell_sort": 2}
+        # launches per profiled phase: the sort phase holds 3 digit passes, the
+        # run finish and the gated full sort (keys, scan, 8 passes, gather)
+        kernels_per_phase = {"radix_sort": 15}
         launches_per_step = sum(v[1] * kernels_per_phase.get(k, 1)
                                 for k, v in phases.items()) / args.steps
         line = {

@@ -152,14 +152,8 @@ nl_status sort_impl(nl_ctx *ctx, int64_t n, const float *pos, const float *box, 
     {
         ProfScope ps(ctx, PH_SORT, s);
         const SortRecompute rk{p4, n, box[0], box[1], box[2], sx, sy, sz, curve};
-        if (launch_radix_passes(ctx, n, keys_out, reinterpret_cast<uint32_t *>(perm), s, rk) !=
-            cudaSuccess)
-            return NL_ERR_CUDA;
-    }
-    {
-        ProfScope ps(ctx, PH_GATHER, s);
-        if (launch_gather(n, p4, perm, reinterpret_cast<float4 *>(pos_sorted), ctx->flags, s) !=
-            cudaSuccess)
+        if (launch_radix_passes(ctx, n, keys_out, reinterpret_cast<uint32_t *>(perm), s, rk,
+                                reinterpret_cast<float4 *>(pos_sorted)) != cudaSuccess)
             return NL_ERR_CUDA;
     }
     return NL_OK;

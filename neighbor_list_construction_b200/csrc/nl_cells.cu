@@ -11,8 +11,12 @@
 namespace nl {
 namespace {
 
-// Largest cell the in-cell sort handles (8 atoms per lane).
-constexpr int kCellSortMax = 256;
+// Largest cell the in-cell sort handles: its table counts must fit a byte.
+constexpr int kCellSortMax = 255;
+// In-cell sort: cells per CTA, atoms a CTA stages at once, threads.
+constexpr int kSortCells = 128;
+constexpr int kSortCap = 2048;
+constexpr int kSortThreads2 = 256;
 
 __global__ void __launch_bounds__(256)
 k_bin_count(const float4 *__restrict__ pos, int64_t n, CellGrid g, uint32_t *__restrict__ atom_cell,
@@ -144,141 +148,96 @@ __device__ __forceinline__ bool before_xi(float xa, int ia, float xb, int ib)
     return xa < xb || (xa == xb && ia < ib);
 }
 
-// Sorts the atoms of cell c by (x, index) in place and writes the cell's x
+// In-cell sort, one CTA per run of kSortCells consecutive cells (a
+// contiguous range of the cell-ordered array).  The CTA stages the range's
+// atoms in shared memory with coalesced loads -- whole cells, at most
+// kSortCap atoms at a time -- ranks each atom by (x, index) inside its cell,
+// writes the cell back sorted (coalesced again) and writes each cell's x
 // sub-bin table: byte b (b = 0..15) = number of the cell's atoms whose x is
 // below the cell's low x face plus b/16 of its width (bin of an atom =
-// floor((x - face) * 16 / width), clamped to 0..15).  The pair search reads
-// these to find x-windows.  Half-warp version for cells of at most 16 atoms:
-// lane hl of the half owns atom hl, ranks it with shuffles inside the half
-// and computes table entry hl.
-__device__ __forceinline__ void sort_small_cell(float4 *__restrict__ cell_pos, int32_t s, int m,
-                                                float face, float inv_bin, uint8_t *tab, int hl,
-                                                bool real)
-{
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (hl < m) v = cell_pos[s + hl];
-    const int id = __float_as_int(v.w);
-    const int bin = max(0, min(15, (int)floorf((v.x - face) * inv_bin)));
-    int r = 0, below = 0;
-    // both halves run to the larger of their two cells
-    const int mm = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
-    for (int j = 0; j < mm; ++j) {
-        const float xj = __shfl_sync(0xffffffffu, v.x, j, 16);
-        const int ij = __shfl_sync(0xffffffffu, id, j, 16);
-        const int bj = __shfl_sync(0xffffffffu, bin, j, 16);
-        if (j < m) {
-            r += before_xi(xj, ij, v.x, id) ? 1 : 0;
-            below += bj < hl ? 1 : 0;
-        }
-    }
-    __syncwarp();
-    if (!real) return;   // a half with no cell only takes part in the shuffles
-    if (hl < m && m > 1) cell_pos[s + r] = v;
-    tab[hl] = (uint8_t)below;
-}
-
-// Full-warp version for cells of 17..kCellSortMax atoms (8 atoms per lane).
-__device__ __forceinline__ void sort_large_cell(float4 *__restrict__ cell_pos, int32_t s, int m,
-                                                float face, float inv_bin, uint8_t *tab, int lane)
-{
-    constexpr int E = kCellSortMax / 32;
-    float4 v[E];
-    int r[E], bin[E];
-    int below = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        r[e] = 0;
-        v[e] = e * 32 + lane < m ? cell_pos[s + e * 32 + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-        bin[e] = max(0, min(15, (int)floorf((v[e].x - face) * inv_bin)));
-    }
-#pragma unroll
-    for (int es = 0; es < E; ++es) {
-        if (es * 32 >= m) break;
-        const float xs = v[es].x;
-        const int is = __float_as_int(v[es].w);
-        const int bs = bin[es];
-        const int lim = m - es * 32 < 32 ? m - es * 32 : 32;
-        for (int l = 0; l < lim; ++l) {
-            const float xj = __shfl_sync(0xffffffffu, xs, l);
-            const int ij = __shfl_sync(0xffffffffu, is, l);
-            const int bj = __shfl_sync(0xffffffffu, bs, l);
-            below += bj < lane ? 1 : 0;
-#pragma unroll
-            for (int e = 0; e < E; ++e)
-                r[e] += before_xi(xj, ij, v[e].x, __float_as_int(v[e].w)) ? 1 : 0;
-        }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        if (e * 32 + lane < m) cell_pos[s + r[e]] = v[e];
-    if (lane < 16) tab[lane] = (uint8_t)below;
-}
-
-// Two cells per warp, one per half.  A cell of at most 16 atoms is sorted
-// here; a larger one (up to kCellSortMax) is listed for k_cell_sort_large,
-// and one above kCellSortMax stays in scatter order and raises `unsorted`.
-// Keeping the large path out of this kernel keeps its register count low, so
-// enough warps are resident to cover the two dependent global loads per cell.
-__global__ void __launch_bounds__(256)
+// floor((x - face) * 16 / width), clamped to 0..15), staged in shared memory
+// and stored 16 bytes per cell.  The pair search reads these to find
+// x-windows.  A cell of more than kCellSortMax atoms (its table counts would
+// not fit a byte) stays in scatter order and raises `unsorted`, which sends
+// the pair search to its per-atom path.
+__global__ void __launch_bounds__(kSortThreads2)
 k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell,
             int nx, float side_x, float inv_bin, uint8_t *__restrict__ cell_tab,
-            uint32_t *__restrict__ large_list, uint32_t *large_count, uint32_t *unsorted,
-            const uint32_t *flags)
+            uint32_t *unsorted, const uint32_t *flags)
 {
-    if (timed_out(flags)) return;
-    const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    // the next iteration's cell range is loaded one iteration ahead, so only
-    // the position load stays on each iteration's dependent chain
-    int32_t s_next = 0, e_next = 0;
-    if (2 * warp + half < ncell) {
-        s_next = cell_start[2 * warp + half];
-        e_next = cell_start[2 * warp + half + 1];
-    }
-    for (int64_t c0 = 2 * warp; c0 < ncell; c0 += 2 * nwarps) {
-        const int64_t c = c0 + half;
-        const bool have = c < ncell;
-        const int32_t s = have ? s_next : 0;
-        const int m = have ? e_next - s_next : 0;
-        const int64_t cn = c + 2 * nwarps;
-        if (cn < ncell) {
-            s_next = cell_start[cn];
-            e_next = cell_start[cn + 1];
+    // cell starts may not be monotonic; one decision for the whole CTA
+    if (__syncthreads_or(timed_out(flags))) return;
+    __shared__ float4 s_pos[kSortCap];
+    __shared__ uint8_t s_sbin[kSortCap];                     // bins in sorted order
+    __shared__ __align__(16) uint8_t s_tab[kSortCells][16];
+    __shared__ int32_t s_cs[kSortCells + 1];
+    const int64_t c0 = (int64_t)blockIdx.x * kSortCells;
+    const int nc = (int)(ncell - c0 < kSortCells ? ncell - c0 : kSortCells);
+    for (int k = threadIdx.x; k <= nc; k += blockDim.x) s_cs[k] = cell_start[c0 + k];
+    __syncthreads();
+    int cb = 0;
+    while (cb < nc) {
+        // the longest run of whole cells from cb whose atoms fit the stage
+        // (at least one cell; a cell alone beyond the stage is left unsorted)
+        const int t = threadIdx.x;
+        const int fit = __syncthreads_count(t >= cb && t < nc &&
+                                            s_cs[t + 1] - s_cs[cb] <= kSortCap);
+        const int ce = cb + (fit > 0 ? fit : 1);
+        const int a0 = s_cs[cb];
+        const int m = s_cs[ce] - a0;
+        if (m > kSortCap) {
+            if (threadIdx.x == 0) atomicOr(unsorted, 1u);
+            cb = ce;
+            continue;
         }
-        const float face = (float)(int)(c % nx) * side_x;
-        const bool small = m <= 16;
-        sort_small_cell(cell_pos, s, small ? m : 0, face, inv_bin, cell_tab + (have ? c : 0) * 16,
-                        hl, have && small);
-        if (have && !small && hl == 0) {
-            if (m > kCellSortMax)
-                atomicOr(unsorted, 1u);
-            else
-                large_list[atomicAdd(large_count, 1u)] = (uint32_t)c;
+        for (int k = threadIdx.x; k < m; k += blockDim.x) s_pos[k] = cell_pos[a0 + k];
+        __syncthreads();
+        // each atom: its cell (binary search of the stage's cell starts), its
+        // bin, and its rank by (x, index) among the cell's atoms
+        for (int k = threadIdx.x; k < m; k += blockDim.x) {
+            int lo = cb, hi = ce - 1;   // cell of atom k: s_cs[c] <= a0 + k < s_cs[c + 1]
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_cs[mid] <= a0 + k) lo = mid; else hi = mid - 1;
+            }
+            const int c = lo;
+            const int s0 = s_cs[c] - a0, s1 = s_cs[c + 1] - a0;
+            if (s1 - s0 > kCellSortMax) continue;   // too large: left in scatter order
+            const float4 v = s_pos[k];
+            const int id = __float_as_int(v.w);
+            int r = 0;
+            for (int q = s0; q < s1; ++q) {
+                const float4 u = s_pos[q];
+                r += before_xi(u.x, __float_as_int(u.w), v.x, id) ? 1 : 0;
+            }
+            const float face = (float)(int)((c0 + c) % nx) * side_x;
+            s_sbin[s0 + r] = (uint8_t)max(0, min(15, (int)floorf((v.x - face) * inv_bin)));
+            cell_pos[a0 + s0 + r] = v;
         }
+        __syncthreads();
+        // tables from the bins in sorted order: entry b of a cell = number of
+        // its atoms with bin < b = the first sorted position whose bin >= b
+        for (int e = threadIdx.x; e < (ce - cb) * 16; e += blockDim.x) {
+            const int c = cb + (e >> 4), b = e & 15;
+            const int s0 = s_cs[c] - a0, s1 = s_cs[c + 1] - a0;
+            if (s1 - s0 > kCellSortMax) {
+                if (b == 0) atomicOr(unsorted, 1u);
+                s_tab[c][b] = 0;
+                continue;
+            }
+            int l = s0, h = s1;   // lower bound of b in s_sbin[s0, s1)
+            while (l < h) {
+                const int mid = (l + h) >> 1;
+                if (s_sbin[mid] < b) l = mid + 1; else h = mid;
+            }
+            s_tab[c][b] = (uint8_t)(l - s0);
+        }
+        __syncthreads();   // the stage is reused by the next run of cells
+        cb = ce;
     }
-}
-
-// The listed cells of 17..kCellSortMax atoms, one warp per cell.
-__global__ void __launch_bounds__(256)
-k_cell_sort_large(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int nx,
-                  float side_x, float inv_bin, uint8_t *__restrict__ cell_tab,
-                  const uint32_t *__restrict__ large_list, const uint32_t *large_count,
-                  const uint32_t *flags)
-{
-    if (timed_out(flags)) return;
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const uint32_t nlisted = *large_count;
-    for (int64_t e = warp; e < (int64_t)nlisted; e += nwarps) {
-        const int64_t c = large_list[e];
-        const int32_t s = cell_start[c];
-        const int m = cell_start[c + 1] - s;
-        const float face = (float)(int)(c % nx) * side_x;
-        sort_large_cell(cell_pos, s, m, face, inv_bin, cell_tab + c * 16, lane);
-    }
+    // the CTA's tables, 16 bytes per cell
+    for (int c = threadIdx.x; c < nc; c += blockDim.x)
+        reinterpret_cast<uint4 *>(cell_tab)[c0 + c] = *reinterpret_cast<const uint4 *>(s_tab[c]);
 }
 
 }  // namespace
@@ -313,22 +272,12 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
         NL_CUDA_TRY(cudaGetLastError());
     }
     {
-        // cells above 16 atoms are listed in fb_list (free until the pair
-        // search, which resets fb_count before it lists its own tiles)
         ProfScope ps(ctx, PH_CELL_SORT, s);
         const float side_x = g.Lx / (float)g.nx;
-        NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, sizeof(uint32_t), s));
-        // several waves of CTAs over the cells: measured faster than one
-        // resident wave striding over them
-        int64_t sort_blocks = (g.ncell * 16 + 255) / 256;
-        if (sort_blocks > (int64_t)ctx->sm_count * 32) sort_blocks = (int64_t)ctx->sm_count * 32;
-        k_cell_sort<<<(unsigned)sort_blocks, 256, 0, s>>>(
+        const int64_t blocks = (g.ncell + kSortCells - 1) / kSortCells;
+        k_cell_sort<<<(unsigned)blocks, kSortThreads2, 0, s>>>(
             ctx->cell_pos, ctx->cell_start, g.ncell, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
-            ctx->fb_list, ctx->fb_count, ctx->unsorted, ctx->flags);
-        NL_CUDA_TRY(cudaGetLastError());
-        k_cell_sort_large<<<(unsigned)(ctx->sm_count * 2), 256, 0, s>>>(
-            ctx->cell_pos, ctx->cell_start, g.nx, side_x, 16.0f / side_x, ctx->cell_tab,
-            ctx->fb_list, ctx->fb_count, ctx->flags);
+            ctx->unsorted, ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
     }
     return cudaSuccess;

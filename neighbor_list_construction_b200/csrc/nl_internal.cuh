@@ -111,12 +111,16 @@ struct SortRecompute {
 // passes over the top kTopPasses digits and the prefix-run finish; behind
 // them a gated full sort (keys recomputed, 8 passes) that runs only when a
 // prefix run was longer than kRunMax.  Writes keys to keys_final (NULL: not
-// kept) and indices to vals_final.
+// kept) and indices to vals_final; with pos_sorted, also the positions in
+// that order, (rk.pos[index].xyz, index) (the gather fused into the run
+// finish, and a gated gather behind the full sort).
 cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
-                                uint32_t *vals_final, cudaStream_t s, const SortRecompute &rk);
-// Returns at once when `flags` holds kFlagTimeout (perm may then be stale).
+                                uint32_t *vals_final, cudaStream_t s, const SortRecompute &rk,
+                                float4 *pos_sorted = nullptr);
+// out[k] = (pos[perm[k]].xyz, perm[k]).  Returns at once when `flags` holds
+// kFlagTimeout (perm may then be stale), or when gate is given and *gate == 0.
 cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, float4 *out,
-                          const uint32_t *flags, cudaStream_t s);
+                          const uint32_t *flags, cudaStream_t s, const uint32_t *gate = nullptr);
 
 // Cell binning of `pos` into ctx->cell_pos (cell order, x-sorted in cells).
 cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const CellGrid &g,

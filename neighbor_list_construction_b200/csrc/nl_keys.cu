@@ -212,8 +212,9 @@ constexpr int kGatherItems = 4;
 
 __global__ void __launch_bounds__(256)
 k_gather(int64_t n, const float4 *__restrict__ pos, const int32_t *__restrict__ perm,
-         float4 *__restrict__ out, const uint32_t *flags)
+         float4 *__restrict__ out, const uint32_t *flags, const uint32_t *gate)
 {
+    if (gate && ld_volatile_u32(gate) == 0u) return;   // gated gather not needed
     if (timed_out(flags)) return;   // perm may not be a permutation
     const int64_t base = (int64_t)blockIdx.x * (256 * kGatherItems) + threadIdx.x;
     int32_t i[kGatherItems];
@@ -261,11 +262,11 @@ cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s, const uint32_t *gate)
 }
 
 cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, float4 *out,
-                          const uint32_t *flags, cudaStream_t s)
+                          const uint32_t *flags, cudaStream_t s, const uint32_t *gate)
 {
     if (n <= 0) return cudaSuccess;
     const int64_t blocks = (n + 256 * kGatherItems - 1) / (256 * kGatherItems);
-    k_gather<<<(unsigned)blocks, 256, 0, s>>>(n, pos, perm, out, flags);
+    k_gather<<<(unsigned)blocks, 256, 0, s>>>(n, pos, perm, out, flags, gate);
     return cudaGetLastError();
 }
 

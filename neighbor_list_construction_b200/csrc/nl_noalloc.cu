@@ -133,11 +133,7 @@ extern "C" nl_status nl_sort_hilbert_noalloc(int64_t n, const float *pos, const 
         if (nl::launch_hist_scan(&view, s) != cudaSuccess) return NL_ERR_CUDA;
         const nl::SortRecompute rk{p4, n, box[0], box[1], box[2], sx, sy, sz, 0};
         if (nl::launch_radix_passes(&view, n, keys_out, reinterpret_cast<uint32_t *>(perm_out), s,
-                                    rk) != cudaSuccess)
-            return NL_ERR_CUDA;
-        if (nl::launch_gather(n, p4, perm_out, reinterpret_cast<float4 *>(pos_sorted_out),
-                              view.flags, s) !=
-            cudaSuccess)
+                                    rk, reinterpret_cast<float4 *>(pos_sorted_out)) != cudaSuccess)
             return NL_ERR_CUDA;
     }
     if (status_out) {

@@ -190,7 +190,8 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
 // sorts a whole run.  A CTA stages its tile of kRunTile keys plus kRunMax + 1
 // on either side in shared memory; a run that reaches the end of that window
 // is longer than kRunMax and sets *gate instead (the full sort then redoes
-// everything).
+// everything).  With gdst, each placed element also gathers its position:
+// gdst[out] = (gsrc[index].xyz, index).
 constexpr int kRunThreads = 256;
 constexpr int kRunItems = 8;
 constexpr int kRunTile = kRunThreads * kRunItems;
@@ -199,7 +200,7 @@ constexpr int kRunHalo = kRunMax + 1;
 __global__ void __launch_bounds__(kRunThreads)
 k_run_sort(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ vals, int64_t n,
            uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, uint32_t *gate,
-           const uint32_t *flags)
+           const uint32_t *flags, const float4 *__restrict__ gsrc, float4 *__restrict__ gdst)
 {
     if (timed_out(flags)) return;
     __shared__ uint64_t s_k[kRunTile + 2 * kRunHalo];
@@ -214,10 +215,14 @@ k_run_sort(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ vals,
     }
     __syncthreads();
     bool too_long = false;
-#pragma unroll 1
+    int64_t outs[kRunItems];
+    uint32_t vps[kRunItems];
+#pragma unroll
     for (int u = 0; u < kRunItems; ++u) {
+        outs[u] = -1;
+        vps[u] = 0u;
         const int64_t p = t0 + threadIdx.x + (int64_t)kRunThreads * u;
-        if (p >= n) break;
+        if (p >= n) continue;
         const int a = (int)(p - lo);
         const uint64_t kp = s_k[a];
         const uint32_t vp = s_v[a];
@@ -240,6 +245,18 @@ k_run_sort(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ vals,
         const int64_t out = lo + h + rank;
         if (keys_out) keys_out[out] = kp;
         vals_out[out] = vp;
+        outs[u] = out;
+        vps[u] = vp;
+    }
+    if (gdst) {   // the gather, fused: every random load issued before any store
+        float4 g[kRunItems];
+#pragma unroll
+        for (int u = 0; u < kRunItems; ++u)
+            if (outs[u] >= 0) g[u] = gsrc[vps[u]];
+#pragma unroll
+        for (int u = 0; u < kRunItems; ++u)
+            if (outs[u] >= 0)
+                gdst[outs[u]] = make_float4(g[u].x, g[u].y, g[u].z, __int_as_float((int)vps[u]));
     }
     if (__any_sync(0xffffffffu, too_long) && (threadIdx.x & 31) == 0) atomicOr(gate, 1u);
 }
@@ -247,7 +264,8 @@ k_run_sort(const uint64_t *__restrict__ keys, const uint32_t *__restrict__ vals,
 }  // namespace
 
 cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
-                                uint32_t *vals_final, cudaStream_t s, const SortRecompute &rk)
+                                uint32_t *vals_final, cudaStream_t s, const SortRecompute &rk,
+                                float4 *pos_sorted)
 {
     if (n <= 0) return cudaSuccess;
     const int64_t tiles = (n + kSortTile - 1) / kSortTile;
@@ -275,7 +293,7 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
         const int64_t blocks = (n + kRunTile - 1) / kRunTile;
         k_run_sort<<<(unsigned)blocks, kRunThreads, 0, s>>>(ctx->keys[src], ctx->vals[src], n,
                                                            keys_final, vals_final, ctx->sort_gate,
-                                                           ctx->flags);
+                                                           ctx->flags, rk.pos, pos_sorted);
         NL_CUDA_TRY(cudaGetLastError());
     }
     // full sort, gated: runs only when a prefix run was too long
@@ -299,6 +317,10 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
         NL_CUDA_TRY(cudaGetLastError());
         src = 1 - src;
     }
+    // the gather of the full sort's order, gated like its passes
+    if (pos_sorted)
+        NL_CUDA_TRY(launch_gather(n, rk.pos, reinterpret_cast<const int32_t *>(vals_final),
+                                  pos_sorted, ctx->flags, s, ctx->sort_gate));
     return cudaSuccess;
 }
 
