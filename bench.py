@@ -427,25 +427,27 @@ def sharded_timing(torch, ctx, ps, w, K, nranks: int = 8, reps: int = 2) -> dict
     """The curve-sharded build of the whole system with nranks equal-count
     shards, all in this process on this GPU (collectives routed in memory):
     halo sizes, and the time of the whole sharded build (all shards, their
-    host round trips included) against one nl_build of the whole system."""
+    no host reads once the halo block is agreed) against one nl_build of the
+    whole system."""
     from neighbor_list_construction_b200 import shard
     n = ps.shape[0]
     p = shard.with_ids(ps, 0)
     bounds = shard.shard_bounds(n, nranks)
     shards = [p[s:e] for s, e in bounds]
     res = shard.build_sharded_local(ctx, shards, w.box, w.cutoff, w.skin, K)
-    halos = [r[2] for r in res]
+    halos = [int(r[2].item()) for r in res]
+    block = res[0][3]
     del res
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(reps):
-        res = shard.build_sharded_local(ctx, shards, w.box, w.cutoff, w.skin, K)
+        res = shard.build_sharded_local(ctx, shards, w.box, w.cutoff, w.skin, K, block)
         del res
     e1.record()
     torch.cuda.synchronize()
     return {"shards": nranks, "atoms_per_shard": [e - s for s, e in bounds],
-            "halo_atoms": halos, "halo_fraction": sum(halos) / n,
+            "halo_atoms": halos, "halo_fraction": sum(halos) / n, "halo_block": block,
             "ms_all_shards_one_gpu": e0.elapsed_time(e1) / reps}
 
 
@@ -725,11 +727,15 @@ def run_sharded(args, rank: int, world: int, local_rank: int) -> None:
     own = shard.with_ids(ps[s0:s1].contiguous(), s0)
     del perm, ps, pos
     comm = shard.DistExchange() if world > 1 else None
+    block = [None]   # agreed by the first (warm-up) build, reused after
 
     def step():
         if comm is not None:
-            return shard.build_sharded(ctx, own, w.box, w.cutoff, w.skin, K, comm)
-        return shard.build_sharded_local(ctx, [own], w.box, w.cutoff, w.skin, K)[0]
+            r = shard.build_sharded(ctx, own, w.box, w.cutoff, w.skin, K, comm, block[0])
+        else:
+            r = shard.build_sharded_local(ctx, [own], w.box, w.cutoff, w.skin, K, block[0])[0]
+        block[0] = r[3]
+        return r
 
     def barrier():
         if world > 1:
@@ -738,7 +744,7 @@ def run_sharded(args, rank: int, world: int, local_rank: int) -> None:
 
     for _ in range(args.warmup):
         res = step()
-    halo = res[2]
+    halo = int(res[2].item())
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_host0 = time.monotonic()

@@ -57,7 +57,12 @@ typedef enum {
     NL_ERR_CUDA = -3,      /* a CUDA runtime call failed */
     NL_ERR_TIMEOUT = -4,   /* a bounded device-side wait gave up; results of
                               that call are not valid */
-    NL_ERR_CAPACITY = -5   /* n > max_atoms or capacity > max_capacity */
+    NL_ERR_CAPACITY = -5,  /* n > max_atoms or capacity > max_capacity */
+    NL_ERR_HALO = -6       /* a halo block or the halo buffer of a sharded build
+                              was too small (nl_halo_fill_blocks,
+                              nl_halo_pack): atoms were dropped and the rows
+                              of that build are incomplete; retry with larger
+                              blocks */
 } nl_status;
 
 /* Creates a context on the current CUDA device and allocates all scratch for
@@ -112,6 +117,20 @@ nl_status nl_build(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
 nl_status nl_build_rows(nl_ctx *ctx, int64_t n, int64_t n_rows, const float *pos,
                         const float *box, float cutoff, float skin, int32_t capacity,
                         int32_t *nbr_out, int32_t *counts_out, void *stream);
+
+/* nl_build_rows whose atom count lives in device memory: *n_dev (int64,
+ * device, read by the kernels; values outside [0, n_max] are clamped) atoms
+ * of `pos` take part, pos holding room for n_max.  n_max bounds every launch
+ * and the context check (n_max <= max_atoms), so the host never reads the
+ * count: a sharded build can size its halo on the device and build without a
+ * synchronization.  The pair search's shared-memory stages are sized for
+ * n_max atoms in the box.  n_rows <= n_max rows are written; a NULL n_dev or
+ * n_rows outside [0, n_max] is NL_ERR_ARG.  Everything else as
+ * nl_build_rows. */
+nl_status nl_build_rows_dev(nl_ctx *ctx, int64_t n_max, const int64_t *n_dev, int64_t n_rows,
+                            const float *pos, const float *box, float cutoff, float skin,
+                            int32_t capacity, int32_t *nbr_out, int32_t *counts_out,
+                            void *stream);
 
 /* nl_build with a close-pair detector as a by-product (Tessera abstract:
  * the simulations show no anomalously close pairs; this reports them while

@@ -20,9 +20,11 @@
  *              NL_ERR_CUDA if a launch fails.  No call synchronizes.
  * The steps, per rank: nl_halo_mark -> sum of all ranks' occ (all-reduce;
  * the rank bits are distinct, so the sum is their or) -> nl_halo_needed ->
- * nl_halo_count -> exchange counts, exclusive offsets -> nl_halo_fill ->
- * all-to-all of the send buffer -> nl_build_rows on [own atoms; received
- * halo] with n_rows = own atoms -> nl_map_ids.
+ * nl_halo_count -> exchange counts -> nl_halo_fill_blocks -> all-to-all of
+ * the fixed blocks -> nl_halo_pack -> nl_build_rows_dev on [own atoms;
+ * received halo] with n_rows = own atoms -> nl_map_ids.  No step needs a
+ * count on the host.  (nl_halo_fill with exact offsets remains for callers
+ * that size the exchange on the host.)
  */
 #ifndef NL_SHARD_H
 #define NL_SHARD_H
@@ -65,6 +67,30 @@ nl_status nl_halo_fill(nl_ctx *ctx, int64_t n, const float *pos, const float *bo
                        const int32_t dims[3], const int32_t *need, int32_t rank, int32_t nranks,
                        const int32_t *offsets, const int32_t *counts, int32_t *cursor,
                        float *send_out, void *stream);
+
+/* nl_halo_fill into fixed blocks, so that nothing on the host depends on
+ * the counts: the atoms for rank q go to send_out[q * block ..], at most
+ * `block` of them (send_out: device, 16-byte aligned, nranks * block x 4
+ * float32; the blocks are exchanged by an all-to-all of equal splits).  A
+ * count above `block` drops the excess and makes nl_sync_status report
+ * NL_ERR_HALO.  block < 1 or a NULL buffer is NL_ERR_ARG. */
+nl_status nl_halo_fill_blocks(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                              const int32_t dims[3], const int32_t *need, int32_t rank,
+                              int32_t nranks, int32_t block, const int32_t *counts,
+                              int32_t *cursor, float *send_out, void *stream);
+
+/* Appends the halo received as fixed blocks to the own atoms, on the device:
+ * recv (device, nranks * block x 4 float32) holds in block q the
+ * min(recv_counts[q], block) atoms rank q sent (recv_counts: device
+ * int32[nranks], the all-to-all of the senders' counts); they are written
+ * to pos_all after its first n_own (own) atoms, block after block, and the
+ * total atom count to *n_all_out (device int64), clamped to n_max (pos_all
+ * holds room for n_max atoms).  A count above `block` or a total above
+ * n_max makes nl_sync_status report NL_ERR_HALO.  The count is meant for
+ * nl_build_rows_dev. */
+nl_status nl_halo_pack(nl_ctx *ctx, int32_t nranks, int32_t block, const int32_t *recv_counts,
+                       const float *recv, int64_t n_own, int64_t n_max, float *pos_all,
+                       int64_t *n_all_out, void *stream);
 
 /* In place: every entry j >= 0 of the n_rows x capacity rows nbr (indices
  * into pos_all, n_all atoms) becomes the global id in pos_all[j]'s fourth

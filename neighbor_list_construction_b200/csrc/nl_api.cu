@@ -67,6 +67,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 nl_status make_grid(nl_ctx *ctx, const float *box, float cutoff, float skin, CellGrid *g)
 {
     g->n_rows = INT64_MAX;
+    g->n_dev = nullptr;
     if (!std::isfinite(cutoff) || !std::isfinite(skin) || cutoff < 0.0f || skin < 0.0f)
         return NL_ERR_ARG;
     volatile float rl = cutoff + skin;
@@ -375,6 +376,7 @@ const char *nl_status_string(nl_status s)
     case NL_ERR_CUDA: return "NL_ERR_CUDA: CUDA runtime error";
     case NL_ERR_TIMEOUT: return "NL_ERR_TIMEOUT: a bounded device wait gave up";
     case NL_ERR_CAPACITY: return "NL_ERR_CAPACITY: n or capacity above the context maximum";
+    case NL_ERR_HALO: return "NL_ERR_HALO: a halo block or buffer was too small; rows incomplete";
     }
     return "unknown nl_status";
 }
@@ -474,6 +476,27 @@ nl_status nl_build(nl_ctx *ctx, int64_t n, const float *pos, const float *box, f
     if (st != NL_OK) return st;
     ctx->last_n = n;
     ctx->last_grid = g;
+    ctx->last_fast = fast;
+    return NL_OK;
+}
+
+nl_status nl_build_rows_dev(nl_ctx *ctx, int64_t n_max, const int64_t *n_dev, int64_t n_rows,
+                            const float *pos, const float *box, float cutoff, float skin,
+                            int32_t capacity, int32_t *nbr_out, int32_t *counts_out, void *stream)
+{
+    if (!n_dev || n_rows < 0 || n_rows > n_max) return NL_ERR_ARG;
+    CellGrid g;
+    nl_status st = build_checked(ctx, n_max, pos, box, cutoff, skin, capacity, nbr_out,
+                                 counts_out, &g, n_rows > 0);
+    if (st != NL_OK) return st;
+    g.n_rows = n_rows;
+    g.n_dev = n_dev;
+    int fast = 0;
+    st = build_enqueue(ctx, n_max, pos, g, capacity, nbr_out, counts_out, S(stream), &fast);
+    if (st != NL_OK) return st;
+    ctx->last_n = n_max;
+    ctx->last_grid = g;
+    ctx->last_grid.n_dev = nullptr;   // the pointer is the caller's
     ctx->last_fast = fast;
     return NL_OK;
 }
@@ -716,6 +739,7 @@ nl_status nl_sync_status(nl_ctx *ctx, void *stream)
         return NL_ERR_CUDA;
     if (f && cudaMemset(ctx->flags, 0, sizeof(uint32_t)) != cudaSuccess) return NL_ERR_CUDA;
     if (f & kFlagTimeout) return NL_ERR_TIMEOUT;
+    if (f & kFlagHalo) return NL_ERR_HALO;
     if (f & kFlagOverflow) return NL_OVERFLOW;
     return NL_OK;
 }

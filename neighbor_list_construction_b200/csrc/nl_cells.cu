@@ -23,6 +23,7 @@ k_bin_count(const float4 *__restrict__ pos, int64_t n, CellGrid g, uint32_t *__r
             uint32_t *__restrict__ atom_rank, int32_t *__restrict__ cell_count,
             float4 *__restrict__ ref)
 {
+    n = atoms_of(g, n);
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) - lane;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -134,6 +135,7 @@ k_bin_scatter(const float4 *__restrict__ pos, int64_t n, CellGrid g,
               const uint32_t *flags)
 {
     if (timed_out(flags)) return;   // cell starts may not be monotonic
+    n = atoms_of(g, n);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const float4 p = pos[i];

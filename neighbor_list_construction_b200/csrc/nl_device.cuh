@@ -40,6 +40,7 @@ constexpr uint32_t kSpinLimit = 1u << 22;
 // Device-detected conditions, accumulated in ctx->flags.
 constexpr uint32_t kFlagOverflow = 1u;
 constexpr uint32_t kFlagTimeout = 2u;
+constexpr uint32_t kFlagHalo = 4u;       // a halo block or buffer was too small
 
 enum Phase {
     PH_KEYS = 0,
@@ -67,7 +68,16 @@ struct CellGrid {
     int wy, wz;              // stencil half-width in y and z (x is always 1)
     int literal;             // 1: literal minimum image (small boxes)
     int64_t n_rows;          // rows are written for atoms of index < n_rows only
+    const int64_t *n_dev;    // when set: the atom count, read on the device (at most n)
 };
+
+// Atoms of a build: n, or the device-side count when the grid carries one.
+__device__ __forceinline__ int64_t atoms_of(const CellGrid &g, int64_t n)
+{
+    if (!g.n_dev) return n;
+    const int64_t d = *g.n_dev;
+    return d < 0 ? 0 : (d < n ? d : n);
+}
 
 
 // ------------------------------------------------------- device helpers

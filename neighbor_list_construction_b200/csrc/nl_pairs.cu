@@ -119,6 +119,7 @@ k_pairs_per_atom(const float4 *__restrict__ cell_pos, const int32_t *__restrict_
                  float close_d2, uint32_t *min_bits, unsigned long long *n_close)
 {
     if (timed_out(flags)) return;   // cell starts may not be monotonic
+    n = atoms_of(g, n);
     CloseAcc cl{__int_as_float(0x7f800000), 0u};
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride)

@@ -93,11 +93,17 @@ __global__ void k_halo_count(const float4 *__restrict__ pos, int64_t n, Coarse C
 
 // Writes the atoms counted by k_halo_count to send[offset[q] + k], k from
 // the cursor of q (zero before); order inside a destination is arbitrary.
+// block > 0: fixed blocks instead, destination q at q * block, at most
+// `block` atoms each; a count above it raises kFlagHalo in flags.
 __global__ void k_halo_fill(const float4 *__restrict__ pos, int64_t n, Coarse C,
                             const int32_t *__restrict__ need, int rank, int nranks,
                             const int32_t *__restrict__ offset, const int32_t *__restrict__ counts,
-                            int32_t *__restrict__ cursor, float4 *__restrict__ send)
+                            int32_t *__restrict__ cursor, float4 *__restrict__ send, int32_t block,
+                            uint32_t *flags)
 {
+    if (block > 0 && blockIdx.x == 0 && threadIdx.x < (unsigned)nranks &&
+        counts[threadIdx.x] > block)
+        atomicOr(flags, kFlagHalo);
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t n_up = (n + 31) & ~int64_t(31);
@@ -119,8 +125,48 @@ __global__ void k_halo_fill(const float4 *__restrict__ pos, int64_t n, Coarse C,
             base = __shfl_sync(0xffffffffu, base, leader);
             const int32_t k = base + __popc(b & lanemask_lt());
             // k < counts[q] unless the inputs changed since k_halo_count
-            if (mine && k < counts[q]) send[offset[q] + k] = p;
+            if (block > 0) {
+                if (mine && k < counts[q] && k < block) send[(int64_t)q * block + k] = p;
+            } else if (mine && k < counts[q]) {
+                send[offset[q] + k] = p;
+            }
         }
+    }
+}
+
+// Appends the received blocks to the own atoms: block q (recv[q * block ..])
+// holds min(recv_counts[q], block) atoms, which go to pos_all after the
+// n_own own atoms and the blocks before q; the total lands in *n_all_out.
+// A count above `block`, or a total above n_max, raises kFlagHalo (atoms
+// past n_max are dropped).
+__global__ void k_halo_pack(int nranks, int32_t block, const int32_t *__restrict__ recv_counts,
+                            const float4 *__restrict__ recv, int64_t n_own, int64_t n_max,
+                            float4 *__restrict__ pos_all, int64_t *n_all_out, uint32_t *flags)
+{
+    __shared__ int64_t s_off[33];
+    if (threadIdx.x == 0) {
+        int64_t off = 0;
+        bool bad = false;
+        for (int q = 0; q < nranks; ++q) {
+            const int32_t c = recv_counts[q];
+            bad |= c > block || c < 0;
+            s_off[q] = off;
+            off += c < 0 ? 0 : (c < block ? c : block);
+        }
+        s_off[nranks] = off;
+        if (n_own + off > n_max) bad = true;
+        if (bad && blockIdx.x == 0) atomicOr(flags, kFlagHalo);
+        if (blockIdx.x == 0) *n_all_out = n_own + off < n_max ? n_own + off : n_max;
+    }
+    __syncthreads();
+    const int64_t total = (int64_t)nranks * block;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+        const int q = (int)(e / block);
+        const int32_t k = (int32_t)(e - (int64_t)q * block);
+        const int64_t c = s_off[q + 1] - s_off[q];
+        const int64_t dst = n_own + s_off[q] + k;
+        if (k < c && dst < n_max) pos_all[dst] = recv[e];
     }
 }
 
@@ -264,7 +310,43 @@ nl_status nl_halo_fill(nl_ctx *ctx, int64_t n, const float *pos, const float *bo
     if (n > 0 && send_out)
         k_halo_fill<<<resident_grid(ctx, k_halo_fill, 256, 0, (n + 255) / 256), 256, 0, s>>>(
             reinterpret_cast<const float4 *>(pos), n, C, need, rank, nranks, offsets, counts,
-            cursor, reinterpret_cast<float4 *>(send_out));
+            cursor, reinterpret_cast<float4 *>(send_out), 0, ctx->flags);
+    return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
+}
+
+nl_status nl_halo_fill_blocks(nl_ctx *ctx, int64_t n, const float *pos, const float *box,
+                              const int32_t dims[3], const int32_t *need, int32_t rank,
+                              int32_t nranks, int32_t block, const int32_t *counts,
+                              int32_t *cursor, float *send_out, void *stream)
+{
+    Coarse C;
+    if (!ctx || n < 0 || nranks < 1 || nranks > 32 || rank < 0 || rank >= nranks || block < 1 ||
+        !need || !counts || !cursor || !send_out || !make_coarse(box, dims, &C))
+        return NL_ERR_ARG;
+    if (n > 0 && (!pos || (reinterpret_cast<uintptr_t>(pos) & 15u))) return NL_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(send_out) & 15u) return NL_ERR_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(cursor, 0, sizeof(int32_t) * nranks, s) != cudaSuccess) return NL_ERR_CUDA;
+    const int64_t want = n > 0 ? (n + 255) / 256 : 1;
+    k_halo_fill<<<resident_grid(ctx, k_halo_fill, 256, 0, want), 256, 0, s>>>(
+        reinterpret_cast<const float4 *>(pos), n, C, need, rank, nranks, nullptr, counts, cursor,
+        reinterpret_cast<float4 *>(send_out), block, ctx->flags);
+    return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
+}
+
+nl_status nl_halo_pack(nl_ctx *ctx, int32_t nranks, int32_t block, const int32_t *recv_counts,
+                       const float *recv, int64_t n_own, int64_t n_max, float *pos_all,
+                       int64_t *n_all_out, void *stream)
+{
+    if (!ctx || nranks < 1 || nranks > 32 || block < 1 || n_own < 0 || n_max < n_own ||
+        !recv_counts || !recv || !pos_all || !n_all_out ||
+        (reinterpret_cast<uintptr_t>(recv) & 15u) || (reinterpret_cast<uintptr_t>(pos_all) & 15u))
+        return NL_ERR_ARG;
+    const int64_t total = (int64_t)nranks * block;
+    k_halo_pack<<<resident_grid(ctx, k_halo_pack, 256, 0, (total + 255) / 256), 256, 0,
+                  reinterpret_cast<cudaStream_t>(stream)>>>(
+        nranks, block, recv_counts, reinterpret_cast<const float4 *>(recv), n_own, n_max,
+        reinterpret_cast<float4 *>(pos_all), n_all_out, ctx->flags);
     return cudaGetLastError() == cudaSuccess ? NL_OK : NL_ERR_CUDA;
 }
 

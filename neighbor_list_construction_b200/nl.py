@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libnl.so")
 
 NL_OK, NL_OVERFLOW = 0, 1
 NL_ERR_ARG, NL_ERR_BOX, NL_ERR_CUDA, NL_ERR_TIMEOUT, NL_ERR_CAPACITY = -1, -2, -3, -4, -5
+NL_ERR_HALO = -6
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libnl.so not built at {LIB_PATH}; run "
@@ -34,6 +35,8 @@ _SIGS = {
     "nl_sort_morton": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_build": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
     "nl_build_rows": (_i32, [_vp, _i64, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
+    "nl_build_rows_dev": (_i32, [_vp, _i64, _vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp,
+                                 _vp]),
     "nl_build_close": (_i32, [_vp, _i64, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _f32, _vp, _vp,
                               _vp]),
     "nl_skin_check": (_i32, [_vp, _i64, _vp, _vp, _f32, _vp, _vp, _vp]),
@@ -57,6 +60,9 @@ _SIGS = {
     "nl_halo_needed": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "nl_halo_count": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp]),
     "nl_halo_fill": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "nl_halo_fill_blocks": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp,
+                                   _vp, _vp]),
+    "nl_halo_pack": (_i32, [_vp, _i32, _i32, _vp, _vp, _i64, _i64, _vp, _vp, _vp]),
     "nl_map_ids": (_i32, [_vp, _i64, _i32, _vp, _vp, _i64, _vp, _vp]),
     "nls_displace": (_i32, [_i64, _vp, _u64, _i64, _vp, _f32, _vp]),
     "nls_step_graph": (_i32, [ctypes.POINTER(_vp), _i64, _vp, _u64, _vp, _f32]),
@@ -317,6 +323,19 @@ def nl_halo_needed(ctx, box, dims, occ_all, need_out, stream=None) -> int:
                   "nl_halo_needed")
 
 
+def nl_build_rows_dev(ctx, pos, n_dev, n_rows, box, cutoff, skin, capacity, nbr_out, counts_out,
+                      stream=None) -> int:
+    """pos holds room for n_max = pos.shape[0] atoms; n_dev (int64 [1], device)
+    says how many take part."""
+    _pos(pos)
+    rows = min(max(int(n_rows), 0), pos.shape[0])
+    return _check(_lib.nl_build_rows_dev(ctx, pos.shape[0], _buf(n_dev, "n_dev", _I64, 1),
+                                         int(n_rows), _ptr(pos), _box(box), float(cutoff),
+                                         float(skin), int(capacity),
+                                         *_rows_outs(rows, capacity, nbr_out, counts_out),
+                                         _stream(stream)), "nl_build_rows_dev")
+
+
 def nl_halo_count(ctx, pos, box, dims, need, rank, nranks, counts_out, stream=None) -> int:
     _pos(pos)
     return _check(_lib.nl_halo_count(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
@@ -335,6 +354,31 @@ def nl_halo_fill(ctx, pos, box, dims, need, rank, nranks, offsets, counts, curso
                                     _buf(offsets, "offsets", _I32, q), _buf(counts, "counts", _I32, q),
                                     _buf(cursor, "cursor", _I32, q), _buf(send_out, "send_out", _F32),
                                     _stream(stream)), "nl_halo_fill")
+
+
+def nl_halo_fill_blocks(ctx, pos, box, dims, need, rank, nranks, block, counts, cursor, send_out,
+                        stream=None) -> int:
+    _pos(pos)
+    q = int(nranks)
+    return _check(_lib.nl_halo_fill_blocks(ctx, pos.shape[0], _ptr(pos), _box(box), _dims(dims),
+                                           _buf(need, "need", _I32, _cells(dims)), int(rank), q,
+                                           int(block), _buf(counts, "counts", _I32, q),
+                                           _buf(cursor, "cursor", _I32, q),
+                                           _buf(send_out, "send_out", _F32, q * int(block) * 4),
+                                           _stream(stream)), "nl_halo_fill_blocks")
+
+
+def nl_halo_pack(ctx, nranks, block, recv_counts, recv, n_own, pos_all, n_all_out,
+                 stream=None) -> int:
+    """pos_all holds room for n_max = pos_all.shape[0] atoms, its first n_own
+    the own ones."""
+    _pos(pos_all)
+    q, blk = int(nranks), int(block)
+    return _check(_lib.nl_halo_pack(ctx, q, blk, _buf(recv_counts, "recv_counts", _I32, q),
+                                    _buf(recv, "recv", _F32, q * blk * 4), int(n_own),
+                                    pos_all.shape[0], _ptr(pos_all),
+                                    _buf(n_all_out, "n_all_out", _I64, 1), _stream(stream)),
+                  "nl_halo_pack")
 
 
 def nl_map_ids(ctx, nbr, pos_all, counts=None, stream=None) -> int:

@@ -10,10 +10,20 @@ halo).  One rank's build, in the order the steps run:
 3. ``nl_halo_needed``, ``nl_halo_count``: per destination rank, how many of
    its atoms lie next to a cell of that rank; the counts go round
    (all-to-all), so each rank knows how many atoms it will receive;
-4. ``nl_halo_fill`` and an all-to-all of those atoms: the halo;
-5. ``nl_build_rows`` over [own atoms; halo], rows for the own atoms only;
-6. ``nl_map_ids``: row entries become global ids (carried in the fourth
+4. ``nl_halo_fill_blocks`` and an all-to-all of equal splits: every rank
+   sends a fixed block of ``halo_block`` atoms to every other rank;
+5. ``nl_halo_pack``: the received blocks are appended to the own atoms on
+   the device, and the atom count stays in device memory;
+6. ``nl_build_rows_dev`` over [own atoms; halo], rows for the own atoms only;
+7. ``nl_map_ids``: row entries become global ids (carried in the fourth
    float of each position).
+
+No step reads a count on the host, so a build enqueues without waiting for
+the GPU.  The block size is agreed once: the first build of a driver (when
+no block is given) takes the largest count over all ranks (an all-reduce of
+maxima, one host read) with a quarter to spare, and later builds reuse it.
+A count above the block drops atoms and makes ``sync_status`` report
+``NL_ERR_HALO``; the caller then rebuilds with a larger block.
 
 Every step that touches atoms runs in libnl's kernels; this module only
 moves buffers between ranks.  The steps are written once, as a generator
@@ -53,10 +63,18 @@ def with_ids(pos: torch.Tensor, first_id: int) -> torch.Tensor:
     return out
 
 
-def _steps(ctx, pos_own, box, cutoff, skin, capacity, rank, nranks):
-    """One rank's halo build; yields ("sum", occ), ("counts", counts) and
-    ("atoms", send, send_splits, recv_splits) for the driver to answer with
-    the combined result, and returns (nbr, counts, n_halo)."""
+def block_for(max_count: int) -> int:
+    """Halo block for a largest per-destination count: a quarter to spare,
+    rounded up to 64 atoms."""
+    want = int(max_count) + int(max_count) // 4 + 64
+    return (want + 63) // 64 * 64
+
+
+def _steps(ctx, pos_own, box, cutoff, skin, capacity, rank, nranks, block=None):
+    """One rank's halo build; yields ("sum", occ), ("counts", counts),
+    ("max", local max) when no block is given, and ("blocks", send) for the
+    driver to answer with the combined result, and returns (nbr, counts,
+    halo atoms as a device int64 tensor, block)."""
     dev = pos_own.device
     n_own = pos_own.shape[0]
     dims = nl.nl_halo_grid(box, cutoff, skin)
@@ -69,22 +87,26 @@ def _steps(ctx, pos_own, box, cutoff, skin, capacity, rank, nranks):
     counts = torch.empty(nranks, dtype=torch.int32, device=dev)
     nl.nl_halo_count(ctx.handle, pos_own, box, dims, need, rank, nranks, counts)
     recv_counts = yield ("counts", counts)
-    send_splits = [int(v) for v in counts.tolist()]
-    recv_splits = [int(v) for v in recv_counts.tolist()]
-    offsets = torch.zeros(nranks, dtype=torch.int32, device=dev)
-    if nranks > 1:
-        offsets[1:] = torch.cumsum(counts, 0, dtype=torch.int32)[:-1]
-    send = torch.empty(max(sum(send_splits), 1), 4, dtype=torch.float32, device=dev)
+    if block is None:   # agree on a block: the one host read, first build only
+        top = yield ("max", counts.max().reshape(1))
+        block = block_for(int(top.item()))
+    send = torch.empty(nranks * block, 4, dtype=torch.float32, device=dev)
     cursor = torch.empty(nranks, dtype=torch.int32, device=dev)
-    nl.nl_halo_fill(ctx.handle, pos_own, box, dims, need, rank, nranks, offsets, counts, cursor,
-                    send)
-    send = send[: sum(send_splits)]
-    halo = yield ("atoms", send, send_splits, recv_splits)
-    pos_all = torch.cat([pos_own, halo]) if halo.shape[0] else pos_own
-    nbr, cnt = ctx.build_rows(pos_all, n_own, box, cutoff, skin, capacity)
+    nl.nl_halo_fill_blocks(ctx.handle, pos_own, box, dims, need, rank, nranks, block, counts,
+                           cursor, send)
+    recv = yield ("blocks", send)
+    n_max = n_own + (nranks - 1) * block
+    pos_all = torch.empty(n_max, 4, dtype=torch.float32, device=dev)
+    pos_all[:n_own] = pos_own
+    n_all = torch.empty(1, dtype=torch.int64, device=dev)
+    nl.nl_halo_pack(ctx.handle, nranks, block, recv_counts, recv, n_own, pos_all, n_all)
+    nbr = torch.empty(n_own, capacity, dtype=torch.int32, device=dev)
+    cnt = torch.empty(n_own, dtype=torch.int32, device=dev)
+    nl.nl_build_rows_dev(ctx.handle, pos_all, n_all, n_own, box, cutoff, skin, capacity,
+                         nbr if n_own else None, cnt if n_own else None)
     if n_own:
         nl.nl_map_ids(ctx.handle, nbr, pos_all, cnt)
-    return nbr, cnt, int(halo.shape[0])
+    return nbr, cnt, n_all - n_own, block
 
 
 class DistExchange:
@@ -107,10 +129,15 @@ class DistExchange:
         self.dist.all_to_all_single(out, c.contiguous(), group=self.group)
         return out
 
-    def atoms(self, send: torch.Tensor, send_splits, recv_splits) -> torch.Tensor:
-        out = torch.empty(sum(recv_splits), 4, dtype=send.dtype, device=send.device)
-        self.dist.all_to_all_single(out, send.contiguous(), output_split_sizes=list(recv_splits),
-                                    input_split_sizes=list(send_splits), group=self.group)
+    def max(self, t: torch.Tensor) -> torch.Tensor:
+        out = t.clone()
+        self.dist.all_reduce(out, op=self.dist.ReduceOp.MAX, group=self.group)
+        return out
+
+    def blocks(self, send: torch.Tensor) -> torch.Tensor:
+        """All-to-all of equal splits: block q of send goes to rank q."""
+        out = torch.empty_like(send)
+        self.dist.all_to_all_single(out, send.contiguous(), group=self.group)
         return out
 
     def run(self, gen):
@@ -120,18 +147,24 @@ class DistExchange:
                 ans = self.sum(req[1])
             elif req[0] == "counts":
                 ans = self.counts(req[1])
+            elif req[0] == "max":
+                ans = self.max(req[1])
             else:
-                ans = self.atoms(req[1], req[2], req[3])
+                ans = self.blocks(req[1])
             try:
                 req = gen.send(ans)
             except StopIteration as fin:
                 return fin.value
 
 
-def build_sharded(ctx, pos_own, box, cutoff, skin, capacity, comm: DistExchange):
+def build_sharded(ctx, pos_own, box, cutoff, skin, capacity, comm: DistExchange,
+                  halo_block: int | None = None):
     """This rank's rows over its own atoms (pos_own, global ids in the fourth
-    float): (nbr [n_own, capacity] of global ids, counts [n_own], halo size)."""
-    return comm.run(_steps(ctx, pos_own, box, cutoff, skin, capacity, comm.rank, comm.size))
+    float): (nbr [n_own, capacity] of global ids, counts [n_own], halo atoms
+    (device int64 [1]), the halo block used).  Pass the returned block back
+    to later builds: they then need no host read."""
+    return comm.run(_steps(ctx, pos_own, box, cutoff, skin, capacity, comm.rank, comm.size,
+                           halo_block))
 
 
 def route_local(reqs):
@@ -149,22 +182,23 @@ def route_local(reqs):
     if kind == "counts":
         mat = torch.stack([r[1] for r in reqs])      # [source, destination]
         return [mat[:, q].contiguous() for q in range(nranks)]
-    pieces = []
-    for r in reqs:
-        send, splits = r[1], r[2]
-        offs = [0]
-        for v in splits:
-            offs.append(offs[-1] + int(v))
-        pieces.append([send[offs[q]:offs[q + 1]] for q in range(nranks)])
+    if kind == "max":
+        top = reqs[0][1].clone()
+        for r in reqs[1:]:
+            top = torch.maximum(top, r[1])
+        return [top for _ in reqs]
+    # blocks: equal splits, block q of rank p's send goes to rank q
+    pieces = [r[1].chunk(nranks) for r in reqs]
     return [torch.cat([pieces[p][q] for p in range(nranks)]) for q in range(nranks)]
 
 
-def build_sharded_local(ctx, shards, box, cutoff, skin, capacity):
+def build_sharded_local(ctx, shards, box, cutoff, skin, capacity, halo_block: int | None = None):
     """All shards' halo builds in one process (one context, one GPU): the
     same steps as build_sharded, with the collectives answered by
-    route_local.  Returns one (nbr, counts, halo size) per shard."""
+    route_local.  Returns one (nbr, counts, halo atoms, block) per shard."""
     nranks = len(shards)
-    gens = [_steps(ctx, p, box, cutoff, skin, capacity, r, nranks) for r, p in enumerate(shards)]
+    gens = [_steps(ctx, p, box, cutoff, skin, capacity, r, nranks, halo_block)
+            for r, p in enumerate(shards)]
     reqs = [next(g) for g in gens]
     while True:
         answers = route_local(reqs)

@@ -48,22 +48,24 @@ def assert_rows_match(g_nbr, g_cnt, o_nbr, o_cnt, full_sets=None):
             assert set(row.tolist()) <= full_sets[r]
 
 
-def assert_all_rows_match(oracle, nbr_t, cnt_t, pos, box, cutoff, skin, K, chunk=1 << 21):
+def assert_all_rows_match(oracle, nbr_t, cnt_t, pos, box, cutoff, skin, K, chunk=1 << 21,
+                          row_offset=0):
     """Every row and count of a GPU build (device tensors, any slot order)
-    against the oracle, element by element, in chunks of rows.
+    against the oracle, element by element, in chunks of rows.  Row r of the
+    GPU tensors is atom row_offset + r of pos (a shard's rows).
 
     The GPU rows are put in canonical order (ascending, -1 padding last) with
     torch.sort on the device; the oracle's rows come from oracle.rows on the
     same positions.  Rows whose count passes K must hold K distinct members of
     the atom's full neighbor set.  Returns True when any row overflowed."""
     import torch
-    n = pos.shape[0]
+    n = nbr_t.shape[0]
     cnt = cnt_t.cpu().numpy()
     big = torch.iinfo(torch.int32).max
     overflow = False
     for s in range(0, n, chunk):
         e = min(n, s + chunk)
-        which = np.arange(s, e, dtype=np.int64)
+        which = np.arange(row_offset + s, row_offset + e, dtype=np.int64)
         o_nbr, o_cnt, o_ov = oracle.rows(pos, box, cutoff, skin, K, which)
         np.testing.assert_array_equal(cnt[s:e], o_cnt)
         g = nbr_t[s:e]

@@ -50,7 +50,8 @@ def bufs():
              rb=i32(1), md=torch.zeros(1), row_ptr=torch.zeros(N + 1, dtype=torch.int64),
              col=i32(N * K), edges=torch.zeros(N * K, 4), edges3=torch.zeros(N, K, 4),
              dec=i32(STEPS), ids=i32(N), aux=torch.zeros(N, 4), occ=i32(12), need=i32(12),
-             cnt2=i32(2), offs=i32(2), cursor=i32(2), send=torch.zeros(N, 4))
+             cnt2=i32(2), offs=i32(2), cursor=i32(2), send=torch.zeros(N, 4),
+             ndev=torch.zeros(1, dtype=torch.int64), blocks=torch.zeros(2 * 3, 4))
     return b
 
 
@@ -83,6 +84,13 @@ def calls(b):
                                                   b["cnt2"]),
         "nl_halo_fill": lambda: nl.nl_halo_fill(ctx, b["pos"], BOX, DIMS, b["need"], 0, 2,
                                                 b["offs"], b["cnt2"], b["cursor"], b["send"]),
+        "nl_halo_fill_blocks": lambda: nl.nl_halo_fill_blocks(ctx, b["pos"], BOX, DIMS, b["need"],
+                                                              0, 2, 3, b["cnt2"], b["cursor"],
+                                                              b["blocks"]),
+        "nl_halo_pack": lambda: nl.nl_halo_pack(ctx, 2, 3, b["cnt2"], b["blocks"], 4, b["pos"],
+                                                b["ndev"]),
+        "nl_build_rows_dev": lambda: nl.nl_build_rows_dev(ctx, b["pos"], b["ndev"], 5, BOX, 2.0,
+                                                          0.5, K, b["nbr5"], b["cnt5"]),
         "nl_map_ids": lambda: nl.nl_map_ids(ctx, b["nbr"], b["pos"], b["cnt"]),
         "nl_wait_selftest": lambda: nl.nl_wait_selftest(ctx, 1000),
     }
@@ -119,6 +127,11 @@ BAD = [
     ("nl_halo_count", "cnt2", torch.zeros(1, dtype=torch.int32)),
     ("nl_halo_fill", "cursor", torch.zeros(1, dtype=torch.int32)),
     ("nl_map_ids", "cnt", torch.zeros(N - 1, dtype=torch.int32)),
+    ("nl_halo_fill_blocks", "blocks", torch.zeros(5, 4)),
+    ("nl_halo_pack", "ndev", torch.zeros(1, dtype=torch.int32)),
+    ("nl_halo_pack", "cnt2", torch.zeros(1, dtype=torch.int32)),
+    ("nl_build_rows_dev", "ndev", torch.zeros(0, dtype=torch.int64)),
+    ("nl_build_rows_dev", "nbr5", torch.zeros(4, K, dtype=torch.int32)),
 ]
 
 

@@ -1,7 +1,7 @@
 """Host side of the sharded build, on CPU: the equal-count cut, the id lane,
-and the collectives -- DistExchange over gloo with two ranks must answer
-every request exactly as route_local (the single-process routing that the
-one-GPU tests use) does."""
+and the collectives -- DistExchange over gloo with two and three ranks
+must answer every request exactly as route_local (the single-process
+routing that the one-GPU tests use) does."""
 import os
 import socket
 
@@ -32,18 +32,20 @@ def test_with_ids_puts_id_bits_in_the_fourth_float():
     assert q[:, 3].view(torch.int32).tolist() == [1000, 1001, 1002, 1003, 1004]
 
 
+BLOCK = 6
+
+
 def fake_requests(rank, nranks):
-    """The three collectives of one rank, with rank-dependent payloads."""
+    """The four collectives of one rank, with rank-dependent payloads: the
+    occupancy marks, the per-destination counts, the local maximum count and
+    the fixed blocks of atoms (BLOCK per destination)."""
     g = torch.Generator().manual_seed(rank)
     occ = (torch.randint(0, 2, (50,), generator=g, dtype=torch.int32) << rank).to(torch.int32)
     counts = torch.tensor([(rank * 3 + q * 5) % 7 if q != rank else 0 for q in range(nranks)],
                           dtype=torch.int32)
-    send = torch.rand(int(counts.sum()), 4, generator=g)
-    return occ, counts, send
-
-
-def recv_splits_of(rank, nranks):
-    return [fake_requests(p, nranks)[1][rank].item() for p in range(nranks)]
+    top = counts.max().reshape(1)
+    send = torch.rand(nranks * BLOCK, 4, generator=g)
+    return occ, counts, top, send
 
 
 def _gloo_rank(rank, nranks, port, out_dir):
@@ -53,16 +55,18 @@ def _gloo_rank(rank, nranks, port, out_dir):
     dist.init_process_group("gloo", rank=rank, world_size=nranks)
     try:
         ex = shard.DistExchange()
-        occ, counts, send = fake_requests(rank, nranks)
+        occ, counts, top, send = fake_requests(rank, nranks)
 
         def steps():
             a = yield ("sum", occ)
             b = yield ("counts", counts)
-            c = yield ("atoms", send, counts.tolist(), b.tolist())
-            return a, b, c
+            m = yield ("max", top)
+            c = yield ("blocks", send)
+            return a, b, m, c
 
-        a, b, c = ex.run(steps())
-        torch.save({"sum": a, "counts": b, "atoms": c}, os.path.join(out_dir, f"r{rank}.pt"))
+        a, b, m, c = ex.run(steps())
+        torch.save({"sum": a, "counts": b, "max": m, "blocks": c},
+                   os.path.join(out_dir, f"r{rank}.pt"))
     finally:
         dist.destroy_process_group()
 
@@ -80,13 +84,25 @@ def test_dist_exchange_matches_local_routing(tmp_path, nranks):
     reqs = [fake_requests(r, nranks) for r in range(nranks)]
     sums = shard.route_local([("sum", r[0]) for r in reqs])
     cnts = shard.route_local([("counts", r[1]) for r in reqs])
-    atoms = shard.route_local([("atoms", r[2], r[1].tolist(), recv_splits_of(k, nranks))
-                               for k, r in enumerate(reqs)])
+    tops = shard.route_local([("max", r[2]) for r in reqs])
+    blocks = shard.route_local([("blocks", r[3]) for r in reqs])
     for k in range(nranks):
         got = torch.load(os.path.join(tmp_path, f"r{k}.pt"))
         assert torch.equal(got["sum"], sums[k])
         assert torch.equal(got["counts"], cnts[k])
-        assert torch.equal(got["atoms"], atoms[k])
+        assert torch.equal(got["max"], tops[k])
+        assert torch.equal(got["blocks"], blocks[k])
+        # block q of rank p's send is block p of rank q's receive
+        for p in range(nranks):
+            assert torch.equal(got["blocks"][p * BLOCK:(p + 1) * BLOCK],
+                               reqs[p][3][k * BLOCK:(k + 1) * BLOCK])
+        assert got["max"].item() == max(int(r[1].max()) for r in reqs)
         # the sum of distinct rank bits is their bitwise or
         ors = np.bitwise_or.reduce(np.stack([r[0].numpy() for r in reqs]), axis=0)
         assert np.array_equal(got["sum"].numpy(), ors)
+
+
+def test_block_for_leaves_room():
+    for top in (0, 1, 63, 64, 1000, 301_000):
+        b = shard.block_for(top)
+        assert b % 64 == 0 and b >= top + top // 4 and b >= 64
