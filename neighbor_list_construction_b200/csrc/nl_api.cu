@@ -32,7 +32,7 @@ void free_ctx(nl_ctx *c)
     void *bufs[] = {c->keys[0], c->keys[1], c->vals[0], c->vals[1], c->hist, c->sort_status,
                     c->sort_ctr, c->cell_count, c->cell_start, c->scan_status, c->scan_ctr,
                     c->atom_cell, c->atom_rank, c->cell_pos, c->ref, c->zero_block,
-                    c->fb_list, c->cell_tab};
+                    c->fb_list, c->fb_list2, c->cell_tab};
     for (void *b : bufs)
         if (b) cudaFree(b);
     if (c->prof_ev) {
@@ -419,6 +419,7 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
     ok &= alloc(&c->ref, N) == cudaSuccess;
     ok &= alloc(&c->zero_block, 64) == cudaSuccess;
     ok &= alloc(&c->fb_list, c->max_cells) == cudaSuccess;
+    ok &= alloc(&c->fb_list2, c->max_cells) == cudaSuccess;
     ok &= alloc(&c->cell_tab, (size_t)c->max_cells * 16) == cudaSuccess;
     if (ok) {
         c->flags = c->zero_block;
@@ -428,8 +429,10 @@ nl_status nl_create(nl_ctx **out, int64_t max_atoms, int32_t max_capacity)
         c->unsorted = c->zero_block + 12;
         c->fb_count = c->zero_block + 13;
         c->tile_ctr = c->zero_block + 14;
-        c->sort_gate = c->zero_block + 15;
-        c->probe_word = c->zero_block + 16;
+        c->fb_count2 = c->zero_block + 15;
+        c->tile_ctr2 = c->zero_block + 16;
+        c->sort_gate = c->zero_block + 17;
+        c->probe_word = c->zero_block + 18;
         ok &= pairs_set_attributes() == cudaSuccess;
         ok &= cudaMemset(c->zero_block, 0, 64 * sizeof(uint32_t)) == cudaSuccess;
         ok &= cudaDeviceSynchronize() == cudaSuccess;
@@ -802,7 +805,7 @@ const char *nl_profile_phase_name(int32_t phase)
 {
     static const char *names[PH_COUNT] = {"keys",        "key_scan",   "radix_sort", "gather",
                                           "bin_count",   "cell_scan",  "bin_scatter",
-                                          "cell_sort",   "pair_search", "pair_search_per_atom",
+                                          "cell_sort",   "pair_search", "pair_search_listed",
                                           "skin_check",  "edge_features"};
     if (phase < 0 || phase >= PH_COUNT) return "";
     return names[phase];

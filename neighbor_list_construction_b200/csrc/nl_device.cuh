@@ -52,7 +52,7 @@ enum Phase {
     PH_BIN_SCATTER,
     PH_CELL_SORT,
     PH_PAIRS,
-    PH_PAIRS_FALLBACK,
+    PH_PAIRS_LISTED,
     PH_SKIN,
     PH_EDGES,
     PH_COUNT

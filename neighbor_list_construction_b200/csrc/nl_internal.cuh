@@ -47,6 +47,9 @@ struct nl_ctx {
     uint32_t *unsorted = nullptr;      // [1] 1 if a cell was too large for the in-cell sort
     uint32_t *fb_count = nullptr;      // [1] tiles listed for the larger-stage launch
     uint32_t *tile_ctr = nullptr;      // [1] next tile of the persistent pair search (after fb_count)
+    uint32_t *fb_count2 = nullptr;     // [1] tiles listed by the two-stage pass (after tile_ctr)
+    uint32_t *tile_ctr2 = nullptr;     // [1] next list entry of the two-stage pass
+    uint32_t *fb_list2 = nullptr;      // [max_cells] their ids
     uint32_t *probe_word = nullptr;    // [1] a word nothing writes (bounded-wait self-test)
     uint32_t *sort_gate = nullptr;     // [1] set when the sort needs its full path
     uint32_t *fb_list = nullptr;       // [max_cells] their ids

@@ -165,12 +165,18 @@ static_assert(kHome <= 32, "home rows are counted one per lane");
 constexpr int kSCells = kTX + 2;            // conceptual cells per staged row
 constexpr int kBinsPerCell = 16;            // x sub-bins per cell (tables built by k_cell_sort)
 constexpr int kRowTab = kSCells * kBinsPerCell;
-constexpr int kFlushAt = 8;                 // pending hits that make the warp flush
-constexpr int kBuf = kFlushAt + 4;          // entries of a lane's hit buffer (7 pending + 4 new)
+// A warp flush costs the same whatever it moves, so hits are flushed late:
+// kFlushAt pending entries in some lane.  The buffer then holds at most
+// kFlushAt - 1 pending plus one group of 4 new.  Measured on saltwater10m
+// (pair search, ms): flush at 8 with 24 searching warps 5.11; at 16, 4.79;
+// at 24 with 20 warps 4.45 (16 warps 4.73; larger buffers leave stages too
+// small for the densest tiles).
+constexpr int kFlushAt = 24;                // pending hits that make the warp flush
+constexpr int kBuf = kFlushAt + 4;          // entries of a lane's hit buffer
 constexpr uint32_t kHitStride = 128;        // bytes between a lane's buffer entries (32 lanes x 4)
-constexpr int kPipeStages = 3;              // staged tiles per CTA of the persistent launch
+constexpr int kPipeStages = 3;              // most staged tiles per CTA of the persistent launch
 constexpr int kPipeMeta = kPipeStages + 1;  // tile descriptions: one ahead of the stages
-constexpr int kPipeConsumers = 24;          // searching warps per CTA (plus one staging warp)
+constexpr int kPipeConsumers = 20;          // searching warps per CTA (plus one staging warp)
 constexpr int kPipeThreads = 32 * (1 + kPipeConsumers);
 constexpr int kQueue = 512;                 // chunk-queue entries
 constexpr uint32_t kQueueEnd = 0xffffffffu;
@@ -211,7 +217,10 @@ struct TileParams {
     const uint32_t *unsorted;
     uint32_t *fb_list;
     uint32_t *fb_count;
-    uint32_t *tile_ctr;             // next tile of the persistent launch
+    uint32_t *tile_ctr;             // next tile (or list entry) of the persistent launch
+    const uint32_t *tile_list;      // the tiles to take, or NULL: every tile in order
+    const uint32_t *tile_list_count;
+    int stages;                     // shared-memory stages of a persistent CTA (1..kPipeStages)
     int tiles_x, tiles_y;
     int ntiles;
     int K;
@@ -1054,16 +1063,17 @@ k_pairs_pipe(const CellGrid g, const TileParams P)
     if (__syncthreads_or(timed_out(P.flags))) return;
     extern __shared__ __align__(16) unsigned char pipe_smem[];
     __shared__ PipeShared sh;
+    const int S = P.stages;
     float4 *stages = reinterpret_cast<float4 *>(pipe_smem);                       // [S][stage_max]
-    uint8_t *tabs = pipe_smem + sizeof(float4) * (size_t)kPipeStages * P.stage_max;   // [S][kSRows][kRowTab]
-    int32_t *hits = reinterpret_cast<int32_t *>(tabs + kPipeStages * kSRows * kRowTab);
+    uint8_t *tabs = pipe_smem + sizeof(float4) * (size_t)S * P.stage_max;          // [S][kSRows][kRowTab]
+    int32_t *hits = reinterpret_cast<int32_t *>(tabs + S * kSRows * kRowTab);
     int32_t *negs = hits + kPipeConsumers * 32 * kBuf;                           // P.K entries of -1
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < P.K; e += blockDim.x) negs[e] = -1;
     fence_proxy_async_smem();   // -1 block is read by bulk copies of any thread
     if (threadIdx.x == 0) {
-        for (int st = 0; st < kPipeStages; ++st) {
+        for (int st = 0; st < S; ++st) {
             mbar_init(&sh.full[st], 1);
             mbar_init(&sh.empty[st], kEmptyCount);
         }
@@ -1079,21 +1089,31 @@ k_pairs_pipe(const CellGrid g, const TileParams P)
         uint32_t tail = 0u;
         int k = 0, mi = 0;               // fills issued; description slot of the next fill
         bool gave_up = false;
-        int t = lane == 0 ? (int)atomicAdd(P.tile_ctr, 1u) : 0;
-        t = __shfl_sync(0xffffffffu, t, 0);
-        while (t < P.ntiles) {
+        // the next tile: in order, or the next entry of the list; -1 when done
+        auto next_tile = [&]() {
+            int tt = -1;
+            if (lane == 0) {
+                const uint32_t e = atomicAdd(P.tile_ctr, 1u);
+                if (P.tile_list)
+                    tt = e < ld_volatile_u32(P.tile_list_count) ? (int)P.tile_list[e] : -1;
+                else
+                    tt = e < (uint32_t)P.ntiles ? (int)e : -1;
+            }
+            return __shfl_sync(0xffffffffu, tt, 0);
+        };
+        int t = next_tile();
+        while (t >= 0) {
             RowSrc ra, rb;
             const uint32_t bytes = describe_tile(t, g, P, sh.tr[mi], sh.rinfo[mi], sh.meta[mi], ra, rb);
             const int tile = t;
-            t = lane == 0 ? (int)atomicAdd(P.tile_ctr, 1u) : 0;
-            t = __shfl_sync(0xffffffffu, t, 0);
+            t = next_tile();
             const int nhome = sh.tr[mi].home_pref[kHome];
             if (sh.tr[mi].fallback) {
-                if (lane == 0) P.fb_list[atomicAdd(P.fb_count, 1u)] = (uint32_t)tile;
+                if (lane == 0) P.fb_list[atomicAdd(P.fb_count, 1u)] = (uint32_t)tile;   // out list
                 continue;
             }
             if (nhome == 0) continue;
-            const int st = k % kPipeStages;
+            const int st = k % S;
             if (used >> st & 1u) {   // the stage's previous tile must be searched out
                 bool done = false;
                 for (uint32_t spins = 0; spins < 4096u && !done; ++spins)
@@ -1277,11 +1297,27 @@ k_pairs_listed(const CellGrid g, const TileParams P)
 
 constexpr int kSlotLimit = 65000;   // slot-table entries are 16 bits
 
-// Dynamic shared memory of the two launches besides their stages.
-size_t pipe_fixed_smem(int K)
+// Dynamic shared memory of the persistent launch with S stages of
+// stage_max slots: the stages, their row tables, the hit buffers, the -1
+// block.
+size_t pipe_smem_bytes(int K, int S, int stage_max)
 {
-    return (size_t)kPipeStages * kSRows * kRowTab +
+    return (size_t)S * ((size_t)stage_max * sizeof(float4) + (size_t)kSRows * kRowTab) +
            (size_t)kPipeConsumers * 32 * kBuf * sizeof(int32_t) + (size_t)K * sizeof(int32_t);
+}
+
+// Stage slots of the persistent launch with S stages, from what shared
+// memory leaves after its static part; also bounded by the chunk queue
+// (every chunk of S tiles plus the end entries) and the 16-bit slot tables.
+// 0 when too small to be worth a launch.
+int pipe_stage_slots(int optin, int static_smem, int K, int S)
+{
+    const long budget = (long)optin - static_smem - (long)pipe_smem_bytes(K, S, 0);
+    long fit = budget > 0 ? budget / ((long)sizeof(float4) * S) : 0;
+    const long qcap = (long)(kQueue - kPipeConsumers - 8) / S * 32;
+    if (fit > qcap) fit = qcap;
+    if (fit > kSlotLimit) fit = kSlotLimit;
+    return fit >= 256 ? (int)(fit & ~31L) : 0;
 }
 
 size_t listed_fixed_smem(int K)
@@ -1329,7 +1365,7 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
     // shared memory; a stage should hold a typical tile (kSRows rows x
     // (kTX + 2) cells at the mean cell occupancy) with 10 % to spare.  Denser
     // tiles are listed for a second launch with larger stages.
-    int stage_max = 0;
+    int stage3 = 0, stage2 = 0;   // stage slots with three and with two stages per CTA
     int need = 0, per_sm = 0, reserved = 0, optin = 0;
     if (g.wy == 2 && g.wz == 2 && !g.literal && capacity % 4 == 0 &&
         (reinterpret_cast<uintptr_t>(nbr) & 15u) == 0 && n < (int64_t(1) << 31)) {
@@ -1343,15 +1379,10 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         const double per_cell = (double)n / (double)g.ncell;
         const int want = (int)(1.1 * per_cell * kSRows * kSCells) + 32;
         need = want > kStageMin ? want : kStageMin;
-        const long budget = (long)optin - (long)fa.sharedSizeBytes - (long)pipe_fixed_smem(capacity);
-        long fit = budget > 0 ? budget / ((long)sizeof(float4) * kPipeStages) : 0;
-        // the chunk queue holds every chunk of kPipeStages tiles plus the end entries
-        const long qcap = (long)(kQueue - kPipeConsumers - 8) / kPipeStages * 32;
-        if (fit > qcap) fit = qcap;
-        if (fit > kSlotLimit) fit = kSlotLimit;
-        stage_max = fit >= 256 ? (int)(fit & ~31L) : 0;
+        stage3 = pipe_stage_slots(optin, (int)fa.sharedSizeBytes, capacity, 3);
+        stage2 = pipe_stage_slots(optin, (int)fa.sharedSizeBytes, capacity, 2);
     }
-    if (stage_max > 0) {
+    if (stage2 > 0) {
         TileParams P;
         P.close_d2 = CLOSE ? close->close_d2 : 0.0f;
         P.min_bits = CLOSE ? reinterpret_cast<uint32_t *>(close->min_d2) : nullptr;
@@ -1364,15 +1395,11 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         P.counts = counts;
         P.flags = ctx->flags;
         P.unsorted = ctx->unsorted;
-        P.fb_list = ctx->fb_list;
-        P.fb_count = ctx->fb_count;
-        P.tile_ctr = ctx->tile_ctr;
         P.tiles_x = (g.nx + kTX - 1) / kTX;
         P.tiles_y = (g.ny + kTY - 1) / kTY;
         const int tiles_z = (g.nz + kTZ - 1) / kTZ;
         P.ntiles = P.tiles_x * P.tiles_y * tiles_z;
         P.K = capacity;
-        P.stage_max = stage_max;
         P.side_x = g.Lx / (float)g.nx;
         P.side_y = g.Ly / (float)g.ny;
         P.side_z = g.Lz / (float)g.nz;
@@ -1381,18 +1408,53 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         const float Lmax = fmaxf(g.Lx, fmaxf(g.Ly, g.Lz));
         P.eps = 1e-3f * rl + 4e-6f * Lmax;
         P.rl2_margin = g.rl2 * (1.0f + 1e-4f);
-        const size_t smem = sizeof(float4) * (size_t)kPipeStages * stage_max + pipe_fixed_smem(capacity);
-        NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, 2 * sizeof(uint32_t), s));   // and tile_ctr
-        {
+        // fb_count, tile_ctr, fb_count2, tile_ctr2
+        NL_CUDA_TRY(cudaMemsetAsync(ctx->fb_count, 0, 4 * sizeof(uint32_t), s));
+        // Three stages when a typical tile fits them: every tile is taken in
+        // order and a tile beyond the stage is listed; a second persistent
+        // launch with two larger stages takes the listed tiles.  Systems
+        // denser than that start with the two-stage launch over every tile.
+        // Tiles beyond even those stages go to k_pairs_listed.
+        TileParams P2 = P;
+        P2.stages = 2;
+        P2.stage_max = stage2;
+        P2.tile_ctr = ctx->tile_ctr2;
+        P2.fb_list = ctx->fb_list2;
+        P2.fb_count = ctx->fb_count2;
+        if (stage3 > 0 && (double)need <= 1.1 * stage3) {
+            TileParams P3 = P;
+            P3.stages = 3;
+            P3.stage_max = stage3;
+            P3.tile_ctr = ctx->tile_ctr;
+            P3.tile_list = nullptr;
+            P3.tile_list_count = nullptr;
+            P3.fb_list = ctx->fb_list;
+            P3.fb_count = ctx->fb_count;
+            {
+                ProfScope ps(ctx, PH_PAIRS, s);
+                k_pairs_pipe<CLOSE><<<(unsigned)ctx->sm_count, kPipeThreads,
+                                      pipe_smem_bytes(capacity, 3, stage3), s>>>(g, P3);
+                NL_CUDA_TRY(cudaGetLastError());
+            }
+            P2.tile_list = ctx->fb_list;
+            P2.tile_list_count = ctx->fb_count;
+            ProfScope ps(ctx, PH_PAIRS_LISTED, s);
+            k_pairs_pipe<CLOSE><<<(unsigned)ctx->sm_count, kPipeThreads,
+                                  pipe_smem_bytes(capacity, 2, stage2), s>>>(g, P2);
+            NL_CUDA_TRY(cudaGetLastError());
+        } else {
+            P2.tile_list = nullptr;
+            P2.tile_list_count = nullptr;
             ProfScope ps(ctx, PH_PAIRS, s);
-            k_pairs_pipe<CLOSE><<<(unsigned)ctx->sm_count, kPipeThreads, smem, s>>>(g, P);
+            k_pairs_pipe<CLOSE><<<(unsigned)ctx->sm_count, kPipeThreads,
+                                  pipe_smem_bytes(capacity, 2, stage2), s>>>(g, P2);
             NL_CUDA_TRY(cudaGetLastError());
         }
         *used_fast = 1;
-        // the listed tiles: as many CTAs per SM (up to kListedCtas) as still
-        // give each a stage of twice a typical tile; one CTA with the
-        // largest stage when none does.  A tile beyond its stage is searched
-        // per atom from global memory in the same kernel.
+        // tiles beyond the two-stage launch: as many CTAs per SM (up to
+        // kListedCtas) as still give each a stage of twice a typical tile;
+        // one CTA with the largest stage when none does.  A tile beyond its
+        // stage is searched per atom from global memory in the same kernel.
         cudaFuncAttributes fl;
         NL_CUDA_TRY(cudaFuncGetAttributes(&fl, k_pairs_listed<CLOSE>));
         const long lfixed = (long)listed_fixed_smem(capacity);
@@ -1419,12 +1481,14 @@ cudaError_t launch_pairs_t(nl_ctx *ctx, int64_t n, const CellGrid &g, int32_t ca
         }
         TileParams PL = P;
         PL.stage_max = (int)(lfit < kSlotLimit ? lfit : kSlotLimit);
-        ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
+        PL.fb_list = ctx->fb_list2;
+        PL.fb_count = ctx->fb_count2;
+        ProfScope ps(ctx, PH_PAIRS_LISTED, s);
         k_pairs_listed<CLOSE><<<(unsigned)(ctx->sm_count * lctas), kListedWarps * 32,
                                 sizeof(float4) * (size_t)PL.stage_max + (size_t)lfixed, s>>>(g, PL);
         return cudaGetLastError();
     }
-    ProfScope ps(ctx, PH_PAIRS_FALLBACK, s);
+    ProfScope ps(ctx, PH_PAIRS_LISTED, s);
     const unsigned blocks =
         g.literal ? resident_grid(ctx, k_pairs_per_atom<true, CLOSE>, 128, 0, (n + 127) / 128)
                   : resident_grid(ctx, k_pairs_per_atom<false, CLOSE>, 128, 0, (n + 127) / 128);
