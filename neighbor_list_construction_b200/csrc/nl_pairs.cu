@@ -738,40 +738,44 @@ __device__ __forceinline__ void scan_rows(const float4 *__restrict__ stage,
     float4 c[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) c[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    // rows by dz, then dy: the z distance to a row's column once per dz
 #pragma unroll 1
-    for (int r = 0; r < 25; ++r) {
-        const int dy = r % 5 - 2, dz = r / 5 - 2;
-        const int R = Rh + dy + kSY * dz;
-        float py = dy > 0 ? dy_hi + (float)(dy - 1) * P.side_y
-                          : (dy < 0 ? dy_lo + (float)(-dy - 1) * P.side_y : 0.0f);
+    for (int dz = -2; dz <= 2; ++dz) {
         float pz = dz > 0 ? dz_hi + (float)(dz - 1) * P.side_z
                           : (dz < 0 ? dz_lo + (float)(-dz - 1) * P.side_z : 0.0f);
-        py = fmaxf(py - P.eps, 0.0f);
         pz = fmaxf(pz - P.eps, 0.0f);
-        const float h2 = P.rl2_margin - (py * py + pz * pz);
-        const bool ok = valid && h2 > 0.0f;
-        // approximate root (relative error ~1e-6): the margin absorbs it
-        const float hc = fmaxf(h2, 1e-20f);
-        const float hw = hc * rsqrtf(hc) + P.eps;
-        const int b0 = min(max(__float2int_rd((mxr - hw) * P.inv_bin), 0), nbins - 1);
-        const int b1 = min(max(__float2int_rd((mxr + hw) * P.inv_bin) + 1, 0), nbins);
-        // first staged slot at or above a bin: start of its cell + the cell's
-        // table entry; past the last bin, the row end
-        const uint8_t *tb = tabs + R * kRowTab;
-        const int off = tr.off[R];
-        const int lo = off + tr.cell[R][b0 >> 4] + tb[b0];
-        const int hi = off + (b1 < nbins ? tr.cell[R][b1 >> 4] + tb[b1] : tr.len[R]);
-        const int4 ri = GEN ? rinfo[R] : make_int4(0, 0, 0, 0);
-        if (r == 12) {
-            const int e1 = min(hi, slot);
-            scan_checked<GEN, CLOSE>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, c,
-                                     close_d2, cl, o);
-            const int s1 = max(lo, slot + 1);
-            scan_checked<GEN, CLOSE>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, c,
-                                     close_d2, cl, o);
-        } else {
-            scan_checked<GEN, CLOSE>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, c,
-                                     close_d2, cl, o);
+        const float pz2 = pz * pz;
+#pragma unroll 1
+        for (int dy = -2; dy <= 2; ++dy) {
+            const int R = Rh + dy + kSY * dz;
+            float py = dy > 0 ? dy_hi + (float)(dy - 1) * P.side_y
+                              : (dy < 0 ? dy_lo + (float)(-dy - 1) * P.side_y : 0.0f);
+            py = fmaxf(py - P.eps, 0.0f);
+            const float h2 = P.rl2_margin - (py * py + pz2);
+            const bool ok = valid && h2 > 0.0f;
+            // approximate root (relative error ~1e-6): the margin absorbs it
+            const float hc = fmaxf(h2, 1e-20f);
+            const float hw = hc * rsqrtf(hc) + P.eps;
+            const int b0 = min(max(__float2int_rd((mxr - hw) * P.inv_bin), 0), nbins - 1);
+            const int b1 = min(max(__float2int_rd((mxr + hw) * P.inv_bin) + 1, 0), nbins);
+            // first staged slot at or above a bin: start of its cell + the cell's
+            // table entry; past the last bin, the row end
+            const uint8_t *tb = tabs + R * kRowTab;
+            const int off = tr.off[R];
+            const int lo = off + tr.cell[R][b0 >> 4] + tb[b0];
+            const int hi = off + (b1 < nbins ? tr.cell[R][b1 >> 4] + tb[b1] : tr.len[R]);
+            const int4 ri = GEN ? rinfo[R] : make_int4(0, 0, 0, 0);
+            if (dy == 0 && dz == 0) {   // the home row
+                const int e1 = min(hi, slot);
+                scan_checked<GEN, CLOSE>(stage, lo, ok && e1 > lo ? e1 - lo : 0, me, rl2, ri, Lx, c,
+                                         close_d2, cl, o);
+                const int s1 = max(lo, slot + 1);
+                scan_checked<GEN, CLOSE>(stage, s1, ok && hi > s1 ? hi - s1 : 0, me, rl2, ri, Lx, c,
+                                         close_d2, cl, o);
+            } else {
+                scan_checked<GEN, CLOSE>(stage, lo, ok && hi > lo ? hi - lo : 0, me, rl2, ri, Lx, c,
+                                         close_d2, cl, o);
+            }
         }
     }
     flush_check(o);
