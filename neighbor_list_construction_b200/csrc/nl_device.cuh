@@ -22,7 +22,7 @@ constexpr int kRunMax = 64;                   // longest prefix run the run fini
 
 // Onesweep tile: 256 threads x 8 keys.
 constexpr int kSortThreads = 256;
-constexpr int kSortItems = 8;
+constexpr int kSortItems = 12;
 constexpr int kSortTile = kSortThreads * kSortItems;
 
 // Cell-count scan tile: 256 threads x 16 cells.

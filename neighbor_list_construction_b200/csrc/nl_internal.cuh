@@ -96,10 +96,11 @@ struct ProfScope {
 // Curve keys of all atoms into ctx->keys[0]/vals[0] and the histograms of
 // the top kTopPasses digits into ctx->hist (which must be zero); curve 0
 // Hilbert, 1 Morton.  With a gate: only when *gate != 0, and the histograms
-// of the other digits.
+// of the other digits, and then it also clears zero[0, zero_words).
 cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly,
                         float Lz, float Sx, float Sy, float Sz, int curve, cudaStream_t s,
-                        const uint32_t *gate = nullptr);
+                        const uint32_t *gate = nullptr, uint32_t *zero = nullptr,
+                        int64_t zero_words = 0);
 // Exclusive scan of the 8 histograms in place; with a gate, only when
 // *gate != 0 and only the digits below the top kTopPasses.
 cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s, const uint32_t *gate = nullptr);
@@ -122,8 +123,9 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
                                 float4 *pos_sorted = nullptr);
 // out[k] = (pos[perm[k]].xyz, perm[k]).  Returns at once when `flags` holds
 // kFlagTimeout (perm may then be stale), or when gate is given and *gate == 0.
-cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, float4 *out,
-                          const uint32_t *flags, cudaStream_t s, const uint32_t *gate = nullptr);
+cudaError_t launch_gather(nl_ctx *ctx, int64_t n, const float4 *pos, const int32_t *perm,
+                          float4 *out, const uint32_t *flags, cudaStream_t s,
+                          const uint32_t *gate = nullptr);
 
 // Cell binning of `pos` into ctx->cell_pos (cell order, x-sorted in cells).
 cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const CellGrid &g,

@@ -144,11 +144,13 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
                                               float Sy, float Sz, uint64_t *__restrict__ keys,
                                               uint32_t *__restrict__ vals,
                                               uint32_t *__restrict__ hist,
-                                              const uint32_t *gate)
+                                              const uint32_t *gate, uint32_t *zero,
+                                              int64_t zero_words)
 {
     // First pass: the histograms of the top kTopPasses digits, which the
     // fast sort uses.  Gated recompute (the full sort's keys): only when the
-    // gate is set, with the histograms of the remaining low digits.
+    // gate is set, with the histograms of the remaining low digits; it also
+    // clears zero[0, zero_words) (the full sort's look-back status).
     const bool recompute = gate != nullptr;
     if (recompute && ld_volatile_u32(gate) == 0u) return;
     constexpr int kLow = kKeyPasses - kTopPasses;
@@ -164,6 +166,8 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
     for (int i = threadIdx.x; i < kKeyPasses * kRadixBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < zero_words; i += stride)
+        zero[i] = 0u;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const float4 p = pos[i];
         const uint32_t qx = quantize(wrap_coord(p.x, Lx), Sx);
@@ -216,21 +220,23 @@ k_gather(int64_t n, const float4 *__restrict__ pos, const int32_t *__restrict__ 
 {
     if (gate && ld_volatile_u32(gate) == 0u) return;   // gated gather not needed
     if (timed_out(flags)) return;   // perm may not be a permutation
-    const int64_t base = (int64_t)blockIdx.x * (256 * kGatherItems) + threadIdx.x;
-    int32_t i[kGatherItems];
+    for (int64_t base = (int64_t)blockIdx.x * (256 * kGatherItems) + threadIdx.x; base < n;
+         base += (int64_t)gridDim.x * (256 * kGatherItems)) {
+        int32_t i[kGatherItems];
 #pragma unroll
-    for (int u = 0; u < kGatherItems; ++u) {
-        const int64_t k = base + 256 * u;
-        i[u] = k < n ? perm[k] : -1;
-    }
-    float4 p[kGatherItems];
+        for (int u = 0; u < kGatherItems; ++u) {
+            const int64_t k = base + 256 * u;
+            i[u] = k < n ? perm[k] : -1;
+        }
+        float4 p[kGatherItems];
 #pragma unroll
-    for (int u = 0; u < kGatherItems; ++u)
-        if (i[u] >= 0) p[u] = pos[i[u]];
+        for (int u = 0; u < kGatherItems; ++u)
+            if (i[u] >= 0) p[u] = pos[i[u]];
 #pragma unroll
-    for (int u = 0; u < kGatherItems; ++u) {
-        const int64_t k = base + 256 * u;
-        if (k < n) out[k] = make_float4(p[u].x, p[u].y, p[u].z, __int_as_float(i[u]));
+        for (int u = 0; u < kGatherItems; ++u) {
+            const int64_t k = base + 256 * u;
+            if (k < n) out[k] = make_float4(p[u].x, p[u].y, p[u].z, __int_as_float(i[u]));
+        }
     }
 }
 
@@ -238,7 +244,7 @@ k_gather(int64_t n, const float4 *__restrict__ pos, const int32_t *__restrict__ 
 
 cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, float Ly, float Lz,
                         float Sx, float Sy, float Sz, int curve, cudaStream_t s,
-                        const uint32_t *gate)
+                        const uint32_t *gate, uint32_t *zero, int64_t zero_words)
 {
     if (n <= 0) return cudaSuccess;
     const int64_t want = (n + 255) / 256;
@@ -246,10 +252,12 @@ cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
                                        : resident_grid(ctx, k_keys<1>, 256, 0, want);
     if (curve == 0)
         k_keys<0><<<(unsigned)blocks, 256, 0, s>>>(pos, n, Lx, Ly, Lz, Sx, Sy, Sz, ctx->keys[0],
-                                                    ctx->vals[0], ctx->hist, gate);
+                                                    ctx->vals[0], ctx->hist, gate, zero,
+                                                    zero_words);
     else
         k_keys<1><<<(unsigned)blocks, 256, 0, s>>>(pos, n, Lx, Ly, Lz, Sx, Sy, Sz, ctx->keys[0],
-                                                    ctx->vals[0], ctx->hist, gate);
+                                                    ctx->vals[0], ctx->hist, gate, zero,
+                                                    zero_words);
     return cudaGetLastError();
 }
 
@@ -261,12 +269,14 @@ cudaError_t launch_hist_scan(nl_ctx *ctx, cudaStream_t s, const uint32_t *gate)
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather(int64_t n, const float4 *pos, const int32_t *perm, float4 *out,
-                          const uint32_t *flags, cudaStream_t s, const uint32_t *gate)
+cudaError_t launch_gather(nl_ctx *ctx, int64_t n, const float4 *pos, const int32_t *perm,
+                          float4 *out, const uint32_t *flags, cudaStream_t s, const uint32_t *gate)
 {
     if (n <= 0) return cudaSuccess;
-    const int64_t blocks = (n + 256 * kGatherItems - 1) / (256 * kGatherItems);
-    k_gather<<<(unsigned)blocks, 256, 0, s>>>(n, pos, perm, out, flags, gate);
+    const int64_t want = (n + 256 * kGatherItems - 1) / (256 * kGatherItems);
+    // gated: one resident wave, so a clear gate costs few CTAs
+    const unsigned blocks = gate ? resident_grid(ctx, k_gather, 256, 0, want) : (unsigned)want;
+    k_gather<<<blocks, 256, 0, s>>>(n, pos, perm, out, flags, gate);
     return cudaGetLastError();
 }
 

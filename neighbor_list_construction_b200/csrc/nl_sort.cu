@@ -12,16 +12,17 @@
 // redoes the whole order; when the gate is clear those launches return at
 // once.
 //
-// One kernel launch per 8-bit digit.  Each CTA takes the next tile from an
-// atomic ticket (so a tile only ever waits on tiles whose CTAs are already
-// running), ranks its keys stably with warp match/popc, publishes its per-
-// digit counts, and finds the counts of all earlier tiles by decoupled
-// look-back over per-(tile, digit) status words.  The global digit starts
-// come from histograms made by the key kernel (those of the low digits only
-// by its gated recompute).  Waits on a status
-// word are bounded: past kSpinLimit polls the kernel records kFlagTimeout
-// and carries on, so a stuck predecessor cannot hang the device; every later
-// pass, the run finish and the gather then return at entry (timed_out).
+// One kernel launch per 8-bit digit, one resident wave of CTAs.  A CTA takes
+// tiles of kSortTile keys from an atomic ticket until none is left (so a tile
+// only ever waits on tiles whose CTAs are already running), ranks each
+// tile's keys stably with warp match/popc, publishes its per-digit counts,
+// and finds the counts of all earlier tiles by decoupled look-back over
+// per-(tile, digit) status words.  The global digit starts come from
+// histograms made by the key kernel (those of the low digits only by its
+// gated recompute).  Waits on a status word are bounded: past kSpinLimit
+// polls the kernel records kFlagTimeout and carries on, so a stuck
+// predecessor cannot hang the device; every later pass, the run finish and
+// the gather then return at entry (timed_out).
 #include "nl_internal.cuh"
 
 namespace nl {
@@ -32,7 +33,7 @@ constexpr int kLookBack = 8;   // predecessor status words read per look-back ro
 constexpr size_t kSortDynSmem = (size_t)kSortTile * (sizeof(uint64_t) + sizeof(uint32_t));
 
 template <bool WRITE_KEYS>
-__global__ void __launch_bounds__(kSortThreads, 4)
+__global__ void __launch_bounds__(kSortThreads, 3)
 k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
            uint64_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out, int64_t n,
            int shift, const uint32_t *__restrict__ digit_start, uint32_t *status,
@@ -52,134 +53,139 @@ k_onesweep(const uint64_t *__restrict__ keys_in, const uint32_t *__restrict__ va
     __shared__ uint32_t s_tile;
 
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    if (t == 0) s_tile = atomicAdd(ticket, 1u);
-    for (int i = t; i < kWarps * kRadixBins; i += kSortThreads) (&s_whist[0][0])[i] = 0u;
-    __syncthreads();
-    const uint32_t tile = s_tile;
-    const int64_t base = (int64_t)tile * kSortTile;
+    const int64_t ntiles = (n + kSortTile - 1) / kSortTile;
+    for (;;) {   // tiles by ticket until none is left
+        if (t == 0) s_tile = atomicAdd(ticket, 1u);
+        for (int i = t; i < kWarps * kRadixBins; i += kSortThreads) (&s_whist[0][0])[i] = 0u;
+        __syncthreads();
+        const uint32_t tile = s_tile;
+        if ((int64_t)tile >= ntiles) return;
+        const int64_t base = (int64_t)tile * kSortTile;
 
-    // warp w owns elements [base + Ew, base + Ew + E), E = 32 kSortItems; item
-    // k of lane l is element base + Ew + 32k + l, so (k, lane) order is index
-    // order.
-    uint64_t key[kSortItems];
-    uint32_t val[kSortItems];
-    uint32_t rank[kSortItems];
+        // warp w owns elements [base + Ew, base + Ew + E), E = 32 kSortItems; item
+        // k of lane l is element base + Ew + 32k + l, so (k, lane) order is index
+        // order.
+        uint64_t key[kSortItems];
+        uint32_t val[kSortItems];
+        uint32_t rank[kSortItems];
 #pragma unroll
-    for (int k = 0; k < kSortItems; ++k) {
-        const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
-        if (idx < n) {
-            key[k] = keys_in[idx];
-            val[k] = vals_in[idx];
+        for (int k = 0; k < kSortItems; ++k) {
+            const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
+            if (idx < n) {
+                key[k] = keys_in[idx];
+                val[k] = vals_in[idx];
+            } else {
+                key[k] = ~0ull;  // digit 255 in every pass, never written
+                val[k] = 0u;
+            }
+        }
+        const uint32_t lt = lanemask_lt();
+#pragma unroll
+        for (int k = 0; k < kSortItems; ++k) {
+            const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
+            const uint32_t d = idx < n ? (uint32_t)(key[k] >> shift) & 0xffu : 0x100u;
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            const int leader = __ffs(peers) - 1;
+            uint32_t before = 0u;
+            if (lane == leader && d < 0x100u) {
+                before = s_whist[w][d];
+                s_whist[w][d] = before + __popc(peers);
+            }
+            before = __shfl_sync(0xffffffffu, before, leader);
+            rank[k] = before + __popc(peers & lt);
+            __syncwarp();
+        }
+        __syncthreads();
+
+        // thread t now owns digit t
+        uint32_t cnt = 0u;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+            const uint32_t c = s_whist[ww][t];
+            s_whist[ww][t] = cnt;
+            cnt += c;
+        }
+        uint32_t *st = status + (size_t)tile * kRadixBins + t;
+        uint32_t excl = 0u;
+        if (tile == 0) {
+            st_volatile_u32(st, kStPrefix | cnt);
         } else {
-            key[k] = ~0ull;  // digit 255 in every pass, never written
-            val[k] = 0u;
-        }
-    }
-    const uint32_t lt = lanemask_lt();
+            st_volatile_u32(st, kStAggregate | cnt);
+            // look back kLookBack predecessors per round: their status words are
+            // read with independent loads, then taken in order until a prefix
+            // (done) or a word not yet published (poll again from there)
+            int64_t j = (int64_t)tile - 1;
+            uint32_t spins = 0u;
+            bool done = false;
+            while (!done) {
+                uint32_t sw[kLookBack];
 #pragma unroll
-    for (int k = 0; k < kSortItems; ++k) {
-        const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
-        const uint32_t d = idx < n ? (uint32_t)(key[k] >> shift) & 0xffu : 0x100u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, d);
-        const int leader = __ffs(peers) - 1;
-        uint32_t before = 0u;
-        if (lane == leader && d < 0x100u) {
-            before = s_whist[w][d];
-            s_whist[w][d] = before + __popc(peers);
-        }
-        before = __shfl_sync(0xffffffffu, before, leader);
-        rank[k] = before + __popc(peers & lt);
-        __syncwarp();
-    }
-    __syncthreads();
-
-    // thread t now owns digit t
-    uint32_t cnt = 0u;
+                for (int q = 0; q < kLookBack; ++q)
+                    sw[q] = j - q >= 0 ? ld_volatile_u32(status + (size_t)(j - q) * kRadixBins + t)
+                                       : kStPrefix;
+                int q = 0;
 #pragma unroll
-    for (int ww = 0; ww < kWarps; ++ww) {
-        const uint32_t c = s_whist[ww][t];
-        s_whist[ww][t] = cnt;
-        cnt += c;
-    }
-    uint32_t *st = status + (size_t)tile * kRadixBins + t;
-    uint32_t excl = 0u;
-    if (tile == 0) {
-        st_volatile_u32(st, kStPrefix | cnt);
-    } else {
-        st_volatile_u32(st, kStAggregate | cnt);
-        // look back kLookBack predecessors per round: their status words are
-        // read with independent loads, then taken in order until a prefix
-        // (done) or a word not yet published (poll again from there)
-        int64_t j = (int64_t)tile - 1;
-        uint32_t spins = 0u;
-        bool done = false;
-        while (!done) {
-            uint32_t sw[kLookBack];
-#pragma unroll
-            for (int q = 0; q < kLookBack; ++q)
-                sw[q] = j - q >= 0 ? ld_volatile_u32(status + (size_t)(j - q) * kRadixBins + t)
-                                   : kStPrefix;
-            int q = 0;
-#pragma unroll
-            for (int qq = 0; qq < kLookBack; ++qq) {
-                if (q == qq && !done) {
-                    const uint32_t f = sw[qq] & ~kStValue;
-                    if (f != 0u) {
-                        excl += sw[qq] & kStValue;
-                        done = f == kStPrefix;
-                        ++q;
+                for (int qq = 0; qq < kLookBack; ++qq) {
+                    if (q == qq && !done) {
+                        const uint32_t f = sw[qq] & ~kStValue;
+                        if (f != 0u) {
+                            excl += sw[qq] & kStValue;
+                            done = f == kStPrefix;
+                            ++q;
+                        }
                     }
                 }
-            }
-            j -= q;
-            if (!done && q < kLookBack) {   // word j not yet published
-                if (++spins >= kSpinLimit) {
-                    atomicOr(flags, kFlagTimeout);
-                    break;
+                j -= q;
+                if (!done && q < kLookBack) {   // word j not yet published
+                    if (++spins >= kSpinLimit) {
+                        atomicOr(flags, kFlagTimeout);
+                        break;
+                    }
+                    if (spins > 64u) __nanosleep(64);
                 }
-                if (spins > 64u) __nanosleep(64);
+            }
+            st_volatile_u32(st, kStPrefix | ((excl + cnt) & kStValue));
+        }
+        s_gbase[t] = digit_start[t] + excl;
+
+        // exclusive scan of the tile's digit counts
+        uint32_t x = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) s_wtot[w] = x;
+        __syncthreads();
+        uint32_t before = 0u;
+        for (int i = 0; i < w; ++i) before += s_wtot[i];
+        s_tdig[t] = before + x - cnt;
+        __syncthreads();
+
+        // stage the tile in digit order
+#pragma unroll
+        for (int k = 0; k < kSortItems; ++k) {
+            const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
+            if (idx < n) {
+                const uint32_t d = (uint32_t)(key[k] >> shift) & 0xffu;
+                const uint32_t p = s_tdig[d] + s_whist[w][d] + rank[k];
+                s_keys[p] = key[k];
+                s_vals[p] = val[k];
             }
         }
-        st_volatile_u32(st, kStPrefix | ((excl + cnt) & kStValue));
-    }
-    s_gbase[t] = digit_start[t] + excl;
+        __syncthreads();
 
-    // exclusive scan of the tile's digit counts
-    uint32_t x = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_wtot[w] = x;
-    __syncthreads();
-    uint32_t before = 0u;
-    for (int i = 0; i < w; ++i) before += s_wtot[i];
-    s_tdig[t] = before + x - cnt;
-    __syncthreads();
-
-    // stage the tile in digit order
-#pragma unroll
-    for (int k = 0; k < kSortItems; ++k) {
-        const int64_t idx = base + (int64_t)w * (32 * kSortItems) + k * 32 + lane;
-        if (idx < n) {
-            const uint32_t d = (uint32_t)(key[k] >> shift) & 0xffu;
-            const uint32_t p = s_tdig[d] + s_whist[w][d] + rank[k];
-            s_keys[p] = key[k];
-            s_vals[p] = val[k];
+        // runs of equal digits go to consecutive global addresses
+        const int64_t rem = n - base;
+        const int tile_n = rem < kSortTile ? (int)rem : kSortTile;
+        for (int p = t; p < tile_n; p += kSortThreads) {
+            const uint64_t k = s_keys[p];
+            const uint32_t d = (uint32_t)(k >> shift) & 0xffu;
+            const uint32_t out = s_gbase[d] + ((uint32_t)p - s_tdig[d]);
+            if (WRITE_KEYS) keys_out[out] = k;
+            vals_out[out] = s_vals[p];
         }
-    }
-    __syncthreads();
-
-    // runs of equal digits go to consecutive global addresses
-    const int64_t rem = n - base;
-    const int tile_n = rem < kSortTile ? (int)rem : kSortTile;
-    for (int p = t; p < tile_n; p += kSortThreads) {
-        const uint64_t k = s_keys[p];
-        const uint32_t d = (uint32_t)(k >> shift) & 0xffu;
-        const uint32_t out = s_gbase[d] + ((uint32_t)p - s_tdig[d]);
-        if (WRITE_KEYS) keys_out[out] = k;
-        vals_out[out] = s_vals[p];
+        __syncthreads();   // the next tile reuses the shared arrays
     }
 }
 
@@ -269,20 +275,28 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
 {
     if (n <= 0) return cudaSuccess;
     const int64_t tiles = (n + kSortTile - 1) / kSortTile;
-    // kSortDynSmem (24 KB) is below the default dynamic shared-memory limit,
-    // so the passes need no per-device attribute
-    static_assert(kSortDynSmem <= 48 * 1024, "onesweep tile needs the opt-in shared memory");
-    NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_status, 0,
-                                sizeof(uint32_t) * kStatusPasses * tiles * kRadixBins, s));
+    // the tile (36 KB) and the static arrays (10 KB) fit the 48 KB a CTA gets
+    // without opt-in, so the passes need no per-device attribute
+    static_assert(kSortDynSmem + 4 * (kWarps * kRadixBins + 2 * kRadixBins + kWarps + 1) + 64 <=
+                      48 * 1024,
+                  "onesweep tile needs the opt-in shared memory");
+    // look-back status: the fast path's slots now; the full sort's slots are
+    // cleared by its gated key recompute, so a clear gate costs no clearing
+    const size_t slot_words = (size_t)tiles * kRadixBins;
+    NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_status + kKeyPasses * slot_words, 0,
+                                sizeof(uint32_t) * kTopPasses * slot_words, s));
     NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_ctr, 0, sizeof(uint32_t) * kStatusPasses, s));
     NL_CUDA_TRY(cudaMemsetAsync(ctx->sort_gate, 0, sizeof(uint32_t), s));
+    // every pass is one resident wave whose CTAs loop over tile tickets, so
+    // a gated pass whose gate is clear costs one wave of CTAs that return
+    const unsigned grid = resident_grid(ctx, k_onesweep<true>, kSortThreads, kSortDynSmem, tiles);
     // fast path: the top kTopPasses digits, then the prefix runs
     int src = 0;
     for (int q = 0; q < kTopPasses; ++q) {
         const int p = kKeyPasses - kTopPasses + q;   // digit
         const int slot = kKeyPasses + q;             // status slot of the fast path
-        uint32_t *status = ctx->sort_status + (size_t)slot * tiles * kRadixBins;
-        k_onesweep<true><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
+        uint32_t *status = ctx->sort_status + (size_t)slot * slot_words;
+        k_onesweep<true><<<grid, kSortThreads, kSortDynSmem, s>>>(
             ctx->keys[src], ctx->vals[src], ctx->keys[1 - src], ctx->vals[1 - src], n,
             kRadixBits * p, ctx->hist + p * kRadixBins, status, ctx->sort_ctr + slot, ctx->flags,
             nullptr);
@@ -297,21 +311,22 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
         NL_CUDA_TRY(cudaGetLastError());
     }
     // full sort, gated: runs only when a prefix run was too long
-    NL_CUDA_TRY(launch_keys(ctx, rk.n, rk.pos, rk.Lx, rk.Ly, rk.Lz, rk.Sx, rk.Sy, rk.Sz, rk.curve, s,
-                            ctx->sort_gate));
+    NL_CUDA_TRY(launch_keys(ctx, rk.n, rk.pos, rk.Lx, rk.Ly, rk.Lz, rk.Sx, rk.Sy, rk.Sz,
+                            rk.curve, s, ctx->sort_gate, ctx->sort_status,
+                            (int64_t)(kKeyPasses * slot_words)));
     NL_CUDA_TRY(launch_hist_scan(ctx, s, ctx->sort_gate));
     src = 0;
     for (int p = 0; p < kKeyPasses; ++p) {
         const bool last = p == kKeyPasses - 1;
         uint64_t *ko = last ? (keys_final ? keys_final : ctx->keys[1 - src]) : ctx->keys[1 - src];
         uint32_t *vo = last ? vals_final : ctx->vals[1 - src];
-        uint32_t *status = ctx->sort_status + (size_t)p * tiles * kRadixBins;
+        uint32_t *status = ctx->sort_status + (size_t)p * slot_words;
         if (last && !keys_final)
-            k_onesweep<false><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
+            k_onesweep<false><<<grid, kSortThreads, kSortDynSmem, s>>>(
                 ctx->keys[src], ctx->vals[src], ko, vo, n, kRadixBits * p,
                 ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags, ctx->sort_gate);
         else
-            k_onesweep<true><<<(unsigned)tiles, kSortThreads, kSortDynSmem, s>>>(
+            k_onesweep<true><<<grid, kSortThreads, kSortDynSmem, s>>>(
                 ctx->keys[src], ctx->vals[src], ko, vo, n, kRadixBits * p,
                 ctx->hist + p * kRadixBins, status, ctx->sort_ctr + p, ctx->flags, ctx->sort_gate);
         NL_CUDA_TRY(cudaGetLastError());
@@ -319,7 +334,7 @@ cudaError_t launch_radix_passes(nl_ctx *ctx, int64_t n, uint64_t *keys_final,
     }
     // the gather of the full sort's order, gated like its passes
     if (pos_sorted)
-        NL_CUDA_TRY(launch_gather(n, rk.pos, reinterpret_cast<const int32_t *>(vals_final),
+        NL_CUDA_TRY(launch_gather(ctx, n, rk.pos, reinterpret_cast<const int32_t *>(vals_final),
                                   pos_sorted, ctx->flags, s, ctx->sort_gate));
     return cudaSuccess;
 }
