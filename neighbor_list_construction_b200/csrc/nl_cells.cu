@@ -15,7 +15,7 @@ namespace {
 constexpr int kCellSortMax = 255;
 // In-cell sort: cells per CTA, atoms a CTA stages at once, threads.
 constexpr int kSortCells = 128;
-constexpr int kSortCap = 2048;
+constexpr int kSortCap = 1024;
 constexpr int kSortThreads2 = 256;
 
 __global__ void __launch_bounds__(256)

@@ -325,6 +325,9 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                                       float sy, float sz, float close_d2, CloseAcc &cl,
                                       uint32_t &bp)
 {
+    // (me.x, me.y) as one packed pair for the f32x2 forms: x in the low half
+    const unsigned long long mxy =
+        ((unsigned long long)__float_as_uint(me.y) << 32) | __float_as_uint(me.x);
     if (GEN && CLOSE)
         asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3, qc;\n\t"
                      "setp.gt.s32 q0, %19, 0;\n\t"
@@ -476,7 +479,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
                      : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(sx0), "f"(sx1), "f"(sx2), "f"(sx3), "f"(sy), "f"(sz));
     if (!GEN && CLOSE)
-        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3, qc;\n\t"
+        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .b64 cxy, dxy;\n\t.reg .pred q0, q1, q2, q3, qc;\n\t"
                      "setp.gt.s32 q0, %19, 0;\n\t"
                      "setp.gt.s32 q1, %19, 1;\n\t"
                      "setp.gt.s32 q2, %19, 2;\n\t"
@@ -485,11 +488,11 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%20+16];\n\t"
                      "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%20+32];\n\t"
                      "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%20+48];\n\t"
-                     "sub.rn.f32 dx, %1, %21;\n\t"
-                     "sub.rn.f32 dy, %2, %22;\n\t"
+                     "mov.b64 cxy, {%1, %2};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %26;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %3, %23;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
@@ -499,11 +502,11 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "@q0 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q0;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
-                     "sub.rn.f32 dx, %5, %21;\n\t"
-                     "sub.rn.f32 dy, %6, %22;\n\t"
+                     "mov.b64 cxy, {%5, %6};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %26;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %7, %23;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
@@ -513,11 +516,11 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "@q1 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q1;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
-                     "sub.rn.f32 dx, %9, %21;\n\t"
-                     "sub.rn.f32 dy, %10, %22;\n\t"
+                     "mov.b64 cxy, {%9, %10};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %26;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %11, %23;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
@@ -527,11 +530,11 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "@q2 min.f32 %17, %17, dx;\n\t"
                      "setp.lt.and.f32 qc, dx, %25, q2;\n\t"
                      "@qc add.u32 %18, %18, 1;\n\t"
-                     "sub.rn.f32 dx, %13, %21;\n\t"
-                     "sub.rn.f32 dy, %14, %22;\n\t"
+                     "mov.b64 cxy, {%13, %14};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %26;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %15, %23;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
@@ -543,9 +546,10 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "@qc add.u32 %18, %18, 1;\n\t"
                      "}"
                      : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w), "+f"(cl.mn), "+r"(cl.nc)
-                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(close_d2));
+                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "f"(close_d2),
+                       "l"(mxy));
     if (!GEN && !CLOSE)
-        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .pred q0, q1, q2, q3;\n\t"
+        asm volatile("{\n\t.reg .f32 dx, dy, dz;\n\t.reg .b64 cxy, dxy;\n\t.reg .pred q0, q1, q2, q3;\n\t"
                      "setp.gt.s32 q0, %17, 0;\n\t"
                      "setp.gt.s32 q1, %17, 1;\n\t"
                      "setp.gt.s32 q2, %17, 2;\n\t"
@@ -554,44 +558,44 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "@q1 ld.shared.v4.f32 {%5, %6, %7, %8}, [%18+16];\n\t"
                      "@q2 ld.shared.v4.f32 {%9, %10, %11, %12}, [%18+32];\n\t"
                      "@q3 ld.shared.v4.f32 {%13, %14, %15, %16}, [%18+48];\n\t"
-                     "sub.rn.f32 dx, %1, %19;\n\t"
-                     "sub.rn.f32 dy, %2, %20;\n\t"
+                     "mov.b64 cxy, {%1, %2};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %23;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %3, %21;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q0, dx, %22, q0;\n\t"
                      "@q0 st.shared.b32 [%0], %4;\n\t"
                      "@q0 add.u32 %0, %0, 128;\n\t"
-                     "sub.rn.f32 dx, %5, %19;\n\t"
-                     "sub.rn.f32 dy, %6, %20;\n\t"
+                     "mov.b64 cxy, {%5, %6};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %23;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %7, %21;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q1, dx, %22, q1;\n\t"
                      "@q1 st.shared.b32 [%0], %8;\n\t"
                      "@q1 add.u32 %0, %0, 128;\n\t"
-                     "sub.rn.f32 dx, %9, %19;\n\t"
-                     "sub.rn.f32 dy, %10, %20;\n\t"
+                     "mov.b64 cxy, {%9, %10};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %23;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %11, %21;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
                      "setp.lt.and.f32 q2, dx, %22, q2;\n\t"
                      "@q2 st.shared.b32 [%0], %12;\n\t"
                      "@q2 add.u32 %0, %0, 128;\n\t"
-                     "sub.rn.f32 dx, %13, %19;\n\t"
-                     "sub.rn.f32 dy, %14, %20;\n\t"
+                     "mov.b64 cxy, {%13, %14};\n\t"
+                     "sub.rn.f32x2 dxy, cxy, %23;\n\t"
+                     "mul.rn.f32x2 dxy, dxy, dxy;\n\t"
+                     "mov.b64 {dx, dy}, dxy;\n\t"
                      "sub.rn.f32 dz, %15, %21;\n\t"
-                     "mul.rn.f32 dx, dx, dx;\n\t"
-                     "mul.rn.f32 dy, dy, dy;\n\t"
                      "mul.rn.f32 dz, dz, dz;\n\t"
                      "add.rn.f32 dx, dx, dy;\n\t"
                      "add.rn.f32 dx, dx, dz;\n\t"
@@ -600,7 +604,7 @@ __device__ __forceinline__ void scan4(uint32_t addr, int act, float4 (&c)[4], co
                      "@q3 add.u32 %0, %0, 128;\n\t"
                      "}"
                      : "+r"(bp), "+f"(c[0].x), "+f"(c[0].y), "+f"(c[0].z), "+f"(c[0].w), "+f"(c[1].x), "+f"(c[1].y), "+f"(c[1].z), "+f"(c[1].w), "+f"(c[2].x), "+f"(c[2].y), "+f"(c[2].z), "+f"(c[2].w), "+f"(c[3].x), "+f"(c[3].y), "+f"(c[3].z), "+f"(c[3].w)
-                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2));
+                     : "r"(act), "r"(addr), "f"(me.x), "f"(me.y), "f"(me.z), "f"(rl2), "l"(mxy));
     (void)close_d2;
     (void)cl;
     (void)sx0;

@@ -272,6 +272,56 @@ def test_build_cutoff_shell_pairs(ctx, oracle):
     gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
 
 
+def test_build_pairs_that_a_fused_sum_would_flip(ctx, oracle):
+    """The predicate is r2 = (dx*dx + dy*dy) + dz*dz with every product and
+    sum rounded to fp32.  Pairs are chosen (from many near the cutoff radius)
+    whose decision r2 < rl2 changes if either sum were fused with the product
+    before it (one rounding instead of two); the GPU rows must equal the
+    oracle's (unfused) on all of them."""
+    rng = np.random.default_rng(29)
+    L, cutoff, skin = 96.0, 5.75, 1.0
+    rl2 = np.float32(np.float32(cutoff + skin) * np.float32(cutoff + skin))
+    rl = np.float64(np.float32(cutoff + skin))
+    nb = 20000
+    base = rng.random((nb, 3)) * L
+    u = rng.normal(size=(nb, 3))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    r = rl * (1.0 + rng.uniform(-3e-7, 3e-7, size=(nb, 1)))
+    a = np.float32(base)
+    b = np.float32(base + r * u) % np.float32(L)
+    d = (b - a).astype(np.float32)                       # fp32 differences
+    d -= np.float32(L) * np.round(d / np.float32(L)).astype(np.float32)
+    sq = (d * d).astype(np.float32)
+    s_xy = (sq[:, 0] + sq[:, 1]).astype(np.float32)
+    plain = (s_xy + sq[:, 2]).astype(np.float32)
+
+    def fma(x, y, z):   # one rounding (exact product in fp64, then to fp32)
+        return np.float32(np.float64(x) * np.float64(y) + np.float64(z))
+
+    f_xy = fma(d[:, 0], d[:, 0], sq[:, 1])
+    fused = [(f_xy + sq[:, 2]).astype(np.float32), fma(d[:, 2], d[:, 2], s_xy),
+             fma(d[:, 2], d[:, 2], f_xy)]
+    flips = np.zeros(nb, bool)
+    for f in fused:
+        flips |= (f < rl2) != (plain < rl2)
+    assert flips.sum() >= 50                              # the test has teeth
+    pos = np.zeros((2 * nb, 4), np.float32)
+    pos[:nb, :3] = a
+    pos[nb:, :3] = b
+    box = np.array([L, L, L], np.float32)
+    nbr, cnt, st = gpu_build(ctx, pos, box, cutoff, skin, 256)
+    o_nbr, o_cnt, o_ov = oracle.build(pos, box, cutoff, skin, 256)
+    assert st == (1 if o_ov else 0)
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt)
+    # each flip-prone pair: the oracle's r2 is the plain sum, and the pair is
+    # in both rows exactly when that sum is below rl2
+    can = gu.canonical(np.asarray(nbr))
+    for k in np.nonzero(flips)[0]:
+        assert oracle.r2(a[k], b[k], box) == plain[k]
+        inside = plain[k] < rl2
+        assert (nb + k in can[k]) == inside and (k in can[nb + k]) == inside
+
+
 def test_build_mixed_density_uses_both_paths(ctx, nl, oracle):
     """A dense slab whose tiles overflow the shared-memory stage (listed for
     the per-atom search) beside sparse tiles that are staged; rows with more
