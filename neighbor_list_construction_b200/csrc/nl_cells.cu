@@ -15,8 +15,13 @@ namespace {
 constexpr int kCellSortMax = 255;
 // In-cell sort: cells per CTA, atoms a CTA stages at once, threads.
 constexpr int kSortCells = 128;
-constexpr int kSortCap = 1024;
+constexpr int kSortCap = 768;
 constexpr int kSortThreads2 = 256;
+
+// Binning kernels: each warp takes kBinUnroll groups of 32 consecutive
+// atoms per round and issues all their loads (and atomics) before using any,
+// so several memory round trips are in flight per warp.
+constexpr int kBinUnroll = 4;
 
 __global__ void __launch_bounds__(256)
 k_bin_count(const float4 *__restrict__ pos, int64_t n, CellGrid g, uint32_t *__restrict__ atom_cell,
@@ -25,30 +30,41 @@ k_bin_count(const float4 *__restrict__ pos, int64_t n, CellGrid g, uint32_t *__r
 {
     n = atoms_of(g, n);
     const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) - lane;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t stride = ((int64_t)gridDim.x * blockDim.x) * kBinUnroll;
     const uint32_t lt = lanemask_lt();
-    for (int64_t b = warp0; b < n; b += stride) {
-        const int64_t i = b + lane;
-        uint32_t c = 0xffffffffu;
-        if (i < n) {
-            const float4 p = pos[i];
-            ref[i] = p;
-            const int cx = cell_coord(wrap_coord(p.x, g.Lx), g.Tx, g.nx);
-            const int cy = cell_coord(wrap_coord(p.y, g.Ly), g.Ty, g.ny);
-            const int cz = cell_coord(wrap_coord(p.z, g.Lz), g.Tz, g.nz);
-            c = (uint32_t)(((int64_t)cz * g.ny + cy) * g.nx + cx);
+    for (int64_t b = warp * 32 * kBinUnroll; b < n; b += stride) {
+        uint32_t c[kBinUnroll];
+#pragma unroll
+        for (int u = 0; u < kBinUnroll; ++u) {
+            const int64_t i = b + 32 * u + lane;
+            c[u] = 0xffffffffu;
+            if (i < n) {
+                const float4 p = pos[i];
+                ref[i] = p;
+                const int cx = cell_coord(wrap_coord(p.x, g.Lx), g.Tx, g.nx);
+                const int cy = cell_coord(wrap_coord(p.y, g.Ly), g.Ty, g.ny);
+                const int cz = cell_coord(wrap_coord(p.z, g.Lz), g.Tz, g.nz);
+                c[u] = (uint32_t)(((int64_t)cz * g.ny + cy) * g.nx + cx);
+            }
         }
-        // warp-aggregated increment: one atomic per distinct cell
-        const uint32_t peers = __match_any_sync(0xffffffffu, c);
-        const int leader = __ffs(peers) - 1;
-        uint32_t old = 0u;
-        if (lane == leader && c != 0xffffffffu)
-            old = (uint32_t)atomicAdd(&cell_count[c], __popc(peers));
-        old = __shfl_sync(0xffffffffu, old, leader);
-        if (i < n) {
-            atom_cell[i] = c;
-            atom_rank[i] = old + __popc(peers & lt);
+        // warp-aggregated increments: one atomic per distinct cell and group
+        uint32_t peers[kBinUnroll], old[kBinUnroll];
+#pragma unroll
+        for (int u = 0; u < kBinUnroll; ++u) {
+            peers[u] = __match_any_sync(0xffffffffu, c[u]);
+            old[u] = 0u;
+            if (lane == __ffs(peers[u]) - 1 && c[u] != 0xffffffffu)
+                old[u] = (uint32_t)atomicAdd(&cell_count[c[u]], __popc(peers[u]));
+        }
+#pragma unroll
+        for (int u = 0; u < kBinUnroll; ++u) {
+            const int64_t i = b + 32 * u + lane;
+            const uint32_t o = __shfl_sync(0xffffffffu, old[u], __ffs(peers[u]) - 1);
+            if (i < n) {
+                atom_cell[i] = c[u];
+                atom_rank[i] = o + __popc(peers[u] & lt);
+            }
         }
     }
 }
@@ -136,18 +152,42 @@ k_bin_scatter(const float4 *__restrict__ pos, int64_t n, CellGrid g,
 {
     if (timed_out(flags)) return;   // cell starts may not be monotonic
     n = atoms_of(g, n);
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-        const float4 p = pos[i];
-        const int64_t dst = (int64_t)cell_start[atom_cell[i]] + atom_rank[i];
-        cell_pos[dst] = make_float4(wrap_coord(p.x, g.Lx), wrap_coord(p.y, g.Ly),
-                                    wrap_coord(p.z, g.Lz), __int_as_float((int)i));
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t stride = ((int64_t)gridDim.x * blockDim.x) * kBinUnroll;
+    for (int64_t b = warp * 32 * kBinUnroll; b < n; b += stride) {
+        float4 p[kBinUnroll];
+        uint32_t c[kBinUnroll], r[kBinUnroll];
+#pragma unroll
+        for (int u = 0; u < kBinUnroll; ++u) {
+            const int64_t i = b + 32 * u + lane;
+            if (i < n) {
+                p[u] = pos[i];
+                c[u] = atom_cell[i];
+                r[u] = atom_rank[i];
+            }
+        }
+        int32_t st[kBinUnroll];
+#pragma unroll
+        for (int u = 0; u < kBinUnroll; ++u)
+            if (b + 32 * u + lane < n) st[u] = cell_start[c[u]];
+#pragma unroll
+        for (int u = 0; u < kBinUnroll; ++u) {
+            const int64_t i = b + 32 * u + lane;
+            if (i < n)
+                cell_pos[(int64_t)st[u] + r[u]] =
+                    make_float4(wrap_coord(p[u].x, g.Lx), wrap_coord(p[u].y, g.Ly),
+                                wrap_coord(p[u].z, g.Lz), __int_as_float((int)i));
+        }
     }
 }
 
-__device__ __forceinline__ bool before_xi(float xa, int ia, float xb, int ib)
+// (x, index) order of wrapped atoms as one unsigned 64-bit key: x is in
+// [0, L), where the bits of a float (sign cleared, so -0 equals +0) order
+// as the values do, and indices are non-negative.
+__device__ __forceinline__ uint64_t xi_key(float x, int i)
 {
-    return xa < xb || (xa == xb && ia < ib);
+    return ((uint64_t)(__float_as_uint(x) & 0x7fffffffu) << 32) | (uint32_t)i;
 }
 
 // In-cell sort, one CTA per run of kSortCells consecutive cells (a
@@ -157,11 +197,15 @@ __device__ __forceinline__ bool before_xi(float xa, int ia, float xb, int ib)
 // writes the cell back sorted (coalesced again) and writes each cell's x
 // sub-bin table: byte b (b = 0..15) = number of the cell's atoms whose x is
 // below the cell's low x face plus b/16 of its width (bin of an atom =
-// floor((x - face) * 16 / width), clamped to 0..15), staged in shared memory
-// and stored 16 bytes per cell.  The pair search reads these to find
-// x-windows.  A cell of more than kCellSortMax atoms (its table counts would
-// not fit a byte) stays in scatter order and raises `unsorted`, which sends
-// the pair search to its per-atom path.
+// floor((x - face) * 16 / width), clamped to 0..15), stored 16 bytes per
+// cell.  The pair search reads these to find x-windows.  Entry b is also the
+// in-cell index of the first sorted atom whose bin is b or more, so the
+// atoms write the table: sorted atom k covers the entries after its
+// predecessor's bin up to its own, and the last atom the entries above its
+// bin (with the cell's count); entries before the first atom's bin stay 0.
+// A cell of more than kCellSortMax atoms (its table counts would not fit a
+// byte) stays in scatter order with a zero table and raises `unsorted`,
+// which sends the pair search to its per-atom path.
 __global__ void __launch_bounds__(kSortThreads2)
 k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_start, int64_t ncell,
             int nx, float side_x, float inv_bin, uint8_t *__restrict__ cell_tab,
@@ -169,76 +213,78 @@ k_cell_sort(float4 *__restrict__ cell_pos, const int32_t *__restrict__ cell_star
 {
     // cell starts may not be monotonic; one decision for the whole CTA
     if (__syncthreads_or(timed_out(flags))) return;
+    static_assert(kSortCells <= 256, "a staged atom's cell is kept in a byte");
     __shared__ float4 s_pos[kSortCap];
+    __shared__ uint64_t s_key[kSortCap];                     // (x bits, index): the sort key
     __shared__ uint8_t s_sbin[kSortCap];                     // bins in sorted order
+    __shared__ uint8_t s_cof[kSortCap];                      // cell of each staged slot
     __shared__ __align__(16) uint8_t s_tab[kSortCells][16];
     __shared__ int32_t s_cs[kSortCells + 1];
+    __shared__ float s_face[kSortCells];                     // low x face of each cell
+    const int t = threadIdx.x;
     const int64_t c0 = (int64_t)blockIdx.x * kSortCells;
     const int nc = (int)(ncell - c0 < kSortCells ? ncell - c0 : kSortCells);
-    for (int k = threadIdx.x; k <= nc; k += blockDim.x) s_cs[k] = cell_start[c0 + k];
+    for (int k = t; k <= nc; k += blockDim.x) s_cs[k] = cell_start[c0 + k];
+    for (int k = t; k < nc; k += blockDim.x) {
+        s_face[k] = (float)(int)((c0 + k) % nx) * side_x;
+        *reinterpret_cast<uint4 *>(s_tab[k]) = make_uint4(0u, 0u, 0u, 0u);
+    }
     __syncthreads();
     int cb = 0;
     while (cb < nc) {
         // the longest run of whole cells from cb whose atoms fit the stage
         // (at least one cell; a cell alone beyond the stage is left unsorted)
-        const int t = threadIdx.x;
         const int fit = __syncthreads_count(t >= cb && t < nc &&
                                             s_cs[t + 1] - s_cs[cb] <= kSortCap);
         const int ce = cb + (fit > 0 ? fit : 1);
         const int a0 = s_cs[cb];
         const int m = s_cs[ce] - a0;
         if (m > kSortCap) {
-            if (threadIdx.x == 0) atomicOr(unsorted, 1u);
+            if (t == 0) atomicOr(unsorted, 1u);
             cb = ce;
             continue;
         }
-        for (int k = threadIdx.x; k < m; k += blockDim.x) s_pos[k] = cell_pos[a0 + k];
+        for (int k = t; k < m; k += blockDim.x) {
+            const float4 v = cell_pos[a0 + k];
+            s_pos[k] = v;
+            s_key[k] = xi_key(v.x, __float_as_int(v.w));
+        }
+        for (int c = cb + t; c < ce; c += blockDim.x)
+            for (int q = s_cs[c] - a0; q < s_cs[c + 1] - a0; ++q) s_cof[q] = (uint8_t)c;
         __syncthreads();
-        // each atom: its cell (binary search of the stage's cell starts), its
-        // bin, and its rank by (x, index) among the cell's atoms
-        for (int k = threadIdx.x; k < m; k += blockDim.x) {
-            int lo = cb, hi = ce - 1;   // cell of atom k: s_cs[c] <= a0 + k < s_cs[c + 1]
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s_cs[mid] <= a0 + k) lo = mid; else hi = mid - 1;
-            }
-            const int c = lo;
+        // each atom: its bin and its rank by (x, index) among its cell's atoms
+        for (int k = t; k < m; k += blockDim.x) {
+            const int c = s_cof[k];
             const int s0 = s_cs[c] - a0, s1 = s_cs[c + 1] - a0;
             if (s1 - s0 > kCellSortMax) continue;   // too large: left in scatter order
             const float4 v = s_pos[k];
-            const int id = __float_as_int(v.w);
+            const uint64_t key = s_key[k];
             int r = 0;
-            for (int q = s0; q < s1; ++q) {
-                const float4 u = s_pos[q];
-                r += before_xi(u.x, __float_as_int(u.w), v.x, id) ? 1 : 0;
-            }
-            const float face = (float)(int)((c0 + c) % nx) * side_x;
-            s_sbin[s0 + r] = (uint8_t)max(0, min(15, (int)floorf((v.x - face) * inv_bin)));
+            for (int q = s0; q < s1; ++q) r += s_key[q] < key ? 1 : 0;
+            s_sbin[s0 + r] = (uint8_t)max(0, min(15, (int)floorf((v.x - s_face[c]) * inv_bin)));
             cell_pos[a0 + s0 + r] = v;
         }
         __syncthreads();
-        // tables from the bins in sorted order: entry b of a cell = number of
-        // its atoms with bin < b = the first sorted position whose bin >= b
-        for (int e = threadIdx.x; e < (ce - cb) * 16; e += blockDim.x) {
-            const int c = cb + (e >> 4), b = e & 15;
+        // the tables, written by the sorted atoms (a cell's slots are the
+        // same before and after its sort)
+        for (int k = t; k < m; k += blockDim.x) {
+            const int c = s_cof[k];
             const int s0 = s_cs[c] - a0, s1 = s_cs[c + 1] - a0;
             if (s1 - s0 > kCellSortMax) {
-                if (b == 0) atomicOr(unsorted, 1u);
-                s_tab[c][b] = 0;
+                if (k == s0) atomicOr(unsorted, 1u);
                 continue;
             }
-            int l = s0, h = s1;   // lower bound of b in s_sbin[s0, s1)
-            while (l < h) {
-                const int mid = (l + h) >> 1;
-                if (s_sbin[mid] < b) l = mid + 1; else h = mid;
-            }
-            s_tab[c][b] = (uint8_t)(l - s0);
+            const int kk = k - s0, b1 = s_sbin[k];
+            for (int b = kk > 0 ? s_sbin[k - 1] + 1 : b1 + 1; b <= b1; ++b)
+                s_tab[c][b] = (uint8_t)kk;
+            if (k == s1 - 1)
+                for (int b = b1 + 1; b < 16; ++b) s_tab[c][b] = (uint8_t)(s1 - s0);
         }
         __syncthreads();   // the stage is reused by the next run of cells
         cb = ce;
     }
     // the CTA's tables, 16 bytes per cell
-    for (int c = threadIdx.x; c < nc; c += blockDim.x)
+    for (int c = t; c < nc; c += blockDim.x)
         reinterpret_cast<uint4 *>(cell_tab)[c0 + c] = *reinterpret_cast<const uint4 *>(s_tab[c]);
 }
 
@@ -255,7 +301,9 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
     {
         ProfScope ps(ctx, PH_BIN_COUNT, s);
         if (n > 0)
-            k_bin_count<<<resident_grid(ctx, k_bin_count, 256, 0, (n + 255) / 256), 256, 0, s>>>(
+            k_bin_count<<<resident_grid(ctx, k_bin_count, 256, 0,
+                                        (n + 256 * kBinUnroll - 1) / (256 * kBinUnroll)),
+                          256, 0, s>>>(
                 pos, n, g, ctx->atom_cell, ctx->atom_rank, ctx->cell_count, ctx->ref);
         NL_CUDA_TRY(cudaGetLastError());
     }
@@ -268,9 +316,10 @@ cudaError_t launch_binning(nl_ctx *ctx, int64_t n, const float4 *pos, const Cell
     if (n <= 0) return cudaSuccess;
     {
         ProfScope ps(ctx, PH_BIN_SCATTER, s);
-        k_bin_scatter<<<resident_grid(ctx, k_bin_scatter, 256, 0, (n + 255) / 256), 256, 0, s>>>(pos, n, g, ctx->atom_cell,
-                                                             ctx->atom_rank, ctx->cell_start,
-                                                             ctx->cell_pos, ctx->flags);
+        k_bin_scatter<<<resident_grid(ctx, k_bin_scatter, 256, 0,
+                                      (n + 256 * kBinUnroll - 1) / (256 * kBinUnroll)),
+                        256, 0, s>>>(pos, n, g, ctx->atom_cell, ctx->atom_rank, ctx->cell_start,
+                                     ctx->cell_pos, ctx->flags);
         NL_CUDA_TRY(cudaGetLastError());
     }
     {
