@@ -106,33 +106,43 @@ k_cell_scan(const int32_t *__restrict__ count, int32_t *__restrict__ start, int6
         if (i < w) wbefore += s_wtot[i];
         total += s_wtot[i];
     }
-    if (t == 0) {
+    if (w == 0) {
+        // look-back by the first warp: lane l reads the status of tile
+        // j - l, so 32 predecessors are read per round; the words before the
+        // first prefix or unpublished one are aggregates to add
         uint32_t excl = 0u;
         uint32_t *st = status + tile;
         if (tile == 0) {
-            st_volatile_u32(st, kStPrefix | total);
+            if (lane == 0) st_volatile_u32(st, kStPrefix | total);
         } else {
-            st_volatile_u32(st, kStAggregate | total);
+            if (lane == 0) st_volatile_u32(st, kStAggregate | total);
             int64_t j = (int64_t)tile - 1;
             uint32_t spins = 0u;
-            while (j >= 0) {
-                const uint32_t s = ld_volatile_u32(status + j);
+            for (;;) {
+                const int64_t jj = j - lane;
+                const uint32_t s = jj >= 0 ? ld_volatile_u32(status + jj) : kStPrefix;
                 const uint32_t f = s & ~kStValue;
-                if (f == 0u) {
+                const uint32_t pre = __ballot_sync(0xffffffffu, f == kStPrefix);
+                const uint32_t stop = pre | __ballot_sync(0xffffffffu, f == 0u);
+                const int first = stop ? __ffs(stop) - 1 : 32;
+                const bool done = first < 32 && ((pre >> first) & 1u);
+                uint32_t v = (lane < first || (done && lane == first)) ? (s & kStValue) : 0u;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                excl += v;
+                if (done) break;
+                j -= first;
+                if (first < 32) {   // tile j not yet published: poll it again
                     if (++spins >= kSpinLimit) {
-                        atomicOr(flags, kFlagTimeout);
+                        if (lane == 0) atomicOr(flags, kFlagTimeout);
                         break;
                     }
                     if (spins > 64u) __nanosleep(64);
-                    continue;
                 }
-                excl += s & kStValue;
-                if (f == kStPrefix) break;
-                --j;
             }
-            st_volatile_u32(st, kStPrefix | ((excl + total) & kStValue));
+            if (lane == 0) st_volatile_u32(st, kStPrefix | ((excl + total) & kStValue));
         }
-        s_excl = excl;
+        if (lane == 0) s_excl = excl;
     }
     __syncthreads();
     uint32_t run = s_excl + wbefore + x - sum;

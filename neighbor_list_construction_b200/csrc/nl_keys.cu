@@ -138,6 +138,8 @@ __device__ __forceinline__ uint32_t quantize(float w, float S)
     return q > kQMax ? kQMax : q;
 }
 
+constexpr int kKeysUnroll = 2;
+
 template <int CURVE>
 __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, int64_t n,
                                               float Lx, float Ly, float Lz, float Sx,
@@ -168,17 +170,30 @@ __global__ void __launch_bounds__(256) k_keys(const float4 *__restrict__ pos, in
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < zero_words; i += stride)
         zero[i] = 0u;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-        const float4 p = pos[i];
-        const uint32_t qx = quantize(wrap_coord(p.x, Lx), Sx);
-        const uint32_t qy = quantize(wrap_coord(p.y, Ly), Sy);
-        const uint32_t qz = quantize(wrap_coord(p.z, Lz), Sz);
-        const uint64_t m = morton_index(qx, qy, qz);
-        const uint64_t k = CURVE == 0 ? hilbert_index(m, s_one, s_two) : m;
-        keys[i] = k;
-        vals[i] = (uint32_t)i;
-        for (int d = d0; d < d1; ++d)
-            atomicAdd(&sh[d * kRadixBins + (uint32_t)((k >> (kRadixBits * d)) & 0xffu)], 1u);
+    // kKeysUnroll atoms per thread and round: their loads first, then their
+    // table walks side by side
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n;
+         i0 += stride * kKeysUnroll) {
+        float4 p[kKeysUnroll];
+#pragma unroll
+        for (int u = 0; u < kKeysUnroll; ++u)
+            if (i0 + stride * u < n) p[u] = pos[i0 + stride * u];
+#pragma unroll
+        for (int u = 0; u < kKeysUnroll; ++u) {
+            const int64_t i = i0 + stride * u;
+            if (i < n) {
+                const uint32_t qx = quantize(wrap_coord(p[u].x, Lx), Sx);
+                const uint32_t qy = quantize(wrap_coord(p[u].y, Ly), Sy);
+                const uint32_t qz = quantize(wrap_coord(p[u].z, Lz), Sz);
+                const uint64_t m = morton_index(qx, qy, qz);
+                const uint64_t k = CURVE == 0 ? hilbert_index(m, s_one, s_two) : m;
+                keys[i] = k;
+                vals[i] = (uint32_t)i;
+                for (int d = d0; d < d1; ++d)
+                    atomicAdd(&sh[d * kRadixBins + (uint32_t)((k >> (kRadixBits * d)) & 0xffu)],
+                              1u);
+            }
+        }
     }
     __syncthreads();
     for (int i = d0 * kRadixBins + threadIdx.x; i < d1 * kRadixBins; i += blockDim.x) {
@@ -247,7 +262,7 @@ cudaError_t launch_keys(nl_ctx *ctx, int64_t n, const float4 *pos, float Lx, flo
                         const uint32_t *gate, uint32_t *zero, int64_t zero_words)
 {
     if (n <= 0) return cudaSuccess;
-    const int64_t want = (n + 255) / 256;
+    const int64_t want = (n + 256 * kKeysUnroll - 1) / (256 * kKeysUnroll);
     const unsigned blocks = curve == 0 ? resident_grid(ctx, k_keys<0>, 256, 0, want)
                                        : resident_grid(ctx, k_keys<1>, 256, 0, want);
     if (curve == 0)
