@@ -265,7 +265,7 @@ nl_status nl_last_build_info(nl_ctx *ctx, int64_t out[8]);
  * inside a framework that owns all device memory, or a plugin whose host
  * forbids allocation).  It computes exactly what nl_sort_hilbert computes,
  * with the same arguments and outputs and no context; its scratch lives in a
- * static device array inside libnl.so (about 30 MiB, held by every GPU that
+ * static device array inside libnl.so (about 28 MiB, held by every GPU that
  * loads the library until the process exits), which bounds n to at most
  * 2^20 = 1,048,576 atoms: larger n returns NL_ERR_CAPACITY without touching
  * the GPU.  The first call on each device looks up the array's device

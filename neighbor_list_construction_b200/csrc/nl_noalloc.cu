@@ -9,7 +9,7 @@
 // index ping-pong buffers, digit histograms, look-back words, tile tickets,
 // status word) in one file-scope __device__ array below instead of in a
 // context.  The array is part of the library image: every GPU that loads
-// libnl.so holds it (kNoallocScratchBytes, about 30 MiB) until the process
+// libnl.so holds it (kNoallocScratchBytes, about 28 MiB) until the process
 // exits.
 //
 // Host code cannot use the array's name as a device address (in host code it
