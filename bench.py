@@ -492,7 +492,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
     clocks.start()
     torch.cuda.set_device(local_rank)
     w = workloads.make(args.workload)
-    n, K = w.n, w.capacity
+    n, K = w.n, (args.capacity or w.capacity)
     box = w.box
     pos_host = torch.from_numpy(w.pos).pin_memory()
     pos = pos_host.cuda()
@@ -638,7 +638,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int) -> None:
         bytes_per_atom = 16 + 4 * K + 4
         alg_bytes = n * bytes_per_atom
         achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
-        traffic = pair_traffic(args.workload)
+        traffic = pair_traffic(args.workload) if K == w.capacity else None
         build_ms = sum(phases.get(p, (0.0, 0))[0] for p in
                        ("bin_count", "cell_scan", "bin_scatter", "cell_sort", "pair_search",
                         "pair_search_listed")) / args.steps
@@ -798,6 +798,9 @@ def main():
     ap.add_argument("--sharded", action="store_true",
                     help="time the pages' multi-GPU design instead of replicas: equal-count "
                          "curve shards of the one workload, halo exchange over NCCL")
+    ap.add_argument("--capacity", type=int, default=0,
+                    help="row capacity K instead of the workload's (for profiling captures that "
+                         "must stay small on the device; rows past K only count)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the rows timed after the step (replayed interval vs eager, "
                          "Hilbert vs Morton, close pairs, edge features and CSR, 8 shards)")
