@@ -232,6 +232,31 @@ def test_overflow_status_and_rows(ctx, oracle):
     gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt, full_sets=sets)
 
 
+@pytest.mark.parametrize("m", [255, 256, 700, 800])
+def test_build_crowded_cell(ctx, oracle, m):
+    """One cell holding m atoms among a uniform background: 255 is the
+    largest cell the in-cell sort orders (its sub-bin counts fill a byte),
+    256 stays in scatter order and sends the build to the per-atom search,
+    700 still fits the sort's shared-memory stage (768 atoms), 800 does
+    not.  Rows past the capacity must be members of the full sets."""
+    rng = np.random.default_rng(m)
+    L, cutoff, skin, K = 30.0, 2.5, 0.5, 320
+    bg = 2000
+    pos = np.zeros((bg + m, 4), np.float32)
+    pos[:bg, :3] = rng.random((bg, 3)) * L
+    # cells are 30/9 wide in x and 30/19 in y and z: the crowd sits inside
+    # cell (4, 9, 9), whose centre is (15, 15, 15)
+    pos[bg:, :3] = 14.8 + rng.random((m, 3)) * 0.4
+    box = np.array([L, L, L], np.float32)
+    nbr, cnt, st = gpu_build(ctx, pos, box, cutoff, skin, K)
+    full, fcnt, _ = oracle.build(pos, box, cutoff, skin, 1024)
+    assert fcnt.max() < 1024
+    o_nbr, o_cnt, o_ov = oracle.build(pos, box, cutoff, skin, K)
+    assert st == (1 if o_ov else 0)
+    sets = [set(full[i, :fcnt[i]].tolist()) for i in range(pos.shape[0])]
+    gu.assert_rows_match(nbr, cnt, o_nbr, o_cnt, full_sets=sets)
+
+
 @pytest.mark.parametrize("K", [102, 104])
 def test_build_capacity_not_multiple_of_vector(ctx, oracle, K):
     """A box large enough for the staged kernel, with a capacity that is
